@@ -1,0 +1,340 @@
+"""Pins for the fp64 oracle: checks that do not reuse its own formulas.
+
+Each test ties one oracle step to something fixed from outside it: the page
+arithmetic printed by the WorldAttention pages, closed forms, brute force on tiny
+inputs, invariants, and the textbook softmax attention of torch's
+``scaled_dot_product_attention`` (fp64 on CPU) where the method reduces to it
+(tau = 1 for the sparse branch; E = I or a row-selection E for the linear branch).
+"""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+import torch.nn.functional as F
+
+from oracle import hsa_oracle as O
+from linear_attention_paged_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def sdpa(q, k, v, mask=None):
+    """Textbook attention softmax(q k^T / sqrt(d)) v from torch, fp64, [n,d],[m,d],[m,d]."""
+    q = torch.as_tensor(q, dtype=torch.float64)[None, None]
+    k = torch.as_tensor(k, dtype=torch.float64)[None, None]
+    v = torch.as_tensor(v, dtype=torch.float64)[None, None]
+    m = None if mask is None else torch.as_tensor(mask)[None, None]
+    return F.scaled_dot_product_attention(q, k, v, attn_mask=m)[0, 0].numpy()
+
+
+def rng(seed):
+    return np.random.default_rng(seed)
+
+
+# ----------------------------------------------------------------- page arithmetic
+def test_page_arithmetic_matches_pages():
+    g = json.load(open(os.path.join(GOLDEN, "page_arithmetic.json")))
+    assert g["K_p"] * g["frames_per_page"] * g["tokens_per_frame"] == g["active_tokens"]
+    assert g["fps"] * g["seconds"] == g["frames_60s"]
+    assert g["frames_60s"] // g["frames_per_page"] == g["pages_60s"]
+    assert g["frames_60s"] * g["tokens_per_frame"] == g["tokens_60s"]
+    c1 = W.C1
+    assert c1.T_p == g["frames_per_page"] * g["tokens_per_frame"]
+    assert c1.L == g["active_tokens"]
+    assert c1.B == g["B_intra"]
+    assert c1.T_p // c1.B == g["blocks_per_page_B64"] and c1.T_p % c1.B == 0
+    assert W.C3.n_pool_pages == g["pages_60s"]
+
+
+# ----------------------------------------------------------------------------- S0
+def test_prompt_select_closed_form_angles():
+    # e_cur along axis 0; chunk m at angle theta_m in the (0,1) plane, cos = cos(theta_m)
+    D = 16
+    thetas = [1.2, 0.4, 2.5, 0.9, 0.41]
+    e_cur = np.zeros(D); e_cur[0] = 3.0
+    E = np.zeros((len(thetas), D))
+    for m, t in enumerate(thetas):
+        E[m, 0], E[m, 1] = math.cos(t) * (m + 1), math.sin(t) * (m + 1)
+    assert O.prompt_select(e_cur, E) == 1
+    assert O.prompt_margin(e_cur, E) == pytest.approx(math.cos(0.4) - math.cos(0.41), rel=1e-9)
+
+
+def test_prompt_select_scale_invariance_and_ties():
+    r = rng(1)
+    e = r.normal(size=64); E = r.normal(size=(9, 64))
+    m = O.prompt_select(e, E)
+    scales = r.uniform(0.1, 10, size=9)
+    assert O.prompt_select(e * 7.5, E * scales[:, None]) == m
+    # exact copies of the best chunk: the lowest index wins
+    E2 = np.concatenate([E[:2], E[m:m + 1], E[m:m + 1]])
+    E2[0] = -E[m]
+    assert O.prompt_select(e, E2) == 2
+    with pytest.raises(ValueError):
+        O.prompt_select(np.zeros(64), E)
+
+
+# ----------------------------------------------------------------------------- S1
+def test_page_scores_equal_mean_of_pairwise_dots():
+    # bilinearity: Qbar.Kbar = mean over all (query, key) pairs of q.k -- a different
+    # computation (pairs, not means) that pins the means, the 1/sqrt(d) and the head average
+    r = rng(2)
+    Nq, n_c, T_p, H, d = 5, 4, 6, 3, 8
+    q = r.normal(size=(Nq, H, d)); k = r.normal(size=(n_c, T_p, H, d))
+    alpha = O.page_scores(q, k)
+    for j in range(n_c):
+        acc = 0.0
+        for n in range(Nq):
+            for t in range(T_p):
+                for h in range(H):
+                    acc += float(np.dot(q[n, h], k[j, t, h]))
+        assert alpha[j] == pytest.approx(acc / (Nq * T_p * H * math.sqrt(d)), rel=1e-12, abs=1e-14)
+
+
+def test_page_scores_closed_form_constant_pages():
+    H, d, T_p = 2, 16, 10
+    u = np.linspace(-1, 1, d)
+    c = np.array([0.5, -2.0, 3.0, 1.0])
+    q = np.tile(u, (7, H, 1))
+    k = np.stack([np.tile(cj * u, (T_p, H, 1)) for cj in c])
+    alpha = O.page_scores(q, k)
+    np.testing.assert_allclose(alpha, c * float(u @ u) / math.sqrt(d), rtol=1e-13)
+    assert O.select_pages(alpha, 2) == [2, 3]
+    assert O.page_margin(alpha, 2) == pytest.approx((1.0 - 0.5) * float(u @ u) / 4.0)
+
+
+def test_select_pages_brute_force_and_invariants():
+    r = rng(3)
+    for trial in range(30):
+        n_c = int(r.integers(2, 9)); K_p = int(r.integers(1, n_c + 1))
+        alpha = r.normal(size=n_c)
+        got = O.select_pages(alpha, K_p)
+        best = max(itertools.combinations(range(n_c), K_p), key=lambda s: sum(alpha[list(s)]))
+        assert got == sorted(best)
+        # positive scaling keeps the set; negation picks the bottom-K_p
+        assert O.select_pages(alpha * 3.3, K_p) == got
+        worst = min(itertools.combinations(range(n_c), K_p), key=lambda s: sum(alpha[list(s)]))
+        assert O.select_pages(-alpha, K_p) == sorted(worst)
+    # ties go to the lower position
+    assert O.select_pages([1.0, 2.0, 1.0, 1.0], 2) == [0, 1]
+    with pytest.raises(ValueError):
+        O.select_pages([1.0, 2.0], 3)
+
+
+def test_page_selection_permutation_invariant():
+    r = rng(4)
+    Nq, n_c, T_p, H, d = 6, 6, 5, 2, 4
+    q = r.normal(size=(Nq, H, d)); k = r.normal(size=(n_c, T_p, H, d)) + r.normal(size=(n_c, 1, H, d))
+    sel = O.select_pages(O.page_scores(q, k), 3)
+    perm = r.permutation(n_c)
+    sel_p = O.select_pages(O.page_scores(q, k[perm]), 3)
+    assert sorted(perm[sel_p].tolist()) == sel
+
+
+# ----------------------------------------------------------------------------- S2
+def test_gather_is_exact_copy():
+    pool = torch.randn(6, 5, 2, 3).to(torch.bfloat16)
+    out = O.gather_pages(pool, [4, 1, 5])
+    assert out.dtype == torch.bfloat16 and out.shape == (15, 2, 3)
+    assert torch.equal(out[0:5], pool[4]) and torch.equal(out[5:10], pool[1]) and torch.equal(out[10:], pool[5])
+
+
+# ----------------------------------------------------------------------------- S3
+def test_block_means_ragged_tail_closed_form():
+    N, B = 10, 4
+    x = np.arange(N, dtype=np.float64).reshape(N, 1, 1) * np.ones((1, 2, 3))
+    m = O.block_means(x, B)
+    assert m.shape == (3, 2, 3)
+    np.testing.assert_array_equal(m[:, 0, 0], [1.5, 5.5, 8.5])  # last block = rows 8, 9 only
+
+
+def test_block_scores_equal_mean_pairwise_dots():
+    r = rng(5)
+    Nq, L, H, d, B = 7, 9, 2, 4, 4
+    q = r.normal(size=(Nq, H, d)); k = r.normal(size=(L, H, d))
+    s = O.block_scores(q, k, B)
+    for h in range(H):
+        for i in range(2):
+            rows = range(i * B, min(Nq, (i + 1) * B))
+            for j in range(3):
+                keys = range(j * B, min(L, (j + 1) * B))
+                acc = sum(float(q[a, h] @ k[b, h]) for a in rows for b in keys)
+                assert s[h, i, j] == pytest.approx(acc / (len(rows) * len(keys) * math.sqrt(d)), rel=1e-12, abs=1e-14)
+
+
+def test_select_row_brute_force_minimal_set():
+    r = rng(6)
+    for trial in range(200):
+        n = int(r.integers(1, 11))
+        s = r.normal(size=n) * r.uniform(0.1, 4)
+        tau = float(r.uniform(0.05, 0.999))
+        kept, margin = O.select_row(s, tau)
+        p = np.exp(s - s.max()); p /= p.sum()
+        assert abs(p.sum() - 1.0) < 1e-12
+        feasible = [c for m in range(1, n + 1) for c in itertools.combinations(range(n), m)
+                    if p[list(c)].sum() >= tau]
+        best_size = min(len(c) for c in feasible)
+        best_mass = max(p[list(c)].sum() for c in feasible if len(c) == best_size)
+        if margin > 1e-9:
+            assert len(kept) == best_size
+            assert p[kept].sum() == pytest.approx(best_mass, abs=1e-12)
+        assert kept == sorted(kept)
+
+
+def test_select_row_limits():
+    r = rng(7)
+    s = r.normal(size=40)
+    assert O.select_row(s, 1e-12)[0] == [int(np.argmax(s))]
+    assert O.select_row(s, 1.0)[0] == list(range(40))
+    assert O.select_row(s, 1.5)[0] == list(range(40))
+    # known weights: p = w exactly up to rounding of log/exp
+    w = np.array([0.05, 0.5, 0.15, 0.3])
+    s = np.log(w)
+    assert O.select_row(s, 0.7)[0] == [1, 3]
+    assert O.select_row(s, 0.81)[0] == [1, 2, 3]
+    assert O.select_row(s, 0.4)[0] == [1]
+    # equal scores: ties go to the lower block index
+    assert O.select_row(np.zeros(8), 0.3)[0] == [0, 1, 2]
+
+
+# ----------------------------------------------------------------------------- S4
+def test_linear_branch_identity_projection_is_dense_attention():
+    r = rng(8)
+    Nq, L, H, d = 9, 12, 2, 8
+    q = r.normal(size=(Nq, H, d)); k = r.normal(size=(L, H, d)); v = r.normal(size=(L, H, d))
+    I = np.eye(L)
+    kt, vt = O.linear_project(k, v, I, I)
+    o = O.linear_attention(q, kt, vt)
+    for h in range(H):
+        np.testing.assert_allclose(o[:, h], sdpa(q[:, h], k[:, h], v[:, h]), rtol=1e-12, atol=1e-12)
+
+
+def test_linear_branch_row_selection_pins_orientation():
+    # E[l, c] = 1 if l == idx[c]: K~ = K[idx_k], V~ = V[idx_v]  (E_K != E_V)
+    r = rng(9)
+    Nq, L, H, d, rr = 6, 20, 2, 4, 7
+    q = r.normal(size=(Nq, H, d)); k = r.normal(size=(L, H, d)); v = r.normal(size=(L, H, d))
+    ik = r.choice(L, rr, replace=False); iv = r.choice(L, rr, replace=False)
+    EK = np.zeros((L, rr)); EK[ik, np.arange(rr)] = 1
+    EV = np.zeros((L, rr)); EV[iv, np.arange(rr)] = 1
+    kt, vt = O.linear_project(k, v, EK, EV)
+    o = O.linear_attention(q, kt, vt)
+    for h in range(H):
+        np.testing.assert_allclose(o[:, h], sdpa(q[:, h], k[ik, h], v[iv, h]), rtol=1e-12, atol=1e-12)
+
+
+def test_linear_branch_rank_one_closed_form():
+    r = rng(10)
+    Nq, L, H, d, rr = 5, 16, 2, 4, 3
+    q = r.normal(size=(Nq, H, d)); k = r.normal(size=(L, H, d)); v = r.normal(size=(L, H, d))
+    E = np.ones((L, rr)) / math.sqrt(L)
+    kt, vt = O.linear_project(k, v, E, E)
+    np.testing.assert_allclose(kt[1], math.sqrt(L) * k.mean(axis=0), rtol=1e-12)
+    o = O.linear_attention(q, kt, vt)
+    # all K~ rows are equal -> uniform weights -> O_lin = V~ row = sqrt(L) * mean V
+    np.testing.assert_allclose(o, np.broadcast_to(math.sqrt(L) * v.mean(axis=0), o.shape), rtol=1e-12)
+
+
+def test_linear_project_is_linear_in_E():
+    r = rng(11)
+    L, H, d, rr = 10, 2, 3, 4
+    k = r.normal(size=(L, H, d)); v = r.normal(size=(L, H, d))
+    E1, E2 = r.normal(size=(L, rr)), r.normal(size=(L, rr))
+    a1, b1 = O.linear_project(k, v, E1, E2)
+    a2, b2 = O.linear_project(k, v, E2, E1)
+    a3, b3 = O.linear_project(k, v, E1 - 2 * E2, E2 + 0.5 * E1)
+    np.testing.assert_allclose(a3, a1 - 2 * a2, atol=1e-12)
+    np.testing.assert_allclose(b3, b1 + 0.5 * b2, atol=1e-12)
+
+
+# ----------------------------------------------------------------------------- S5
+def test_sparse_branch_all_blocks_is_dense_attention():
+    r = rng(12)
+    Nq, L, H, d, B = 11, 14, 2, 8, 4       # ragged query and key tails
+    q = r.normal(size=(Nq, H, d)); k = r.normal(size=(L, H, d)); v = r.normal(size=(L, H, d))
+    tau = np.ones(H)
+    kept, _ = O.block_select(q, k, tau, B)
+    assert all(kept[h][i] == [0, 1, 2, 3] for h in range(H) for i in range(3))
+    o = O.sparse_attention(q, k, v, kept, B)
+    for h in range(H):
+        np.testing.assert_allclose(o[:, h], sdpa(q[:, h], k[:, h], v[:, h]), rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_branch_matches_masked_dense_attention():
+    r = rng(13)
+    Nq, L, H, d, B = 10, 22, 3, 4, 4
+    q = r.normal(size=(Nq, H, d)); k = r.normal(size=(L, H, d)); v = r.normal(size=(L, H, d))
+    n_qb, n_kb = 3, 6
+    kept = [[sorted(r.choice(n_kb, int(r.integers(1, n_kb + 1)), replace=False).tolist())
+             for _ in range(n_qb)] for _ in range(H)]
+    o = O.sparse_attention(q, k, v, kept, B)
+    for h in range(H):
+        mask = np.zeros((Nq, L), dtype=bool)
+        for i in range(n_qb):
+            for j in kept[h][i]:
+                mask[i * B:(i + 1) * B, j * B:(j + 1) * B] = True
+        np.testing.assert_allclose(o[:, h], sdpa(q[:, h], k[:, h], v[:, h], mask), rtol=1e-12, atol=1e-12)
+
+
+def test_sparse_branch_single_block_identical_keys():
+    r = rng(14)
+    B, H, d = 4, 1, 6
+    q = r.normal(size=(B, H, d)); k = np.tile(r.normal(size=(1, H, d)), (3 * B, 1, 1))
+    v = r.normal(size=(3 * B, H, d))
+    o = O.sparse_attention(q, k, v, [[[1]]], B)
+    np.testing.assert_allclose(o[:, 0], np.broadcast_to(v[B:2 * B, 0].mean(axis=0), (B, d)), rtol=1e-12)
+
+
+# ----------------------------------------------------------------------------- S6
+def test_gate_limits():
+    r = rng(15)
+    a = r.normal(size=(4, 2, 3)); b = r.normal(size=(4, 2, 3))
+    np.testing.assert_allclose(O.gate_fuse(a, b, np.full((4, 2), 60.0)), a, atol=1e-20)
+    np.testing.assert_allclose(O.gate_fuse(a, b, np.full((4, 2), -60.0)), b, atol=1e-20)
+    np.testing.assert_allclose(O.gate_fuse(a, b, np.zeros((4, 2))), 0.5 * (a + b), rtol=1e-15)
+    g = r.normal(size=(4, 2))
+    np.testing.assert_allclose(O.sigmoid(g) + O.sigmoid(-g), 1.0, rtol=1e-15)
+
+
+# ----------------------------------------------------------------------------- step
+def test_step_composes_pinned_parts_on_tiny_workload():
+    cfg = W.C0.with_(T_p=64, Nq=72)
+    inp = W.make_inputs(cfg)
+    res = O.hsa_step(inp, cfg.B, cfg.K_p)
+    assert len(res["sel"]) == cfg.K_p and res["sel"] == sorted(res["sel"])
+    k_act = torch.cat([inp["k_pool"][p] for p in res["sel"]]).double().numpy()
+    v_act = torch.cat([inp["v_pool"][p] for p in res["sel"]]).double().numpy()
+    q = inp["q"].double().numpy()
+    # sparse branch = masked textbook attention; linear branch = textbook attention over
+    # the projected keys; gate by the sigmoid of g
+    h = 0
+    mask = np.zeros((cfg.Nq, cfg.L), dtype=bool)
+    for i, ks in enumerate(res["kept"][h]):
+        for j in ks:
+            mask[i * cfg.B:(i + 1) * cfg.B, j * cfg.B:(j + 1) * cfg.B] = True
+    o_sp = sdpa(q[:, h], k_act[:, h], v_act[:, h], mask)
+    EK = inp["e_k"].double().numpy(); EV = inp["e_v"].double().numpy()
+    o_lin = sdpa(q[:, h], EK.T @ k_act[:, h], EV.T @ v_act[:, h])
+    s = 1.0 / (1.0 + np.exp(-inp["gate"].double().numpy()[:, h:h + 1]))
+    np.testing.assert_allclose(res["o"][:, h], s * o_sp + (1 - s) * o_lin, rtol=1e-10, atol=1e-12)
+
+
+def test_step_sampled_rows_equal_full():
+    cfg = W.C0.with_(T_p=64, Nq=100)
+    inp = W.make_inputs(cfg)
+    full = O.hsa_step(inp, cfg.B, cfg.K_p)
+    part = O.hsa_step(inp, cfg.B, cfg.K_p, rows_of_blocks=[(0, 1), (0, 0)])
+    for (h, i), blk in part["blocks"].items():
+        np.testing.assert_allclose(blk["o"], full["o"][i * cfg.B:(i + 1) * cfg.B, h], rtol=1e-13, atol=1e-14)
+
+
+def test_prompt_selected_chunk_drives_candidates():
+    cfg = W.C0.with_(T_p=64, Nq=64, n_chunks=3, prompt_dim=32)
+    inp = W.make_inputs(cfg)
+    inp["e_cur"] = inp["e_chunks"][2] * 2.0
+    res = O.hsa_step(inp, cfg.B, cfg.K_p)
+    assert res["chunk"] == 2
+    assert set(res["sel"]) <= set(range(2 * cfg.n_c, 3 * cfg.n_c))
