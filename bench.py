@@ -1,0 +1,407 @@
+#!/usr/bin/env python
+"""Benchmark of the HSA decode step (one chunk-layer) on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one call of wa_hsa_step -- page scoring + top-4 pages, page-table
+addressing (no gather copy), head-adaptive block selection, the Linformer
+projection, the linear and block-sparse attention branches and the sigmoid gate --
+on the one-layer bf16 workload: 12 heads, d=128, 8-frame pages of 1560-token
+frames, a candidate chunk of 8 pages resident in HBM, a 3-frame query chunk (4680
+tokens), top-4 pages -> 49,920 keys, B=64, r=256.  Inputs are seeded synthetic
+tensors (see linear_attention_paged_b200/workloads.py) already resident in HBM;
+the pool read per step (>600 MB) is larger than the 126 MB L2, so no flush is
+needed between steps.
+
+Metric: attention frames/s = frames per chunk (3) / (120 chunk-layers per chunk:
+30 layers x 4 denoising steps) / ms per chunk-layer, summed over ranks (each rank
+runs its own layer: weak scaling, no data-path collective).
+
+The JSON line also carries: per-stage ms (CUDA events recorded by the library on
+the launching stream), the roofline of the dominant kernel (the block-sparse
+attention, counting selected-block FLOPs only), the HBM fraction of the page
+scoring pass, an end-to-end number through the public API with pinned host
+buffers (H2D of the step's q and gate, D2H of its output, inside the timed
+region), the clock record, and the fp64 oracle timed on the host cores on a
+bounded sample of the same workload (rank 0, N=1 only).
+
+--impl reference times that oracle alone (the reference arm: there is no
+upstream implementation of this path to install).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "HSA ms/chunk-layer & attention frames/s; % of BF16 tensor / HBM roofline"
+FRAMES_PER_CHUNK = 3
+CHUNK_LAYERS_PER_CHUNK = 30 * 4
+STAGES = ["page_retrieval", "gather", "block_select", "projection", "linear_branch", "work_list",
+          "sparse_branch_gate"]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def workload_desc(cfg):
+    return (f"{cfg.name}: one HSA decode step (chunk-layer), H={cfg.H}, d={cfg.d}, T_p={cfg.T_p} "
+            f"(8 frames x 1560 tokens), n_c={cfg.n_c} candidate pages, Nq={cfg.Nq}, K_p={cfg.K_p} "
+            f"-> L={cfg.L}, B={cfg.B}, r={cfg.r}, tau_h=0.80+0.15h/11, bf16")
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.proc = None
+        sel = []
+        try:
+            props = torch.cuda.get_device_properties(device_index)
+            bus = getattr(props, "pci_bus_id", None)
+            dom = getattr(props, "pci_domain_id", None)
+            dev = getattr(props, "pci_device_id", None)
+            if bus is not None and dom is not None and dev is not None:
+                sel = ["-i", f"{dom:08X}:{bus:02X}:{dev:02X}.0"]
+        except Exception:
+            sel = []
+        self.cmd = ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                    "-lms", "100"] + sel
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(self.cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        sm, mx, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx.append(float(r[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- oracle
+def oracle_sample(inp, cfg, n_blocks=2, head_frac=1, l_slices=8, seed=0):
+    """Time the fp64 oracle on a bounded sample of one step and scale each part to
+    the full step: page scores in full, block selection for one head (x H), the
+    projection on 1/l_slices of L (x l_slices), both attention branches for
+    n_blocks sampled (head, query block) pairs (x H*n_qb).  Returns seconds per
+    full step (estimate) and a description."""
+    from oracle import hsa_oracle as O
+    rng = np.random.default_rng(seed)
+    t = {}
+    t0 = time.perf_counter()
+    cand = [int(x) for x in inp["cand"]]
+    k_cand = np.stack([O.f64(inp["k_pool"][p]) for p in cand])
+    alpha = O.page_scores(inp["q"], k_cand)
+    sel = [cand[j] for j in O.select_pages(alpha, cfg.K_p)]
+    del k_cand
+    t["page_retrieval"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    k_act = O.gather_pages(inp["k_pool"], sel)
+    v_act = O.gather_pages(inp["v_pool"], sel)
+    t["gather"] = time.perf_counter() - t0
+    t0 = time.perf_counter()
+    h = int(rng.integers(cfg.H))
+    s = O.block_scores(inp["q"][:, h:h + 1], k_act[:, h:h + 1], cfg.B)
+    kept, _ = O.block_select(None, None, O.f64(inp["tau"])[h:h + 1], cfg.B, scores=s)
+    t["block_select"] = (time.perf_counter() - t0) * cfg.H
+    t0 = time.perf_counter()
+    Ls = cfg.L // l_slices
+    # a partial sum over L/l_slices rows: same cost per row, same output shape
+    kt, vt = O.linear_project(k_act[:Ls], v_act[:Ls], inp["e_k"][:Ls], inp["e_v"][:Ls])
+    t["projection"] = (time.perf_counter() - t0) * l_slices
+    t0 = time.perf_counter()
+    for _ in range(n_blocks):
+        i = int(rng.integers(cfg.n_qb))
+        O.sparse_attention_block(inp["q"], k_act, v_act, h, i, kept[0][i], cfg.B)
+        r0, r1 = i * cfg.B, min(cfg.Nq, (i + 1) * cfg.B)
+        O.linear_attention(O.f64(inp["q"][r0:r1, h:h + 1]), kt[:, h:h + 1], vt[:, h:h + 1])
+    t["attention"] = (time.perf_counter() - t0) / n_blocks * cfg.H * cfg.n_qb
+    total = sum(t.values())
+    desc = (f"fp64 numpy oracle on a bounded sample of one step: page scores in full, block "
+            f"selection for 1 of {cfg.H} heads (x{cfg.H}), projection on L/{l_slices} (x{l_slices}), "
+            f"both branches for {n_blocks} of {cfg.H * cfg.n_qb} (head, query block) pairs "
+            f"(x{cfg.H * cfg.n_qb // n_blocks}); per-step time extrapolated")
+    return total, desc, t
+
+
+def cores():
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count()
+
+
+def frames_per_s(ms_per_chunk_layer, n=1):
+    return n * FRAMES_PER_CHUNK / (CHUNK_LAYERS_PER_CHUNK * ms_per_chunk_layer / 1000.0)
+
+
+# ----------------------------------------------------------------------------- reference arm
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    from linear_attention_paged_b200 import workloads as W
+    cfg = W.C1
+    inp = W.make_inputs(cfg, device="cpu")
+    for _ in range(args.warmup):
+        oracle_sample(inp, cfg, n_blocks=1, seed=0)
+    ts = []
+    desc = ""
+    for k in range(args.steps):
+        tot, desc, _ = oracle_sample(inp, cfg, n_blocks=1, seed=k + 1)
+        ts.append(tot)
+    sec = float(np.mean(ts))
+    ms = sec * 1000.0
+    v = frames_per_s(ms)
+    line = {"impl": "reference", "metric": METRIC, "value": v, "unit": "frames/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg), "device": "host cpu"},
+            "cpu_baseline": {"value": v, "unit": "frames/s", "cores": cores(), "kind": "oracle",
+                             "sample": desc},
+            "e2e": {"value": v, "unit": "frames/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "gpu_launches": 0}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- our arm
+def selected_flops(mask, cfg):
+    """4 * b_q(i) * b_k(j) * d summed over kept (head, query block, key block)."""
+    m = mask.cpu().numpy().astype(np.uint32)
+    H, n_qb, W_ = m.shape
+    bq = np.array([min(cfg.Nq, (i + 1) * cfg.B) - i * cfg.B for i in range(n_qb)], dtype=np.float64)
+    bk = np.array([min(cfg.L, (j + 1) * cfg.B) - j * cfg.B for j in range(cfg.n_kb)], dtype=np.float64)
+    total = 0.0
+    kept = 0
+    for h in range(H):
+        for i in range(n_qb):
+            bits = np.unpackbits(m[h, i].view(np.uint8), bitorder="little")[:cfg.n_kb].astype(bool)
+            kept += int(bits.sum())
+            total += 4.0 * bq[i] * float(bk[bits].sum()) * cfg.d
+    return total, kept / float(H * n_qb * cfg.n_kb)
+
+
+def run_ours(args, rank, world, local_rank):
+    from linear_attention_paged_b200 import build as wb
+    if rank == 0:
+        wb.build()
+    if world > 1:
+        torch.distributed.barrier()
+    from linear_attention_paged_b200 import wa, workloads as W
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    base = W.C1
+    cfg = base.with_(seed=base.seed + 1000 * rank)     # each rank: its own layer
+    inp = W.make_inputs(cfg, device="cuda", gen_device="cuda")
+    tau = inp["tau"].cuda()
+    stream = torch.cuda.current_stream()
+
+    step = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"], inp["e_v"],
+                      tau, inp["gate"], cfg.K_p, cfg.B, fused_gather=True, keep_intermediates=True)
+    step()
+    torch.cuda.synchronize()
+    flags = wa.wa_device_error()
+    if flags:
+        raise RuntimeError(f"device error flags 0x{flags:x}")
+    flops, kept_frac = selected_flops(step.inter["blk_mask"], cfg)
+    launches_per_step = 12
+
+    n_ev = 8  # WA_STEP_EVENTS
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
+    for row in ev:                 # torch creates the CUDA event on first record
+        for e in row:
+            e.record(stream)
+    torch.cuda.synchronize()
+    ev_ptrs = [ctypes_void_array(e) for e in ev]
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+
+    clk = ClockSampler(local_rank)
+    clk.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    t_start.record(stream)
+    for k in range(args.steps):
+        step.args.stage_events = ev_ptrs[k][0]
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = clk.stop()
+    step.args.stage_events = None
+    elapsed = t_start.elapsed_time(t_end)
+    el = torch.tensor([elapsed], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(el, op=torch.distributed.ReduceOp.MAX)
+    elapsed_max = float(el.item())
+    ms_step = elapsed_max / args.steps
+
+    stage_ms = {}
+    for j, name in enumerate(STAGES):
+        stage_ms[name] = float(np.mean([ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(args.steps)]))
+    attn_ms = stage_ms["sparse_branch_gate"]
+    peaks, peak_src = load_peaks()
+    peak_t = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+    achieved_t = flops / (attn_ms * 1e-3) / 1e12
+    page_bytes = (cfg.Nq * cfg.H * cfg.d + cfg.n_c * cfg.T_p * cfg.H * cfg.d) * 2
+    hbm_achieved = page_bytes / (stage_ms["page_retrieval"] * 1e-3) / 1e9
+
+    # end to end through the public API: pinned host q/gate in, output back to the host
+    e2e_steps = max(3, min(args.steps, 50))
+    q_host = inp["q"].cpu().pin_memory()
+    g_host = inp["gate"].cpu().pin_memory()
+    o_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
+    for _ in range(2):
+        inp["q"].copy_(q_host, non_blocking=True)
+        inp["gate"].copy_(g_host, non_blocking=True)
+        step()
+        o_host.copy_(step.out, non_blocking=True)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        inp["q"].copy_(q_host, non_blocking=True)
+        inp["gate"].copy_(g_host, non_blocking=True)
+        step()
+        o_host.copy_(step.out, non_blocking=True)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_el = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(e2e_el, op=torch.distributed.ReduceOp.MAX)
+    e2e_ms = float(e2e_el.item()) / e2e_steps
+    h2d = q_host.numel() * q_host.element_size() + g_host.numel() * g_host.element_size()
+    d2h = o_host.numel() * o_host.element_size()
+
+    line = None
+    if rank == 0:
+        cpu = None
+        if world == 1 and not args.no_cpu_baseline:
+            inp_cpu = {k: (v.cpu() if isinstance(v, torch.Tensor) else v) for k, v in inp.items()}
+            sec, desc, parts = oracle_sample(inp_cpu, cfg, n_blocks=2)
+            cpu = {"value": frames_per_s(sec * 1000.0), "unit": "frames/s", "cores": cores(),
+                   "kind": "oracle", "sample": desc, "ms_per_step": sec * 1000.0,
+                   "parts_s": {k: round(v, 3) for k, v in parts.items()}}
+        line = {
+            "metric": METRIC, "value": frames_per_s(ms_step, world), "unit": "frames/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "ms_per_chunk_layer": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": workload_desc(cfg),
+                       "l2": "no flush: each step reads >600 MB (candidate keys + selected K/V), "
+                             "larger than the 126 MB L2",
+                       "parallelism": f"replicas x{world} (one layer per rank, no collective)"},
+            "roofline": {"bound": "tensor", "achieved": achieved_t, "peak": peak_t, "unit": "TFLOP/s",
+                         "frac": achieved_t / peak_t, "traffic": None,
+                         "kernel": "k_umma_attention (sparse branch + gate)",
+                         "flops_per_launch": flops, "kept_fraction": kept_frac,
+                         "peak_source": f"bf16_tflops_sustained, of {peak_src}",
+                         "frac_of_burst": achieved_t / float(peaks["bf16_tflops"])},
+            "hbm_page_scoring": {"achieved": hbm_achieved, "peak": float(peaks["hbm_gbs"]),
+                                 "unit": "GB/s", "frac": hbm_achieved / float(peaks["hbm_gbs"]),
+                                 "bytes_per_launch": page_bytes},
+            "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
+            "e2e": {"value": frames_per_s(e2e_ms, world), "unit": "frames/s", "ms_per_step": e2e_ms,
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "cpu_baseline": cpu,
+            "clocks": clocks,
+            "gpu_launches": launches_per_step * args.steps,
+            "context": {"pages_end_to_end_fps_h100": 22.0, "pages_e2e_speedup_h100": 2.21,
+                        "pages_sparse_kernel_speedup_vs_fa3_hopper": 14.02,
+                        "note": "the pages' numbers are end-to-end or relative on H100 with trained "
+                                "weights; context only, not this metric"},
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def ctypes_void_array(events):
+    import ctypes
+    arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
+    return (ctypes.cast(arr, ctypes.c_void_p), arr)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        return run_reference(args, rank, world)
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        return run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    sys.exit(main())

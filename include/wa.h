@@ -1,0 +1,238 @@
+/*
+ * wa.h -- C ABI of libwa: the Hybrid Sparse Attention (HSA) decode step of
+ * WorldAttention over Hierarchical-KV-Cache pages, for NVIDIA B200 (sm_100a).
+ *
+ * Method: "WorldAttention: An Efficient Attention Architecture for Interactive
+ * Video World Models".  Each entry point below names the section of that paper
+ * that defines what it computes.
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ *  - Tensor pointers are DEVICE pointers, owned by the caller.  The library never
+ *    allocates device memory on these paths: scratch comes from a caller-provided
+ *    workspace `ws` of at least `*_workspace_size(...)` bytes (256-byte aligned).
+ *  - `stream` is a cudaStream_t passed as void* (NULL = the legacy default stream).
+ *    Every call is asynchronous on that stream; nothing synchronises.
+ *  - Layouts are dense and token-major, row-major in the order written:
+ *      q, out          [Nq][H][d]
+ *      k_pool, v_pool  [n_pool_pages][T_p][H][d]
+ *      k_act, v_act    [L][H][d]            (L = K_p * T_p)
+ *      e_k, e_v        [L][r]               (shared by all heads)
+ *      k_til, v_til    [r][H][d]
+ *      gate            [Nq][H]   float32    (gate logits g)
+ *      tau             [H]       float32
+ *    Block b of a sequence covers rows [b*B, min(N, (b+1)*B)); the last block may be
+ *    ragged.  n_qb = ceil(Nq/B), n_kb = ceil(L/B), W = ceil(n_kb/32).
+ *  - `dtype` (WA_F32 or WA_BF16) applies to q, k/v, e_k/e_v, k_til/v_til and out.
+ *    Scores, page/block means and every quantity that decides an index (page or
+ *    block selection) are computed in float64; attention accumulates in float32.
+ *  - Supported shapes: d in {64, 128}; B = 64; for WA_BF16 also r % 64 == 0 and
+ *    r <= 256.  Others return WA_ERR_UNSUPPORTED.
+ *  - Errors: every call validates its scalar arguments on the host and returns a
+ *    wa_status; no C++ exception crosses the ABI.  `wa_last_error()` returns a
+ *    message for the calling thread's last failure.  Index arguments that live in
+ *    device memory (page ids) are checked by the kernels: an out-of-range id is
+ *    skipped and recorded in a device error word that `wa_device_error()` reads.
+ */
+#ifndef WA_H_
+#define WA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum wa_status {
+  WA_OK = 0,
+  WA_ERR_INVALID_ARG = 1,  /* a size, pointer or count is invalid                 */
+  WA_ERR_UNSUPPORTED = 2,  /* valid, but outside the shapes this build implements */
+  WA_ERR_CUDA = 3,         /* a CUDA runtime call or kernel launch failed          */
+  WA_ERR_DEVICE = 4,       /* a kernel recorded a bad device-side index            */
+  WA_ERR_WORKSPACE = 5     /* workspace NULL, too small or misaligned              */
+} wa_status;
+
+typedef enum wa_dtype { WA_F32 = 0, WA_BF16 = 1 } wa_dtype;
+
+/* Device error word bits, returned through wa_device_error's *flags. */
+#define WA_DEVERR_PAGE_ID   0x1u  /* a page id outside [0, n_pool_pages)            */
+#define WA_DEVERR_ZERO_NORM 0x2u  /* a zero-norm prompt embedding in prompt select  */
+#define WA_DEVERR_TIMEOUT   0x4u  /* a bounded wait inside a kernel gave up         */
+
+/* Message describing the calling thread's most recent failure ("" if none). */
+const char* wa_last_error(void);
+
+/* Library version string. */
+const char* wa_version(void);
+
+/* Synchronise `stream`, read and clear the current device's error word.
+ * *flags (may be NULL) receives the WA_DEVERR_* bits.  Returns WA_ERR_DEVICE when
+ * any bit was set, WA_OK otherwise. */
+wa_status wa_device_error(void* stream, uint32_t* flags);
+
+/* ---------------------------------------------------------------------------
+ * S0 -- prompt-level retrieval (WorldAttention §3.2, "Stage 1: prompt-level
+ * retrieval"): the index of the history chunk whose prompt embedding has the
+ * largest cosine similarity with the current prompt embedding (ties -> lowest).
+ *   e_cur    [D] float32        current prompt embedding
+ *   e_chunks [n_chunks][D] f32  one embedding per history chunk
+ *   chunk_out[1] int32          the chosen chunk; -1 and WA_DEVERR_ZERO_NORM when a
+ *                               norm is zero
+ * Computed in float64.  INVALID_ARG: NULL pointer, n_chunks < 1, D < 1. */
+wa_status wa_prompt_select(const float* e_cur, const float* e_chunks, int n_chunks, int D,
+                           int32_t* chunk_out, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * S1 -- page-level retrieval (WorldAttention §3.2, "Stage 2: page-level
+ * retrieval", the equation alpha_{m,j} = Qbar^T Kbar_{m,j} / sqrt(d_k)): with
+ * Qbar_h the mean query of head h over the chunk and Kbar_{h,j} the mean key of
+ * candidate page j,  alpha_j = (1/H) sum_h Qbar_h . Kbar_{h,j} / sqrt(d); the
+ * top-K_p pages (ties -> lower candidate position) are kept.
+ *   q          [Nq][H][d]                queries of the current chunk
+ *   k_pool     [n_pool_pages][T_p][H][d] key page pool
+ *   cand_pages [n_c] int32 (device)      pool page ids of the candidate chunk
+ *   alpha      [n_c] float64 (out)       page scores
+ *   sel        [K_p] int32 (out)         chosen POOL PAGE IDS, in ascending
+ *                                        candidate position (chronological order)
+ *   k_blockmean[n_c][T_p/B][H][d] f64    (out, nullable) mean key of every B-row
+ *                                        block of every candidate page; needs
+ *                                        T_p % B == 0
+ * One HBM pass over q and the candidate pages.  INVALID_ARG: K_p > n_c, sizes < 1,
+ * NULL required pointer.  A candidate id outside the pool sets WA_DEVERR_PAGE_ID. */
+size_t wa_page_score_workspace_size(int Nq, int H, int d, int n_c, int T_p, int B);
+wa_status wa_page_score(const void* q, int Nq, int H, int d,
+                        const void* k_pool, int n_pool_pages, int T_p,
+                        const int32_t* cand_pages, int n_c, int K_p, int B, wa_dtype dtype,
+                        double* alpha, int32_t* sel, double* k_blockmean,
+                        void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * S2 -- active KV construction (WorldAttention §3.2, "Active KV construction";
+ * summary step 4, the concatenation of the selected pages into K_active and
+ * V_active): k_act[s*T_p + t] = k_pool[sel[s]][t], likewise for V.  A bit-exact
+ * copy.  A page id outside the pool sets WA_DEVERR_PAGE_ID and that page is
+ * skipped. */
+wa_status wa_gather_pages(const void* k_pool, const void* v_pool, int n_pool_pages, int T_p,
+                          int H, int d, const int32_t* sel, int K_p, wa_dtype dtype,
+                          void* k_act, void* v_act, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * S3 -- head-adaptive block selection (WorldAttention §3.3, "Head-level sparsity
+ * adaptation": per head the minimal set of blocks whose cumulative attention mass
+ * reaches tau_h; summary step 5, block-pooled coarse selection).  For head h and
+ * query block i: qbar, kbar are the means over the valid rows of each block;
+ * s_j = qbar_i . kbar_j / sqrt(d); p = softmax_j(s); blocks sorted by s descending
+ * (ties -> lower j); the shortest prefix whose mass sum reaches tau_h (>=) is kept.
+ * tau_h >= 1, or a prefix sum that never reaches tau_h, keeps every block.
+ *   q           [Nq][H][d]
+ *   k_act       [L][H][d]        keys whose block means are pooled, or NULL
+ *   k_blockmean [n_kb][H][d] f64 precomputed key block means, or NULL
+ *                                (exactly one of k_act, k_blockmean is non-NULL)
+ *   tau         [H] float32
+ *   blk_idx     [H][n_qb][n_kb] int32 (out, nullable) kept blocks ascending, then -1
+ *   blk_cnt     [H][n_qb] int32 (out, nullable)       number of kept blocks
+ *   blk_mask    [H][n_qb][W] uint32 (out, nullable)   bit j of word j/32 = kept
+ * INVALID_ARG: both or neither key sources, NULL q/tau, n_kb > 8192. */
+size_t wa_block_select_workspace_size(int Nq, int H, int d, int L, int B);
+wa_status wa_block_select(const void* q, int Nq, int H, int d,
+                          const void* k_act, const double* k_blockmean, int L, int B,
+                          wa_dtype dtype, const float* tau,
+                          int32_t* blk_idx, int32_t* blk_cnt, uint32_t* blk_mask,
+                          void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * S4a -- Linformer projection of the linear branch (WorldAttention §3.3, "Linear
+ * branch": K~ = E_K^T K, V~ = E_V^T V with rank r << L, following Wang et al.
+ * 2020): k_til[c][h][:] = sum_l e_k[l][c] * k_act[l][h][:], likewise v_til.
+ * E is shared by all heads.  Accumulates in float32 (bf16 inputs on tcgen05
+ * tensor cores with split-L and an ordered reduction); the result is rounded to
+ * dtype. */
+size_t wa_linear_project_workspace_size(int L, int H, int d, int r, wa_dtype dtype);
+wa_status wa_linear_project(const void* k_act, const void* v_act, const void* e_k,
+                            const void* e_v, int L, int H, int d, int r, wa_dtype dtype,
+                            void* k_til, void* v_til, void* ws, size_t ws_bytes,
+                            void* stream);
+
+/* ---------------------------------------------------------------------------
+ * S4b + S5 + S6 -- the two attention branches and their gate (WorldAttention
+ * §3.3: "Linear branch" O_lin = softmax(Q K~^T / sqrt(d)) V~; "Sparse branch",
+ * exact attention restricted to the selected key blocks, Appendix A.1.3;
+ * "Gated fusion of two branches" with a sigmoid gate):
+ *   out[n][h] = sigmoid(g[n][h]) * O_sp[n][h] + (1 - sigmoid(g[n][h])) * O_lin[n][h]
+ *   q        [Nq][H][d]
+ *   k_act, v_act [L][H][d]
+ *   blk_mask [H][n_qb][W] uint32   key blocks kept for each (head, query block)
+ *   k_til, v_til [r][H][d]
+ *   gate     [Nq][H] float32
+ *   out      [Nq][H][d] (dtype)
+ *   o_sp, o_lin [Nq][H][d] float32 (out, nullable): the two branch outputs before
+ *                                  the gate, for identity checks
+ * A (head, query block) whose mask is empty gets O_sp = 0.  Masked key rows of a
+ * ragged last block never enter a softmax. */
+size_t wa_hsa_attention_workspace_size(int Nq, int H, int d, int L, int B, int r, wa_dtype dtype);
+wa_status wa_hsa_attention(const void* q, int Nq, int H, int d,
+                           const void* k_act, const void* v_act, int L, int B,
+                           const uint32_t* blk_mask,
+                           const void* k_til, const void* v_til, int r,
+                           const float* gate, wa_dtype dtype,
+                           void* out, float* o_sp, float* o_lin,
+                           void* ws, size_t ws_bytes, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * The whole decode step (WorldAttention §3.2 + §3.3; summary steps 2-6):
+ * S0 (when e_cur != NULL) -> S1 -> S2 (or page-table addressing) -> S3 -> S4 ->
+ * S5 -> S6, all on the device with no host round trip.
+ * With fused_gather != 0 (needs T_p % B == 0) the projection and the sparse
+ * branch read K/V straight from the pool pages through `sel`, so no K_active /
+ * V_active copy is made; otherwise the selected pages are first gathered into
+ * the workspace. */
+typedef struct wa_step_args {
+  /* S0, optional: when e_cur is NULL the candidate chunk is row 0 of chunk_pages */
+  const float* e_cur;          /* [D] float32                                  */
+  const float* e_chunks;       /* [n_chunks][D] float32                        */
+  int n_chunks;
+  int D;
+  const int32_t* chunk_pages;  /* [n_chunks][n_c] pool page ids (device)       */
+  int n_c;
+  /* queries, pool and parameters */
+  const void* q;               /* [Nq][H][d]                                   */
+  int Nq, H, d;
+  const void* k_pool;          /* [n_pool_pages][T_p][H][d]                    */
+  const void* v_pool;
+  int n_pool_pages, T_p;
+  int K_p, B, r;
+  const void* e_k;             /* [K_p*T_p][r]                                 */
+  const void* e_v;
+  const float* tau;            /* [H]                                          */
+  const float* gate;           /* [Nq][H]                                      */
+  wa_dtype dtype;
+  int fused_gather;
+  /* output */
+  void* out;                   /* [Nq][H][d]                                   */
+  /* optional outputs (NULL to skip) */
+  int32_t* chunk_out;          /* [1]                                          */
+  double* alpha_out;           /* [n_c]                                        */
+  int32_t* sel_out;            /* [K_p]                                        */
+  uint32_t* blk_mask_out;      /* [H][n_qb][W]                                 */
+  void* k_til_out;             /* [r][H][d]                                    */
+  void* v_til_out;
+  /* optional timing: NULL, or WA_STEP_EVENTS cudaEvent_t handles (as void*) that
+     are recorded on `stream` at the stage boundaries listed below */
+  void* const* stage_events;
+} wa_step_args;
+
+/* Stage boundaries recorded into wa_step_args.stage_events:
+ *   0 start | 1 after S0+S1 (page retrieval) | 2 after S2 (gather; = 1 when fused)
+ *   3 after S3 (block selection) | 4 after S4a (projection) | 5 after S4b (linear
+ *   branch) | 6 after the work list | 7 after S5+S6 (sparse branch + gate) */
+#define WA_STEP_EVENTS 8
+
+size_t wa_hsa_step_workspace_size(const wa_step_args* a);
+wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* stream);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* WA_H_ */

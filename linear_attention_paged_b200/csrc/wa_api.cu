@@ -1,0 +1,587 @@
+// wa_api.cu -- the extern "C" entry points of libwa (declared in include/wa.h):
+// host-side argument validation, workspace carving, error reporting, tensor-map
+// creation, and the sequencing of the kernels of one HSA decode step on a stream.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "wa_internal.h"
+
+#define WA_VERSION "wa 0.1.0 (sm_100a)"
+
+namespace wa {
+
+namespace {
+thread_local std::string g_last_error;
+
+// Device error word: one per device, read and cleared by wa_device_error().
+__device__ uint32_t g_err_word;
+
+std::mutex g_mu;
+uint32_t* g_err_ptr[64] = {};
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+constexpr size_t kAlign = 256;
+size_t align_up(size_t x) { return (x + kAlign - 1) & ~(kAlign - 1); }
+
+// Bump allocator over the caller's workspace (sizes are computed with the same
+// carving, so "measure" mode just counts).
+struct Carver {
+  char* base;
+  size_t used = 0;
+  explicit Carver(void* b) : base(static_cast<char*>(b)) {}
+  template <typename T>
+  T* take(size_t count) {
+    const size_t off = used;
+    used = align_up(used + count * sizeof(T));
+    return base ? reinterpret_cast<T*>(base + off) : nullptr;
+  }
+};
+
+size_t elem_size(wa_dtype dt) { return dt == WA_BF16 ? 2 : 4; }
+int ceil_div(int a, int b) { return (a + b - 1) / b; }
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+}  // namespace
+
+wa_status set_error(wa_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+wa_status check_launch(const char* what) {
+  const cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+  return WA_OK;
+}
+
+uint32_t* device_error_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_err_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_err_word) != cudaSuccess) return nullptr;
+    g_err_ptr[dev] = static_cast<uint32_t*>(p);
+  }
+  return g_err_ptr[dev];
+}
+
+bool make_tmap_bf16_2d(void* tmap, const void* base, uint64_t inner, uint64_t outer,
+                       uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer) {
+  {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_encode) {
+      void* fn = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) !=
+              cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+        return false;
+      g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    }
+  }
+  if (!aligned16(base) || row_bytes % 16 != 0) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {row_bytes};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = g_encode(static_cast<CUtensorMap*>(tmap), CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                              const_cast<void*>(base), dims, strides, box, estr,
+                              CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                              CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+}  // namespace wa
+
+using namespace wa;
+
+#define WA_REQUIRE(cond, ...)                                     \
+  do {                                                            \
+    if (!(cond)) return set_error(WA_ERR_INVALID_ARG, __VA_ARGS__); \
+  } while (0)
+#define WA_TRY(expr)                    \
+  do {                                  \
+    const wa_status s_ = (expr);        \
+    if (s_ != WA_OK) return s_;         \
+  } while (0)
+
+namespace wa_detail {
+
+wa_status check_shape(int H, int d, int B, wa_dtype dt) {
+  WA_REQUIRE(H >= 1, "H must be >= 1");
+  WA_REQUIRE(dt == WA_F32 || dt == WA_BF16, "dtype must be WA_F32 or WA_BF16");
+  if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
+  if (B != 64) return set_error(WA_ERR_UNSUPPORTED, "B must be 64 (got %d)", B);
+  const int vec = dt == WA_BF16 ? 8 : 4;
+  if ((H * d) / vec > 1024) return set_error(WA_ERR_UNSUPPORTED, "H*d too large");
+  return WA_OK;
+}
+
+wa_status check_ws(void* ws, size_t have, size_t need) {
+  if (need == 0) return WA_OK;
+  if (!ws || have < need || (reinterpret_cast<uintptr_t>(ws) & 255u))
+    return set_error(WA_ERR_WORKSPACE, "workspace needs %zu bytes, 256-byte aligned (got %zu)", need,
+                     have);
+  return WA_OK;
+}
+
+uint32_t* errw() { return device_error_word(); }
+
+// ---- S1 internals (shared by wa_page_score and wa_hsa_step)
+struct PageScoreWs {
+  double* q_blocksum;   // [n_qb][cols]
+  double* q_partial;    // [q_split][cols]
+  double* k_blocksum;   // [n_c][nbp][cols] (nullable)
+  double* k_partial;    // [n_c][k_split][cols]
+  int q_split, k_split;
+};
+
+PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks) {
+  PageScoreWs w{};
+  const int cols = H * d;
+  const int n_qb = ceil_div(Nq, B);
+  w.q_split = rowsum_splits(1, Nq, B);
+  w.k_split = rowsum_splits(n_c, T_p, B);
+  w.q_blocksum = c.take<double>(static_cast<size_t>(n_qb) * cols);
+  w.q_partial = c.take<double>(static_cast<size_t>(w.q_split) * cols);
+  w.k_blocksum = k_blocks ? c.take<double>(static_cast<size_t>(n_c) * ceil_div(T_p, B) * cols) : nullptr;
+  w.k_partial = c.take<double>(static_cast<size_t>(n_c) * w.k_split * cols);
+  return w;
+}
+
+wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int d,
+                         const void* k_pool, int n_pool_pages, int T_p, const int32_t* cand,
+                         int n_c, int K_p, int B, wa_dtype dt, double* alpha, int32_t* sel,
+                         int32_t* sel_pos, cudaStream_t st) {
+  const int cols = H * d;
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no device error word (is a CUDA device present?)");
+  WA_TRY(launch_rowblock_sum(q, dt, nullptr, 1, 1, Nq, cols, B, w.q_blocksum, w.q_partial,
+                             w.q_split, err, st));
+  WA_TRY(launch_rowblock_sum(k_pool, dt, cand, n_c, n_pool_pages, T_p, cols, B, w.k_blocksum,
+                             w.k_partial, w.k_split, err, st));
+  return launch_page_alpha_topk(w.q_partial, w.q_split, Nq, w.k_partial, w.k_split, T_p, n_c, H,
+                                d, K_p, cand, alpha, sel, sel_pos, st);
+}
+
+}  // namespace wa_detail
+using namespace wa_detail;
+
+extern "C" {
+
+const char* wa_last_error(void) { return g_last_error.c_str(); }
+const char* wa_version(void) { return WA_VERSION; }
+
+wa_status wa_device_error(void* stream, uint32_t* flags) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  uint32_t* p = errw();
+  if (!p) return set_error(WA_ERR_CUDA, "no CUDA device");
+  cudaError_t e = cudaStreamSynchronize(st);
+  if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "stream sync: %s", cudaGetErrorString(e));
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, p, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "read error word: %s", cudaGetErrorString(e));
+  if (v) cudaMemset(p, 0, sizeof(uint32_t));
+  if (flags) *flags = v;
+  if (v) return set_error(WA_ERR_DEVICE, "device error flags 0x%x", v);
+  return WA_OK;
+}
+
+// ------------------------------------------------------------------ S0
+wa_status wa_prompt_select(const float* e_cur, const float* e_chunks, int n_chunks, int D,
+                           int32_t* chunk_out, void* stream) {
+  WA_REQUIRE(e_cur && e_chunks && chunk_out, "NULL pointer");
+  WA_REQUIRE(n_chunks >= 1 && D >= 1, "n_chunks and D must be >= 1");
+  WA_REQUIRE(n_chunks <= 4096, "at most 4096 chunks");
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  return launch_prompt_select(e_cur, e_chunks, n_chunks, D, chunk_out, err,
+                              static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------ S1
+size_t wa_page_score_workspace_size(int Nq, int H, int d, int n_c, int T_p, int B) {
+  if (Nq < 1 || H < 1 || d < 1 || n_c < 1 || T_p < 1 || B < 1) return 0;
+  Carver c(nullptr);
+  carve_page_score(c, Nq, H, d, n_c, T_p, B, true);
+  c.take<int32_t>(n_c);
+  return c.used;
+}
+
+wa_status wa_page_score(const void* q, int Nq, int H, int d, const void* k_pool, int n_pool_pages,
+                        int T_p, const int32_t* cand_pages, int n_c, int K_p, int B, wa_dtype dtype,
+                        double* alpha, int32_t* sel, double* k_blockmean, void* ws, size_t ws_bytes,
+                        void* stream) {
+  WA_REQUIRE(q && k_pool && cand_pages && alpha && sel, "NULL pointer");
+  WA_REQUIRE(Nq >= 1 && T_p >= 1 && n_pool_pages >= 1 && n_c >= 1, "sizes must be >= 1");
+  WA_REQUIRE(K_p >= 1 && K_p <= n_c, "need 1 <= K_p <= n_c (K_p=%d, n_c=%d)", K_p, n_c);
+  WA_REQUIRE(n_c <= 4096, "n_c must be <= 4096");
+  WA_TRY(check_shape(H, d, B, dtype));
+  if (k_blockmean && T_p % B != 0)
+    return set_error(WA_ERR_UNSUPPORTED, "k_blockmean needs T_p %% B == 0");
+  WA_TRY(check_ws(ws, ws_bytes, wa_page_score_workspace_size(Nq, H, d, n_c, T_p, B)));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c(ws);
+  PageScoreWs w = carve_page_score(c, Nq, H, d, n_c, T_p, B, true);
+  int32_t* sel_pos = c.take<int32_t>(n_c);
+  WA_TRY(run_page_score(w, q, Nq, H, d, k_pool, n_pool_pages, T_p, cand_pages, n_c, K_p, B, dtype,
+                        alpha, sel, sel_pos, st));
+  if (k_blockmean) {
+    const size_t n = static_cast<size_t>(n_c) * (T_p / B) * H * d;
+    WA_TRY(launch_scale_copy(w.k_blocksum, k_blockmean, n, 1.0 / B, st));
+  }
+  return WA_OK;
+}
+
+// ------------------------------------------------------------------ S2
+wa_status wa_gather_pages(const void* k_pool, const void* v_pool, int n_pool_pages, int T_p, int H,
+                          int d, const int32_t* sel, int K_p, wa_dtype dtype, void* k_act,
+                          void* v_act, void* stream) {
+  WA_REQUIRE(k_pool && v_pool && sel && k_act && v_act, "NULL pointer");
+  WA_REQUIRE(n_pool_pages >= 1 && T_p >= 1 && H >= 1 && d >= 1 && K_p >= 1, "sizes must be >= 1");
+  WA_REQUIRE(dtype == WA_F32 || dtype == WA_BF16, "bad dtype");
+  const size_t page_bytes = static_cast<size_t>(T_p) * H * d * elem_size(dtype);
+  if (page_bytes % 16 != 0 || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(k_act) ||
+      !aligned16(v_act))
+    return set_error(WA_ERR_UNSUPPORTED, "gather needs 16-byte aligned pages");
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  return launch_gather(k_pool, v_pool, n_pool_pages, page_bytes, sel, K_p, k_act, v_act, err,
+                       static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------ S3
+size_t wa_block_select_workspace_size(int Nq, int H, int d, int L, int B) {
+  if (Nq < 1 || H < 1 || d < 1 || L < 1 || B < 1) return 0;
+  Carver c(nullptr);
+  const int cols = H * d;
+  c.take<double>(static_cast<size_t>(ceil_div(Nq, B)) * cols);           // q block sums
+  c.take<double>(static_cast<size_t>(rowsum_splits(1, Nq, B)) * cols);   // q partials
+  c.take<double>(static_cast<size_t>(ceil_div(L, B)) * cols);            // k block sums
+  c.take<double>(static_cast<size_t>(rowsum_splits(1, L, B)) * cols);    // k partials
+  return c.used;
+}
+
+wa_status wa_block_select(const void* q, int Nq, int H, int d, const void* k_act,
+                          const double* k_blockmean, int L, int B, wa_dtype dtype, const float* tau,
+                          int32_t* blk_idx, int32_t* blk_cnt, uint32_t* blk_mask, void* ws,
+                          size_t ws_bytes, void* stream) {
+  WA_REQUIRE(q && tau, "NULL pointer");
+  WA_REQUIRE((k_act != nullptr) != (k_blockmean != nullptr),
+             "exactly one of k_act and k_blockmean must be given");
+  WA_REQUIRE(Nq >= 1 && L >= 1, "sizes must be >= 1");
+  WA_TRY(check_shape(H, d, B, dtype));
+  const int n_kb = ceil_div(L, B);
+  WA_REQUIRE(n_kb <= 8192, "at most 8192 key blocks");
+  WA_TRY(check_ws(ws, ws_bytes, wa_block_select_workspace_size(Nq, H, d, L, B)));
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c(ws);
+  const int cols = H * d;
+  const int q_split = rowsum_splits(1, Nq, B);
+  double* qsum = c.take<double>(static_cast<size_t>(ceil_div(Nq, B)) * cols);
+  double* qpart = c.take<double>(static_cast<size_t>(q_split) * cols);
+  double* ksum = c.take<double>(static_cast<size_t>(n_kb) * cols);
+  const int k_split = rowsum_splits(1, L, B);
+  double* kpart = c.take<double>(static_cast<size_t>(k_split) * cols);
+  WA_TRY(launch_rowblock_sum(q, dtype, nullptr, 1, 1, Nq, cols, B, qsum, qpart, q_split, err, st));
+  KeyMeans km;
+  km.L = L;
+  if (k_act) {
+    WA_TRY(launch_rowblock_sum(k_act, dtype, nullptr, 1, 1, L, cols, B, ksum, kpart, k_split, err, st));
+    km.data = ksum;
+    km.is_sum = 1;
+  } else {
+    km.data = k_blockmean;
+    km.is_sum = 0;
+  }
+  return launch_block_select(qsum, Nq, H, d, B, km, n_kb, tau, blk_idx, blk_cnt, blk_mask, st);
+}
+
+// ------------------------------------------------------------------ S4a
+size_t wa_linear_project_workspace_size(int L, int H, int d, int r, wa_dtype dtype) {
+  if (L < 1 || H < 1 || d < 1 || r < 1) return 0;
+  if (dtype == WA_BF16) return align_up(umma_project_ws_bytes(L, H, d, r));
+  return 0;
+}
+
+wa_status wa_linear_project(const void* k_act, const void* v_act, const void* e_k, const void* e_v,
+                            int L, int H, int d, int r, wa_dtype dtype, void* k_til, void* v_til,
+                            void* ws, size_t ws_bytes, void* stream) {
+  WA_REQUIRE(k_act && v_act && e_k && e_v && k_til && v_til, "NULL pointer");
+  WA_REQUIRE(L >= 1 && r >= 1, "sizes must be >= 1");
+  WA_TRY(check_shape(H, d, 64, dtype));
+  WA_TRY(check_ws(ws, ws_bytes, wa_linear_project_workspace_size(L, H, d, r, dtype)));
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RowSource rs;
+  rs.k = k_act; rs.v = v_act; rs.page_rows = L; rs.n_pages = 1; rs.L = L;
+  if (dtype == WA_BF16)
+    return launch_umma_project(k_act, v_act, rs, e_k, e_v, L, H, d, r, k_til, v_til, ws, err, st);
+  WA_TRY(launch_simt_project(static_cast<const float*>(k_act), nullptr, L, 1,
+                             static_cast<const float*>(e_k), L, H * d, r,
+                             static_cast<float*>(k_til), err, st));
+  return launch_simt_project(static_cast<const float*>(v_act), nullptr, L, 1,
+                             static_cast<const float*>(e_v), L, H * d, r,
+                             static_cast<float*>(v_til), err, st);
+}
+
+// ------------------------------------------------------------------ S4b+S5+S6
+size_t wa_hsa_attention_workspace_size(int Nq, int H, int d, int L, int B, int r, wa_dtype dtype) {
+  if (Nq < 1 || H < 1 || d < 1 || L < 1 || B < 1 || r < 1) return 0;
+  Carver c(nullptr);
+  c.take<float>(static_cast<size_t>(Nq) * H * d);                  // gated linear branch
+  if (dtype == WA_BF16) c.take<char>(attn_items_ws_bytes(H, ceil_div(Nq, B)));
+  return c.used;
+}
+
+namespace wa_detail {
+wa_status run_attention(const void* q, int Nq, int H, int d, RowSource rs, int B,
+                        const uint32_t* blk_mask, const void* k_til, const void* v_til, int r,
+                        const float* gate, wa_dtype dtype, void* out, float* o_sp, float* o_lin,
+                        float* lin_ws, int4* items, cudaStream_t st,
+                        void* const* events = nullptr) {
+  auto mark = [&](int k) {
+    if (events && events[k]) cudaEventRecord(static_cast<cudaEvent_t>(events[k]), st);
+  };
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  const int n_qb = ceil_div(Nq, B);
+  const int n_kb = ceil_div(rs.L, B);
+  const int W = ceil_div(n_kb, 32);
+  RowSource lin;
+  lin.k = k_til; lin.v = v_til; lin.page_rows = r; lin.n_pages = 1; lin.L = r;
+  if (dtype == WA_BF16) {
+    WA_TRY(launch_umma_attention(0, q, Nq, H, d, lin, B, nullptr, 0, nullptr, 0, gate, lin_ws,
+                                 nullptr, o_lin, err, st));
+    mark(5);
+    WA_TRY(launch_attn_items(blk_mask, H, n_qb, n_kb, items, nullptr, st));
+    mark(6);
+    return launch_umma_attention(1, q, Nq, H, d, rs, B, blk_mask, W, items, H * ((n_qb + 1) / 2),
+                                 gate, lin_ws, out, o_sp, err, st);
+  }
+  WA_TRY(launch_simt_attention(0, static_cast<const float*>(q), Nq, H, d, lin, B, nullptr, 0, gate,
+                               lin_ws, nullptr, o_lin, err, st));
+  mark(5);
+  mark(6);
+  return launch_simt_attention(1, static_cast<const float*>(q), Nq, H, d, rs, B, blk_mask, W, gate,
+                               lin_ws, static_cast<float*>(out), o_sp, err, st);
+}
+
+wa_status check_rank(int r, wa_dtype dt) {
+  if (dt == WA_BF16 && r != 128 && r != 256)
+    return set_error(WA_ERR_UNSUPPORTED, "bf16 path needs r in {128, 256} (got %d)", r);
+  if (dt == WA_F32 && (r > 4096)) return set_error(WA_ERR_UNSUPPORTED, "r too large");
+  return WA_OK;
+}
+}  // namespace wa_detail
+using namespace wa_detail;
+
+wa_status wa_hsa_attention(const void* q, int Nq, int H, int d, const void* k_act, const void* v_act,
+                           int L, int B, const uint32_t* blk_mask, const void* k_til,
+                           const void* v_til, int r, const float* gate, wa_dtype dtype, void* out,
+                           float* o_sp, float* o_lin, void* ws, size_t ws_bytes, void* stream) {
+  WA_REQUIRE(q && k_act && v_act && blk_mask && k_til && v_til && gate && out, "NULL pointer");
+  WA_REQUIRE(Nq >= 1 && L >= 1 && r >= 1, "sizes must be >= 1");
+  WA_TRY(check_shape(H, d, B, dtype));
+  WA_TRY(check_rank(r, dtype));
+  WA_REQUIRE(ceil_div(L, B) <= 8192, "at most 8192 key blocks");
+  WA_TRY(check_ws(ws, ws_bytes, wa_hsa_attention_workspace_size(Nq, H, d, L, B, r, dtype)));
+  Carver c(ws);
+  float* lin_ws = c.take<float>(static_cast<size_t>(Nq) * H * d);
+  int4* items = dtype == WA_BF16 ? reinterpret_cast<int4*>(c.take<char>(attn_items_ws_bytes(H, ceil_div(Nq, B)))) : nullptr;
+  RowSource rs;
+  rs.k = k_act; rs.v = v_act; rs.page_rows = L; rs.n_pages = 1; rs.L = L;
+  return run_attention(q, Nq, H, d, rs, B, blk_mask, k_til, v_til, r, gate, dtype, out, o_sp, o_lin,
+                       lin_ws, items, static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------ step
+namespace wa_detail {
+struct StepWs {
+  int32_t* chunk;
+  int32_t* cand;       // candidate page ids copied from chunk_pages row
+  PageScoreWs ps;
+  double* alpha;
+  int32_t* sel;
+  int32_t* sel_pos;
+  uint32_t* mask;
+  void* k_til;
+  void* v_til;
+  void* proj;
+  float* lin;
+  int4* items;
+  void* k_act;
+  void* v_act;
+  double* ksum;     // non-fused: block sums of the gathered keys
+  double* kpart;
+};
+
+wa_status validate_step(const wa_step_args* a) {
+  WA_REQUIRE(a, "NULL args");
+  WA_REQUIRE(a->q && a->k_pool && a->v_pool && a->e_k && a->e_v && a->tau && a->gate && a->out &&
+                 a->chunk_pages,
+             "NULL pointer in wa_step_args");
+  WA_REQUIRE(a->Nq >= 1 && a->T_p >= 1 && a->n_pool_pages >= 1 && a->n_c >= 1, "sizes must be >= 1");
+  WA_REQUIRE(a->K_p >= 1 && a->K_p <= a->n_c, "need 1 <= K_p <= n_c");
+  WA_REQUIRE(a->n_c <= 4096, "n_c must be <= 4096");
+  WA_REQUIRE(!a->e_cur || (a->e_chunks && a->n_chunks >= 1 && a->n_chunks <= 4096 && a->D >= 1),
+             "bad prompt arguments");
+  WA_TRY(check_shape(a->H, a->d, a->B, a->dtype));
+  WA_TRY(check_rank(a->r, a->dtype));
+  const long long L = static_cast<long long>(a->K_p) * a->T_p;
+  WA_REQUIRE(L < (1LL << 31), "K_p*T_p too large");
+  WA_REQUIRE(ceil_div(static_cast<int>(L), a->B) <= 8192, "at most 8192 key blocks");
+  if (a->fused_gather && a->T_p % a->B != 0)
+    return set_error(WA_ERR_UNSUPPORTED, "fused gather needs T_p %% B == 0");
+  WA_REQUIRE(static_cast<long long>(a->n_pool_pages) * a->T_p < (1LL << 31), "pool too large");
+  return WA_OK;
+}
+
+StepWs carve_step(Carver& c, const wa_step_args* a) {
+  StepWs w{};
+  const int cols = a->H * a->d;
+  const int L = a->K_p * a->T_p;
+  const int n_qb = ceil_div(a->Nq, a->B), n_kb = ceil_div(L, a->B), W = ceil_div(n_kb, 32);
+  const size_t es = elem_size(a->dtype);
+  w.chunk = c.take<int32_t>(1);
+  w.cand = c.take<int32_t>(a->n_c);
+  // block sums of the candidate pages are only needed when selection reads them
+  w.ps = carve_page_score(c, a->Nq, a->H, a->d, a->n_c, a->T_p, a->B, a->fused_gather != 0);
+  w.alpha = c.take<double>(a->n_c);
+  w.sel = c.take<int32_t>(a->K_p);
+  w.sel_pos = c.take<int32_t>(a->K_p);
+  w.mask = c.take<uint32_t>(static_cast<size_t>(a->H) * n_qb * W);
+  w.k_til = c.take<char>(static_cast<size_t>(a->r) * cols * es);
+  w.v_til = c.take<char>(static_cast<size_t>(a->r) * cols * es);
+  w.proj = c.take<char>(a->dtype == WA_BF16 ? umma_project_ws_bytes(L, a->H, a->d, a->r) : 0);
+  w.lin = c.take<float>(static_cast<size_t>(a->Nq) * cols);
+  w.items = reinterpret_cast<int4*>(c.take<char>(attn_items_ws_bytes(a->H, n_qb)));
+  if (!a->fused_gather) {
+    w.k_act = c.take<char>(static_cast<size_t>(L) * cols * es);
+    w.v_act = c.take<char>(static_cast<size_t>(L) * cols * es);
+    // k block sums of the gathered buffer for selection
+    w.ksum = c.take<double>(static_cast<size_t>(n_kb) * cols);
+    w.kpart = c.take<double>(static_cast<size_t>(rowsum_splits(1, L, a->B)) * cols);
+  }
+  return w;
+}
+
+__global__ void k_pick_chunk(const int32_t* chunk_pages, int n_c, const int32_t* chunk,
+                             int n_chunks, int32_t* cand) {
+  int m = chunk ? *chunk : 0;
+  if (m < 0 || m >= n_chunks) m = 0;
+  for (int j = threadIdx.x; j < n_c; j += blockDim.x) cand[j] = chunk_pages[static_cast<size_t>(m) * n_c + j];
+}
+}  // namespace wa_detail
+using namespace wa_detail;
+
+size_t wa_hsa_step_workspace_size(const wa_step_args* a) {
+  if (!a || validate_step(a) != WA_OK) return 0;
+  Carver c(nullptr);
+  carve_step(c, a);
+  return c.used;
+}
+
+wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* stream) {
+  WA_TRY(validate_step(a));
+  const size_t need = wa_hsa_step_workspace_size(a);
+  WA_TRY(check_ws(ws, ws_bytes, need));
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Carver c(ws);
+  StepWs w = carve_step(c, a);
+  auto mark = [&](int k) {
+    if (a->stage_events && a->stage_events[k])
+      cudaEventRecord(static_cast<cudaEvent_t>(a->stage_events[k]), st);
+  };
+  mark(0);
+  const int cols = a->H * a->d;
+  const int L = a->K_p * a->T_p;
+  const int n_qb = ceil_div(a->Nq, a->B), n_kb = ceil_div(L, a->B), W = ceil_div(n_kb, 32);
+
+  // S0: candidate chunk
+  int32_t* chunk = a->chunk_out ? a->chunk_out : w.chunk;
+  const int n_chunks = a->e_cur ? a->n_chunks : 1;
+  if (a->e_cur)
+    WA_TRY(launch_prompt_select(a->e_cur, a->e_chunks, a->n_chunks, a->D, chunk, err, st));
+  k_pick_chunk<<<1, 256, 0, st>>>(a->chunk_pages, a->n_c, a->e_cur ? chunk : nullptr, n_chunks, w.cand);
+  WA_TRY(check_launch("pick_chunk"));
+  if (!a->e_cur && a->chunk_out) cudaMemsetAsync(a->chunk_out, 0, sizeof(int32_t), st);
+
+  // S1: page scores + top-K_p (+ the candidate pages' block sums, fused path)
+  double* alpha = a->alpha_out ? a->alpha_out : w.alpha;
+  int32_t* sel = a->sel_out ? a->sel_out : w.sel;
+  WA_TRY(run_page_score(w.ps, a->q, a->Nq, a->H, a->d, a->k_pool, a->n_pool_pages, a->T_p, w.cand,
+                        a->n_c, a->K_p, a->B, a->dtype, alpha, sel, w.sel_pos, st));
+
+  mark(1);
+  // S2: page table (fused) or explicit gather
+  RowSource rs;
+  KeyMeans km;
+  km.L = L;
+  km.is_sum = 1;
+  if (a->fused_gather) {
+    rs.k = a->k_pool; rs.v = a->v_pool; rs.page_ids = sel; rs.page_rows = a->T_p;
+    rs.n_pages = a->n_pool_pages; rs.L = L;
+    km.data = w.ps.k_blocksum;
+    km.page_pos = w.sel_pos;
+    km.nbp = a->T_p / a->B;
+  } else {
+    const size_t page_bytes = static_cast<size_t>(a->T_p) * cols * elem_size(a->dtype);
+    WA_TRY(launch_gather(a->k_pool, a->v_pool, a->n_pool_pages, page_bytes, sel, a->K_p, w.k_act,
+                         w.v_act, err, st));
+    rs.k = w.k_act; rs.v = w.v_act; rs.page_rows = L; rs.n_pages = 1; rs.L = L;
+    WA_TRY(launch_rowblock_sum(w.k_act, a->dtype, nullptr, 1, 1, L, cols, a->B, w.ksum, w.kpart,
+                               rowsum_splits(1, L, a->B), err, st));
+    km.data = w.ksum;
+  }
+
+  mark(2);
+  // S3: block selection
+  uint32_t* mask = a->blk_mask_out ? a->blk_mask_out : w.mask;
+  WA_TRY(launch_block_select(w.ps.q_blocksum, a->Nq, a->H, a->d, a->B, km, n_kb, a->tau, nullptr,
+                             nullptr, mask, st));
+  (void)W;
+  (void)n_qb;
+
+  mark(3);
+  // S4a: projection
+  void* kt = a->k_til_out ? a->k_til_out : w.k_til;
+  void* vt = a->v_til_out ? a->v_til_out : w.v_til;
+  if (a->dtype == WA_BF16) {
+    WA_TRY(launch_umma_project(rs.k, rs.v, rs, a->e_k, a->e_v, L, a->H, a->d, a->r, kt, vt, w.proj,
+                               err, st));
+  } else {
+    WA_TRY(launch_simt_project(static_cast<const float*>(rs.k), rs.page_ids, rs.page_rows,
+                               rs.n_pages, static_cast<const float*>(a->e_k), L, cols, a->r,
+                               static_cast<float*>(kt), err, st));
+    WA_TRY(launch_simt_project(static_cast<const float*>(rs.v), rs.page_ids, rs.page_rows,
+                               rs.n_pages, static_cast<const float*>(a->e_v), L, cols, a->r,
+                               static_cast<float*>(vt), err, st));
+  }
+  mark(4);
+  // S4b + S5 + S6
+  WA_TRY(run_attention(a->q, a->Nq, a->H, a->d, rs, a->B, mask, kt, vt, a->r, a->gate, a->dtype,
+                       a->out, nullptr, nullptr, w.lin, w.items, st, a->stage_events));
+  mark(7);
+  return WA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,108 @@
+// wa_internal.h -- declarations shared by the translation units of libwa.
+// Not part of the public ABI (see include/wa.h).
+#pragma once
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "../../include/wa.h"
+
+namespace wa {
+
+// Where the rows of a key/value sequence live.  Block j (B rows) of the active
+// sequence starts at row
+//     page_ids[j / blocks_per_page] * page_rows + (j % blocks_per_page) * B
+// of the base arrays; with page_ids == nullptr the sequence is one contiguous
+// buffer (row = j * B).  page_ids are checked against n_pages.
+struct RowSource {
+  const void* k = nullptr;
+  const void* v = nullptr;
+  const int32_t* page_ids = nullptr;  // device, nullable
+  int page_rows = 0;                  // T_p (paged) or L (contiguous)
+  int n_pages = 1;                    // pool pages addressable from k / v
+  int L = 0;                          // rows of the active sequence
+};
+
+// Status of an internal launch: WA_OK or WA_ERR_CUDA with a message set.
+wa_status set_error(wa_status s, const char* fmt, ...);
+wa_status check_launch(const char* what);
+uint32_t* device_error_word();  // current device's error word (device address)
+
+// ---------------------------------------------------------------- selection
+// S0: cosine of every chunk embedding with the current one, argmax -> chunk_out.
+wa_status launch_prompt_select(const float* e_cur, const float* e_chunks, int n_chunks, int D,
+                               int32_t* chunk_out, uint32_t* err, cudaStream_t st);
+
+// Row-block sums in float64.  Sums B-row blocks of `n_src` sources of `rows`
+// rows each (a source is a pool page given by src_ids, or the buffer itself when
+// src_ids == nullptr) over cols = H*d columns:
+//   blocksum[s][b][c]    (nullable)   sum of rows [b*B, min(rows,(b+1)*B)) of source s
+//   partial [s][split][c]             per-CTA running sums (page totals = sum over split)
+// Returns the number of splits in *n_split.
+int rowsum_splits(int n_src, int rows, int B);
+wa_status launch_rowblock_sum(const void* x, wa_dtype dt, const int32_t* src_ids, int n_src,
+                              int n_pages, int rows, int cols, int B, double* blocksum,
+                              double* partial, int n_split, uint32_t* err, cudaStream_t st);
+
+// S1 tail: alpha[c] from the q / k partials, then top-K_p -> sel (pool ids) and
+// sel_pos (candidate positions), both in ascending position.
+wa_status launch_page_alpha_topk(const double* q_partial, int q_split, int Nq,
+                                 const double* k_partial, int k_split, int T_p, int n_c,
+                                 int H, int d, int K_p, const int32_t* cand, double* alpha,
+                                 int32_t* sel, int32_t* sel_pos, cudaStream_t st);
+
+// Write k_blockmean[c][b][:] = blocksum / B for the candidate pages (T_p % B == 0).
+wa_status launch_scale_copy(const double* src, double* dst, size_t n, double scale,
+                            cudaStream_t st);
+
+// Key block means source for block selection.
+struct KeyMeans {
+  const double* data = nullptr;   // [*][cols] fp64 means or sums
+  const int32_t* page_pos = nullptr;  // nullable: block j -> row page_pos[j/nbp]*nbp + j%nbp
+  int nbp = 0;                    // blocks per page (when page_pos != nullptr)
+  int is_sum = 0;                 // data holds sums: divide by the block's row count
+  int L = 0;                      // rows of the key sequence (for ragged counts)
+};
+// S3: per (head, query block) block selection from float64 pooled means.
+size_t block_select_smem_bytes(int d, int n_kb, int* G_out);
+wa_status launch_block_select(const double* q_blocksum, int Nq, int H, int d, int B,
+                              KeyMeans km, int n_kb, const float* tau, int32_t* blk_idx,
+                              int32_t* blk_cnt, uint32_t* blk_mask, cudaStream_t st);
+
+// ---------------------------------------------------------------- gather
+wa_status launch_gather(const void* k_pool, const void* v_pool, int n_pages, size_t page_bytes,
+                        const int32_t* sel, int K_p, void* k_act, void* v_act, uint32_t* err,
+                        cudaStream_t st);
+
+// ---------------------------------------------------------------- fp32 SIMT path
+wa_status launch_simt_project(const float* x, const int32_t* page_ids, int page_rows, int n_pages,
+                              const float* e, int L, int cols, int r, float* out,
+                              uint32_t* err, cudaStream_t st);
+// mode 0: linear branch over (k_til, v_til), writes lin_ws = (1-sigmoid(g))*O_lin
+// mode 1: sparse branch over blk_mask, writes out = sigmoid(g)*O_sp + lin_ws
+wa_status launch_simt_attention(int mode, const float* q, int Nq, int H, int d, RowSource rs,
+                                int B, const uint32_t* blk_mask, int W, const float* gate,
+                                float* lin_ws, float* out, float* o_branch, uint32_t* err,
+                                cudaStream_t st);
+
+// ---------------------------------------------------------------- bf16 tcgen05 path
+size_t umma_project_ws_bytes(int L, int H, int d, int r);
+wa_status launch_umma_project(const void* k, const void* v, RowSource rs, const void* e_k,
+                              const void* e_v, int L, int H, int d, int r, void* k_til,
+                              void* v_til, void* ws, uint32_t* err, cudaStream_t st);
+
+// Work items of the tcgen05 attention: (head, query block 0, query block 1 or -1,
+// number of key blocks in the union), longest first.
+size_t attn_items_ws_bytes(int H, int n_qb);
+wa_status launch_attn_items(const uint32_t* blk_mask, int H, int n_qb, int n_kb, int4* items,
+                            void* scratch, cudaStream_t st);
+// mode 0 (linear branch): keys = k_til/v_til [r][H][d], every block, writes
+//   lin_ws[n][h][:] = (1 - sigmoid(g)) * O_lin (fp32) and o_branch (nullable).
+// mode 1 (sparse branch): keys from rs, blocks = union of the item's masks, writes
+//   out = bf16(sigmoid(g) * O_sp + lin_ws) and o_branch (nullable, O_sp fp32).
+wa_status launch_umma_attention(int mode, const void* q, int Nq, int H, int d, RowSource rs,
+                                int B, const uint32_t* blk_mask, int W, const int4* items,
+                                int n_items, const float* gate, float* lin_ws, void* out,
+                                float* o_branch, uint32_t* err, cudaStream_t st);
+
+}  // namespace wa

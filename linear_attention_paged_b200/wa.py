@@ -1,0 +1,313 @@
+"""ctypes binding of libwa (include/wa.h) with the same function names.
+
+Argument marshalling only: every step runs in the CUDA kernels of libwa.so.
+Tensors are torch tensors on the current CUDA device (contiguous, token-major,
+see include/wa.h); workspaces are carved from a per-device cached torch buffer,
+so the library itself never allocates.  Importing this module raises ImportError
+when libwa.so has not been built -- there is no fallback path.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libwa.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "wa.h")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(f"{LIB_PATH} is missing: build it with `python -m linear_attention_paged_b200.build`")
+lib = ctypes.CDLL(LIB_PATH)
+
+WA_OK, WA_ERR_INVALID_ARG, WA_ERR_UNSUPPORTED, WA_ERR_CUDA, WA_ERR_DEVICE, WA_ERR_WORKSPACE = range(6)
+WA_F32, WA_BF16 = 0, 1
+DEVERR_PAGE_ID, DEVERR_ZERO_NORM, DEVERR_TIMEOUT = 1, 2, 4
+
+c_void_p, c_int, c_size_t = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+P = c_void_p
+
+
+class WAError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed with status {status}: {msg}")
+        self.status = status
+
+
+class StepArgs(ctypes.Structure):
+    """Mirror of ``wa_step_args`` (field order and types must match include/wa.h)."""
+    _fields_ = [
+        ("e_cur", P), ("e_chunks", P), ("n_chunks", c_int), ("D", c_int),
+        ("chunk_pages", P), ("n_c", c_int),
+        ("q", P), ("Nq", c_int), ("H", c_int), ("d", c_int),
+        ("k_pool", P), ("v_pool", P), ("n_pool_pages", c_int), ("T_p", c_int),
+        ("K_p", c_int), ("B", c_int), ("r", c_int),
+        ("e_k", P), ("e_v", P), ("tau", P), ("gate", P),
+        ("dtype", c_int), ("fused_gather", c_int),
+        ("out", P),
+        ("chunk_out", P), ("alpha_out", P), ("sel_out", P), ("blk_mask_out", P),
+        ("k_til_out", P), ("v_til_out", P),
+        ("stage_events", P),
+    ]
+
+
+_SIGS = {
+    "wa_last_error": (ctypes.c_char_p, []),
+    "wa_version": (ctypes.c_char_p, []),
+    "wa_device_error": (c_int, [P, P]),
+    "wa_prompt_select": (c_int, [P, P, c_int, c_int, P, P]),
+    "wa_page_score_workspace_size": (c_size_t, [c_int] * 6),
+    "wa_page_score": (c_int, [P, c_int, c_int, c_int, P, c_int, c_int, P, c_int, c_int, c_int,
+                              c_int, P, P, P, P, c_size_t, P]),
+    "wa_gather_pages": (c_int, [P, P, c_int, c_int, c_int, c_int, P, c_int, c_int, P, P, P]),
+    "wa_block_select_workspace_size": (c_size_t, [c_int] * 5),
+    "wa_block_select": (c_int, [P, c_int, c_int, c_int, P, P, c_int, c_int, c_int, P, P, P, P,
+                                P, c_size_t, P]),
+    "wa_linear_project_workspace_size": (c_size_t, [c_int] * 5),
+    "wa_linear_project": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, c_int, P, P, P,
+                                  c_size_t, P]),
+    "wa_hsa_attention_workspace_size": (c_size_t, [c_int] * 7),
+    "wa_hsa_attention": (c_int, [P, c_int, c_int, c_int, P, P, c_int, c_int, P, P, P, c_int, P,
+                                 c_int, P, P, P, P, c_size_t, P]),
+    "wa_hsa_step_workspace_size": (c_size_t, [ctypes.POINTER(StepArgs)]),
+    "wa_hsa_step": (c_int, [ctypes.POINTER(StepArgs), P, c_size_t, P]),
+}
+for _name, (_res, _args) in _SIGS.items():
+    _f = getattr(lib, _name)
+    _f.restype = _res
+    _f.argtypes = _args
+
+
+def header_functions() -> list:
+    """Names of the functions declared in include/wa.h."""
+    txt = open(HEADER_PATH).read()
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(wa_\w+)\s*\(", txt, re.M)))
+
+
+def last_error() -> str:
+    return lib.wa_last_error().decode()
+
+
+def version() -> str:
+    return lib.wa_version().decode()
+
+
+def _check(fn: str, status: int) -> None:
+    if status != WA_OK:
+        raise WAError(fn, status, last_error())
+
+
+def _p(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return WA_F32
+    if t.dtype == torch.bfloat16:
+        return WA_BF16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+_WS: dict = {}
+
+
+def workspace(nbytes: int, device=None) -> torch.Tensor:
+    """Cached per-device scratch buffer of at least ``nbytes`` (256-byte aligned)."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    buf = _WS.get(dev)
+    if buf is None or buf.numel() < nbytes:
+        _WS.pop(dev, None)
+        buf = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
+        assert buf.data_ptr() % 256 == 0
+        _WS[dev] = buf
+    return buf
+
+
+def _need_cuda(*ts):
+    for t in ts:
+        if t is not None:
+            assert t.is_cuda and t.is_contiguous(), "tensors must be contiguous CUDA tensors"
+
+
+# --------------------------------------------------------------------- S0
+def wa_prompt_select(e_cur: torch.Tensor, e_chunks: torch.Tensor, stream=None) -> torch.Tensor:
+    _need_cuda(e_cur, e_chunks)
+    out = torch.empty(1, dtype=torch.int32, device=e_cur.device)
+    _check("wa_prompt_select", lib.wa_prompt_select(_p(e_cur), _p(e_chunks), e_chunks.shape[0],
+                                                    e_chunks.shape[1], _p(out), _stream(stream)))
+    return out
+
+
+# --------------------------------------------------------------------- S1
+def wa_page_score(q, k_pool, cand_pages, K_p: int, B: int = 64, want_blockmean: bool = False,
+                  stream=None):
+    _need_cuda(q, k_pool, cand_pages)
+    Nq, H, d = q.shape
+    P_, T_p = k_pool.shape[0], k_pool.shape[1]
+    n_c = cand_pages.numel()
+    alpha = torch.empty(n_c, dtype=torch.float64, device=q.device)
+    sel = torch.empty(K_p, dtype=torch.int32, device=q.device)
+    kbm = (torch.empty((n_c, T_p // B, H, d), dtype=torch.float64, device=q.device)
+           if want_blockmean else None)
+    nbytes = lib.wa_page_score_workspace_size(Nq, H, d, n_c, T_p, B)
+    ws = workspace(nbytes, q.device)
+    _check("wa_page_score", lib.wa_page_score(
+        _p(q), Nq, H, d, _p(k_pool), P_, T_p, _p(cand_pages), n_c, K_p, B, dtype_code(q),
+        _p(alpha), _p(sel), _p(kbm), _p(ws), nbytes, _stream(stream)))
+    return alpha, sel, kbm
+
+
+# --------------------------------------------------------------------- S2
+def wa_gather_pages(k_pool, v_pool, sel, stream=None):
+    _need_cuda(k_pool, v_pool, sel)
+    P_, T_p, H, d = k_pool.shape
+    K_p = sel.numel()
+    k_act = torch.empty((K_p * T_p, H, d), dtype=k_pool.dtype, device=k_pool.device)
+    v_act = torch.empty_like(k_act)
+    _check("wa_gather_pages", lib.wa_gather_pages(
+        _p(k_pool), _p(v_pool), P_, T_p, H, d, _p(sel), K_p, dtype_code(k_pool), _p(k_act),
+        _p(v_act), _stream(stream)))
+    return k_act, v_act
+
+
+# --------------------------------------------------------------------- S3
+def wa_block_select(q, tau, B: int = 64, k_act=None, k_blockmean=None, L: Optional[int] = None,
+                    stream=None):
+    _need_cuda(q, tau, k_act, k_blockmean)
+    Nq, H, d = q.shape
+    if L is None:
+        L = k_act.shape[0] if k_act is not None else k_blockmean.shape[0] * B
+    n_qb, n_kb = -(-Nq // B), -(-L // B)
+    W = -(-n_kb // 32)
+    idx = torch.empty((H, n_qb, n_kb), dtype=torch.int32, device=q.device)
+    cnt = torch.empty((H, n_qb), dtype=torch.int32, device=q.device)
+    mask = torch.empty((H, n_qb, W), dtype=torch.int32, device=q.device)
+    nbytes = lib.wa_block_select_workspace_size(Nq, H, d, L, B)
+    ws = workspace(nbytes, q.device)
+    _check("wa_block_select", lib.wa_block_select(
+        _p(q), Nq, H, d, _p(k_act), _p(k_blockmean), L, B, dtype_code(q), _p(tau), _p(idx),
+        _p(cnt), _p(mask), _p(ws), nbytes, _stream(stream)))
+    return idx, cnt, mask
+
+
+# --------------------------------------------------------------------- S4a
+def wa_linear_project(k_act, v_act, e_k, e_v, stream=None):
+    _need_cuda(k_act, v_act, e_k, e_v)
+    L, H, d = k_act.shape
+    r = e_k.shape[1]
+    k_til = torch.empty((r, H, d), dtype=k_act.dtype, device=k_act.device)
+    v_til = torch.empty_like(k_til)
+    dt = dtype_code(k_act)
+    nbytes = lib.wa_linear_project_workspace_size(L, H, d, r, dt)
+    ws = workspace(nbytes, k_act.device)
+    _check("wa_linear_project", lib.wa_linear_project(
+        _p(k_act), _p(v_act), _p(e_k), _p(e_v), L, H, d, r, dt, _p(k_til), _p(v_til), _p(ws),
+        nbytes, _stream(stream)))
+    return k_til, v_til
+
+
+# --------------------------------------------------------------------- S4b+S5+S6
+def wa_hsa_attention(q, k_act, v_act, blk_mask, k_til, v_til, gate, B: int = 64,
+                     want_branches: bool = False, stream=None):
+    _need_cuda(q, k_act, v_act, blk_mask, k_til, v_til, gate)
+    Nq, H, d = q.shape
+    L = k_act.shape[0]
+    r = k_til.shape[0]
+    dt = dtype_code(q)
+    out = torch.empty_like(q)
+    o_sp = torch.empty(q.shape, dtype=torch.float32, device=q.device) if want_branches else None
+    o_lin = torch.empty(q.shape, dtype=torch.float32, device=q.device) if want_branches else None
+    nbytes = lib.wa_hsa_attention_workspace_size(Nq, H, d, L, B, r, dt)
+    ws = workspace(nbytes, q.device)
+    _check("wa_hsa_attention", lib.wa_hsa_attention(
+        _p(q), Nq, H, d, _p(k_act), _p(v_act), L, B, _p(blk_mask), _p(k_til), _p(v_til), r,
+        _p(gate), dt, _p(out), _p(o_sp), _p(o_lin), _p(ws), nbytes, _stream(stream)))
+    return (out, o_sp, o_lin) if want_branches else out
+
+
+# --------------------------------------------------------------------- step
+class HSAStep:
+    """A prepared decode step: the argument block, outputs and workspace are built
+    once; ``__call__`` is a single wa_hsa_step launch sequence on the stream."""
+
+    def __init__(self, q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 4,
+                 B: int = 64, e_cur=None, e_chunks=None, fused_gather: bool = True,
+                 keep_intermediates: bool = False, out=None):
+        _need_cuda(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, e_cur, e_chunks)
+        Nq, H, d = q.shape
+        P_, T_p = k_pool.shape[0], k_pool.shape[1]
+        if chunk_pages.dim() == 1:
+            chunk_pages = chunk_pages.reshape(1, -1)
+        n_chunks, n_c = chunk_pages.shape
+        r = e_k.shape[1]
+        L = K_p * T_p
+        n_qb, n_kb = -(-Nq // B), -(-L // B)
+        W = -(-n_kb // 32)
+        dev = q.device
+        self.out = out if out is not None else torch.empty_like(q)
+        self._keep = [q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, e_cur, e_chunks]
+        a = StepArgs()
+        a.e_cur, a.e_chunks = _p(e_cur), _p(e_chunks)
+        a.n_chunks = n_chunks if e_cur is not None else 0
+        a.D = e_cur.numel() if e_cur is not None else 0
+        a.chunk_pages, a.n_c = _p(chunk_pages), n_c
+        a.q, a.Nq, a.H, a.d = _p(q), Nq, H, d
+        a.k_pool, a.v_pool, a.n_pool_pages, a.T_p = _p(k_pool), _p(v_pool), P_, T_p
+        a.K_p, a.B, a.r = K_p, B, r
+        a.e_k, a.e_v, a.tau, a.gate = _p(e_k), _p(e_v), _p(tau), _p(gate)
+        a.dtype, a.fused_gather = dtype_code(q), int(bool(fused_gather))
+        a.out = _p(self.out)
+        self.inter = {}
+        if keep_intermediates:
+            self.inter = dict(
+                chunk=torch.empty(1, dtype=torch.int32, device=dev),
+                alpha=torch.empty(n_c, dtype=torch.float64, device=dev),
+                sel=torch.empty(K_p, dtype=torch.int32, device=dev),
+                blk_mask=torch.empty((H, n_qb, W), dtype=torch.int32, device=dev),
+                k_til=torch.empty((r, H, d), dtype=q.dtype, device=dev),
+                v_til=torch.empty((r, H, d), dtype=q.dtype, device=dev))
+            a.chunk_out = _p(self.inter["chunk"])
+            a.alpha_out = _p(self.inter["alpha"])
+            a.sel_out = _p(self.inter["sel"])
+            a.blk_mask_out = _p(self.inter["blk_mask"])
+            a.k_til_out = _p(self.inter["k_til"])
+            a.v_til_out = _p(self.inter["v_til"])
+        self.args = a
+        nbytes = lib.wa_hsa_step_workspace_size(ctypes.byref(a))
+        if nbytes == 0:
+            # a zero size means validation failed: surface the reason
+            _check("wa_hsa_step_workspace_size", lib.wa_hsa_step(ctypes.byref(a), None, 0, None))
+        self.nbytes = nbytes
+        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        assert self.ws.data_ptr() % 256 == 0
+
+    def __call__(self, stream=None):
+        _check("wa_hsa_step", lib.wa_hsa_step(ctypes.byref(self.args), _p(self.ws), self.nbytes,
+                                              _stream(stream)))
+        return self.out
+
+
+def wa_hsa_step(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 4, B: int = 64,
+                e_cur=None, e_chunks=None, fused_gather: bool = True, keep_intermediates: bool = False,
+                stream=None):
+    """One HSA decode step; returns ``out`` (and the intermediates when asked)."""
+    st = HSAStep(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p, B, e_cur, e_chunks,
+                 fused_gather, keep_intermediates)
+    out = st(stream)
+    return (out, st.inter) if keep_intermediates else out
+
+
+def wa_device_error(stream=None) -> int:
+    """Synchronise, read and clear the device error word; returns its WA_DEVERR_* bits."""
+    flags = ctypes.c_uint32(0)
+    lib.wa_device_error(_stream(stream), ctypes.byref(flags))
+    return int(flags.value)

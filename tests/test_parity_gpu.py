@@ -1,0 +1,273 @@
+"""GPU parity: every libwa entry point against the float64 oracle on the same seeded
+inputs.  Small shapes span several tiles with ragged query (and key) tails; the
+one-layer bf16 workload runs at full size in the launch configuration the bench
+times (the fused page-table step) and is checked on sampled (head, query block)
+outputs plus every page / block selection."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import hsa_oracle as O
+from linear_attention_paged_b200 import workloads as W
+from tests.helpers import (assert_close, compare_selection, mask_to_sets, kept_fraction, to64)
+
+pytestmark = pytest.mark.gpu
+
+# small multi-tile shapes (ragged query tails; odd n_qb leaves one unpaired block)
+SMALL_BF16 = W.HSAConfig("small_bf16", H=2, d=128, T_p=1280, n_c=6, Nq=520, K_p=3, B=64, r=128,
+                         dtype="bf16", seed=11, recipe="offset")
+SMALL_BF16_D64 = W.HSAConfig("small_bf16_d64", H=4, d=64, T_p=640, n_c=5, Nq=300, K_p=2, B=64,
+                             r=256, dtype="bf16", seed=12, recipe="offset")
+SMALL_STRESS = W.HSAConfig("small_stress", H=4, d=128, T_p=1280, n_c=4, Nq=640, K_p=2, B=64, r=128,
+                           dtype="bf16", seed=13, recipe="stress", hot_beta_scale=12.0)
+SMALL_F32 = W.HSAConfig("small_f32", H=2, d=128, T_p=320, n_c=4, Nq=150, K_p=2, B=64, r=48,
+                        dtype="f32", seed=14, recipe="offset")
+
+
+@pytest.fixture(scope="module")
+def wa():
+    from linear_attention_paged_b200 import build
+    build.build()
+    from linear_attention_paged_b200 import wa as _wa
+    return _wa
+
+
+def inputs(cfg, device="cuda"):
+    return W.make_inputs(cfg, device=device)
+
+
+def dkey(cfg):
+    return "f32" if cfg.dtype == "f32" else "bf16"
+
+
+def check_device_ok(wa):
+    flags = wa.wa_device_error()
+    assert flags == 0, f"device error flags 0x{flags:x}"
+
+
+# ---------------------------------------------------------------- S0
+def test_prompt_select(wa):
+    g = torch.Generator().manual_seed(5)
+    e = torch.randn(4096, generator=g)
+    E = torch.randn(15, 4096, generator=g)
+    E[9] = e * 0.5 + E[9] * 0.1
+    got = int(wa.wa_prompt_select(e.cuda(), E.cuda()).item())
+    assert got == O.prompt_select(e, E) == 9
+    for s in range(5):
+        E = torch.randn(40, 512, generator=g)
+        e = torch.randn(512, generator=g)
+        assert int(wa.wa_prompt_select(e.cuda(), E.cuda()).item()) == O.prompt_select(e, E)
+    check_device_ok(wa)
+
+
+def test_prompt_select_zero_norm_flags(wa):
+    E = torch.randn(4, 64)
+    E[2] = 0
+    out = wa.wa_prompt_select(torch.randn(64).cuda(), E.cuda())
+    assert int(out.item()) == -1
+    assert wa.wa_device_error() & wa.DEVERR_ZERO_NORM
+
+
+# ---------------------------------------------------------------- S1 + S2
+@pytest.mark.parametrize("cfg", [W.C0, SMALL_BF16, SMALL_BF16_D64, SMALL_F32], ids=lambda c: c.name)
+def test_page_score_and_gather(wa, cfg):
+    inp = inputs(cfg)
+    alpha, sel, kbm = wa.wa_page_score(inp["q"], inp["k_pool"], inp["cand"], cfg.K_p, cfg.B,
+                                       want_blockmean=True)
+    k_cand = np.stack([to64(inp["k_pool"][int(p)]) for p in inp["cand"].cpu()])
+    a_ref = O.page_scores(inp["q"], k_cand)
+    np.testing.assert_allclose(to64(alpha), a_ref, rtol=1e-10, atol=1e-13)
+    margin = O.page_margin(a_ref, cfg.K_p)
+    ref_sel = [int(inp["cand"][j]) for j in O.select_pages(a_ref, cfg.K_p)]
+    if margin >= 1e-5:
+        assert sel.cpu().tolist() == ref_sel
+    # block means of every candidate page
+    ref_bm = np.stack([O.block_means(k_cand[c], cfg.B) for c in range(cfg.n_c)])
+    np.testing.assert_allclose(to64(kbm), ref_bm, rtol=1e-10, atol=1e-13)
+    # gather: a bit-exact copy
+    k_act, v_act = wa.wa_gather_pages(inp["k_pool"], inp["v_pool"], sel)
+    assert torch.equal(k_act, O.gather_pages(inp["k_pool"], sel.cpu().tolist()))
+    assert torch.equal(v_act, O.gather_pages(inp["v_pool"], sel.cpu().tolist()))
+    check_device_ok(wa)
+
+
+def test_page_score_bad_page_id_is_flagged(wa):
+    cfg = SMALL_BF16
+    inp = inputs(cfg)
+    cand = inp["cand"].clone()
+    cand[1] = cfg.n_pool_pages + 5            # outside the pool: skipped and recorded
+    wa.wa_page_score(inp["q"], inp["k_pool"], cand, cfg.K_p, cfg.B)
+    assert wa.wa_device_error() & wa.DEVERR_PAGE_ID
+    sel = torch.tensor([0, 99], dtype=torch.int32, device="cuda")
+    wa.wa_gather_pages(inp["k_pool"], inp["v_pool"], sel)
+    assert wa.wa_device_error() & wa.DEVERR_PAGE_ID
+
+
+# ---------------------------------------------------------------- S3
+@pytest.mark.parametrize("cfg", [W.C0, SMALL_BF16, SMALL_BF16_D64, SMALL_STRESS, SMALL_F32],
+                         ids=lambda c: c.name)
+def test_block_select(wa, cfg):
+    inp = inputs(cfg)
+    sel = [int(x) for x in inp["cand"][: cfg.K_p].cpu()]
+    k_act = O.gather_pages(inp["k_pool"], sel)
+    kept, margin = O.block_select(inp["q"], k_act, inp["tau"], cfg.B)
+    idx, cnt, mask = wa.wa_block_select(inp["q"], inp["tau"].cuda(), cfg.B, k_act=k_act)
+    gpu = mask_to_sets(mask, cfg.n_kb)
+    compare_selection(gpu, kept, margin, f"{cfg.name} block masks")
+    # index lists and counts agree with the mask
+    idx_c, cnt_c = idx.cpu().numpy(), cnt.cpu().numpy()
+    for h in range(cfg.H):
+        for i in range(cfg.n_qb):
+            c = int(cnt_c[h, i])
+            assert idx_c[h, i, :c].tolist() == gpu[h][i]
+            assert (idx_c[h, i, c:] == -1).all()
+    print(f"[info] {cfg.name} kept fraction per head: {np.round(kept_fraction(kept, cfg.n_kb), 3)}")
+    # the same from precomputed block means
+    kbm = torch.from_numpy(O.block_means(k_act, cfg.B)).cuda()
+    _, _, mask2 = wa.wa_block_select(inp["q"], inp["tau"].cuda(), cfg.B, k_blockmean=kbm, L=cfg.L)
+    compare_selection(mask_to_sets(mask2, cfg.n_kb), kept, margin, f"{cfg.name} masks from means")
+    check_device_ok(wa)
+
+
+def test_block_select_limits(wa):
+    cfg = SMALL_BF16
+    inp = inputs(cfg)
+    k_act = O.gather_pages(inp["k_pool"], [0, 1, 2])
+    for tval, expect in ((1.0, "all"), (1e-9, "one")):
+        tau = torch.full((cfg.H,), tval, dtype=torch.float32, device="cuda")
+        _, cnt, mask = wa.wa_block_select(inp["q"], tau, cfg.B, k_act=k_act)
+        c = cnt.cpu().numpy()
+        if expect == "all":
+            assert (c == cfg.n_kb).all()
+        else:
+            assert (c == 1).all()
+            s = O.block_scores(inp["q"], k_act, cfg.B)
+            gpu = mask_to_sets(mask, cfg.n_kb)
+            for h in range(cfg.H):
+                for i in range(cfg.n_qb):
+                    assert gpu[h][i] == [int(np.argmax(s[h, i]))]
+
+
+# ---------------------------------------------------------------- S4a
+@pytest.mark.parametrize("cfg", [W.C0, SMALL_BF16, SMALL_BF16_D64, SMALL_F32], ids=lambda c: c.name)
+def test_linear_project(wa, cfg):
+    inp = inputs(cfg)
+    sel = [int(x) for x in inp["cand"][: cfg.K_p].cpu()]
+    k_act = O.gather_pages(inp["k_pool"], sel)
+    v_act = O.gather_pages(inp["v_pool"], sel)
+    kt, vt = wa.wa_linear_project(k_act, v_act, inp["e_k"], inp["e_v"])
+    kr, vr = O.linear_project(k_act, v_act, inp["e_k"], inp["e_v"])
+    assert_close(kt, kr, dkey(cfg), f"{cfg.name} K~")
+    assert_close(vt, vr, dkey(cfg), f"{cfg.name} V~")
+    check_device_ok(wa)
+
+
+# ---------------------------------------------------------------- S4b + S5 + S6
+@pytest.mark.parametrize("cfg", [W.C0, SMALL_BF16, SMALL_BF16_D64, SMALL_STRESS, SMALL_F32],
+                         ids=lambda c: c.name)
+def test_hsa_attention(wa, cfg):
+    inp = inputs(cfg)
+    sel = [int(x) for x in inp["cand"][: cfg.K_p].cpu()]
+    k_act = O.gather_pages(inp["k_pool"], sel)
+    v_act = O.gather_pages(inp["v_pool"], sel)
+    kept, margin = O.block_select(inp["q"], k_act, inp["tau"], cfg.B)
+    _, _, mask = wa.wa_block_select(inp["q"], inp["tau"].cuda(), cfg.B, k_act=k_act)
+    compare_selection(mask_to_sets(mask, cfg.n_kb), kept, margin, f"{cfg.name} masks")
+    kt, vt = O.linear_project(k_act, v_act, inp["e_k"], inp["e_v"])
+    # the branches take the projected keys in the input dtype
+    kt_in = torch.from_numpy(kt).to(cfg.torch_dtype).cuda()
+    vt_in = torch.from_numpy(vt).to(cfg.torch_dtype).cuda()
+    out, o_sp, o_lin = wa.wa_hsa_attention(inp["q"], k_act, v_act, mask, kt_in, vt_in, inp["gate"],
+                                           cfg.B, want_branches=True)
+    ref_sp = O.sparse_attention(inp["q"], k_act, v_act, kept, cfg.B)
+    ref_lin = O.linear_attention(inp["q"], kt_in, vt_in)
+    ref = O.gate_fuse(ref_sp, ref_lin, inp["gate"])
+    assert_close(o_lin, ref_lin, dkey(cfg), f"{cfg.name} O_lin")
+    assert_close(o_sp, ref_sp, dkey(cfg), f"{cfg.name} O_sp")
+    assert_close(out, ref, dkey(cfg), f"{cfg.name} O")
+    check_device_ok(wa)
+
+
+def test_hsa_attention_identities(wa):
+    """tau = 1 gives dense attention; an empty mask gives O_sp = 0; a ragged key tail."""
+    cfg = SMALL_BF16.with_(seed=21)
+    inp = inputs(cfg)
+    L = 1000                                      # not a multiple of B: masked key tail
+    k_act = O.gather_pages(inp["k_pool"], [0])[:L].contiguous()
+    v_act = O.gather_pages(inp["v_pool"], [0])[:L].contiguous()
+    n_kb = -(-L // cfg.B)
+    ones = torch.ones(cfg.H, dtype=torch.float32, device="cuda")
+    _, cnt, mask = wa.wa_block_select(inp["q"], ones, cfg.B, k_act=k_act)
+    assert (cnt.cpu() == n_kb).all()
+    e = torch.randn(L, cfg.r, generator=torch.Generator().manual_seed(3)) / math.sqrt(L)
+    e = e.to(torch.bfloat16).cuda()
+    kt, vt = wa.wa_linear_project(k_act, v_act, e, e)
+    out, o_sp, o_lin = wa.wa_hsa_attention(inp["q"], k_act, v_act, mask, kt, vt, inp["gate"], cfg.B,
+                                           want_branches=True)
+    dense = O.sparse_attention(inp["q"], k_act, v_act, [[list(range(n_kb))] * cfg.n_qb] * cfg.H, cfg.B)
+    assert_close(o_sp, dense, "bf16", "tau=1 sparse branch = dense attention")
+    zero = torch.zeros_like(mask)
+    out0, o_sp0, o_lin0 = wa.wa_hsa_attention(inp["q"], k_act, v_act, zero, kt, vt, inp["gate"], cfg.B,
+                                              want_branches=True)
+    assert float(o_sp0.abs().max()) == 0.0
+    s = torch.sigmoid(inp["gate"]).unsqueeze(-1)
+    assert_close(out0, (1 - s) * o_lin0, "bf16", "empty mask -> (1 - sigmoid(g)) O_lin")
+    check_device_ok(wa)
+
+
+# ---------------------------------------------------------------- whole step
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "gathered"])
+@pytest.mark.parametrize("cfg", [W.C0, SMALL_BF16, SMALL_BF16_D64, SMALL_F32], ids=lambda c: c.name)
+def test_hsa_step_small(wa, cfg, fused):
+    inp = inputs(cfg)
+    out, inter = wa.wa_hsa_step(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"],
+                                inp["e_v"], inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B,
+                                fused_gather=fused, keep_intermediates=True)
+    res = O.hsa_step(inp, cfg.B, cfg.K_p)
+    if res["page_margin"] >= 1e-5:
+        assert inter["sel"].cpu().tolist() == res["sel"]
+    compare_selection(mask_to_sets(inter["blk_mask"], cfg.n_kb), res["kept"], res["block_margin"],
+                      f"{cfg.name} step masks")
+    assert_close(inter["k_til"], res["k_til"], dkey(cfg), f"{cfg.name} step K~")
+    assert_close(out, res["o"], dkey(cfg), f"{cfg.name} step O ({'fused' if fused else 'gathered'})")
+    check_device_ok(wa)
+
+
+def _full_size_step(wa, cfg, samples, gen_device="cuda"):
+    inp = W.make_inputs(cfg, device="cuda", gen_device=gen_device)
+    e_cur = inp.get("e_cur")
+    step = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"], inp["e_v"],
+                      inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B, e_cur=e_cur,
+                      e_chunks=inp.get("e_chunks"), fused_gather=True, keep_intermediates=True)
+    out = step()
+    torch.cuda.synchronize()
+    res = O.hsa_step(inp, cfg.B, cfg.K_p, rows_of_blocks=samples)
+    if "chunk" in res:
+        assert int(step.inter["chunk"].item()) == res["chunk"]
+    np.testing.assert_allclose(to64(step.inter["alpha"]), res["alpha"], rtol=1e-9, atol=1e-13)
+    if res["page_margin"] >= 1e-5:
+        assert step.inter["sel"].cpu().tolist() == res["sel"]
+    compare_selection(mask_to_sets(step.inter["blk_mask"], cfg.n_kb), res["kept"], res["block_margin"],
+                      f"{cfg.name} masks")
+    print(f"[info] {cfg.name} kept fraction per head: {np.round(kept_fraction(res['kept'], cfg.n_kb), 3)}")
+    assert_close(step.inter["k_til"], res["k_til"], "bf16", f"{cfg.name} K~")
+    assert_close(step.inter["v_til"], res["v_til"], "bf16", f"{cfg.name} V~")
+    for (h, i), blk in res["blocks"].items():
+        r0, r1 = i * cfg.B, min(cfg.Nq, (i + 1) * cfg.B)
+        assert_close(out[r0:r1, h], blk["o"], "bf16", f"{cfg.name} O[h={h}, block {i}]")
+    check_device_ok(wa)
+
+
+def test_full_size_layer_step(wa):
+    cfg = W.C1
+    n_qb = cfg.n_qb
+    samples = [(0, 0), (11, n_qb - 1), (5, 37), (3, n_qb - 2), (8, 12), (11, 0)]
+    _full_size_step(wa, cfg, samples)
+
+
+def test_full_size_stress_step(wa):
+    cfg = W.C2
+    samples = [(0, 0), (4, cfg.n_qb - 1), (7, 20), (11, 50)]
+    _full_size_step(wa, cfg, samples)
