@@ -239,7 +239,7 @@ def run_ours(args, rank, world, local_rank):
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
-    base = W.C1
+    base = W.C1 if args.heads is None else W.C1.with_(name=f"c1_layer_bf16_h{args.heads}", H=args.heads)
     cfg = base.with_(seed=base.seed + 1000 * rank)     # each rank: its own layer
     inp = W.make_inputs(cfg, device="cuda", gen_device="cuda")
     tau = inp["tau"].cuda()
@@ -301,11 +301,11 @@ def run_ours(args, rank, world, local_rank):
     hbm_achieved = page_bytes / (stage_ms["page_retrieval"] * 1e-3) / 1e9
 
     # end to end through the public API: pinned host q/gate in, output back to the host
-    e2e_steps = max(3, min(args.steps, 50))
+    e2e_steps = 0 if args.no_e2e else max(3, min(args.steps, 50))
     q_host = inp["q"].cpu().pin_memory()
     g_host = inp["gate"].cpu().pin_memory()
     o_host = torch.empty(step.out.shape, dtype=step.out.dtype).pin_memory()
-    for _ in range(2):
+    for _ in range(2 if e2e_steps else 0):
         inp["q"].copy_(q_host, non_blocking=True)
         inp["gate"].copy_(g_host, non_blocking=True)
         step()
@@ -326,7 +326,7 @@ def run_ours(args, rank, world, local_rank):
     e2e_el = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
     if world > 1:
         torch.distributed.all_reduce(e2e_el, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = float(e2e_el.item()) / e2e_steps
+    e2e_ms = float(e2e_el.item()) / max(e2e_steps, 1)
     h2d = q_host.numel() * q_host.element_size() + g_host.numel() * g_host.element_size()
     d2h = o_host.numel() * o_host.element_size()
 
@@ -358,8 +358,9 @@ def run_ours(args, rank, world, local_rank):
                                  "unit": "GB/s", "frac": hbm_achieved / float(peaks["hbm_gbs"]),
                                  "bytes_per_launch": page_bytes},
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
-            "e2e": {"value": frames_per_s(e2e_ms, world), "unit": "frames/s", "ms_per_step": e2e_ms,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps},
+            "e2e": ({"value": frames_per_s(e2e_ms, world), "unit": "frames/s", "ms_per_step": e2e_ms,
+                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}
+                    if e2e_steps else None),
             "cpu_baseline": cpu,
             "clocks": clocks,
             "gpu_launches": launches_per_step * args.steps,
@@ -385,6 +386,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end loop (profiling runs)")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="override H of the workload (smaller profiling captures)")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
