@@ -155,6 +155,35 @@ wa_status wa_linear_project(const void* k_act, const void* v_act, const void* e_
                             void* stream);
 
 /* ---------------------------------------------------------------------------
+ * The S4a projection for callers that cannot allocate device memory.  The paper
+ * has no counterpart to this entry point.
+ *
+ * Some callers cannot call cudaMalloc and have no workspace to hand over: code
+ * that runs inside a host framework which owns every device allocation through
+ * its own pool, or a real-time loop where an allocation (which can synchronise
+ * the device) is not allowed.  This call computes exactly what wa_linear_project
+ * computes for bf16 inputs, on the same tcgen05 kernels, but keeps its split-L
+ * partial sums in a fixed 32 MiB array that the library holds as a file-scope
+ * device variable: every GPU that loads libwa holds those 32 MiB until the
+ * process exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ *   - The caller still passes inputs and outputs (same layouts as
+ *     wa_linear_project; contiguous k_act / v_act [L][H][d], e_k / e_v [L][r]).
+ *   - The first call on a device looks the array's device address up
+ *     (cudaGetSymbolAddress, once per device, with that device current); make that
+ *     first call before any stream capture.
+ *   - All calls share the array, which keeps the last call's contents.  Each call
+ *     writes every partial it later reads, so no earlier contents leak into a
+ *     result; but calls that overlap on the GPU (two streams at once) race on it
+ *     and must be ordered by the caller.
+ *   - Sizes whose partials do not fit (2 * r * H * d * 4 bytes per split of L above
+ *     32 MiB) are rejected with WA_ERR_UNSUPPORTED and a message; larger problems use
+ *     fewer splits of L, down to one.
+ *   - dtype must be WA_BF16, d in {64, 128}, r in {128, 256}, H*d % 64 == 0. */
+wa_status wa_linear_project_noalloc(const void* k_act, const void* v_act, const void* e_k,
+                                    const void* e_v, int L, int H, int d, int r, wa_dtype dtype,
+                                    void* k_til, void* v_til, void* stream);
+
+/* ---------------------------------------------------------------------------
  * S4b + S5 + S6 -- the two attention branches and their gate (WorldAttention
  * §3.3: "Linear branch" O_lin = softmax(Q K~^T / sqrt(d)) V~; "Sparse branch",
  * exact attention restricted to the selected key blocks, Appendix A.1.3;

@@ -12,6 +12,8 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+#include <mutex>
+
 #include "sm100.cuh"
 #include "wa_internal.h"
 
@@ -275,3 +277,111 @@ wa_status launch_umma_project(const void* k, const void* v, RowSource rs, const 
 }
 
 }  // namespace wa
+
+// ============================================================================
+// Projection without any allocation.
+//
+// Some callers cannot allocate device memory at all: code that runs inside a
+// host framework which owns every device allocation through its own pool and
+// forbids cudaMalloc, or a real-time loop where an allocation (which can
+// synchronise the device) is not allowed.  They also may not have a workspace to
+// hand over.  wa_linear_project_noalloc serves them: it runs the same tcgen05
+// projection kernels as wa_linear_project, but keeps the split-L partial sums in
+// one fixed, file-scope device array instead of a caller workspace.  The caller
+// still passes its inputs and outputs.
+//
+// The array is kNoAllocScratchBytes (32 MiB) and is held by every GPU that loads
+// this library until the process exits.  All calls share it, so calls that
+// overlap on the GPU (for instance on two streams at once) race on it; callers
+// must order them.  Each call overwrites every partial it reads before reading
+// it, so the contents left by an earlier call never leak into a result.
+// ============================================================================
+namespace wa {
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 32ull << 20;
+static __device__ __align__(256) float g_noalloc_partials[kNoAllocScratchBytes / sizeof(float)];
+
+std::mutex g_noalloc_mu;
+float* g_noalloc_ptr[64] = {};
+
+// Device address of the static array for the current device.  In host code the
+// array's name is only a host-side stand-in; the kernels need the address that
+// cudaGetSymbolAddress returns, looked up once per device with that device current.
+wa_status noalloc_scratch(float** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess || dev < 0 || dev >= 64)
+    return set_error(WA_ERR_CUDA, "cudaGetDevice: %s", cudaGetErrorString(e));
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_partials);
+    if (e != cudaSuccess || p == nullptr)
+      return set_error(WA_ERR_CUDA, "cudaGetSymbolAddress(projection scratch): %s",
+                       cudaGetErrorString(e));
+    g_noalloc_ptr[dev] = static_cast<float*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return WA_OK;
+}
+
+}  // namespace
+}  // namespace wa
+
+extern "C" wa_status wa_linear_project_noalloc(const void* k_act, const void* v_act,
+                                               const void* e_k, const void* e_v, int L, int H,
+                                               int d, int r, wa_dtype dtype, void* k_til,
+                                               void* v_til, void* stream) {
+  using namespace wa;
+  if (!k_act || !v_act || !e_k || !e_v || !k_til || !v_til)
+    return set_error(WA_ERR_INVALID_ARG, "NULL pointer");
+  if (L < 1 || H < 1 || r < 1) return set_error(WA_ERR_INVALID_ARG, "sizes must be >= 1");
+  if (dtype != WA_BF16)
+    return set_error(WA_ERR_UNSUPPORTED, "wa_linear_project_noalloc takes bf16 inputs only");
+  if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "d must be 64 or 128");
+  if (r != 128 && r != 256) return set_error(WA_ERR_UNSUPPORTED, "r must be 128 or 256");
+  const int cols = H * d;
+  const int tn = pick_tn(cols);
+  if (tn == 0) return set_error(WA_ERR_UNSUPPORTED, "H*d must be a multiple of 64");
+  // as many splits of L as the default launch uses, but no more than the static
+  // scratch holds (2 matrices x n_split x r x H*d floats)
+  const size_t per_split = 2ull * r * cols * sizeof(float);
+  const size_t fit = kNoAllocScratchBytes / per_split;
+  if (fit < 1)
+    return set_error(WA_ERR_UNSUPPORTED,
+                     "r*H*d = %zu needs %zu bytes of scratch per split; the static scratch holds %zu",
+                     static_cast<size_t>(r) * cols, per_split, kNoAllocScratchBytes);
+  int n_split = pick_splits(L, r, cols);
+  if (static_cast<size_t>(n_split) > fit) n_split = static_cast<int>(fit);
+  float* part = nullptr;
+  wa_status s = noalloc_scratch(&part);
+  if (s != WA_OK) return s;
+  uint32_t* err = device_error_word();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RowSource rs;
+  rs.k = k_act; rs.v = v_act; rs.page_rows = L; rs.n_pages = 1; rs.L = L;
+  alignas(64) CUtensorMap tek, tev, txk, txv;
+  if (!make_tmap_bf16_2d(&tek, e_k, r, L, static_cast<uint64_t>(r) * 2, 64, 64) ||
+      !make_tmap_bf16_2d(&tev, e_v, r, L, static_cast<uint64_t>(r) * 2, 64, 64) ||
+      !make_tmap_bf16_2d(&txk, k_act, cols, L, static_cast<uint64_t>(cols) * 2, 64, 64) ||
+      !make_tmap_bf16_2d(&txv, v_act, cols, L, static_cast<uint64_t>(cols) * 2, 64, 64))
+    return set_error(WA_ERR_CUDA, "cuTensorMapEncodeTiled failed for the projection operands");
+  dim3 grid(2 * (cols / tn), n_split);
+  if (r == 256) {
+    if (tn == 256) launch_proj<2, 256>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
+    else if (tn == 128) launch_proj<2, 128>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
+    else launch_proj<2, 64>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
+  } else {
+    if (tn == 256) launch_proj<1, 256>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
+    else if (tn == 128) launch_proj<1, 128>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
+    else launch_proj<1, 64>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
+  }
+  s = check_launch("umma_project (no-alloc)");
+  if (s != WA_OK) return s;
+  const size_t per_m = static_cast<size_t>(r) * cols;
+  k_reduce_splits<<<2 * 148, 256, 0, st>>>(part, n_split, per_m, static_cast<__nv_bfloat16*>(k_til),
+                                           static_cast<__nv_bfloat16*>(v_til));
+  return check_launch("reduce_splits (no-alloc)");
+}

@@ -69,6 +69,7 @@ _SIGS = {
     "wa_linear_project_workspace_size": (c_size_t, [c_int] * 5),
     "wa_linear_project": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, c_int, P, P, P,
                                   c_size_t, P]),
+    "wa_linear_project_noalloc": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, c_int, P, P, P]),
     "wa_hsa_attention_workspace_size": (c_size_t, [c_int] * 7),
     "wa_hsa_attention": (c_int, [P, c_int, c_int, c_int, P, P, c_int, c_int, P, P, P, c_int, P,
                                  c_int, P, P, P, P, c_size_t, P]),
@@ -212,6 +213,21 @@ def wa_linear_project(k_act, v_act, e_k, e_v, stream=None):
     _check("wa_linear_project", lib.wa_linear_project(
         _p(k_act), _p(v_act), _p(e_k), _p(e_v), L, H, d, r, dt, _p(k_til), _p(v_til), _p(ws),
         nbytes, _stream(stream)))
+    return k_til, v_til
+
+
+def wa_linear_project_noalloc(k_act, v_act, e_k, e_v, stream=None):
+    """The projection without a workspace: the library keeps the split partials in
+    its own fixed device array (see include/wa.h).  Outputs are new tensors here;
+    the C call itself allocates nothing."""
+    _need_cuda(k_act, v_act, e_k, e_v)
+    L, H, d = k_act.shape
+    r = e_k.shape[1]
+    k_til = torch.empty((r, H, d), dtype=k_act.dtype, device=k_act.device)
+    v_til = torch.empty_like(k_til)
+    _check("wa_linear_project_noalloc", lib.wa_linear_project_noalloc(
+        _p(k_act), _p(v_act), _p(e_k), _p(e_v), L, H, d, r, dtype_code(k_act), _p(k_til),
+        _p(v_til), _stream(stream)))
     return k_til, v_til
 
 
