@@ -103,19 +103,24 @@ k_prompt_select(const float* __restrict__ e_cur, const float* __restrict__ e_chu
 }
 
 // ------------------------------------------------------------------ S1 HBM pass
-// One CTA sums blocks [b0, b1) of one source (pool page or buffer); thread t owns
-// columns [t*V, t*V + V).  Rows are read with 16-byte loads, eight in flight.
+// One CTA sums the B-row blocks [b0, b1) of one source (a pool page, or the buffer
+// itself) over one chunk of columns; thread t owns V consecutive columns.  Rows are
+// read with 16-byte loads, sixteen in flight per thread.  Optionally (qbar != null)
+// the CTA also forms the dot product of its running column sums with qbar, so the
+// page scores need only one scalar per CTA afterwards.
 template <typename T, int V>
-__global__ void __launch_bounds__(1024)
+__global__ void __launch_bounds__(256)
 k_rowblock_sum(const T* __restrict__ x, const int32_t* __restrict__ src_ids, int n_pages,
                int rows, int cols, int B, int nb, int bps, double* __restrict__ blocksum,
-               double* __restrict__ partial, int n_split, uint32_t* err) {
+               const double* __restrict__ qbar, double* __restrict__ kdot, uint32_t* err) {
+  __shared__ double red[32];
   const int s = blockIdx.y, split = blockIdx.x;
+  const int c0 = (blockIdx.z * blockDim.x + threadIdx.x) * V;
   int page = src_ids ? src_ids[s] : s;
   const bool ok = page >= 0 && page < n_pages;
   if (!ok && threadIdx.x == 0) atomicOr(err, WA_DEVERR_PAGE_ID);
   if (!ok) page = 0;
-  const T* base = x + static_cast<size_t>(page) * rows * cols + threadIdx.x * V;
+  const T* base = x + static_cast<size_t>(page) * rows * cols + c0;
   double part[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) part[v] = 0.0;
@@ -127,12 +132,12 @@ k_rowblock_sum(const T* __restrict__ x, const int32_t* __restrict__ src_ids, int
     for (int v = 0; v < V; ++v) acc[v] = 0.0;
     if (ok) {
       int r = r0;
-      for (; r + 8 <= r1; r += 8) {
-        uint4 raw[8];
+      for (; r + 16 <= r1; r += 16) {
+        uint4 raw[16];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) load_raw(base + static_cast<size_t>(r + u) * cols, raw[u]);
+        for (int u = 0; u < 16; ++u) load_raw(base + static_cast<size_t>(r + u) * cols, raw[u]);
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
+        for (int u = 0; u < 16; ++u) {
           double w[V];
           widen(base, raw[u], w);
 #pragma unroll
@@ -149,45 +154,69 @@ k_rowblock_sum(const T* __restrict__ x, const int32_t* __restrict__ src_ids, int
       }
     }
     if (blocksum) {
-      double* o = blocksum + (static_cast<size_t>(s) * nb + b) * cols + threadIdx.x * V;
+      double* o = blocksum + (static_cast<size_t>(s) * nb + b) * cols + c0;
 #pragma unroll
       for (int v = 0; v < V; ++v) o[v] = acc[v];
     }
 #pragma unroll
     for (int v = 0; v < V; ++v) part[v] += acc[v];
   }
-  double* o = partial + (static_cast<size_t>(s) * n_split + split) * cols + threadIdx.x * V;
+  if (qbar) {
+    double dot = 0.0;
 #pragma unroll
-  for (int v = 0; v < V; ++v) o[v] = part[v];
+    for (int v = 0; v < V; ++v) dot += part[v] * qbar[c0 + v];
+    dot = block_sum(dot, red);
+    if (threadIdx.x == 0)
+      kdot[(static_cast<size_t>(s) * gridDim.x + split) * gridDim.z + blockIdx.z] = dot;
+  }
+}
+
+// Qbar[col] = sum of all query rows / Nq; qmean[i][col] = block sum / rows of block i.
+// CTA = 32 columns x 8 row groups; group g sums blocks g, g+8, ...; the eight group
+// sums are added in a fixed order (deterministic).
+__global__ void __launch_bounds__(256)
+k_qmeans(const double* __restrict__ qsum, int n_qb, int Nq, int B, int cols,
+         double* __restrict__ qbar, double* __restrict__ qmean) {
+  __shared__ double red[8][32];
+  const int col = blockIdx.x * 32 + threadIdx.x;
+  const int g = threadIdx.y;
+  double t = 0.0;
+  if (col < cols) {
+#pragma unroll 4
+    for (int i = g; i < n_qb; i += 8) {
+      const double v = qsum[static_cast<size_t>(i) * cols + col];
+      t += v;
+      if (qmean) qmean[static_cast<size_t>(i) * cols + col] = v / (min(Nq, (i + 1) * B) - i * B);
+    }
+  }
+  red[g][threadIdx.x] = t;
+  __syncthreads();
+  if (g == 0 && col < cols) {
+    double s = 0.0;
+    for (int k = 0; k < 8; ++k) s += red[k][threadIdx.x];
+    qbar[col] = s / Nq;
+  }
 }
 
 // ------------------------------------------------------------------ S1 scores
-// alpha[c] = (1/(H*sqrt(d))) * sum_cols Qbar * Kbar_c, with Qbar = sum(q)/Nq and
-// Kbar_c = sum(k_c)/T_p rebuilt from the per-CTA partial sums in a fixed order.
-__global__ void k_page_alpha(const double* __restrict__ q_partial, int q_split, int Nq,
-                             const double* __restrict__ k_partial, int k_split, int T_p, int H,
-                             int d, double* __restrict__ alpha) {
-  __shared__ double red[32];
-  const int c = blockIdx.x, cols = H * d;
-  double acc = 0.0;
-  for (int col = threadIdx.x; col < cols; col += blockDim.x) {
-    double qs = 0.0, ks = 0.0;
-    for (int sp = 0; sp < q_split; ++sp) qs += q_partial[static_cast<size_t>(sp) * cols + col];
-    for (int sp = 0; sp < k_split; ++sp)
-      ks += k_partial[(static_cast<size_t>(c) * k_split + sp) * cols + col];
-    acc += (qs / Nq) * (ks / T_p);
-  }
-  acc = block_sum(acc, red);
-  if (threadIdx.x == 0) alpha[c] = acc / sqrt(static_cast<double>(d)) / H;
-}
-
-// Top-K_p of alpha (ties -> lower position), emitted in ascending position.
-__global__ void k_page_topk(const double* __restrict__ alpha, int n_c, int K_p,
-                            const int32_t* __restrict__ cand, int32_t* sel, int32_t* sel_pos) {
+// alpha[c] = (1/(H*sqrt(d))) * Qbar . Kbar_c, where Kbar_c = (sum of the page's rows)/T_p
+// and Qbar . (sum of rows) arrives as the per-CTA dot products of the K pass.  Then
+// the top-K_p pages (ties -> lower position), emitted in ascending position.
+__global__ void __launch_bounds__(256)
+k_alpha_topk(const double* __restrict__ kdot, int per_page, int n_c, int T_p, int H, int d,
+             int K_p, const int32_t* __restrict__ cand, double* __restrict__ alpha,
+             int32_t* __restrict__ sel, int32_t* __restrict__ sel_pos) {
   extern __shared__ unsigned char chosen[];  // n_c bytes
-  const int lane = threadIdx.x;
-  for (int j = lane; j < n_c; j += 32) chosen[j] = 0;
-  __syncwarp();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  for (int c = warp; c < n_c; c += nw) {
+    double t = 0.0;
+    for (int k = lane; k < per_page; k += 32) t += kdot[static_cast<size_t>(c) * per_page + k];
+    t = warp_sum(t);
+    if (lane == 0) alpha[c] = t / T_p / sqrt(static_cast<double>(d)) / H;
+  }
+  for (int j = threadIdx.x; j < n_c; j += blockDim.x) chosen[j] = 0;
+  __syncthreads();
+  if (warp != 0) return;
   for (int s = 0; s < K_p; ++s) {
     double best = -DBL_MAX;
     int bi = INT_MAX;
@@ -221,181 +250,186 @@ __global__ void k_scale_copy(const double* __restrict__ src, double* __restrict_
     dst[i] = src[i] * scale;
 }
 
-// ------------------------------------------------------------------ S3
-// CTA = (group of G query blocks, head).  Phases: pooled scores for every key block
-// (float64), a bitonic sort per row (descending score, ascending block on ties), a
-// warp scan of the softmax masses to find the shortest prefix reaching tau_h, then
-// the mask / ascending index list.
-constexpr int kSelThreads = 256;
+// ------------------------------------------------------------------ S3 scores
+// s[h][i][j] = qbar_{h,i} . kbar_{h,j} / sqrt(d) in float64.  CTA = (32 key blocks,
+// head): the 32 key-block means are staged in shared memory (row pitch d+1 doubles
+// against bank conflicts), the query means in chunks of 64 blocks; warp w computes
+// 8 query blocks of the chunk against lane l's key block, eight independent
+// accumulators per thread.
+constexpr int kScoreQChunk = 64;
 
-struct SelSmem {
-  double* qb;      // [G][d]
-  double* kc;      // [32][d+1]
-  double* key;     // [G][NP]
-  int* idx;        // [G][NP]
-  uint32_t* maskw; // [G][W]
-  int* mstar;      // [G]
-};
+__global__ void __launch_bounds__(256)
+k_block_scores(const double* __restrict__ qmean, KeyMeans km, int n_qb, int n_kb, int H, int d,
+               int B, double* __restrict__ scores) {
+  extern __shared__ double sm_scores[];
+  double* kc = sm_scores;                    // [32][d+1]
+  double* qs = sm_scores + 32 * (d + 1);     // [kScoreQChunk][d]
+  const int h = blockIdx.y, j0 = blockIdx.x * 32;
+  const int cols = H * d;
+  for (int e = threadIdx.x; e < 32 * d; e += blockDim.x) {
+    const int jj = e / d, c = e - jj * d, j = j0 + jj;
+    double v = 0.0;
+    if (j < n_kb) {
+      size_t row = j;
+      if (km.page_pos) row = static_cast<size_t>(km.page_pos[j / km.nbp]) * km.nbp + j % km.nbp;
+      v = km.data[row * cols + h * d + c];
+      if (km.is_sum) v /= static_cast<double>(min(km.L, (j + 1) * B) - j * B);
+    }
+    kc[jj * (d + 1) + c] = v;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int j = j0 + lane;
+  const double sqrt_d = sqrt(static_cast<double>(d));
+  const double* kr = kc + lane * (d + 1);
+  for (int ic = 0; ic < n_qb; ic += kScoreQChunk) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < kScoreQChunk * d; e += blockDim.x) {
+      const int ii = e / d, c = e - ii * d, i = ic + ii;
+      qs[e] = i < n_qb ? qmean[static_cast<size_t>(i) * cols + h * d + c] : 0.0;
+    }
+    __syncthreads();
+    const double* q0 = qs + (warp * 8) * d;
+    double acc[8];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc[r] = 0.0;
+    for (int c = 0; c < d; ++c) {
+      const double kv = kr[c];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) acc[r] += q0[r * d + c] * kv;
+    }
+    if (j < n_kb) {
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int i = ic + warp * 8 + r;
+        if (i < n_qb) scores[(static_cast<size_t>(h) * n_qb + i) * n_kb + j] = acc[r] / sqrt_d;
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ S3 choice
+// CTA = one (head, query block) row: bitonic sort of the scores (descending,
+// ascending block on ties), softmax masses exp(s - max)/Z, a block-wide scan of the
+// masses in sorted order, the first position whose prefix reaches tau_h, then the
+// mask and the ascending index list.
+constexpr int kChooseThreads = 256;
 
 __device__ __forceinline__ bool before(double ka, int ia, double kb, int ib) {
   return ka > kb || (ka == kb && ia < ib);
 }
 
-__global__ void __launch_bounds__(kSelThreads)
-k_block_select(const double* __restrict__ qsum, int Nq, int H, int d, int B, int n_qb,
-               KeyMeans km, int n_kb, int NP, int G, int W, const float* __restrict__ tau,
-               int32_t* __restrict__ blk_idx, int32_t* __restrict__ blk_cnt,
-               uint32_t* __restrict__ blk_mask) {
+__global__ void __launch_bounds__(kChooseThreads)
+k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int lg_np, int W,
+               const float* __restrict__ tau, int32_t* __restrict__ blk_idx,
+               int32_t* __restrict__ blk_cnt, uint32_t* __restrict__ blk_mask) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  SelSmem sm;
-  sm.qb = reinterpret_cast<double*>(smem_raw);
-  sm.kc = sm.qb + G * d;
-  sm.key = sm.kc + 32 * (d + 1);
-  sm.idx = reinterpret_cast<int*>(sm.key + static_cast<size_t>(G) * NP);
-  sm.maskw = reinterpret_cast<uint32_t*>(sm.idx + static_cast<size_t>(G) * NP);
-  sm.mstar = reinterpret_cast<int*>(sm.maskw + G * W);
-
-  const int h = blockIdx.y, i0 = blockIdx.x * G;
-  const int cols = H * d;
+  const int NP = 1 << lg_np;
+  double* key = reinterpret_cast<double*>(smem_raw);          // [NP]
+  int* idx = reinterpret_cast<int*>(key + NP);                 // [NP]
+  uint32_t* maskw = reinterpret_cast<uint32_t*>(idx + NP);     // [W]
+  __shared__ double wred[kChooseThreads / 32];
+  __shared__ int ired[kChooseThreads / 32];
+  const int h = blockIdx.y, i = blockIdx.x;
+  const size_t rowid = static_cast<size_t>(h) * n_qb + i;
+  const double* srow = scores + rowid * n_kb;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const double sqrt_d = sqrt(static_cast<double>(d));
-
-  // pooled query means
-  for (int e = tid; e < G * d; e += kSelThreads) {
-    const int g = e / d, c = e % d, i = i0 + g;
-    double v = 0.0;
-    if (i < n_qb) {
-      const int cnt = min(Nq, (i + 1) * B) - i * B;
-      v = qsum[static_cast<size_t>(i) * cols + h * d + c] / cnt;
-    }
-    sm.qb[e] = v;
+  for (int e = tid; e < NP; e += kChooseThreads) {
+    key[e] = e < n_kb ? srow[e] : -INFINITY;
+    idx[e] = e < n_kb ? e : INT_MAX;
   }
-  // scores s[g][j] = qbar_g . kbar_j / sqrt(d), 32 key blocks per pass
-  for (int j0 = 0; j0 < n_kb; j0 += 32) {
-    __syncthreads();
-    for (int e = tid; e < 32 * d; e += kSelThreads) {
-      const int jj = e / d, c = e % d, j = j0 + jj;
-      double v = 0.0;
-      if (j < n_kb) {
-        size_t row = j;
-        if (km.page_pos) row = static_cast<size_t>(km.page_pos[j / km.nbp]) * km.nbp + j % km.nbp;
-        v = km.data[row * cols + h * d + c];
-        if (km.is_sum) v /= static_cast<double>(min(km.L, (j + 1) * B) - j * B);
-      }
-      sm.kc[jj * (d + 1) + c] = v;
-    }
-    __syncthreads();
-    const int jj = tid & 31, g = tid >> 5, j = j0 + jj;
-    if (g < G && j < n_kb) {
-      const double* qg = sm.qb + g * d;
-      const double* kr = sm.kc + jj * (d + 1);
-      double s = 0.0;
-      for (int c = 0; c < d; ++c) s += qg[c] * kr[c];
-      sm.key[static_cast<size_t>(g) * NP + j] = s / sqrt_d;
-      sm.idx[static_cast<size_t>(g) * NP + j] = j;
-    }
-  }
-  for (int e = tid; e < G * NP; e += kSelThreads) {
-    if (e % NP >= n_kb) { sm.key[e] = -INFINITY; sm.idx[e] = INT_MAX; }
-  }
+  for (int w = tid; w < W; w += kChooseThreads) maskw[w] = 0u;
   __syncthreads();
-
-  // bitonic sort of every row: "before" order first
-  const int half = NP >> 1;
   for (int k = 2; k <= NP; k <<= 1) {
-    for (int jstep = k >> 1; jstep > 0; jstep >>= 1) {
-      for (int e = tid; e < G * half; e += kSelThreads) {
-        const int g = e / half, p = e % half;
-        const int i = 2 * jstep * (p / jstep) + (p % jstep);
-        const int l = i + jstep;
-        double* kr = sm.key + static_cast<size_t>(g) * NP;
-        int* ir = sm.idx + static_cast<size_t>(g) * NP;
-        const double ki = kr[i], kl = kr[l];
-        const int ii = ir[i], il = ir[l];
-        const bool up = (i & k) == 0;
-        const bool swap = up ? before(kl, il, ki, ii) : before(ki, ii, kl, il);
-        if (swap) { kr[i] = kl; kr[l] = ki; ir[i] = il; ir[l] = ii; }
+    for (int js = k >> 1; js > 0; js >>= 1) {
+      for (int p = tid; p < (NP >> 1); p += kChooseThreads) {
+        const int a = ((p & ~(js - 1)) << 1) | (p & (js - 1));   // bit js of a is 0
+        const int b = a | js;
+        const double ka = key[a], kb = key[b];
+        const int ia = idx[a], ib = idx[b];
+        const bool swap = (a & k) == 0 ? before(kb, ib, ka, ia) : before(ka, ia, kb, ib);
+        if (swap) { key[a] = kb; key[b] = ka; idx[a] = ib; idx[b] = ia; }
       }
       __syncthreads();
     }
   }
-
-  // shortest prefix reaching tau: one warp per row
-  for (int g = warp; g < G; g += kSelThreads / 32) {
-    const int i = i0 + g;
-    if (i >= n_qb) { if (lane == 0) sm.mstar[g] = 0; continue; }
-    const double th = static_cast<double>(tau[h]);
-    const double* kr = sm.key + static_cast<size_t>(g) * NP;
-    int m = n_kb;
-    if (th < 1.0) {
-      const double smax = kr[0];
-      const int per = NP / 32;             // NP >= 32
-      const int t0 = lane * per;
-      double zl = 0.0;
-      for (int t = t0; t < t0 + per && t < n_kb; ++t) zl += exp(kr[t] - smax);
-      const double Z = warp_sum(zl);
-      double pl = 0.0;
-      for (int t = t0; t < t0 + per && t < n_kb; ++t) pl += exp(kr[t] - smax) / Z;
-      // exclusive scan of the lane sums
-      double incl = pl;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const double y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      double c = incl - pl;
-      int first = INT_MAX;
-      for (int t = t0; t < t0 + per && t < n_kb; ++t) {
-        c += exp(kr[t] - smax) / Z;
-        if (c >= th) { first = t; break; }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
-      if (first != INT_MAX) m = first + 1;
+  const double th = static_cast<double>(tau[h]);
+  int m = n_kb;
+  if (th < 1.0) {
+    const double smax = key[0];
+    const int per = NP / kChooseThreads > 0 ? NP / kChooseThreads : 1;
+    const int t0 = tid * per;
+    // z_t = exp(s_t - max), kept in place of the sorted scores
+    double zl = 0.0;
+    for (int t = t0; t < t0 + per && t < NP; ++t) {
+      const double z = t < n_kb ? exp(key[t] - smax) : 0.0;
+      key[t] = z;
+      zl += z;
     }
-    if (lane == 0) sm.mstar[g] = m;
+    zl = warp_sum(zl);
+    if (lane == 0) wred[warp] = zl;
+    __syncthreads();
+    double Z = 0.0;
+    for (int w = 0; w < kChooseThreads / 32; ++w) Z += wred[w];
+    __syncthreads();
+    double pl = 0.0;
+    for (int t = t0; t < t0 + per && t < NP; ++t) {
+      const double pv = key[t] / Z;
+      key[t] = pv;
+      pl += pv;
+    }
+    // exclusive prefix of the per-thread sums, in thread order
+    double incl = pl;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) wred[warp] = incl;
+    __syncthreads();
+    double c = incl - pl;
+    for (int w = 0; w < warp; ++w) c += wred[w];
+    int first = INT_MAX;
+    for (int t = t0; t < t0 + per && t < n_kb; ++t) {
+      c += key[t];
+      if (c >= th) { first = t; break; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+    if (lane == 0) ired[warp] = first;
+    __syncthreads();
+    first = INT_MAX;
+    for (int w = 0; w < kChooseThreads / 32; ++w) first = min(first, ired[w]);
+    if (first != INT_MAX) m = first + 1;
   }
-  for (int e = tid; e < G * W; e += kSelThreads) sm.maskw[e] = 0u;
-  __syncthreads();
-  for (int e = tid; e < G * NP; e += kSelThreads) {
-    const int g = e / NP, t = e % NP;
-    if (t < sm.mstar[g]) {
-      const int j = sm.idx[e];
-      atomicOr(&sm.maskw[g * W + (j >> 5)], 1u << (j & 31));
-    }
+  for (int t = tid; t < m; t += kChooseThreads) {
+    const int j = idx[t];
+    atomicOr(&maskw[j >> 5], 1u << (j & 31));
   }
   __syncthreads();
-  for (int g = warp; g < G; g += kSelThreads / 32) {
-    const int i = i0 + g;
-    if (i >= n_qb) continue;
-    const size_t row = static_cast<size_t>(h) * n_qb + i;
-    if (blk_mask)
-      for (int w = lane; w < W; w += 32) blk_mask[row * W + w] = sm.maskw[g * W + w];
-    if (blk_cnt && lane == 0) blk_cnt[row] = sm.mstar[g];
-    if (blk_idx) {
-      // lane owns words [lane*wpl, lane*wpl + wpl): ascending order follows lane order
-      const int wpl = (W + 31) / 32;
-      int cnt = 0;
-      for (int w = lane * wpl; w < min(W, lane * wpl + wpl); ++w) cnt += __popc(sm.maskw[g * W + w]);
-      int incl = cnt;
+  if (blk_mask)
+    for (int w = tid; w < W; w += kChooseThreads) blk_mask[rowid * W + w] = maskw[w];
+  if (blk_cnt && tid == 0) blk_cnt[rowid] = m;
+  if (blk_idx && warp == 0) {
+    const int wpl = (W + 31) / 32;
+    int cnt = 0;
+    for (int w = lane * wpl; w < min(W, lane * wpl + wpl); ++w) cnt += __popc(maskw[w]);
+    int incl = cnt;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const int y = __shfl_up_sync(0xffffffffu, incl, o);
-        if (lane >= o) incl += y;
-      }
-      int pos = incl - cnt;
-      int32_t* out = blk_idx + row * n_kb;
-      for (int w = lane * wpl; w < min(W, lane * wpl + wpl); ++w) {
-        uint32_t bits = sm.maskw[g * W + w];
-        while (bits) {
-          const int b = __ffs(bits) - 1;
-          bits &= bits - 1;
-          out[pos++] = w * 32 + b;
-        }
-      }
-      const int m = sm.mstar[g];
-      for (int t = m + lane; t < n_kb; t += 32) out[t] = -1;
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
     }
+    int pos = incl - cnt;
+    int32_t* out = blk_idx + rowid * n_kb;
+    for (int w = lane * wpl; w < min(W, lane * wpl + wpl); ++w) {
+      uint32_t bits = maskw[w];
+      while (bits) {
+        const int b = __ffs(bits) - 1;
+        bits &= bits - 1;
+        out[pos++] = w * 32 + b;
+      }
+    }
+    for (int t = m + lane; t < n_kb; t += 32) out[t] = -1;
   }
 }
 
@@ -409,40 +443,52 @@ wa_status launch_prompt_select(const float* e_cur, const float* e_chunks, int n_
   return check_launch("prompt_select");
 }
 
-int rowsum_splits(int n_src, int rows, int B) {
-  const int nb = (rows + B - 1) / B;
-  int want = (kTargetCtas + n_src - 1) / n_src;
-  want = want < 1 ? 1 : (want > nb ? nb : want);
-  const int bps = (nb + want - 1) / want;
-  return (nb + bps - 1) / bps;
+RowsumPlan rowsum_plan(int n_src, int rows, int cols, int B, wa_dtype dt) {
+  RowsumPlan p;
+  const int V = dt == WA_BF16 ? 8 : 4;
+  const int threads_total = cols / V;
+  p.n_cc = 1;
+  p.threads = threads_total;
+  while (p.threads >= 128 && (p.threads % 2) == 0 && n_src * p.n_cc < 16) {  // few sources: split columns
+    p.threads /= 2;
+    p.n_cc *= 2;
+  }
+  p.nb = (rows + B - 1) / B;
+  int want = (kTargetCtas + n_src * p.n_cc - 1) / (n_src * p.n_cc);
+  want = want < 1 ? 1 : (want > p.nb ? p.nb : want);
+  p.bps = (p.nb + want - 1) / want;
+  p.n_split = (p.nb + p.bps - 1) / p.bps;
+  return p;
 }
 
 wa_status launch_rowblock_sum(const void* x, wa_dtype dt, const int32_t* src_ids, int n_src,
                               int n_pages, int rows, int cols, int B, double* blocksum,
-                              double* partial, int n_split, uint32_t* err, cudaStream_t st) {
-  const int nb = (rows + B - 1) / B;
-  const int bps = (nb + n_split - 1) / n_split;
-  dim3 grid(n_split, n_src);
+                              const double* qbar, double* kdot, const RowsumPlan& p, uint32_t* err,
+                              cudaStream_t st) {
+  dim3 grid(p.n_split, n_src, p.n_cc);
   if (dt == WA_BF16) {
-    k_rowblock_sum<__nv_bfloat16, 8><<<grid, cols / 8, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), src_ids, n_pages, rows, cols, B, nb, bps, blocksum,
-        partial, n_split, err);
+    k_rowblock_sum<__nv_bfloat16, 8><<<grid, p.threads, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), src_ids, n_pages, rows, cols, B, p.nb, p.bps, blocksum,
+        qbar, kdot, err);
   } else {
-    k_rowblock_sum<float, 4><<<grid, cols / 4, 0, st>>>(static_cast<const float*>(x), src_ids,
-                                                        n_pages, rows, cols, B, nb, bps, blocksum,
-                                                        partial, n_split, err);
+    k_rowblock_sum<float, 4><<<grid, p.threads, 0, st>>>(static_cast<const float*>(x), src_ids,
+                                                          n_pages, rows, cols, B, p.nb, p.bps,
+                                                          blocksum, qbar, kdot, err);
   }
   return check_launch("rowblock_sum");
 }
 
-wa_status launch_page_alpha_topk(const double* q_partial, int q_split, int Nq,
-                                 const double* k_partial, int k_split, int T_p, int n_c,
-                                 int H, int d, int K_p, const int32_t* cand, double* alpha,
-                                 int32_t* sel, int32_t* sel_pos, cudaStream_t st) {
-  k_page_alpha<<<n_c, 256, 0, st>>>(q_partial, q_split, Nq, k_partial, k_split, T_p, H, d,
-                                    alpha);
-  k_page_topk<<<1, 32, n_c, st>>>(alpha, n_c, K_p, cand, sel, sel_pos);
-  return check_launch("page_alpha_topk");
+wa_status launch_qmeans(const double* qsum, int n_qb, int Nq, int B, int cols, double* qbar,
+                        double* qmean, cudaStream_t st) {
+  k_qmeans<<<(cols + 31) / 32, dim3(32, 8), 0, st>>>(qsum, n_qb, Nq, B, cols, qbar, qmean);
+  return check_launch("qmeans");
+}
+
+wa_status launch_alpha_topk(const double* kdot, int per_page, int n_c, int T_p, int H, int d,
+                            int K_p, const int32_t* cand, double* alpha, int32_t* sel,
+                            int32_t* sel_pos, cudaStream_t st) {
+  k_alpha_topk<<<1, 256, n_c, st>>>(kdot, per_page, n_c, T_p, H, d, K_p, cand, alpha, sel, sel_pos);
+  return check_launch("alpha_topk");
 }
 
 wa_status launch_scale_copy(const double* src, double* dst, size_t n, double scale,
@@ -451,32 +497,31 @@ wa_status launch_scale_copy(const double* src, double* dst, size_t n, double sca
   return check_launch("scale_copy");
 }
 
-size_t block_select_smem_bytes(int d, int n_kb, int* G_out) {
-  int NP = 32;
-  while (NP < n_kb) NP <<= 1;
-  int G = 8;
-  while (G > 1 && static_cast<size_t>(G) * NP * 12 > 98304) G >>= 1;
-  const int W = (n_kb + 31) / 32;
-  if (G_out) *G_out = G;
-  return static_cast<size_t>(G) * d * 8 + 32 * static_cast<size_t>(d + 1) * 8 +
-         static_cast<size_t>(G) * NP * 12 + static_cast<size_t>(G) * W * 4 + G * 4;
+size_t block_scores_bytes(int H, int n_qb, int n_kb) {
+  return static_cast<size_t>(H) * n_qb * n_kb * sizeof(double);
 }
 
-wa_status launch_block_select(const double* q_blocksum, int Nq, int H, int d, int B,
-                              KeyMeans km, int n_kb, const float* tau, int32_t* blk_idx,
-                              int32_t* blk_cnt, uint32_t* blk_mask, cudaStream_t st) {
-  int G = 1;
-  const size_t smem = block_select_smem_bytes(d, n_kb, &G);
-  int NP = 32;
-  while (NP < n_kb) NP <<= 1;
-  const int W = (n_kb + 31) / 32;
+wa_status launch_block_select(const double* q_blockmean, int Nq, int H, int d, int B,
+                              KeyMeans km, int n_kb, const float* tau, double* scores,
+                              int32_t* blk_idx, int32_t* blk_cnt, uint32_t* blk_mask,
+                              cudaStream_t st) {
   const int n_qb = (Nq + B - 1) / B;
-  cudaError_t e = cudaFuncSetAttribute(k_block_select, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
-  if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "block_select smem attr: %s", cudaGetErrorString(e));
-  dim3 grid((n_qb + G - 1) / G, H);
-  k_block_select<<<grid, kSelThreads, smem, st>>>(q_blocksum, Nq, H, d, B, n_qb, km, n_kb, NP, G,
-                                                  W, tau, blk_idx, blk_cnt, blk_mask);
+  const int W = (n_kb + 31) / 32;
+  const size_t smem_s = (32 * static_cast<size_t>(d + 1) + kScoreQChunk * static_cast<size_t>(d)) *
+                        sizeof(double);
+  cudaError_t e = cudaFuncSetAttribute(k_block_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem_s));
+  if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "block_scores smem attr: %s", cudaGetErrorString(e));
+  k_block_scores<<<dim3((n_kb + 31) / 32, H), 256, smem_s, st>>>(q_blockmean, km, n_qb, n_kb, H, d,
+                                                               B, scores);
+  int lg = 5;
+  while ((1 << lg) < n_kb) ++lg;
+  const size_t smem_c = (static_cast<size_t>(1) << lg) * 12 + static_cast<size_t>(W) * 4 + 16;
+  e = cudaFuncSetAttribute(k_block_choose, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem_c));
+  if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "block_choose smem attr: %s", cudaGetErrorString(e));
+  k_block_choose<<<dim3(n_qb, H), kChooseThreads, smem_c, st>>>(scores, n_qb, n_kb, lg, W, tau,
+                                                                blk_idx, blk_cnt, blk_mask);
   return check_launch("block_select");
 }
 

@@ -9,17 +9,22 @@
 //           out = bf16(sigmoid(g) * O_sp + workspace).
 //
 // The pages' kernels tile for Hopper WGMMA with 64-row query blocks.  The B200
-// MMA wants M = 128, so one CTA takes a pair of query blocks of the same head
-// (rows 0-63 and 64-127 of one tile) and walks the union of their two key-block
-// sets, masking each half's unselected blocks to -inf.  Pairs are chosen to
-// overlap as much as possible (k_pair_heads) and run longest first.
+// MMA wants M = 128, so a tile is a pair of query blocks of the same head (rows
+// 0-63 and 64-127) that walks the union of their two key-block sets, each half
+// masking the blocks it did not select.  Pairs are chosen to overlap as much as
+// possible (k_pair_heads).  A pair's key list is split in two work items when it
+// is long enough, so that the work items fill whole waves of CTAs; the two
+// partial results (unnormalised O, running max m, sum l per row) are merged by
+// k_combine, which also applies the gate.  Items run longest first.
 //
-// CTA = 256 threads: warp 0 issues TMA loads (Q once, then K/V blocks through a
-// 2-stage ring, straight from the pool pages via the page table), warp 1 owns
-// TMEM and issues tcgen05.mma (S = Q K^T into one of two TMEM S buffers; O += P V
-// with P read back from TMEM), warps 4-7 run the online softmax, one thread per
-// TMEM lane (= query row), and the epilogue.  Two CTAs fit on an SM, so one CTA's
-// softmax overlaps the other's MMAs.  Every wait is bounded in time.
+// CTA = 256 threads, two CTAs per SM: warp 0 loads Q and the K blocks, warp 2 the
+// V blocks (TMA, 128-byte swizzle, straight from the pool pages through the page
+// table, each through its own 2-slot ring: a K slot frees as soon as its S = Q K^T
+// MMA completes, a V slot when its O += P V MMA completes); warp 1 owns TMEM and
+// issues tcgen05.mma; warps 4-7 run the online softmax with one thread per TMEM
+// lane (query row), write P back as bf16 into the S buffer, rescale O in TMEM only
+// when the running max grows by more than 2^8, and run the epilogue.  One CTA's
+// softmax overlaps the other CTA's MMAs.  Every wait is bounded in time.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -36,31 +41,35 @@ using namespace sm100;
 
 constexpr int kBM = 128;          // query rows per tile (two 64-row blocks)
 constexpr int kBN = 64;           // keys per block
-constexpr int kStages = 2;
+constexpr int kRing = 2;          // slots of the K ring and of the V ring
 constexpr int kThreads = 256;
 constexpr uint32_t kTmemCols = 256;
 constexpr int kColS = 0;          // two S/P buffers at columns 0 and 64
 constexpr int kColO = 128;        // O accumulator at columns 128 .. 128+d
 constexpr int kMaxW = 256;        // up to 8192 key blocks
+constexpr int kSplitMin = 8;      // pairs with at least this many key blocks are split in two
+
+// item.y values
+constexpr int kWhole = -1;        // the whole key list; writes the final output
+constexpr int kEmpty = -2;        // placeholder: nothing to do
 
 template <int D>
 struct Cfg {
   static constexpr int kPanels = D / 64;                 // 128-byte column panels
   static constexpr int kQBytes = kBM * D * 2;
   static constexpr int kKVBytes = kBN * D * 2;
-  static constexpr int kStageBytes = 2 * kKVBytes;
-  static constexpr int kSmem = kQBytes + kStages * kStageBytes + 1024;  // + alignment slack
+  static constexpr int kSmem = kQBytes + 2 * kRing * kKVBytes + 1024;  // + alignment slack
   static constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
   static constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, false, true);
 };
 
 struct Shared {
   uint64_t q_full;
-  uint64_t kv_full[kStages];
-  uint64_t kv_empty[kStages];
+  uint64_t k_full[kRing], k_empty[kRing];
+  uint64_t v_full[kRing], v_empty[kRing];
   uint64_t s_full[2];
   uint64_t p_full[2];
-  uint64_t o_done;
+  uint64_t o_done[2];   // completion of O += P_u V_u, by the parity of u
   uint32_t tmem_base;
   int abort_flag;
   uint32_t mask[2][kMaxW];
@@ -84,17 +93,14 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared&
   }
 }
 
-// Walks the key blocks of a tile in ascending order: the union of the two masks
-// (mode 1) or every block (mode 0).
+// Walks key blocks [k0, k1) of a tile's list in ascending block order: the list is
+// the union of the two masks (mode 1) or every block (mode 0).
 struct BlockIter {
   const uint32_t* a;
   const uint32_t* b;
-  int W, n_kb, w, all;
+  int W, n_kb, w, all, pos, k1;
   uint32_t bits;
-  __device__ void init(const uint32_t* a_, const uint32_t* b_, int W_, int n_kb_, int all_) {
-    a = a_; b = b_; W = W_; n_kb = n_kb_; all = all_; w = -1; bits = 0u;
-  }
-  __device__ int next() {
+  __device__ int next_raw() {
     if (all) { ++w; return w < n_kb ? w : -1; }
     while (bits == 0u) {
       if (++w >= W) return -1;
@@ -104,6 +110,16 @@ struct BlockIter {
     bits &= bits - 1u;
     return j;
   }
+  __device__ void init(const uint32_t* a_, const uint32_t* b_, int W_, int n_kb_, int all_, int k0_,
+                       int k1_) {
+    a = a_; b = b_; W = W_; n_kb = n_kb_; all = all_; w = -1; bits = 0u; pos = 0; k1 = k1_;
+    for (; pos < k0_; ++pos) next_raw();
+  }
+  __device__ int next() {
+    if (pos >= k1) return -1;
+    ++pos;
+    return next_raw();
+  }
 };
 
 __device__ __forceinline__ float ex2(float x) {
@@ -112,42 +128,64 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
+__device__ __forceinline__ int key_row(const RowSource& rs, int bpp, int j, uint32_t* err) {
+  if (!rs.page_ids) return j * kBN;
+  int pg = rs.page_ids[j / bpp];
+  if (pg < 0 || pg >= rs.n_pages) { atomicOr(err, WA_DEVERR_PAGE_ID); pg = 0; }
+  return pg * rs.page_rows + (j % bpp) * kBN;
+}
+
+struct Partials {
+  float* o;    // [slots][128][d]  unnormalised O
+  float* ml;   // [slots][128][2]  running max (log2 units) and sum
+};
+
 template <int D>
 __global__ void __launch_bounds__(kThreads, 2)
 k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, int mode, int Nq, int H, int Lk,
                  RowSource rs, const uint32_t* __restrict__ blk_mask, int W, int n_qb,
-                 const int4* __restrict__ items, const float* __restrict__ gate,
-                 float* __restrict__ lin_ws, __nv_bfloat16* __restrict__ out,
-                 float* __restrict__ o_branch, uint32_t* err) {
+                 const int4* __restrict__ pairs, const int4* __restrict__ items, Partials part,
+                 const float* __restrict__ gate, float* __restrict__ lin_ws,
+                 __nv_bfloat16* __restrict__ out, float* __restrict__ o_branch, uint32_t* err) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_dyn[];
   __shared__ Shared sh;
-  uint8_t* tiles = reinterpret_cast<uint8_t*>(
-      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* Qs = tiles;
-  auto Ks = [&](int s) { return tiles + C::kQBytes + s * C::kStageBytes; };
-  auto Vs = [&](int s) { return tiles + C::kQBytes + s * C::kStageBytes + C::kKVBytes; };
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  int h, i0, i1;
+  const int n_kb = (Lk + kBN - 1) / kBN;
+  int h, i0, i1, k0, k1, kind, slot;
   if (mode == 0) {
     const int n_pairs = (n_qb + 1) / 2;
     h = blockIdx.x / n_pairs;
     const int p = blockIdx.x % n_pairs;
     i0 = 2 * p;
     i1 = (2 * p + 1 < n_qb) ? 2 * p + 1 : -1;
+    k0 = 0; k1 = n_kb; kind = kWhole; slot = 0;
   } else {
     const int4 it = items[blockIdx.x];
-    h = it.x; i0 = it.y; i1 = it.z;
+    kind = it.y;
+    if (kind == kEmpty) return;
+    const int4 pr = pairs[it.x];
+    h = pr.x; i0 = pr.y; i1 = pr.z;
+    k0 = it.z; k1 = it.w;
+    slot = 2 * it.x + (kind < 0 ? 0 : kind);
   }
-  const int n_kb = (Lk + kBN - 1) / kBN;
+  uint8_t* tiles = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* Qs = tiles;
+  auto Ks = [&](int s) { return tiles + C::kQBytes + s * C::kKVBytes; };
+  auto Vs = [&](int s) { return tiles + C::kQBytes + (kRing + s) * C::kKVBytes; };
 
   if (tid == 0) {
     mbar_init(&sh.q_full, 1);
-    for (int s = 0; s < kStages; ++s) { mbar_init(&sh.kv_full[s], 1); mbar_init(&sh.kv_empty[s], 1); }
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&sh.k_full[s], 1); mbar_init(&sh.k_empty[s], 1);
+      mbar_init(&sh.v_full[s], 1); mbar_init(&sh.v_empty[s], 1);
+    }
     for (int b = 0; b < 2; ++b) { mbar_init(&sh.s_full[b], 1); mbar_init(&sh.p_full[b], 128); }
-    mbar_init(&sh.o_done, 1);
+    mbar_init(&sh.o_done[0], 1);
+    mbar_init(&sh.o_done[1], 1);
     sh.abort_flag = 0;
     fence_mbar_init();
   }
@@ -167,22 +205,14 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sh.tmem_base;
-
-  // number of key blocks this tile walks
-  int n_blk = 0;
-  if (mode == 0) {
-    n_blk = n_kb;
-  } else {
-    for (int w = 0; w < W; ++w) n_blk += __popc(sh.mask[0][w] | sh.mask[1][w]);
-  }
+  const int n_blk = k1 - k0;
   const int bpp = rs.page_ids ? rs.page_rows / kBN : 0;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ Q + K producer
     if (lane == 0) {
       prefetch_tmap(&tmQ);
       prefetch_tmap(&tmK);
-      prefetch_tmap(&tmV);
       mbar_arrive_expect_tx(&sh.q_full, C::kQBytes);
       const int y1 = i1 >= 0 ? i1 * 64 : Nq;  // out of range -> zero fill
       for (int p = 0; p < C::kPanels; ++p) {
@@ -190,24 +220,31 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         tma_load_2d(Qs + p * (kBM * 128) + 64 * 128, &tmQ, &sh.q_full, h * D + p * 64, y1);
       }
       BlockIter it;
-      it.init(sh.mask[0], sh.mask[1], W, n_kb, mode == 0);
+      it.init(sh.mask[0], sh.mask[1], W, n_kb, mode == 0, k0, k1);
       int t = 0;
       for (int j = it.next(); j >= 0; j = it.next(), ++t) {
-        const int s = t % kStages;
-        if (!wait_bar(&sh.kv_empty[s], ((t / kStages) & 1) ^ 1, sh, err)) break;
-        int row;
-        if (rs.page_ids) {
-          int pg = rs.page_ids[j / bpp];
-          if (pg < 0 || pg >= rs.n_pages) { atomicOr(err, WA_DEVERR_PAGE_ID); pg = 0; }
-          row = pg * rs.page_rows + (j % bpp) * kBN;
-        } else {
-          row = j * kBN;
-        }
-        mbar_arrive_expect_tx(&sh.kv_full[s], C::kStageBytes);
-        for (int p = 0; p < C::kPanels; ++p) {
-          tma_load_2d(Ks(s) + p * (kBN * 128), &tmK, &sh.kv_full[s], h * D + p * 64, row);
-          tma_load_2d(Vs(s) + p * (kBN * 128), &tmV, &sh.kv_full[s], h * D + p * 64, row);
-        }
+        const int s = t % kRing;
+        if (!wait_bar(&sh.k_empty[s], ((t / kRing) & 1) ^ 1, sh, err)) break;
+        const int row = key_row(rs, bpp, j, err);
+        mbar_arrive_expect_tx(&sh.k_full[s], C::kKVBytes);
+        for (int p = 0; p < C::kPanels; ++p)
+          tma_load_2d(Ks(s) + p * (kBN * 128), &tmK, &sh.k_full[s], h * D + p * 64, row);
+      }
+    }
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ V producer
+    if (lane == 0) {
+      prefetch_tmap(&tmV);
+      BlockIter it;
+      it.init(sh.mask[0], sh.mask[1], W, n_kb, mode == 0, k0, k1);
+      int t = 0;
+      for (int j = it.next(); j >= 0; j = it.next(), ++t) {
+        const int s = t % kRing;
+        if (!wait_bar(&sh.v_empty[s], ((t / kRing) & 1) ^ 1, sh, err)) break;
+        const int row = key_row(rs, bpp, j, err);
+        mbar_arrive_expect_tx(&sh.v_full[s], C::kKVBytes);
+        for (int p = 0; p < C::kPanels; ++p)
+          tma_load_2d(Vs(s) + p * (kBN * 128), &tmV, &sh.v_full[s], h * D + p * 64, row);
       }
     }
   } else if (warp == 1) {
@@ -216,39 +253,41 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       bool ok = wait_bar(&sh.q_full, 0, sh, err);
       tc_fence_after();
       const uint32_t q_base = smem_u32(Qs);
-      auto issue_pv = [&](int u) -> bool {
-        const int su = u & 1;
-        if (!wait_bar(&sh.p_full[su], (u >> 1) & 1, sh, err)) return false;
-        tc_fence_after();
-        const uint32_t v_base = smem_u32(Vs(u % kStages));
+      for (int t = 0; ok && t <= n_blk; ++t) {
+        if (t < n_blk) {
+          // S_t = Q K_t^T into S buffer t % 2 (its previous P was consumed by PV_{t-2},
+          // issued earlier by this thread)
+          const int s = t % kRing;
+          if (!wait_bar(&sh.k_full[s], (t / kRing) & 1, sh, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t k_base = smem_u32(Ks(s));
+          const int sb = t & 1;
 #pragma unroll
-        for (int kk = 0; kk < kBN / 16; ++kk) {
-          const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, 64 * 128, 1024);
-          mma_ts(tbase + kColO, tbase + kColS + su * 64 + kk * 8, bdesc, C::kIdescO,
-                 (u > 0 || kk > 0) ? 1u : 0u);
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t adesc = smem_desc_sw128(q_base + (k >> 2) * (kBM * 128) + (k & 3) * 32, 16, 1024);
+            const uint64_t bdesc = smem_desc_sw128(k_base + (k >> 2) * (kBN * 128) + (k & 3) * 32, 16, 1024);
+            mma_ss(tbase + kColS + sb * 64, adesc, bdesc, C::kIdescS, k > 0 ? 1u : 0u);
+          }
+          mma_commit(&sh.k_empty[s]);
+          mma_commit(&sh.s_full[sb]);
         }
-        mma_commit(&sh.kv_empty[u % kStages]);
-        mma_commit(&sh.o_done);
-        return true;
-      };
-      int t = 0;
-      for (; ok && t < n_blk; ++t) {
-        const int s = t % kStages;
-        if (!wait_bar(&sh.kv_full[s], (t / kStages) & 1, sh, err)) { ok = false; break; }
-        tc_fence_after();
-        const uint32_t k_base = smem_u32(Ks(s));
-        const int sb = t & 1;
+        if (t > 0) {
+          // O += P_u V_u, P read from TMEM
+          const int u = t - 1, su = u & 1, vs = u % kRing;
+          if (!wait_bar(&sh.p_full[su], (u >> 1) & 1, sh, err)) { ok = false; break; }
+          if (!wait_bar(&sh.v_full[vs], (u / kRing) & 1, sh, err)) { ok = false; break; }
+          tc_fence_after();
+          const uint32_t v_base = smem_u32(Vs(vs));
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t adesc = smem_desc_sw128(q_base + (k >> 2) * (kBM * 128) + (k & 3) * 32, 16, 1024);
-          const uint64_t bdesc = smem_desc_sw128(k_base + (k >> 2) * (kBN * 128) + (k & 3) * 32, 16, 1024);
-          mma_ss(tbase + kColS + sb * 64, adesc, bdesc, C::kIdescS, k > 0 ? 1u : 0u);
+          for (int kk = 0; kk < kBN / 16; ++kk) {
+            const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, 64 * 128, 1024);
+            mma_ts(tbase + kColO, tbase + kColS + su * 64 + kk * 8, bdesc, C::kIdescO,
+                   (u > 0 || kk > 0) ? 1u : 0u);
+          }
+          mma_commit(&sh.v_empty[vs]);
+          mma_commit(&sh.o_done[u & 1]);
         }
-        mma_commit(&sh.s_full[sb]);
-        if (t > 0 && !issue_pv(t - 1)) { ok = false; break; }
       }
-      if (ok && n_blk > 0) ok = issue_pv(n_blk - 1);
-      (void)ok;
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
@@ -264,7 +303,7 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
     BlockIter it;
-    it.init(sh.mask[0], sh.mask[1], W, n_kb, mode == 0);
+    it.init(sh.mask[0], sh.mask[1], W, n_kb, mode == 0, k0, k1);
     int t = 0;
     for (int j = it.next(); j >= 0; j = it.next(), ++t) {
       const int sb = t & 1;
@@ -276,14 +315,23 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tmem_wait_ld();
       const bool sel = mode == 0 || ((mymask[j >> 5] >> (j & 31)) & 1u);
       const int valid = min(kBN, Lk - j * kBN);
-      float mx = -INFINITY;
+      if (!sel || valid < kBN) {
+        // a block this half did not select, or the ragged last block: mask columns
 #pragma unroll
-      for (int c = 0; c < 64; ++c) {
-        float s = __uint_as_float(r[c]) * scale_log2;
-        if (!sel || c >= valid) s = -INFINITY;
-        r[c] = __float_as_uint(s);
-        mx = fmaxf(mx, s);
+        for (int c = 0; c < 64; ++c)
+          if (!sel || c >= valid) r[c] = __float_as_uint(-INFINITY);
       }
+      // row max of the raw scores: eight independent chains
+      float mx8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(r[e]);
+#pragma unroll
+      for (int c = 8; c < 64; c += 8)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], __uint_as_float(r[c + e]));
+      const float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
+                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+      const float mx = mraw * scale_log2;   // scale_log2 > 0: the max commutes with it
       float factor = 1.f;
       bool resc = false;
       if (m_run == -INFINITY) {
@@ -293,90 +341,124 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         m_run = mx;
         resc = true;
       }
-      const float m_use = (m_run == -INFINITY) ? 0.f : m_run;
-      float sum = 0.f;
+      const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
+      // p = 2^(s * log2(e)/sqrt(d) - m), summed in eight chains, packed to bf16 pairs
+      float sum8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
 #pragma unroll
       for (int c = 0; c < 64; c += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(__uint_as_float(r[c + 2 * e]) - m_use);
-          const float p1 = ex2(__uint_as_float(r[c + 2 * e + 1]) - m_use);
-          sum += p0 + p1;
+          const float p0 = ex2(fmaf(__uint_as_float(r[c + 2 * e]), scale_log2, neg_m));
+          const float p1 = ex2(fmaf(__uint_as_float(r[c + 2 * e + 1]), scale_log2, neg_m));
+          sum8[e & 7] += p0 + p1;
           pk[e] = pack_bf16x2(p0, p1);
         }
         tmem_st16(tbase + lane_base + kColS + sb * 64 + c / 2, pk);
       }
+      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
+                        ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
       l_run = l_run * factor + sum;
       tmem_wait_st();
-      if (t > 0) {
-        if (!__all_sync(0xffffffffu, wait_bar(&sh.o_done, (t - 1) & 1, sh, err))) { ok = false; break; }
+      if (__any_sync(0xffffffffu, resc)) {
+        // O may be rescaled only once PV_{t-1} has landed in it.  MMAs complete in
+        // issue order and S_{t-1} (already waited for) was issued after PV_{t-3},
+        // so on the barrier of PV_{t-1}'s parity at most PV_{t-1} is outstanding and
+        // this parity wait is unambiguous although iterations without a rescale
+        // skip it; S_t (waited for) also implies PV_{t-2} has landed.
+        const int u = t - 1;
+        if (!__all_sync(0xffffffffu, wait_bar(&sh.o_done[u & 1], (u >> 1) & 1, sh, err))) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, resc)) {
 #pragma unroll
-          for (int c0 = 0; c0 < D; c0 += 32) {
-            uint32_t o[32];
-            tmem_ld32(tbase + lane_base + kColO + c0, o);
-            tmem_wait_ld();
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          uint32_t o[32];
+          tmem_ld32(tbase + lane_base + kColO + c0, o);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-            tmem_st32(tbase + lane_base + kColO + c0, o);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
+          tmem_st32(tbase + lane_base + kColO + c0, o);
         }
+        tmem_wait_st();
       }
       tc_fence_before();
       mbar_arrive(&sh.p_full[sb]);
     }
-    if (ok && t > 0) ok = __all_sync(0xffffffffu, wait_bar(&sh.o_done, (t - 1) & 1, sh, err));
+    // the last two PVs may both be outstanding: one wait on each parity's barrier
+    if (ok && t > 0) ok = __all_sync(0xffffffffu, wait_bar(&sh.o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, sh, err));
+    if (ok && t > 1) ok = __all_sync(0xffffffffu, wait_bar(&sh.o_done[(t - 2) & 1], ((t - 2) >> 1) & 1, sh, err));
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
-    // epilogue
-    const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-    float sg = 0.f;
-    size_t obase = 0;
-    if (row_valid) {
-      const float g = gate[static_cast<size_t>(qrow) * H + h];
-      sg = 1.f / (1.f + expf(-g));
-      obase = static_cast<size_t>(qrow) * H * D + static_cast<size_t>(h) * D;
-    }
+    const bool have_o = ok && t > 0;
+    if (kind >= 0) {
+      // one half of a split key list: hand the unnormalised state to k_combine
+      float* po = part.o + (static_cast<size_t>(slot) * kBM + row) * D;
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
-      uint32_t o[32];
-      if (ok && t > 0) {
-        tmem_ld32(tbase + lane_base + kColO + c0, o);
-        tmem_wait_ld();
-      } else {
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (have_o) {
+          tmem_ld32(tbase + lane_base + kColO + c0, o);
+          tmem_wait_ld();
+        } else {
 #pragma unroll
-        for (int e = 0; e < 32; ++e) o[e] = 0u;
-      }
-      if (!row_valid) continue;
-      float v[32];
-#pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
-      if (o_branch) {
-        float4* ob = reinterpret_cast<float4*>(o_branch + obase + c0);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ob[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
-      }
-      if (mode == 0) {
-        float4* lw = reinterpret_cast<float4*>(lin_ws + obase + c0);
-        const float a = 1.f - sg;
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
+        }
+        float4* p4 = reinterpret_cast<float4*>(po + c0);
 #pragma unroll
         for (int e = 0; e < 8; ++e)
-          lw[e] = make_float4(a * v[4 * e], a * v[4 * e + 1], a * v[4 * e + 2], a * v[4 * e + 3]);
-      } else {
-        const float4* lw = reinterpret_cast<const float4*>(lin_ws + obase + c0);
-        uint32_t pk[16];
+          p4[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
+                              __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+      }
+      *reinterpret_cast<float2*>(part.ml + (static_cast<size_t>(slot) * kBM + row) * 2) =
+          make_float2(m_run, l_run);
+    } else {
+      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      float sg = 0.f;
+      size_t obase = 0;
+      if (row_valid) {
+        const float g = gate[static_cast<size_t>(qrow) * H + h];
+        sg = 1.f / (1.f + expf(-g));
+        obase = static_cast<size_t>(qrow) * H * D + static_cast<size_t>(h) * D;
+      }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) {
-          const float4 l4 = lw[e];
-          pk[2 * e] = pack_bf16x2(sg * v[4 * e] + l4.x, sg * v[4 * e + 1] + l4.y);
-          pk[2 * e + 1] = pack_bf16x2(sg * v[4 * e + 2] + l4.z, sg * v[4 * e + 3] + l4.w);
+      for (int c0 = 0; c0 < D; c0 += 32) {
+        uint32_t o[32];
+        if (have_o) {
+          tmem_ld32(tbase + lane_base + kColO + c0, o);
+          tmem_wait_ld();
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) o[e] = 0u;
         }
-        uint4* op = reinterpret_cast<uint4*>(out + obase + c0);
+        if (!row_valid) continue;
+        float v[32];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) op[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
+        if (o_branch) {
+          float4* ob = reinterpret_cast<float4*>(o_branch + obase + c0);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) ob[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
+        }
+        if (mode == 0) {
+          float4* lw = reinterpret_cast<float4*>(lin_ws + obase + c0);
+          const float a = 1.f - sg;
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            lw[e] = make_float4(a * v[4 * e], a * v[4 * e + 1], a * v[4 * e + 2], a * v[4 * e + 3]);
+        } else {
+          const float4* lw = reinterpret_cast<const float4*>(lin_ws + obase + c0);
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float4 l4 = lw[e];
+            pk[2 * e] = pack_bf16x2(sg * v[4 * e] + l4.x, sg * v[4 * e + 1] + l4.y);
+            pk[2 * e + 1] = pack_bf16x2(sg * v[4 * e + 2] + l4.z, sg * v[4 * e + 3] + l4.w);
+          }
+          uint4* op = reinterpret_cast<uint4*>(out + obase + c0);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) op[e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        }
       }
     }
   }
@@ -388,28 +470,80 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   }
 }
 
+// Merge the two halves of a split pair: M = max(m0, m1), w_s = 2^(m_s - M),
+// O = (w0 O0 + w1 O1) / (w0 l0 + w1 l1); then out = bf16(sigmoid(g) O + lin_ws).
+// One CTA per pair, one thread per tile row.
+template <int D>
+__global__ void __launch_bounds__(128)
+k_combine(const int4* __restrict__ pairs, Partials part, int Nq, int H,
+          const float* __restrict__ gate, const float* __restrict__ lin_ws,
+          __nv_bfloat16* __restrict__ out, float* __restrict__ o_branch) {
+  const int4 pr = pairs[blockIdx.x];
+  if (pr.w < kSplitMin) return;               // written whole by the attention kernel
+  const int row = threadIdx.x;
+  const int half = row >> 6;
+  const int ib = half ? pr.z : pr.y;
+  const int qrow = ib * 64 + (row & 63);
+  if (ib < 0 || qrow >= Nq) return;
+  const int h = pr.x;
+  const size_t s0 = 2 * static_cast<size_t>(blockIdx.x), s1 = s0 + 1;
+  const float2 a = *reinterpret_cast<const float2*>(part.ml + (s0 * kBM + row) * 2);
+  const float2 b = *reinterpret_cast<const float2*>(part.ml + (s1 * kBM + row) * 2);
+  const float M = fmaxf(a.x, b.x);
+  const float w0 = a.x == -INFINITY ? 0.f : exp2f(a.x - M);
+  const float w1 = b.x == -INFINITY ? 0.f : exp2f(b.x - M);
+  const float lsum = w0 * a.y + w1 * b.y;
+  const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
+  const float c0w = w0 * inv, c1w = w1 * inv;
+  const float g = gate[static_cast<size_t>(qrow) * H + h];
+  const float sg = 1.f / (1.f + expf(-g));
+  const float4* o0 = reinterpret_cast<const float4*>(part.o + (s0 * kBM + row) * D);
+  const float4* o1 = reinterpret_cast<const float4*>(part.o + (s1 * kBM + row) * D);
+  const size_t obase = static_cast<size_t>(qrow) * H * D + static_cast<size_t>(h) * D;
+  const float4* lw = reinterpret_cast<const float4*>(lin_ws + obase);
+  uint2* op = reinterpret_cast<uint2*>(out + obase);
+#pragma unroll 4
+  for (int e = 0; e < D / 4; ++e) {
+    const float4 x = o0[e], y = o1[e], l4 = lw[e];
+    const float v0 = c0w * x.x + c1w * y.x, v1 = c0w * x.y + c1w * y.y;
+    const float v2 = c0w * x.z + c1w * y.z, v3 = c0w * x.w + c1w * y.w;
+    if (o_branch) reinterpret_cast<float4*>(o_branch + obase)[e] = make_float4(v0, v1, v2, v3);
+    op[e] = make_uint2(pack_bf16x2(sg * v0 + l4.x, sg * v1 + l4.y),
+                       pack_bf16x2(sg * v2 + l4.z, sg * v3 + l4.w));
+  }
+}
+
 // ------------------------------------------------------------------ work items
 // One CTA per head pairs its query blocks greedily by the smallest symmetric
 // difference of their key-block sets (fewest masked half-blocks), falling back
 // to neighbours when there are too many blocks for the distance table.
-constexpr int kMaxPairTable = 144;  // 144^2 uint16 distances fit in static shared memory
+// pairs[h * n_pairs + k] = (h, first block, second block or -1, union size).
+constexpr int kMaxPairTable = 128;
+constexpr int kMaxPairMaskWords = 3072;   // staged masks of one head (n_qb * W words)
 
-__global__ void k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W,
-                             int4* __restrict__ items) {
+__global__ void __launch_bounds__(256)
+k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W, int4* __restrict__ pairs) {
   __shared__ uint16_t dist[kMaxPairTable * kMaxPairTable];
+  __shared__ uint32_t ms[kMaxPairMaskWords];
   __shared__ unsigned char paired[kMaxPairTable];
+  __shared__ int2 chosen[kMaxPairTable];
   const int h = blockIdx.x;
   const int n_pairs = (n_qb + 1) / 2;
   const uint32_t* mh = mask + static_cast<size_t>(h) * n_qb * W;
+  const bool staged = n_qb * W <= kMaxPairMaskWords;
+  if (staged)
+    for (int e = threadIdx.x; e < n_qb * W; e += blockDim.x) ms[e] = mh[e];
+  __syncthreads();
+  const uint32_t* m = staged ? ms : mh;
   auto union_count = [&](int a, int b) {
     int c = 0;
-    for (int w = 0; w < W; ++w) c += __popc(mh[a * W + w] | (b >= 0 ? mh[b * W + w] : 0u));
+    for (int w = 0; w < W; ++w) c += __popc(m[a * W + w] | (b >= 0 ? m[b * W + w] : 0u));
     return c;
   };
   if (n_qb > kMaxPairTable) {
     for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
       const int a = 2 * p, b = (2 * p + 1 < n_qb) ? 2 * p + 1 : -1;
-      items[static_cast<size_t>(h) * n_pairs + p] = make_int4(h, a, b, union_count(a, b));
+      pairs[static_cast<size_t>(h) * n_pairs + p] = make_int4(h, a, b, union_count(a, b));
     }
     return;
   }
@@ -417,7 +551,7 @@ __global__ void k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W,
     const int a = e / n_qb, b = e % n_qb;
     int c = 0;
     if (a < b)
-      for (int w = 0; w < W; ++w) c += __popc(mh[a * W + w] ^ mh[b * W + w]);
+      for (int w = 0; w < W; ++w) c += __popc(m[a * W + w] ^ m[b * W + w]);
     dist[e] = static_cast<uint16_t>(min(c, 65535));
   }
   for (int a = threadIdx.x; a < n_qb; a += blockDim.x) paired[a] = 0;
@@ -443,7 +577,7 @@ __global__ void k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W,
       if (lane == 0) {
         paired[a] = 1;
         if (bi >= 0) paired[bi] = 1;
-        items[static_cast<size_t>(h) * n_pairs + k] = make_int4(h, a, bi, 0);
+        chosen[k] = make_int2(a, bi);
       }
       __syncwarp();
       ++k;
@@ -451,98 +585,170 @@ __global__ void k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W,
   }
   __syncthreads();
   for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
-    int4 it = items[static_cast<size_t>(h) * n_pairs + p];
-    it.w = union_count(it.y, it.z);
-    items[static_cast<size_t>(h) * n_pairs + p] = it;
+    const int2 c = chosen[p];
+    pairs[static_cast<size_t>(h) * n_pairs + p] = make_int4(h, c.x, c.y, union_count(c.x, c.y));
   }
 }
 
-// Longest-first order (ties by head, then first block) with one CTA's bitonic sort.
-constexpr int kMaxSortItems = 4096;
+// Two work items per pair -- both halves of a split key list, or the whole list
+// and an empty placeholder -- ordered longest first by a counting sort on the
+// item length (order among equal lengths is arbitrary: it affects only the
+// schedule, never a result).  One CTA.
+constexpr int kLenBins = 1024;
 
-__device__ __forceinline__ bool item_before(int4 a, int4 b) {
-  if (a.w != b.w) return a.w > b.w;
-  if (a.x != b.x) return a.x < b.x;
-  return a.y < b.y;
-}
-
-__global__ void __launch_bounds__(1024) k_sort_items(int4* __restrict__ items, int n, int NP) {
-  extern __shared__ int4 buf[];
-  for (int e = threadIdx.x; e < NP; e += blockDim.x)
-    buf[e] = e < n ? items[e] : make_int4(INT_MAX, INT_MAX, INT_MAX, -1);
+__global__ void __launch_bounds__(1024)
+k_make_items(const int4* __restrict__ pairs, int n_pairs, int shift, int4* __restrict__ items) {
+  __shared__ int hist[kLenBins];
+  __shared__ int base[kLenBins];
+  __shared__ int wsum[32];
+  for (int e = threadIdx.x; e < kLenBins; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  for (int k = 2; k <= NP; k <<= 1) {
-    for (int js = k >> 1; js > 0; js >>= 1) {
-      for (int p = threadIdx.x; p < NP / 2; p += blockDim.x) {
-        const int i = 2 * js * (p / js) + (p % js), l = i + js;
-        const int4 a = buf[i], b = buf[l];
-        const bool up = (i & k) == 0;
-        const bool sw = up ? item_before(b, a) : item_before(a, b);
-        if (sw) { buf[i] = b; buf[l] = a; }
-      }
-      __syncthreads();
+  auto bin_of = [&](int len) { return kLenBins - 1 - min(kLenBins - 1, len >> shift); };  // long first
+  for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
+    const int cnt = pairs[p].w;
+    if (cnt >= kSplitMin) {
+      atomicAdd(&hist[bin_of(cnt / 2)], 1);
+      atomicAdd(&hist[bin_of(cnt - cnt / 2)], 1);
+    } else {
+      atomicAdd(&hist[bin_of(cnt)], 1);
+      atomicAdd(&hist[kLenBins - 1], 1);
     }
   }
-  for (int e = threadIdx.x; e < n; e += blockDim.x) items[e] = buf[e];
+  __syncthreads();
+  // exclusive scan of hist (1024 bins, one per thread)
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  const int v = threadIdx.x < kLenBins ? hist[threadIdx.x] : 0;
+  int incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) wsum[wid] = incl;
+  __syncthreads();
+  int off = 0;
+  for (int w = 0; w < wid; ++w) off += wsum[w];
+  if (threadIdx.x < kLenBins) base[threadIdx.x] = off + incl - v;
+  __syncthreads();
+  for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
+    const int cnt = pairs[p].w;
+    if (cnt >= kSplitMin) {
+      const int hlf = cnt / 2;
+      items[atomicAdd(&base[bin_of(hlf)], 1)] = make_int4(p, 0, 0, hlf);
+      items[atomicAdd(&base[bin_of(cnt - hlf)], 1)] = make_int4(p, 1, hlf, cnt);
+    } else {
+      items[atomicAdd(&base[bin_of(cnt)], 1)] = make_int4(p, kWhole, 0, cnt);
+      items[atomicAdd(&base[kLenBins - 1], 1)] = make_int4(p, kEmpty, 0, 0);
+    }
+  }
 }
 
 }  // namespace
 
-size_t attn_items_ws_bytes(int H, int n_qb) {
-  return static_cast<size_t>(H) * ((n_qb + 1) / 2) * sizeof(int4);
-}
-
-wa_status launch_attn_items(const uint32_t* blk_mask, int H, int n_qb, int n_kb, int4* items,
-                            void* /*scratch*/, cudaStream_t st) {
-  const int W = (n_kb + 31) / 32;
-  k_pair_heads<<<H, 256, 0, st>>>(blk_mask, n_qb, W, items);
-  const int n = H * ((n_qb + 1) / 2);
-  if (n <= kMaxSortItems) {
-    int NP = 1;
-    while (NP < n) NP <<= 1;
-    if (NP < 2) NP = 2;
-    cudaFuncSetAttribute(k_sort_items, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                         static_cast<int>(NP * sizeof(int4)));
-    k_sort_items<<<1, 1024, NP * sizeof(int4), st>>>(items, n, NP);
-  }
-  return check_launch("attn_items");
+size_t sparse_attn_ws_bytes(int H, int Nq, int d, int B) {
+  const size_t n_pairs = static_cast<size_t>(H) * (((Nq + B - 1) / B + 1) / 2);
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  return al(n_pairs * sizeof(int4)) + al(2 * n_pairs * sizeof(int4)) +
+         al(2 * n_pairs * kBM * d * sizeof(float)) + al(2 * n_pairs * kBM * 2 * sizeof(float));
 }
 
 bool make_tmap_bf16_2d(void* tmap, const void* base, uint64_t inner, uint64_t outer,
                        uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer);
 
-wa_status launch_umma_attention(int mode, const void* q, int Nq, int H, int d, RowSource rs,
-                                int B, const uint32_t* blk_mask, int W, const int4* items,
-                                int n_items, const float* gate, float* lin_ws, void* out,
-                                float* o_branch, uint32_t* err, cudaStream_t st) {
-  if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
-  if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs d in {64,128}");
-  if (W > kMaxW) return set_error(WA_ERR_UNSUPPORTED, "too many key blocks (max %d)", kMaxW * 32);
+namespace {
+template <int D>
+void launch_attn_kernel(int grid, cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& tk,
+                        const CUtensorMap& tv, int mode, int Nq, int H, RowSource rs,
+                        const uint32_t* blk_mask, int W, int n_qb, const int4* pairs,
+                        const int4* items, Partials part, const float* gate, float* lin_ws,
+                        void* out, float* o_branch, uint32_t* err) {
+  const int smem = Cfg<D>::kSmem;
+  cudaFuncSetAttribute(k_umma_attention<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  k_umma_attention<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, mode, Nq, H, rs.L, rs, blk_mask, W,
+                                                     n_qb, pairs, items, part, gate, lin_ws,
+                                                     static_cast<__nv_bfloat16*>(out), o_branch, err);
+}
+
+wa_status make_maps(const void* q, int Nq, int H, int d, const RowSource& rs, CUtensorMap* tq,
+                    CUtensorMap* tk, CUtensorMap* tv) {
   const int cols = H * d;
-  alignas(64) CUtensorMap tq, tk, tv;
   const uint64_t key_rows = rs.page_ids ? static_cast<uint64_t>(rs.n_pages) * rs.page_rows
                                         : static_cast<uint64_t>(rs.L);
-  if (!make_tmap_bf16_2d(&tq, q, cols, Nq, static_cast<uint64_t>(cols) * 2, 64, 64) ||
-      !make_tmap_bf16_2d(&tk, rs.k, cols, key_rows, static_cast<uint64_t>(cols) * 2, 64, 64) ||
-      !make_tmap_bf16_2d(&tv, rs.v, cols, key_rows, static_cast<uint64_t>(cols) * 2, 64, 64))
+  if (!make_tmap_bf16_2d(tq, q, cols, Nq, static_cast<uint64_t>(cols) * 2, 64, 64) ||
+      !make_tmap_bf16_2d(tk, rs.k, cols, key_rows, static_cast<uint64_t>(cols) * 2, 64, 64) ||
+      !make_tmap_bf16_2d(tv, rs.v, cols, key_rows, static_cast<uint64_t>(cols) * 2, 64, 64))
     return set_error(WA_ERR_CUDA, "cuTensorMapEncodeTiled failed for the attention operands");
+  return WA_OK;
+}
+}  // namespace
+
+wa_status launch_linear_attention(const void* q, int Nq, int H, int d, RowSource lin, int B,
+                                  const float* gate, float* lin_ws, float* o_lin, uint32_t* err,
+                                  cudaStream_t st) {
+  if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
+  if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs d in {64,128}");
+  alignas(64) CUtensorMap tq, tk, tv;
+  wa_status s = make_maps(q, Nq, H, d, lin, &tq, &tk, &tv);
+  if (s != WA_OK) return s;
   const int n_qb = (Nq + B - 1) / B;
-  const int grid = mode == 0 ? H * ((n_qb + 1) / 2) : n_items;
-  if (grid == 0) return WA_OK;
+  const int grid = H * ((n_qb + 1) / 2);
+  Partials none{nullptr, nullptr};
+  if (d == 128)
+    launch_attn_kernel<128>(grid, st, tq, tk, tv, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
+                            none, gate, lin_ws, nullptr, o_lin, err);
+  else
+    launch_attn_kernel<64>(grid, st, tq, tk, tv, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
+                           none, gate, lin_ws, nullptr, o_lin, err);
+  return check_launch("linear attention");
+}
+
+wa_status launch_sparse_attention(const void* q, int Nq, int H, int d, RowSource rs, int B,
+                                  const uint32_t* blk_mask, const float* gate, const float* lin_ws,
+                                  void* out, float* o_sp, void* scratch, uint32_t* err,
+                                  cudaStream_t st, void* const* events) {
+  if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
+  if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs d in {64,128}");
+  const int n_qb = (Nq + B - 1) / B;
+  const int n_kb = (rs.L + B - 1) / B;
+  const int W = (n_kb + 31) / 32;
+  if (W > kMaxW) return set_error(WA_ERR_UNSUPPORTED, "too many key blocks (max %d)", kMaxW * 32);
+  const int n_pairs = H * ((n_qb + 1) / 2);
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  char* p = static_cast<char*>(scratch);
+  int4* pairs = reinterpret_cast<int4*>(p);
+  p += al(n_pairs * sizeof(int4));
+  int4* items = reinterpret_cast<int4*>(p);
+  p += al(2 * static_cast<size_t>(n_pairs) * sizeof(int4));
+  Partials part;
+  part.o = reinterpret_cast<float*>(p);
+  p += al(2 * static_cast<size_t>(n_pairs) * kBM * d * sizeof(float));
+  part.ml = reinterpret_cast<float*>(p);
+
+  k_pair_heads<<<H, 256, 0, st>>>(blk_mask, n_qb, W, pairs);
+  int shift = 0;
+  while ((n_kb >> shift) >= kLenBins) ++shift;
+  k_make_items<<<1, 1024, 0, st>>>(pairs, n_pairs, shift, items);
+  wa_status s = check_launch("attention work list");
+  if (s != WA_OK) return s;
+  if (events && events[6]) cudaEventRecord(static_cast<cudaEvent_t>(events[6]), st);
+
+  alignas(64) CUtensorMap tq, tk, tv;
+  s = make_maps(q, Nq, H, d, rs, &tq, &tk, &tv);
+  if (s != WA_OK) return s;
+  const int grid = 2 * n_pairs;
+  float* lin_rw = const_cast<float*>(lin_ws);
   if (d == 128) {
-    const int smem = Cfg<128>::kSmem;
-    cudaFuncSetAttribute(k_umma_attention<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    k_umma_attention<128><<<grid, kThreads, smem, st>>>(
-        tq, tk, tv, mode, Nq, H, rs.L, rs, blk_mask, W, n_qb, items, gate, lin_ws,
-        static_cast<__nv_bfloat16*>(out), o_branch, err);
+    launch_attn_kernel<128>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, W, n_qb, pairs, items, part,
+                            gate, lin_rw, out, o_sp, err);
+    k_combine<128><<<n_pairs, 128, 0, st>>>(pairs, part, Nq, H, gate, lin_ws,
+                                            static_cast<__nv_bfloat16*>(out), o_sp);
   } else {
-    const int smem = Cfg<64>::kSmem;
-    cudaFuncSetAttribute(k_umma_attention<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-    k_umma_attention<64><<<grid, kThreads, smem, st>>>(
-        tq, tk, tv, mode, Nq, H, rs.L, rs, blk_mask, W, n_qb, items, gate, lin_ws,
-        static_cast<__nv_bfloat16*>(out), o_branch, err);
+    launch_attn_kernel<64>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, W, n_qb, pairs, items, part,
+                           gate, lin_rw, out, o_sp, err);
+    k_combine<64><<<n_pairs, 128, 0, st>>>(pairs, part, Nq, H, gate, lin_ws,
+                                           static_cast<__nv_bfloat16*>(out), o_sp);
   }
-  return check_launch("umma_attention");
+  return check_launch("sparse attention");
 }
 
 }  // namespace wa

@@ -143,25 +143,30 @@ uint32_t* errw() { return device_error_word(); }
 // ---- S1 internals (shared by wa_page_score and wa_hsa_step)
 struct PageScoreWs {
   double* q_blocksum;   // [n_qb][cols]
-  double* q_partial;    // [q_split][cols]
+  double* qbar;         // [cols]
+  double* q_blockmean;  // [n_qb][cols]
   double* k_blocksum;   // [n_c][nbp][cols] (nullable)
-  double* k_partial;    // [n_c][k_split][cols]
-  int q_split, k_split;
+  double* kdot;         // [n_c][k_split * k_cc]
+  RowsumPlan qp, kp;
 };
 
-PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks) {
+PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks,
+                             wa_dtype dt) {
   PageScoreWs w{};
   const int cols = H * d;
   const int n_qb = ceil_div(Nq, B);
-  w.q_split = rowsum_splits(1, Nq, B);
-  w.k_split = rowsum_splits(n_c, T_p, B);
+  w.qp = rowsum_plan(1, Nq, cols, B, dt);
+  w.kp = rowsum_plan(n_c, T_p, cols, B, dt);
   w.q_blocksum = c.take<double>(static_cast<size_t>(n_qb) * cols);
-  w.q_partial = c.take<double>(static_cast<size_t>(w.q_split) * cols);
+  w.qbar = c.take<double>(cols);
+  w.q_blockmean = c.take<double>(static_cast<size_t>(n_qb) * cols);
   w.k_blocksum = k_blocks ? c.take<double>(static_cast<size_t>(n_c) * ceil_div(T_p, B) * cols) : nullptr;
-  w.k_partial = c.take<double>(static_cast<size_t>(n_c) * w.k_split * cols);
+  w.kdot = c.take<double>(static_cast<size_t>(n_c) * w.kp.n_split * w.kp.n_cc);
   return w;
 }
 
+// Q pass (block sums), query means, then the K pass over the candidate pages with
+// the page-score dot products fused in, then alpha and the top-K_p pages.
 wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int d,
                          const void* k_pool, int n_pool_pages, int T_p, const int32_t* cand,
                          int n_c, int K_p, int B, wa_dtype dt, double* alpha, int32_t* sel,
@@ -169,12 +174,13 @@ wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int
   const int cols = H * d;
   uint32_t* err = errw();
   if (!err) return set_error(WA_ERR_CUDA, "no device error word (is a CUDA device present?)");
-  WA_TRY(launch_rowblock_sum(q, dt, nullptr, 1, 1, Nq, cols, B, w.q_blocksum, w.q_partial,
-                             w.q_split, err, st));
-  WA_TRY(launch_rowblock_sum(k_pool, dt, cand, n_c, n_pool_pages, T_p, cols, B, w.k_blocksum,
-                             w.k_partial, w.k_split, err, st));
-  return launch_page_alpha_topk(w.q_partial, w.q_split, Nq, w.k_partial, w.k_split, T_p, n_c, H,
-                                d, K_p, cand, alpha, sel, sel_pos, st);
+  WA_TRY(launch_rowblock_sum(q, dt, nullptr, 1, 1, Nq, cols, B, w.q_blocksum, nullptr, nullptr, w.qp,
+                             err, st));
+  WA_TRY(launch_qmeans(w.q_blocksum, ceil_div(Nq, B), Nq, B, cols, w.qbar, w.q_blockmean, st));
+  WA_TRY(launch_rowblock_sum(k_pool, dt, cand, n_c, n_pool_pages, T_p, cols, B, w.k_blocksum, w.qbar,
+                             w.kdot, w.kp, err, st));
+  return launch_alpha_topk(w.kdot, w.kp.n_split * w.kp.n_cc, n_c, T_p, H, d, K_p, cand, alpha, sel,
+                           sel_pos, st);
 }
 
 }  // namespace wa_detail
@@ -216,9 +222,12 @@ wa_status wa_prompt_select(const float* e_cur, const float* e_chunks, int n_chun
 size_t wa_page_score_workspace_size(int Nq, int H, int d, int n_c, int T_p, int B) {
   if (Nq < 1 || H < 1 || d < 1 || n_c < 1 || T_p < 1 || B < 1) return 0;
   Carver c(nullptr);
-  carve_page_score(c, Nq, H, d, n_c, T_p, B, true);
+  carve_page_score(c, Nq, H, d, n_c, T_p, B, true, WA_BF16);
   c.take<int32_t>(n_c);
-  return c.used;
+  Carver c2(nullptr);
+  carve_page_score(c2, Nq, H, d, n_c, T_p, B, true, WA_F32);
+  c2.take<int32_t>(n_c);
+  return c.used > c2.used ? c.used : c2.used;
 }
 
 wa_status wa_page_score(const void* q, int Nq, int H, int d, const void* k_pool, int n_pool_pages,
@@ -235,7 +244,7 @@ wa_status wa_page_score(const void* q, int Nq, int H, int d, const void* k_pool,
   WA_TRY(check_ws(ws, ws_bytes, wa_page_score_workspace_size(Nq, H, d, n_c, T_p, B)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carver c(ws);
-  PageScoreWs w = carve_page_score(c, Nq, H, d, n_c, T_p, B, true);
+  PageScoreWs w = carve_page_score(c, Nq, H, d, n_c, T_p, B, true, dtype);
   int32_t* sel_pos = c.take<int32_t>(n_c);
   WA_TRY(run_page_score(w, q, Nq, H, d, k_pool, n_pool_pages, T_p, cand_pages, n_c, K_p, B, dtype,
                         alpha, sel, sel_pos, st));
@@ -264,14 +273,34 @@ wa_status wa_gather_pages(const void* k_pool, const void* v_pool, int n_pool_pag
 }
 
 // ------------------------------------------------------------------ S3
+namespace wa_detail {
+struct BlockSelectWs {
+  double* qsum;
+  double* qbar;
+  double* qmean;
+  double* ksum;
+  double* scores;
+  RowsumPlan qp, kp;
+};
+BlockSelectWs carve_block_select(Carver& c, int Nq, int H, int d, int L, int B, wa_dtype dt) {
+  BlockSelectWs w{};
+  const int cols = H * d;
+  const int n_qb = ceil_div(Nq, B), n_kb = ceil_div(L, B);
+  w.qp = rowsum_plan(1, Nq, cols, B, dt);
+  w.kp = rowsum_plan(1, L, cols, B, dt);
+  w.qsum = c.take<double>(static_cast<size_t>(n_qb) * cols);
+  w.qbar = c.take<double>(cols);
+  w.qmean = c.take<double>(static_cast<size_t>(n_qb) * cols);
+  w.ksum = c.take<double>(static_cast<size_t>(n_kb) * cols);
+  w.scores = reinterpret_cast<double*>(c.take<char>(block_scores_bytes(H, n_qb, n_kb)));
+  return w;
+}
+}  // namespace wa_detail
+
 size_t wa_block_select_workspace_size(int Nq, int H, int d, int L, int B) {
   if (Nq < 1 || H < 1 || d < 1 || L < 1 || B < 1) return 0;
   Carver c(nullptr);
-  const int cols = H * d;
-  c.take<double>(static_cast<size_t>(ceil_div(Nq, B)) * cols);           // q block sums
-  c.take<double>(static_cast<size_t>(rowsum_splits(1, Nq, B)) * cols);   // q partials
-  c.take<double>(static_cast<size_t>(ceil_div(L, B)) * cols);            // k block sums
-  c.take<double>(static_cast<size_t>(rowsum_splits(1, L, B)) * cols);    // k partials
+  carve_block_select(c, Nq, H, d, L, B, WA_F32);
   return c.used;
 }
 
@@ -291,25 +320,24 @@ wa_status wa_block_select(const void* q, int Nq, int H, int d, const void* k_act
   if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carver c(ws);
+  BlockSelectWs w = carve_block_select(c, Nq, H, d, L, B, dtype);
   const int cols = H * d;
-  const int q_split = rowsum_splits(1, Nq, B);
-  double* qsum = c.take<double>(static_cast<size_t>(ceil_div(Nq, B)) * cols);
-  double* qpart = c.take<double>(static_cast<size_t>(q_split) * cols);
-  double* ksum = c.take<double>(static_cast<size_t>(n_kb) * cols);
-  const int k_split = rowsum_splits(1, L, B);
-  double* kpart = c.take<double>(static_cast<size_t>(k_split) * cols);
-  WA_TRY(launch_rowblock_sum(q, dtype, nullptr, 1, 1, Nq, cols, B, qsum, qpart, q_split, err, st));
+  WA_TRY(launch_rowblock_sum(q, dtype, nullptr, 1, 1, Nq, cols, B, w.qsum, nullptr, nullptr, w.qp,
+                             err, st));
+  WA_TRY(launch_qmeans(w.qsum, ceil_div(Nq, B), Nq, B, cols, w.qbar, w.qmean, st));
   KeyMeans km;
   km.L = L;
   if (k_act) {
-    WA_TRY(launch_rowblock_sum(k_act, dtype, nullptr, 1, 1, L, cols, B, ksum, kpart, k_split, err, st));
-    km.data = ksum;
+    WA_TRY(launch_rowblock_sum(k_act, dtype, nullptr, 1, 1, L, cols, B, w.ksum, nullptr, nullptr,
+                               w.kp, err, st));
+    km.data = w.ksum;
     km.is_sum = 1;
   } else {
     km.data = k_blockmean;
     km.is_sum = 0;
   }
-  return launch_block_select(qsum, Nq, H, d, B, km, n_kb, tau, blk_idx, blk_cnt, blk_mask, st);
+  return launch_block_select(w.qmean, Nq, H, d, B, km, n_kb, tau, w.scores, blk_idx, blk_cnt,
+                             blk_mask, st);
 }
 
 // ------------------------------------------------------------------ S4a
@@ -346,7 +374,7 @@ size_t wa_hsa_attention_workspace_size(int Nq, int H, int d, int L, int B, int r
   if (Nq < 1 || H < 1 || d < 1 || L < 1 || B < 1 || r < 1) return 0;
   Carver c(nullptr);
   c.take<float>(static_cast<size_t>(Nq) * H * d);                  // gated linear branch
-  if (dtype == WA_BF16) c.take<char>(attn_items_ws_bytes(H, ceil_div(Nq, B)));
+  if (dtype == WA_BF16) c.take<char>(sparse_attn_ws_bytes(H, Nq, d, B));
   return c.used;
 }
 
@@ -354,7 +382,7 @@ namespace wa_detail {
 wa_status run_attention(const void* q, int Nq, int H, int d, RowSource rs, int B,
                         const uint32_t* blk_mask, const void* k_til, const void* v_til, int r,
                         const float* gate, wa_dtype dtype, void* out, float* o_sp, float* o_lin,
-                        float* lin_ws, int4* items, cudaStream_t st,
+                        float* lin_ws, void* scratch, cudaStream_t st,
                         void* const* events = nullptr) {
   auto mark = [&](int k) {
     if (events && events[k]) cudaEventRecord(static_cast<cudaEvent_t>(events[k]), st);
@@ -367,13 +395,10 @@ wa_status run_attention(const void* q, int Nq, int H, int d, RowSource rs, int B
   RowSource lin;
   lin.k = k_til; lin.v = v_til; lin.page_rows = r; lin.n_pages = 1; lin.L = r;
   if (dtype == WA_BF16) {
-    WA_TRY(launch_umma_attention(0, q, Nq, H, d, lin, B, nullptr, 0, nullptr, 0, gate, lin_ws,
-                                 nullptr, o_lin, err, st));
+    WA_TRY(launch_linear_attention(q, Nq, H, d, lin, B, gate, lin_ws, o_lin, err, st));
     mark(5);
-    WA_TRY(launch_attn_items(blk_mask, H, n_qb, n_kb, items, nullptr, st));
-    mark(6);
-    return launch_umma_attention(1, q, Nq, H, d, rs, B, blk_mask, W, items, H * ((n_qb + 1) / 2),
-                                 gate, lin_ws, out, o_sp, err, st);
+    return launch_sparse_attention(q, Nq, H, d, rs, B, blk_mask, gate, lin_ws, out, o_sp, scratch,
+                                   err, st, events);
   }
   WA_TRY(launch_simt_attention(0, static_cast<const float*>(q), Nq, H, d, lin, B, nullptr, 0, gate,
                                lin_ws, nullptr, o_lin, err, st));
@@ -404,11 +429,11 @@ wa_status wa_hsa_attention(const void* q, int Nq, int H, int d, const void* k_ac
   WA_TRY(check_ws(ws, ws_bytes, wa_hsa_attention_workspace_size(Nq, H, d, L, B, r, dtype)));
   Carver c(ws);
   float* lin_ws = c.take<float>(static_cast<size_t>(Nq) * H * d);
-  int4* items = dtype == WA_BF16 ? reinterpret_cast<int4*>(c.take<char>(attn_items_ws_bytes(H, ceil_div(Nq, B)))) : nullptr;
+  void* scratch = dtype == WA_BF16 ? c.take<char>(sparse_attn_ws_bytes(H, Nq, d, B)) : nullptr;
   RowSource rs;
   rs.k = k_act; rs.v = v_act; rs.page_rows = L; rs.n_pages = 1; rs.L = L;
   return run_attention(q, Nq, H, d, rs, B, blk_mask, k_til, v_til, r, gate, dtype, out, o_sp, o_lin,
-                       lin_ws, items, static_cast<cudaStream_t>(stream));
+                       lin_ws, scratch, static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------------ step
@@ -425,11 +450,11 @@ struct StepWs {
   void* v_til;
   void* proj;
   float* lin;
-  int4* items;
+  void* attn;         // sparse-attention work list and partials
   void* k_act;
   void* v_act;
   double* ksum;     // non-fused: block sums of the gathered keys
-  double* kpart;
+  double* scores;   // float64 pooled block scores
 };
 
 wa_status validate_step(const wa_step_args* a) {
@@ -462,7 +487,8 @@ StepWs carve_step(Carver& c, const wa_step_args* a) {
   w.chunk = c.take<int32_t>(1);
   w.cand = c.take<int32_t>(a->n_c);
   // block sums of the candidate pages are only needed when selection reads them
-  w.ps = carve_page_score(c, a->Nq, a->H, a->d, a->n_c, a->T_p, a->B, a->fused_gather != 0);
+  w.ps = carve_page_score(c, a->Nq, a->H, a->d, a->n_c, a->T_p, a->B, a->fused_gather != 0,
+                          a->dtype);
   w.alpha = c.take<double>(a->n_c);
   w.sel = c.take<int32_t>(a->K_p);
   w.sel_pos = c.take<int32_t>(a->K_p);
@@ -471,13 +497,13 @@ StepWs carve_step(Carver& c, const wa_step_args* a) {
   w.v_til = c.take<char>(static_cast<size_t>(a->r) * cols * es);
   w.proj = c.take<char>(a->dtype == WA_BF16 ? umma_project_ws_bytes(L, a->H, a->d, a->r) : 0);
   w.lin = c.take<float>(static_cast<size_t>(a->Nq) * cols);
-  w.items = reinterpret_cast<int4*>(c.take<char>(attn_items_ws_bytes(a->H, n_qb)));
+  w.scores = reinterpret_cast<double*>(c.take<char>(block_scores_bytes(a->H, n_qb, n_kb)));
+  w.attn = c.take<char>(a->dtype == WA_BF16 ? sparse_attn_ws_bytes(a->H, a->Nq, a->d, a->B) : 0);
   if (!a->fused_gather) {
     w.k_act = c.take<char>(static_cast<size_t>(L) * cols * es);
     w.v_act = c.take<char>(static_cast<size_t>(L) * cols * es);
     // k block sums of the gathered buffer for selection
     w.ksum = c.take<double>(static_cast<size_t>(n_kb) * cols);
-    w.kpart = c.take<double>(static_cast<size_t>(rowsum_splits(1, L, a->B)) * cols);
   }
   return w;
 }
@@ -548,16 +574,16 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
     WA_TRY(launch_gather(a->k_pool, a->v_pool, a->n_pool_pages, page_bytes, sel, a->K_p, w.k_act,
                          w.v_act, err, st));
     rs.k = w.k_act; rs.v = w.v_act; rs.page_rows = L; rs.n_pages = 1; rs.L = L;
-    WA_TRY(launch_rowblock_sum(w.k_act, a->dtype, nullptr, 1, 1, L, cols, a->B, w.ksum, w.kpart,
-                               rowsum_splits(1, L, a->B), err, st));
+    WA_TRY(launch_rowblock_sum(w.k_act, a->dtype, nullptr, 1, 1, L, cols, a->B, w.ksum, nullptr,
+                               nullptr, rowsum_plan(1, L, cols, a->B, a->dtype), err, st));
     km.data = w.ksum;
   }
 
   mark(2);
   // S3: block selection
   uint32_t* mask = a->blk_mask_out ? a->blk_mask_out : w.mask;
-  WA_TRY(launch_block_select(w.ps.q_blocksum, a->Nq, a->H, a->d, a->B, km, n_kb, a->tau, nullptr,
-                             nullptr, mask, st));
+  WA_TRY(launch_block_select(w.ps.q_blockmean, a->Nq, a->H, a->d, a->B, km, n_kb, a->tau, w.scores,
+                             nullptr, nullptr, mask, st));
   (void)W;
   (void)n_qb;
 
@@ -579,7 +605,7 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
   mark(4);
   // S4b + S5 + S6
   WA_TRY(run_attention(a->q, a->Nq, a->H, a->d, rs, a->B, mask, kt, vt, a->r, a->gate, a->dtype,
-                       a->out, nullptr, nullptr, w.lin, w.items, st, a->stage_events));
+                       a->out, nullptr, nullptr, w.lin, w.attn, st, a->stage_events));
   mark(7);
   return WA_OK;
 }

@@ -33,25 +33,33 @@ uint32_t* device_error_word();  // current device's error word (device address)
 wa_status launch_prompt_select(const float* e_cur, const float* e_chunks, int n_chunks, int D,
                                int32_t* chunk_out, uint32_t* err, cudaStream_t st);
 
-// Row-block sums in float64.  Sums B-row blocks of `n_src` sources of `rows`
-// rows each (a source is a pool page given by src_ids, or the buffer itself when
-// src_ids == nullptr) over cols = H*d columns:
-//   blocksum[s][b][c]    (nullable)   sum of rows [b*B, min(rows,(b+1)*B)) of source s
-//   partial [s][split][c]             per-CTA running sums (page totals = sum over split)
-// Returns the number of splits in *n_split.
-int rowsum_splits(int n_src, int rows, int B);
+// Row-block sums in float64 over B-row blocks of `n_src` sources of `rows` rows
+// each (a source is a pool page given by src_ids, or the buffer itself when
+// src_ids == nullptr), cols = H*d columns:
+//   blocksum[s][b][c]  (nullable)  sum of rows [b*B, min(rows,(b+1)*B)) of source s
+//   kdot[s][split][cc] (with qbar) dot product of qbar with the CTA's column sums
+struct RowsumPlan {
+  int threads = 0;   // threads per CTA (V columns each)
+  int n_cc = 1;      // column chunks
+  int nb = 0;        // blocks per source
+  int bps = 1;       // blocks per CTA
+  int n_split = 1;   // CTAs per source and column chunk
+};
+RowsumPlan rowsum_plan(int n_src, int rows, int cols, int B, wa_dtype dt);
 wa_status launch_rowblock_sum(const void* x, wa_dtype dt, const int32_t* src_ids, int n_src,
                               int n_pages, int rows, int cols, int B, double* blocksum,
-                              double* partial, int n_split, uint32_t* err, cudaStream_t st);
+                              const double* qbar, double* kdot, const RowsumPlan& p, uint32_t* err,
+                              cudaStream_t st);
+// qbar[c] = sum_i qsum[i][c] / Nq; qmean[i][c] (nullable) = qsum[i][c] / rows of block i.
+wa_status launch_qmeans(const double* qsum, int n_qb, int Nq, int B, int cols, double* qbar,
+                        double* qmean, cudaStream_t st);
+// S1 tail: alpha[c] from the K pass's dot products (per_page scalars per page), then
+// top-K_p -> sel (pool ids) and sel_pos (candidate positions), ascending position.
+wa_status launch_alpha_topk(const double* kdot, int per_page, int n_c, int T_p, int H, int d,
+                            int K_p, const int32_t* cand, double* alpha, int32_t* sel,
+                            int32_t* sel_pos, cudaStream_t st);
 
-// S1 tail: alpha[c] from the q / k partials, then top-K_p -> sel (pool ids) and
-// sel_pos (candidate positions), both in ascending position.
-wa_status launch_page_alpha_topk(const double* q_partial, int q_split, int Nq,
-                                 const double* k_partial, int k_split, int T_p, int n_c,
-                                 int H, int d, int K_p, const int32_t* cand, double* alpha,
-                                 int32_t* sel, int32_t* sel_pos, cudaStream_t st);
-
-// Write k_blockmean[c][b][:] = blocksum / B for the candidate pages (T_p % B == 0).
+// dst[i] = src[i] * scale (float64).
 wa_status launch_scale_copy(const double* src, double* dst, size_t n, double scale,
                             cudaStream_t st);
 
@@ -63,11 +71,13 @@ struct KeyMeans {
   int is_sum = 0;                 // data holds sums: divide by the block's row count
   int L = 0;                      // rows of the key sequence (for ragged counts)
 };
-// S3: per (head, query block) block selection from float64 pooled means.
-size_t block_select_smem_bytes(int d, int n_kb, int* G_out);
-wa_status launch_block_select(const double* q_blocksum, int Nq, int H, int d, int B,
-                              KeyMeans km, int n_kb, const float* tau, int32_t* blk_idx,
-                              int32_t* blk_cnt, uint32_t* blk_mask, cudaStream_t st);
+// S3: float64 pooled block scores into `scores` [H][n_qb][n_kb], then per (head,
+// query block) the shortest descending prefix reaching tau_h.
+size_t block_scores_bytes(int H, int n_qb, int n_kb);
+wa_status launch_block_select(const double* q_blockmean, int Nq, int H, int d, int B,
+                              KeyMeans km, int n_kb, const float* tau, double* scores,
+                              int32_t* blk_idx, int32_t* blk_cnt, uint32_t* blk_mask,
+                              cudaStream_t st);
 
 // ---------------------------------------------------------------- gather
 wa_status launch_gather(const void* k_pool, const void* v_pool, int n_pages, size_t page_bytes,
@@ -91,18 +101,19 @@ wa_status launch_umma_project(const void* k, const void* v, RowSource rs, const 
                               const void* e_v, int L, int H, int d, int r, void* k_til,
                               void* v_til, void* ws, uint32_t* err, cudaStream_t st);
 
-// Work items of the tcgen05 attention: (head, query block 0, query block 1 or -1,
-// number of key blocks in the union), longest first.
-size_t attn_items_ws_bytes(int H, int n_qb);
-wa_status launch_attn_items(const uint32_t* blk_mask, int H, int n_qb, int n_kb, int4* items,
-                            void* scratch, cudaStream_t st);
-// mode 0 (linear branch): keys = k_til/v_til [r][H][d], every block, writes
-//   lin_ws[n][h][:] = (1 - sigmoid(g)) * O_lin (fp32) and o_branch (nullable).
-// mode 1 (sparse branch): keys from rs, blocks = union of the item's masks, writes
-//   out = bf16(sigmoid(g) * O_sp + lin_ws) and o_branch (nullable, O_sp fp32).
-wa_status launch_umma_attention(int mode, const void* q, int Nq, int H, int d, RowSource rs,
-                                int B, const uint32_t* blk_mask, int W, const int4* items,
-                                int n_items, const float* gate, float* lin_ws, void* out,
-                                float* o_branch, uint32_t* err, cudaStream_t st);
+// Linear branch on tcgen05 (keys = k_til/v_til [r][H][d], every block): writes
+//   lin_ws[n][h][:] = (1 - sigmoid(g)) * O_lin (fp32) and o_lin (nullable).
+wa_status launch_linear_attention(const void* q, int Nq, int H, int d, RowSource lin, int B,
+                                  const float* gate, float* lin_ws, float* o_lin, uint32_t* err,
+                                  cudaStream_t st);
+// Sparse branch on tcgen05 over the kept blocks of blk_mask, fused with the gate:
+//   out = bf16(sigmoid(g) * O_sp + lin_ws), o_sp (nullable) = O_sp in fp32.
+// `scratch` holds the work list and the split partials (sparse_attn_ws_bytes).
+// events (nullable, WA_STEP_EVENTS entries): entry 6 is recorded after the work list.
+size_t sparse_attn_ws_bytes(int H, int Nq, int d, int B);
+wa_status launch_sparse_attention(const void* q, int Nq, int H, int d, RowSource rs, int B,
+                                  const uint32_t* blk_mask, const float* gate, const float* lin_ws,
+                                  void* out, float* o_sp, void* scratch, uint32_t* err,
+                                  cudaStream_t st, void* const* events);
 
 }  // namespace wa
