@@ -49,8 +49,12 @@ import torch  # noqa: E402
 METRIC = "HSA ms/chunk-layer & attention frames/s; % of BF16 tensor / HBM roofline"
 FRAMES_PER_CHUNK = 3
 CHUNK_LAYERS_PER_CHUNK = 30 * 4
-STAGES = ["page_retrieval", "gather", "block_select", "projection", "linear_branch", "work_list",
-          "sparse_branch_gate"]
+# stage -> (start event, end event) of the events wa_hsa_step records; the
+# projection and the linear branch run on a side stream concurrently with block
+# selection and the work list, so their stages overlap those
+STAGES = {"page_retrieval": (0, 1), "gather": (1, 2), "block_select": (2, 3),
+          "projection": (2, 4), "linear_branch": (4, 5), "work_list_and_join": (3, 6),
+          "sparse_branch_gate": (6, 7)}
 
 
 def load_peaks():
@@ -291,8 +295,8 @@ def run_ours(args, rank, world, local_rank):
     ms_step = elapsed_max / args.steps
 
     stage_ms = {}
-    for j, name in enumerate(STAGES):
-        stage_ms[name] = float(np.mean([ev[k][j].elapsed_time(ev[k][j + 1]) for k in range(args.steps)]))
+    for name, (a0, a1) in STAGES.items():
+        stage_ms[name] = float(np.mean([ev[k][a0].elapsed_time(ev[k][a1]) for k in range(args.steps)]))
     attn_ms = stage_ms["sparse_branch_gate"]
     peaks, peak_src = load_peaks()
     peak_t = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))

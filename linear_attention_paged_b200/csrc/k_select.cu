@@ -18,7 +18,6 @@
 namespace wa {
 namespace {
 
-constexpr int kTargetCtas = 4 * 148;  // about four resident CTAs per SM on a B200
 
 __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
@@ -251,23 +250,21 @@ __global__ void k_scale_copy(const double* __restrict__ src, double* __restrict_
 }
 
 // ------------------------------------------------------------------ S3 scores
-// s[h][i][j] = qbar_{h,i} . kbar_{h,j} / sqrt(d) in float64.  CTA = (32 key blocks,
-// head): the 32 key-block means are staged in shared memory (row pitch d+1 doubles
-// against bank conflicts), the query means in chunks of 64 blocks; warp w computes
-// 8 query blocks of the chunk against lane l's key block, eight independent
-// accumulators per thread.
-constexpr int kScoreQChunk = 64;
-
+// s[h][i][j] = qbar_{h,i} . kbar_{h,j} / sqrt(d) in float64.  CTA = a 32 x 32 tile
+// of (query block, key block) of one head; both 32-row operand tiles are staged in
+// shared memory (key rows at pitch d+1 doubles against bank conflicts) and each
+// thread accumulates a 2 x 2 register tile: rows ty, ty+16 and key blocks tx, tx+16.
 __global__ void __launch_bounds__(256)
 k_block_scores(const double* __restrict__ qmean, KeyMeans km, int n_qb, int n_kb, int H, int d,
                int B, double* __restrict__ scores) {
   extern __shared__ double sm_scores[];
-  double* kc = sm_scores;                    // [32][d+1]
-  double* qs = sm_scores + 32 * (d + 1);     // [kScoreQChunk][d]
-  const int h = blockIdx.y, j0 = blockIdx.x * 32;
+  double* qs = sm_scores;                    // [32][d]
+  double* kc = sm_scores + 32 * d;           // [32][d+1]
+  const int j0 = blockIdx.x * 32, i0 = blockIdx.y * 32, h = blockIdx.z;
   const int cols = H * d;
   for (int e = threadIdx.x; e < 32 * d; e += blockDim.x) {
-    const int jj = e / d, c = e - jj * d, j = j0 + jj;
+    const int rr = e / d, c = e - rr * d;
+    const int j = j0 + rr, i = i0 + rr;
     double v = 0.0;
     if (j < n_kb) {
       size_t row = j;
@@ -275,36 +272,30 @@ k_block_scores(const double* __restrict__ qmean, KeyMeans km, int n_qb, int n_kb
       v = km.data[row * cols + h * d + c];
       if (km.is_sum) v /= static_cast<double>(min(km.L, (j + 1) * B) - j * B);
     }
-    kc[jj * (d + 1) + c] = v;
+    kc[rr * (d + 1) + c] = v;
+    qs[e] = i < n_qb ? qmean[static_cast<size_t>(i) * cols + h * d + c] : 0.0;
   }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int j = j0 + lane;
+  __syncthreads();
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  const double* q0 = qs + ty * d;
+  const double* q1 = qs + (ty + 16) * d;
+  const double* k0 = kc + tx * (d + 1);
+  const double* k1 = kc + (tx + 16) * (d + 1);
+  double a00 = 0.0, a01 = 0.0, a10 = 0.0, a11 = 0.0;
+#pragma unroll 4
+  for (int c = 0; c < d; ++c) {
+    const double x0 = q0[c], x1 = q1[c], y0 = k0[c], y1 = k1[c];
+    a00 += x0 * y0; a01 += x0 * y1; a10 += x1 * y0; a11 += x1 * y1;
+  }
   const double sqrt_d = sqrt(static_cast<double>(d));
-  const double* kr = kc + lane * (d + 1);
-  for (int ic = 0; ic < n_qb; ic += kScoreQChunk) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < kScoreQChunk * d; e += blockDim.x) {
-      const int ii = e / d, c = e - ii * d, i = ic + ii;
-      qs[e] = i < n_qb ? qmean[static_cast<size_t>(i) * cols + h * d + c] : 0.0;
-    }
-    __syncthreads();
-    const double* q0 = qs + (warp * 8) * d;
-    double acc[8];
+  const double acc[2][2] = {{a00, a01}, {a10, a11}};
 #pragma unroll
-    for (int r = 0; r < 8; ++r) acc[r] = 0.0;
-    for (int c = 0; c < d; ++c) {
-      const double kv = kr[c];
+  for (int u = 0; u < 2; ++u)
 #pragma unroll
-      for (int r = 0; r < 8; ++r) acc[r] += q0[r * d + c] * kv;
+    for (int v = 0; v < 2; ++v) {
+      const int i = i0 + ty + 16 * u, j = j0 + tx + 16 * v;
+      if (i < n_qb && j < n_kb) scores[(static_cast<size_t>(h) * n_qb + i) * n_kb + j] = acc[u][v] / sqrt_d;
     }
-    if (j < n_kb) {
-#pragma unroll
-      for (int r = 0; r < 8; ++r) {
-        const int i = ic + warp * 8 + r;
-        if (i < n_qb) scores[(static_cast<size_t>(h) * n_qb + i) * n_kb + j] = acc[r] / sqrt_d;
-      }
-    }
-  }
 }
 
 // ------------------------------------------------------------------ S3 choice
@@ -444,19 +435,20 @@ wa_status launch_prompt_select(const float* e_cur, const float* e_chunks, int n_
 }
 
 RowsumPlan rowsum_plan(int n_src, int rows, int cols, int B, wa_dtype dt) {
+  // 64-thread CTAs (V columns per thread) over one B-row block each: many small
+  // CTAs keep enough 16-byte loads in flight to cover HBM latency
   RowsumPlan p;
   const int V = dt == WA_BF16 ? 8 : 4;
   const int threads_total = cols / V;
-  p.n_cc = 1;
   p.threads = threads_total;
-  while (p.threads >= 128 && (p.threads % 2) == 0 && n_src * p.n_cc < 16) {  // few sources: split columns
-    p.threads /= 2;
-    p.n_cc *= 2;
+  p.n_cc = 1;
+  if (threads_total % 64 == 0) {
+    p.threads = 64;
+    p.n_cc = threads_total / 64;
   }
   p.nb = (rows + B - 1) / B;
-  int want = (kTargetCtas + n_src * p.n_cc - 1) / (n_src * p.n_cc);
-  want = want < 1 ? 1 : (want > p.nb ? p.nb : want);
-  p.bps = (p.nb + want - 1) / want;
+  const long long ctas = static_cast<long long>(n_src) * p.n_cc * p.nb;
+  p.bps = ctas > 32LL * 148 ? static_cast<int>((ctas + 32LL * 148 - 1) / (32LL * 148)) : 1;
   p.n_split = (p.nb + p.bps - 1) / p.bps;
   return p;
 }
@@ -507,13 +499,13 @@ wa_status launch_block_select(const double* q_blockmean, int Nq, int H, int d, i
                               cudaStream_t st) {
   const int n_qb = (Nq + B - 1) / B;
   const int W = (n_kb + 31) / 32;
-  const size_t smem_s = (32 * static_cast<size_t>(d + 1) + kScoreQChunk * static_cast<size_t>(d)) *
+  const size_t smem_s = (32 * static_cast<size_t>(d + 1) + 32 * static_cast<size_t>(d)) *
                         sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_block_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem_s));
   if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "block_scores smem attr: %s", cudaGetErrorString(e));
-  k_block_scores<<<dim3((n_kb + 31) / 32, H), 256, smem_s, st>>>(q_blockmean, km, n_qb, n_kb, H, d,
-                                                               B, scores);
+  k_block_scores<<<dim3((n_kb + 31) / 32, (n_qb + 31) / 32, H), 256, smem_s, st>>>(
+      q_blockmean, km, n_qb, n_kb, H, d, B, scores);
   int lg = 5;
   while ((1 << lg) < n_kb) ++lg;
   const size_t smem_c = (static_cast<size_t>(1) << lg) * 12 + static_cast<size_t>(W) * 4 + 16;

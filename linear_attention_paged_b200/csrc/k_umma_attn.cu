@@ -321,16 +321,17 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         for (int c = 0; c < 64; ++c)
           if (!sel || c >= valid) r[c] = __float_as_uint(-INFINITY);
       }
-      // row max of the raw scores: eight independent chains
+      // row max of the raw scores: eight independent chains of 3-input maxima
       float mx8[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = __uint_as_float(r[e]);
+      for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(__uint_as_float(r[e]), __uint_as_float(r[8 + e]));
 #pragma unroll
-      for (int c = 8; c < 64; c += 8)
+      for (int c = 16; c < 64; c += 16)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(mx8[e], __uint_as_float(r[c + e]));
-      const float mraw = fmaxf(fmaxf(fmaxf(mx8[0], mx8[1]), fmaxf(mx8[2], mx8[3])),
-                               fmaxf(fmaxf(mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7])));
+        for (int e = 0; e < 8; ++e)
+          mx8[e] = max3f(mx8[e], __uint_as_float(r[c + e]), __uint_as_float(r[c + 8 + e]));
+      const float mraw = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
+                               fmaxf(mx8[6], mx8[7]));
       const float mx = mraw * scale_log2;   // scale_log2 > 0: the max commutes with it
       float factor = 1.f;
       bool resc = false;
@@ -342,24 +343,29 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         resc = true;
       }
       const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-      // p = 2^(s * log2(e)/sqrt(d) - m), summed in eight chains, packed to bf16 pairs
-      float sum8[8];
+      // p = 2^(s * log2(e)/sqrt(d) - m) on column pairs (paired fp32 FMA and add),
+      // summed in four two-lane chains, packed to bf16 pairs
+      const float2 sc2 = make_float2(scale_log2, scale_log2);
+      const float2 nm2 = make_float2(neg_m, neg_m);
+      float2 acc2[4];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) sum8[e] = 0.f;
+      for (int e = 0; e < 4; ++e) acc2[e] = make_float2(0.f, 0.f);
 #pragma unroll
       for (int c = 0; c < 64; c += 32) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2(fmaf(__uint_as_float(r[c + 2 * e]), scale_log2, neg_m));
-          const float p1 = ex2(fmaf(__uint_as_float(r[c + 2 * e + 1]), scale_log2, neg_m));
-          sum8[e & 7] += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          const float2 x = make_float2(__uint_as_float(r[c + 2 * e]), __uint_as_float(r[c + 2 * e + 1]));
+          const float2 y = __ffma2_rn(x, sc2, nm2);
+          const float2 pp = make_float2(ex2(y.x), ex2(y.y));
+          acc2[e & 3] = __fadd2_rn(acc2[e & 3], pp);
+          pk[e] = pack_bf16x2(pp.x, pp.y);
         }
         tmem_st16(tbase + lane_base + kColS + sb * 64 + c / 2, pk);
       }
-      const float sum = ((sum8[0] + sum8[1]) + (sum8[2] + sum8[3])) +
-                        ((sum8[4] + sum8[5]) + (sum8[6] + sum8[7]));
+      const float2 a01 = __fadd2_rn(acc2[0], acc2[1]), a23 = __fadd2_rn(acc2[2], acc2[3]);
+      const float2 a03 = __fadd2_rn(a01, a23);
+      const float sum = a03.x + a03.y;
       l_run = l_run * factor + sum;
       tmem_wait_st();
       if (__any_sync(0xffffffffu, resc)) {
@@ -472,52 +478,63 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
 // Merge the two halves of a split pair: M = max(m0, m1), w_s = 2^(m_s - M),
 // O = (w0 O0 + w1 O1) / (w0 l0 + w1 l1); then out = bf16(sigmoid(g) O + lin_ws).
-// One CTA per pair, one thread per tile row.
+// CTA = (pair, 32 tile rows); each thread takes 16 columns of one row (a warp
+// covers 4 rows x 512 contiguous bytes), all its loads issued up front.
 template <int D>
-__global__ void __launch_bounds__(128)
+__global__ void __launch_bounds__(2 * D)
 k_combine(const int4* __restrict__ pairs, Partials part, int Nq, int H,
           const float* __restrict__ gate, const float* __restrict__ lin_ws,
           __nv_bfloat16* __restrict__ out, float* __restrict__ o_branch) {
+  constexpr int kSeg = D / 16;                 // 16-column segments per row
   const int4 pr = pairs[blockIdx.x];
-  if (pr.w < kSplitMin) return;               // written whole by the attention kernel
-  const int row = threadIdx.x;
+  if (pr.w < kSplitMin) return;                // written whole by the attention kernel
+  const int row = blockIdx.y * 32 + threadIdx.x / kSeg;
+  const int c0 = (threadIdx.x % kSeg) * 16;
   const int half = row >> 6;
   const int ib = half ? pr.z : pr.y;
   const int qrow = ib * 64 + (row & 63);
   if (ib < 0 || qrow >= Nq) return;
   const int h = pr.x;
   const size_t s0 = 2 * static_cast<size_t>(blockIdx.x), s1 = s0 + 1;
+  const float4* o0 = reinterpret_cast<const float4*>(part.o + (s0 * kBM + row) * D + c0);
+  const float4* o1 = reinterpret_cast<const float4*>(part.o + (s1 * kBM + row) * D + c0);
+  const size_t obase = static_cast<size_t>(qrow) * H * D + static_cast<size_t>(h) * D + c0;
+  const float4* lw = reinterpret_cast<const float4*>(lin_ws + obase);
+  float4 x[4], y[4], l4[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) { x[e] = o0[e]; y[e] = o1[e]; l4[e] = lw[e]; }
   const float2 a = *reinterpret_cast<const float2*>(part.ml + (s0 * kBM + row) * 2);
   const float2 b = *reinterpret_cast<const float2*>(part.ml + (s1 * kBM + row) * 2);
+  const float g = gate[static_cast<size_t>(qrow) * H + h];
   const float M = fmaxf(a.x, b.x);
   const float w0 = a.x == -INFINITY ? 0.f : exp2f(a.x - M);
   const float w1 = b.x == -INFINITY ? 0.f : exp2f(b.x - M);
   const float lsum = w0 * a.y + w1 * b.y;
   const float inv = lsum > 0.f ? 1.f / lsum : 0.f;
   const float c0w = w0 * inv, c1w = w1 * inv;
-  const float g = gate[static_cast<size_t>(qrow) * H + h];
   const float sg = 1.f / (1.f + expf(-g));
-  const float4* o0 = reinterpret_cast<const float4*>(part.o + (s0 * kBM + row) * D);
-  const float4* o1 = reinterpret_cast<const float4*>(part.o + (s1 * kBM + row) * D);
-  const size_t obase = static_cast<size_t>(qrow) * H * D + static_cast<size_t>(h) * D;
-  const float4* lw = reinterpret_cast<const float4*>(lin_ws + obase);
-  uint2* op = reinterpret_cast<uint2*>(out + obase);
-#pragma unroll 4
-  for (int e = 0; e < D / 4; ++e) {
-    const float4 x = o0[e], y = o1[e], l4 = lw[e];
-    const float v0 = c0w * x.x + c1w * y.x, v1 = c0w * x.y + c1w * y.y;
-    const float v2 = c0w * x.z + c1w * y.z, v3 = c0w * x.w + c1w * y.w;
+  uint32_t pk[8];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float v0 = c0w * x[e].x + c1w * y[e].x, v1 = c0w * x[e].y + c1w * y[e].y;
+    const float v2 = c0w * x[e].z + c1w * y[e].z, v3 = c0w * x[e].w + c1w * y[e].w;
     if (o_branch) reinterpret_cast<float4*>(o_branch + obase)[e] = make_float4(v0, v1, v2, v3);
-    op[e] = make_uint2(pack_bf16x2(sg * v0 + l4.x, sg * v1 + l4.y),
-                       pack_bf16x2(sg * v2 + l4.z, sg * v3 + l4.w));
+    pk[2 * e] = pack_bf16x2(sg * v0 + l4[e].x, sg * v1 + l4[e].y);
+    pk[2 * e + 1] = pack_bf16x2(sg * v2 + l4[e].z, sg * v3 + l4[e].w);
   }
+  uint4* op = reinterpret_cast<uint4*>(out + obase);
+  op[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  op[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
 // ------------------------------------------------------------------ work items
-// One CTA per head pairs its query blocks greedily by the smallest symmetric
-// difference of their key-block sets (fewest masked half-blocks), falling back
-// to neighbours when there are too many blocks for the distance table.
-// pairs[h * n_pairs + k] = (h, first block, second block or -1, union size).
+// One CTA per head pairs its query blocks by rounds of mutual nearest neighbours:
+// distance = size of the symmetric difference of the two key-block sets (the
+// half-blocks the pair computes and masks), ties broken by the lower block index.
+// Each round pairs every two unpaired blocks that are each other's nearest
+// unpaired neighbour; the closest remaining pair always qualifies, so every round
+// makes progress.  Falls back to neighbours when there are too many blocks for the
+// distance table.  pairs[h * n_pairs + k] = (h, first, second or -1, union size).
 constexpr int kMaxPairTable = 128;
 constexpr int kMaxPairMaskWords = 3072;   // staged masks of one head (n_qb * W words)
 
@@ -525,8 +542,9 @@ __global__ void __launch_bounds__(256)
 k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W, int4* __restrict__ pairs) {
   __shared__ uint16_t dist[kMaxPairTable * kMaxPairTable];
   __shared__ uint32_t ms[kMaxPairMaskWords];
-  __shared__ unsigned char paired[kMaxPairTable];
-  __shared__ int2 chosen[kMaxPairTable];
+  __shared__ int partner[kMaxPairTable];
+  __shared__ int nn[kMaxPairTable];
+  __shared__ int progress;
   const int h = blockIdx.x;
   const int n_pairs = (n_qb + 1) / 2;
   const uint32_t* mh = mask + static_cast<size_t>(h) * n_qb * W;
@@ -548,45 +566,50 @@ k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W, int4* __restric
     return;
   }
   for (int e = threadIdx.x; e < n_qb * n_qb; e += blockDim.x) {
-    const int a = e / n_qb, b = e % n_qb;
+    const int a = e / n_qb, b = e - a * n_qb;
     int c = 0;
-    if (a < b)
+    if (a != b)
       for (int w = 0; w < W; ++w) c += __popc(m[a * W + w] ^ m[b * W + w]);
     dist[e] = static_cast<uint16_t>(min(c, 65535));
   }
-  for (int a = threadIdx.x; a < n_qb; a += blockDim.x) paired[a] = 0;
+  for (int a = threadIdx.x; a < n_qb; a += blockDim.x) partner[a] = -2;   // -2: unpaired
   __syncthreads();
-  if (threadIdx.x < 32) {
-    const int lane = threadIdx.x;
+  for (int round = 0; round < n_qb; ++round) {
+    for (int a = threadIdx.x; a < n_qb; a += blockDim.x) {
+      int best = INT_MAX, bi = -1;
+      if (partner[a] == -2)
+        for (int b = 0; b < n_qb; ++b) {
+          if (b == a || partner[b] != -2) continue;
+          const int dv = dist[a * n_qb + b];
+          if (dv < best) { best = dv; bi = b; }   // increasing b: ties keep the lower index
+        }
+      nn[a] = bi;
+    }
+    if (threadIdx.x == 0) progress = 0;
+    __syncthreads();
+    for (int a = threadIdx.x; a < n_qb; a += blockDim.x) {
+      const int b = nn[a];
+      if (b > a && nn[b] == a) { partner[a] = b; partner[b] = a; progress = 1; }
+    }
+    __syncthreads();
+    if (!progress) break;
+  }
+  // emit pairs in order of their first block (deterministic); a block left alone
+  // (odd count) gets partner -1
+  if (threadIdx.x == 0) {
     int k = 0;
     for (int a = 0; a < n_qb; ++a) {
-      if (paired[a]) continue;
-      int best = INT_MAX, bi = -1;
-      for (int b = a + 1 + lane; b < n_qb; b += 32) {
-        if (paired[b]) continue;
-        const int dv = dist[a * n_qb + b];
-        if (dv < best) { best = dv; bi = b; }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const int ob = __shfl_xor_sync(0xffffffffu, best, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ob < best || (ob == best && oi >= 0 && (bi < 0 || oi < bi))) { best = ob; bi = oi; }
-      }
-      __syncwarp();
-      if (lane == 0) {
-        paired[a] = 1;
-        if (bi >= 0) paired[bi] = 1;
-        chosen[k] = make_int2(a, bi);
-      }
-      __syncwarp();
+      const int b = partner[a];
+      if (b >= 0 && b < a) continue;
+      pairs[static_cast<size_t>(h) * n_pairs + k] = make_int4(h, a, b >= 0 ? b : -1, 0);
       ++k;
     }
   }
   __syncthreads();
   for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
-    const int2 c = chosen[p];
-    pairs[static_cast<size_t>(h) * n_pairs + p] = make_int4(h, c.x, c.y, union_count(c.x, c.y));
+    int4 it = pairs[static_cast<size_t>(h) * n_pairs + p];
+    it.w = union_count(it.y, it.z);
+    pairs[static_cast<size_t>(h) * n_pairs + p] = it;
   }
 }
 
@@ -702,53 +725,78 @@ wa_status launch_linear_attention(const void* q, int Nq, int H, int d, RowSource
   return check_launch("linear attention");
 }
 
+namespace {
+struct SparseLayout {
+  int n_qb, n_kb, W, n_pairs;
+  int4* pairs;
+  int4* items;
+  Partials part;
+};
+SparseLayout sparse_layout(void* scratch, int Nq, int H, int d, int B, int L) {
+  SparseLayout s;
+  s.n_qb = (Nq + B - 1) / B;
+  s.n_kb = (L + B - 1) / B;
+  s.W = (s.n_kb + 31) / 32;
+  s.n_pairs = H * ((s.n_qb + 1) / 2);
+  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+  char* p = static_cast<char*>(scratch);
+  s.pairs = reinterpret_cast<int4*>(p);
+  p += al(s.n_pairs * sizeof(int4));
+  s.items = reinterpret_cast<int4*>(p);
+  p += al(2 * static_cast<size_t>(s.n_pairs) * sizeof(int4));
+  s.part.o = reinterpret_cast<float*>(p);
+  p += al(2 * static_cast<size_t>(s.n_pairs) * kBM * d * sizeof(float));
+  s.part.ml = reinterpret_cast<float*>(p);
+  return s;
+}
+}  // namespace
+
+wa_status launch_attn_worklist(int Nq, int H, int d, int B, int L, const uint32_t* blk_mask,
+                               void* scratch, cudaStream_t st) {
+  if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
+  SparseLayout s = sparse_layout(scratch, Nq, H, d, B, L);
+  if (s.W > kMaxW) return set_error(WA_ERR_UNSUPPORTED, "too many key blocks (max %d)", kMaxW * 32);
+  k_pair_heads<<<H, 256, 0, st>>>(blk_mask, s.n_qb, s.W, s.pairs);
+  int shift = 0;
+  while ((s.n_kb >> shift) >= kLenBins) ++shift;
+  k_make_items<<<1, 1024, 0, st>>>(s.pairs, s.n_pairs, shift, s.items);
+  return check_launch("attention work list");
+}
+
+wa_status launch_attn_sparse(const void* q, int Nq, int H, int d, RowSource rs, int B,
+                             const uint32_t* blk_mask, const float* gate, const float* lin_ws,
+                             void* out, float* o_sp, void* scratch, uint32_t* err, cudaStream_t st) {
+  if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
+  if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs d in {64,128}");
+  SparseLayout s = sparse_layout(scratch, Nq, H, d, B, rs.L);
+  if (s.W > kMaxW) return set_error(WA_ERR_UNSUPPORTED, "too many key blocks (max %d)", kMaxW * 32);
+  alignas(64) CUtensorMap tq, tk, tv;
+  wa_status e = make_maps(q, Nq, H, d, rs, &tq, &tk, &tv);
+  if (e != WA_OK) return e;
+  const int grid = 2 * s.n_pairs;
+  float* lin_rw = const_cast<float*>(lin_ws);
+  if (d == 128) {
+    launch_attn_kernel<128>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
+                            s.part, gate, lin_rw, out, o_sp, err);
+    k_combine<128><<<dim3(s.n_pairs, kBM / 32), 2 * 128, 0, st>>>(s.pairs, s.part, Nq, H, gate, lin_ws,
+                                                                  static_cast<__nv_bfloat16*>(out), o_sp);
+  } else {
+    launch_attn_kernel<64>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
+                           s.part, gate, lin_rw, out, o_sp, err);
+    k_combine<64><<<dim3(s.n_pairs, kBM / 32), 2 * 64, 0, st>>>(s.pairs, s.part, Nq, H, gate, lin_ws,
+                                                                static_cast<__nv_bfloat16*>(out), o_sp);
+  }
+  return check_launch("sparse attention");
+}
+
 wa_status launch_sparse_attention(const void* q, int Nq, int H, int d, RowSource rs, int B,
                                   const uint32_t* blk_mask, const float* gate, const float* lin_ws,
                                   void* out, float* o_sp, void* scratch, uint32_t* err,
                                   cudaStream_t st, void* const* events) {
-  if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
-  if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs d in {64,128}");
-  const int n_qb = (Nq + B - 1) / B;
-  const int n_kb = (rs.L + B - 1) / B;
-  const int W = (n_kb + 31) / 32;
-  if (W > kMaxW) return set_error(WA_ERR_UNSUPPORTED, "too many key blocks (max %d)", kMaxW * 32);
-  const int n_pairs = H * ((n_qb + 1) / 2);
-  auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
-  char* p = static_cast<char*>(scratch);
-  int4* pairs = reinterpret_cast<int4*>(p);
-  p += al(n_pairs * sizeof(int4));
-  int4* items = reinterpret_cast<int4*>(p);
-  p += al(2 * static_cast<size_t>(n_pairs) * sizeof(int4));
-  Partials part;
-  part.o = reinterpret_cast<float*>(p);
-  p += al(2 * static_cast<size_t>(n_pairs) * kBM * d * sizeof(float));
-  part.ml = reinterpret_cast<float*>(p);
-
-  k_pair_heads<<<H, 256, 0, st>>>(blk_mask, n_qb, W, pairs);
-  int shift = 0;
-  while ((n_kb >> shift) >= kLenBins) ++shift;
-  k_make_items<<<1, 1024, 0, st>>>(pairs, n_pairs, shift, items);
-  wa_status s = check_launch("attention work list");
-  if (s != WA_OK) return s;
+  wa_status e = launch_attn_worklist(Nq, H, d, B, rs.L, blk_mask, scratch, st);
+  if (e != WA_OK) return e;
   if (events && events[6]) cudaEventRecord(static_cast<cudaEvent_t>(events[6]), st);
-
-  alignas(64) CUtensorMap tq, tk, tv;
-  s = make_maps(q, Nq, H, d, rs, &tq, &tk, &tv);
-  if (s != WA_OK) return s;
-  const int grid = 2 * n_pairs;
-  float* lin_rw = const_cast<float*>(lin_ws);
-  if (d == 128) {
-    launch_attn_kernel<128>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, W, n_qb, pairs, items, part,
-                            gate, lin_rw, out, o_sp, err);
-    k_combine<128><<<n_pairs, 128, 0, st>>>(pairs, part, Nq, H, gate, lin_ws,
-                                            static_cast<__nv_bfloat16*>(out), o_sp);
-  } else {
-    launch_attn_kernel<64>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, W, n_qb, pairs, items, part,
-                           gate, lin_rw, out, o_sp, err);
-    k_combine<64><<<n_pairs, 128, 0, st>>>(pairs, part, Nq, H, gate, lin_ws,
-                                           static_cast<__nv_bfloat16*>(out), o_sp);
-  }
-  return check_launch("sparse attention");
+  return launch_attn_sparse(q, Nq, H, d, rs, B, blk_mask, gate, lin_ws, out, o_sp, scratch, err, st);
 }
 
 }  // namespace wa

@@ -104,6 +104,31 @@ bool make_tmap_bf16_2d(void* tmap, const void* base, uint64_t inner, uint64_t ou
   return r == CUDA_SUCCESS;
 }
 
+// A second stream (and the fork / join events) per host thread and device, on
+// which the decode step runs the projection and the linear branch concurrently with
+// block selection.  Created on first use; no device memory is allocated.
+struct SideStream {
+  cudaStream_t stream = nullptr;
+  cudaEvent_t fork = nullptr;
+  cudaEvent_t join = nullptr;
+};
+thread_local SideStream t_side[64];
+
+wa_status side_stream(SideStream** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+    return set_error(WA_ERR_CUDA, "cudaGetDevice failed");
+  SideStream& s = t_side[dev];
+  if (!s.stream) {
+    if (cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess)
+      return set_error(WA_ERR_CUDA, "could not create the side stream");
+  }
+  *out = &s;
+  return WA_OK;
+}
+
 }  // namespace wa
 
 using namespace wa;
@@ -580,32 +605,54 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
   }
 
   mark(2);
-  // S3: block selection
   uint32_t* mask = a->blk_mask_out ? a->blk_mask_out : w.mask;
-  WA_TRY(launch_block_select(w.ps.q_blockmean, a->Nq, a->H, a->d, a->B, km, n_kb, a->tau, w.scores,
-                             nullptr, nullptr, mask, st));
-  (void)W;
-  (void)n_qb;
-
-  mark(3);
-  // S4a: projection
   void* kt = a->k_til_out ? a->k_til_out : w.k_til;
   void* vt = a->v_til_out ? a->v_til_out : w.v_til;
+  RowSource lin;
+  lin.k = kt; lin.v = vt; lin.page_rows = a->r; lin.n_pages = 1; lin.L = a->r;
   if (a->dtype == WA_BF16) {
+    // S4a + S4b (HBM-bound projection, then the linear branch) on a side stream,
+    // concurrently with S3 and the work list (latency-bound) on this stream; the
+    // sparse branch joins both.
+    SideStream* side = nullptr;
+    WA_TRY(side_stream(&side));
+    cudaEventRecord(side->fork, st);
+    cudaStreamWaitEvent(side->stream, side->fork, 0);
+    auto mark_side = [&](int k) {
+      if (a->stage_events && a->stage_events[k])
+        cudaEventRecord(static_cast<cudaEvent_t>(a->stage_events[k]), side->stream);
+    };
     WA_TRY(launch_umma_project(rs.k, rs.v, rs, a->e_k, a->e_v, L, a->H, a->d, a->r, kt, vt, w.proj,
-                               err, st));
+                               err, side->stream));
+    mark_side(4);
+    WA_TRY(launch_linear_attention(a->q, a->Nq, a->H, a->d, lin, a->B, a->gate, w.lin, nullptr, err,
+                                   side->stream));
+    mark_side(5);
+    cudaEventRecord(side->join, side->stream);
+    // S3: block selection
+    WA_TRY(launch_block_select(w.ps.q_blockmean, a->Nq, a->H, a->d, a->B, km, n_kb, a->tau, w.scores,
+                               nullptr, nullptr, mask, st));
+    mark(3);
+    WA_TRY(launch_attn_worklist(a->Nq, a->H, a->d, a->B, L, mask, w.attn, st));
+    cudaStreamWaitEvent(st, side->join, 0);
+    mark(6);
+    // S5 + S6
+    WA_TRY(launch_attn_sparse(a->q, a->Nq, a->H, a->d, rs, a->B, mask, a->gate, w.lin, a->out, nullptr,
+                              w.attn, err, st));
   } else {
+    WA_TRY(launch_block_select(w.ps.q_blockmean, a->Nq, a->H, a->d, a->B, km, n_kb, a->tau, w.scores,
+                               nullptr, nullptr, mask, st));
+    mark(3);
     WA_TRY(launch_simt_project(static_cast<const float*>(rs.k), rs.page_ids, rs.page_rows,
                                rs.n_pages, static_cast<const float*>(a->e_k), L, cols, a->r,
                                static_cast<float*>(kt), err, st));
     WA_TRY(launch_simt_project(static_cast<const float*>(rs.v), rs.page_ids, rs.page_rows,
                                rs.n_pages, static_cast<const float*>(a->e_v), L, cols, a->r,
                                static_cast<float*>(vt), err, st));
+    mark(4);
+    WA_TRY(run_attention(a->q, a->Nq, a->H, a->d, rs, a->B, mask, kt, vt, a->r, a->gate, a->dtype,
+                         a->out, nullptr, nullptr, w.lin, w.attn, st, a->stage_events));
   }
-  mark(4);
-  // S4b + S5 + S6
-  WA_TRY(run_attention(a->q, a->Nq, a->H, a->d, rs, a->B, mask, kt, vt, a->r, a->gate, a->dtype,
-                       a->out, nullptr, nullptr, w.lin, w.attn, st, a->stage_events));
   mark(7);
   return WA_OK;
 }

@@ -111,6 +111,13 @@ wa_status launch_linear_attention(const void* q, int Nq, int H, int d, RowSource
 // `scratch` holds the work list and the split partials (sparse_attn_ws_bytes).
 // events (nullable, WA_STEP_EVENTS entries): entry 6 is recorded after the work list.
 size_t sparse_attn_ws_bytes(int H, int Nq, int d, int B);
+// The two halves of launch_sparse_attention: the work list (pairs + items) from the
+// masks, then the attention kernel and the combine.
+wa_status launch_attn_worklist(int Nq, int H, int d, int B, int L, const uint32_t* blk_mask,
+                               void* scratch, cudaStream_t st);
+wa_status launch_attn_sparse(const void* q, int Nq, int H, int d, RowSource rs, int B,
+                             const uint32_t* blk_mask, const float* gate, const float* lin_ws,
+                             void* out, float* o_sp, void* scratch, uint32_t* err, cudaStream_t st);
 wa_status launch_sparse_attention(const void* q, int Nq, int H, int d, RowSource rs, int B,
                                   const uint32_t* blk_mask, const float* gate, const float* lin_ws,
                                   void* out, float* o_sp, void* scratch, uint32_t* err,
