@@ -257,7 +257,10 @@ def run_ours(args, rank, world, local_rank):
     if flags:
         raise RuntimeError(f"device error flags 0x{flags:x}")
     flops, kept_frac = selected_flops(step.inter["blk_mask"], cfg)
-    launches_per_step = 12
+    # per step: pick_chunk, Q row sums, query means, candidate-page row sums, alpha/top-k,
+    # block scores, block choice, pairing, work items, sparse attention, combine on the
+    # caller's stream; projection, split reduction, linear branch on the side stream
+    launches_per_step = 14
 
     n_ev = 8  # WA_STEP_EVENTS
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
@@ -377,6 +380,112 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
+def run_c4(args, rank, world, local_rank):
+    """Full denoise stack: `layers` layers x 4 denoising steps per chunk x `chunks`
+    chunks of 3 frames.  Each layer owns a 16-page pool (8 history pages = the
+    candidate chunk, 8 pages of room for appended chunks), its E_K/E_V and tau, and
+    a float64 page index of its pool.  Per chunk: 4 x layers HSA steps (queries and
+    gates cycle through a resident set of pre-drawn tensors), then every layer's
+    new 4680-token KV is appended to its pool with the index refreshed.  The index
+    of the history pages is built before timing (it belongs to the cache state);
+    appends and all steps are timed."""
+    from linear_attention_paged_b200 import build as wb
+    if rank == 0:
+        wb.build()
+    if world > 1:
+        torch.distributed.barrier()
+    from linear_attention_paged_b200 import wa, workloads as W
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    n_layers, n_steps, n_chunks = args.layers, 4, args.chunks
+    base = W.C1.with_(name="c4_layer", n_chunks=2)
+    layers = []
+    for l in range(n_layers):
+        cfg = base.with_(seed=4000 + 1000 * rank + l)
+        inp = W.make_inputs(cfg, device="cuda", gen_device="cuda")
+        P_ = cfg.n_pool_pages
+        hist = inp["chunk_pages"][0:1].contiguous()
+        idx = wa.wa_pool_index(inp["k_pool"], hist[0].contiguous(), cfg.B,
+                               page_index=torch.zeros((P_, cfg.T_p // cfg.B, cfg.H, cfg.d),
+                                                      dtype=torch.float64, device=dev))
+        g = torch.Generator(device="cuda").manual_seed(cfg.seed + 7)
+        k_new = (torch.randn((cfg.Nq, cfg.H, cfg.d), generator=g, device="cuda") / cfg.d ** 0.5).to(torch.bfloat16)
+        v_new = (torch.randn((cfg.Nq, cfg.H, cfg.d), generator=g, device="cuda") / cfg.d ** 0.5).to(torch.bfloat16)
+        step = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], hist, inp["e_k"], inp["e_v"],
+                          inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B, page_index=idx)
+        for key in ("q", "gate", "e_cur", "e_chunks"):
+            inp.pop(key, None)
+        layers.append(dict(cfg=cfg, inp=inp, idx=idx, step=step, k_new=k_new, v_new=v_new))
+    n_rot = 8
+    gq = torch.Generator(device="cuda").manual_seed(99 + rank)
+    qs = [(torch.randn((base.Nq, base.H, base.d), generator=gq, device="cuda") / base.d ** 0.5).to(torch.bfloat16)
+          for _ in range(n_rot)]
+    gs = [torch.randn((base.Nq, base.H), generator=gq, device="cuda") for _ in range(n_rot)]
+    import ctypes
+    fill0 = base.n_c * base.T_p
+
+    def run(chunks, fill):
+        k = 0
+        for _ in range(chunks):
+            for _ in range(n_steps):
+                for L_ in layers:
+                    a = L_["step"].args
+                    a.q = ctypes.c_void_p(qs[k % n_rot].data_ptr())
+                    a.gate = ctypes.c_void_p(gs[k % n_rot].data_ptr())
+                    L_["step"]()
+                    k += 1
+            for L_ in layers:
+                wa.wa_pool_append(L_["inp"]["k_pool"], L_["inp"]["v_pool"], L_["k_new"], L_["v_new"], fill,
+                                  page_index=L_["idx"], B=base.B)
+            fill += base.Nq
+        return fill
+
+    run(1, fill0)                     # warm-up chunk (writes the first append slot)
+    torch.cuda.synchronize()
+    flags = wa.wa_device_error()
+    if flags:
+        raise RuntimeError(f"device error flags 0x{flags:x}")
+    clk = ClockSampler(local_rank)
+    clk.start()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    run(n_chunks, fill0)              # rewrites the pool tail from the same offset
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = clk.stop()
+    el = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(el, op=torch.distributed.ReduceOp.MAX)
+    total_ms = float(el.item())
+    frames = world * FRAMES_PER_CHUNK * n_chunks
+    if rank == 0:
+        n_step_calls = n_chunks * n_steps * n_layers
+        line = {
+            "metric": METRIC, "value": frames / (total_ms / 1000.0), "unit": "frames/s", "n_gpus": world,
+            "steps": n_step_calls, "warmup": n_steps * n_layers, "ms_per_step": total_ms / n_step_calls,
+            "ms_total": total_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"c4 full denoise stack: {n_layers} layers x {n_steps} denoising steps "
+                                   f"x {n_chunks} chunks of 3 frames, one-layer shapes as C1, pool of "
+                                   f"16 pages per layer with a float64 page index; each chunk's KV "
+                                   f"appended to every layer's pool (index refreshed) inside the "
+                                   f"timed region; queries/gates cycle through {n_rot} resident draws",
+                       "l2": "no flush: each step reads >300 MB of selected K/V",
+                       "parallelism": f"replicas x{world} (independent layer stacks, no collective)"},
+            "clocks": clocks,
+            "gpu_launches": n_step_calls * 14 + n_chunks * n_layers * 3,
+        }
+        print(json.dumps(line), flush=True)
+    return 0
+
+
 def ctypes_void_array(events):
     import ctypes
     arr = (ctypes.c_void_p * len(events))(*[ctypes.c_void_p(e.cuda_event) for e in events])
@@ -393,6 +502,10 @@ def main():
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end loop (profiling runs)")
     ap.add_argument("--heads", type=int, default=None,
                     help="override H of the workload (smaller profiling captures)")
+    ap.add_argument("--config", choices=["c1", "c4"], default="c1",
+                    help="c1: one-layer step (default); c4: the full denoise stack")
+    ap.add_argument("--layers", type=int, default=30, help="c4: layers")
+    ap.add_argument("--chunks", type=int, default=20, help="c4: chunks")
     args = ap.parse_args()
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -405,6 +518,8 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local_rank))
     try:
+        if args.config == "c4":
+            return run_c4(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:

@@ -118,6 +118,29 @@ wa_status wa_gather_pages(const void* k_pool, const void* v_pool, int n_pool_pag
                           void* k_act, void* v_act, void* stream);
 
 /* ---------------------------------------------------------------------------
+ * Page pool maintenance (WorldAttention §3.2, "page-level KV abstraction" and the
+ * L1 tier, which holds the retrieved KV pages "along with ... page indices
+ * constructed from the keys K").
+ *
+ * The page index is a float64 array of B-row block SUMS of the keys:
+ *   page_index [n_pool_pages][T_p/B][H][d]  (needs T_p % B == 0)
+ * Block means, page means and therefore the page scores (S1) and the pooled block
+ * scores (S3) follow from it without re-reading the keys.
+ *
+ * wa_pool_index: (re)compute the index entries of pages[0..n_pages) (device ids).
+ * wa_pool_append: copy n_tokens new rows of K and V (k_new, v_new [n_tokens][H][d])
+ *   into the pool's flat token space at rows [token_offset, token_offset + n_tokens)
+ *   (a chunk may span page boundaries); when page_index is non-NULL, also refresh
+ *   the index entries of every block the write touches (a block's entry is exact
+ *   once all its rows are written).  INVALID_ARG: rows outside the pool. */
+wa_status wa_pool_index(const void* k_pool, int n_pool_pages, int T_p, int H, int d, int B,
+                        wa_dtype dtype, const int32_t* pages, int n_pages, double* page_index,
+                        void* stream);
+wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, int H, int d,
+                         wa_dtype dtype, const void* k_new, const void* v_new, int n_tokens,
+                         long long token_offset, double* page_index, int B, void* stream);
+
+/* ---------------------------------------------------------------------------
  * S3 -- head-adaptive block selection (WorldAttention §3.3, "Head-level sparsity
  * adaptation": per head the minimal set of blocks whose cumulative attention mass
  * reaches tau_h; summary step 5, block-pooled coarse selection).  For head h and
@@ -249,12 +272,18 @@ typedef struct wa_step_args {
   /* optional timing: NULL, or WA_STEP_EVENTS cudaEvent_t handles (as void*) that
      are recorded on `stream` at the stage boundaries listed below */
   void* const* stage_events;
+  /* optional page index (see wa_pool_index), [n_pool_pages][T_p/B][H][d] float64
+     block sums kept current by the caller; with it S1 and S3 read the index instead
+     of re-reducing the candidate pages (needs fused_gather and T_p % B == 0) */
+  const double* page_index;
 } wa_step_args;
 
 /* Stage boundaries recorded into wa_step_args.stage_events:
  *   0 start | 1 after S0+S1 (page retrieval) | 2 after S2 (gather; = 1 when fused)
  *   3 after S3 (block selection) | 4 after S4a (projection) | 5 after S4b (linear
- *   branch) | 6 after the work list | 7 after S5+S6 (sparse branch + gate) */
+ *   branch) | 6 after the work list | 7 after S5+S6 (sparse branch + gate).
+ * With bf16 inputs S4a and S4b run on a second stream that forks after event 2 and
+ * joins before event 6, so events 4 and 5 are recorded on that stream. */
 #define WA_STEP_EVENTS 8
 
 size_t wa_hsa_step_workspace_size(const wa_step_args* a);

@@ -44,7 +44,23 @@ k_gather(const uint4* __restrict__ kp, const uint4* __restrict__ vp, int n_pages
   for (; i < n16; i += stride) st_stream(dst + i, ld_stream(src + i));
 }
 
+__global__ void __launch_bounds__(256)
+k_copy16(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n16) {
+  const size_t stride = static_cast<size_t>(gridDim.x) * blockDim.x;
+  for (size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n16; i += stride)
+    st_stream(dst + i, ld_stream(src + i));
+}
+
 }  // namespace
+
+wa_status launch_copy16(const void* src, void* dst, size_t n16, cudaStream_t st) {
+  size_t blocks = (n16 + 1023) / 1024;
+  if (blocks > 8 * 148) blocks = 8 * 148;
+  if (blocks < 1) blocks = 1;
+  k_copy16<<<static_cast<unsigned>(blocks), 256, 0, st>>>(static_cast<const uint4*>(src),
+                                                          static_cast<uint4*>(dst), n16);
+  return check_launch("copy16");
+}
 
 wa_status launch_gather(const void* k_pool, const void* v_pool, int n_pages, size_t page_bytes,
                         const int32_t* sel, int K_p, void* k_act, void* v_act, uint32_t* err,

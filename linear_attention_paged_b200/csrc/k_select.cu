@@ -110,8 +110,9 @@ k_prompt_select(const float* __restrict__ e_cur, const float* __restrict__ e_chu
 template <typename T, int V>
 __global__ void __launch_bounds__(256)
 k_rowblock_sum(const T* __restrict__ x, const int32_t* __restrict__ src_ids, int n_pages,
-               int rows, int cols, int B, int nb, int bps, double* __restrict__ blocksum,
-               const double* __restrict__ qbar, double* __restrict__ kdot, uint32_t* err) {
+               int rows, int cols, int B, int nb, int bps, int block0, int nb_end, int bs_by_page,
+               double* __restrict__ blocksum, const double* __restrict__ qbar,
+               double* __restrict__ kdot, uint32_t* err) {
   __shared__ double red[32];
   const int s = blockIdx.y, split = blockIdx.x;
   const int c0 = (blockIdx.z * blockDim.x + threadIdx.x) * V;
@@ -123,7 +124,7 @@ k_rowblock_sum(const T* __restrict__ x, const int32_t* __restrict__ src_ids, int
   double part[V];
 #pragma unroll
   for (int v = 0; v < V; ++v) part[v] = 0.0;
-  const int b0 = split * bps, b1 = min(nb, b0 + bps);
+  const int b0 = block0 + split * bps, b1 = min(nb_end, b0 + bps);
   for (int b = b0; b < b1; ++b) {
     const int r0 = b * B, r1 = min(rows, r0 + B);
     double acc[V];
@@ -153,7 +154,7 @@ k_rowblock_sum(const T* __restrict__ x, const int32_t* __restrict__ src_ids, int
       }
     }
     if (blocksum) {
-      double* o = blocksum + (static_cast<size_t>(s) * nb + b) * cols + c0;
+      double* o = blocksum + (static_cast<size_t>(bs_by_page ? page : s) * nb + b) * cols + c0;
 #pragma unroll
       for (int v = 0; v < V; ++v) o[v] = acc[v];
     }
@@ -447,6 +448,7 @@ RowsumPlan rowsum_plan(int n_src, int rows, int cols, int B, wa_dtype dt) {
     p.n_cc = threads_total / 64;
   }
   p.nb = (rows + B - 1) / B;
+  p.n_blocks = p.nb;
   const long long ctas = static_cast<long long>(n_src) * p.n_cc * p.nb;
   p.bps = ctas > 32LL * 148 ? static_cast<int>((ctas + 32LL * 148 - 1) / (32LL * 148)) : 1;
   p.n_split = (p.nb + p.bps - 1) / p.bps;
@@ -460,14 +462,49 @@ wa_status launch_rowblock_sum(const void* x, wa_dtype dt, const int32_t* src_ids
   dim3 grid(p.n_split, n_src, p.n_cc);
   if (dt == WA_BF16) {
     k_rowblock_sum<__nv_bfloat16, 8><<<grid, p.threads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), src_ids, n_pages, rows, cols, B, p.nb, p.bps, blocksum,
-        qbar, kdot, err);
+        static_cast<const __nv_bfloat16*>(x), src_ids, n_pages, rows, cols, B, p.nb, p.bps,
+        p.block0, p.block0 + p.n_blocks, p.by_page, blocksum, qbar, kdot, err);
   } else {
-    k_rowblock_sum<float, 4><<<grid, p.threads, 0, st>>>(static_cast<const float*>(x), src_ids,
-                                                          n_pages, rows, cols, B, p.nb, p.bps,
-                                                          blocksum, qbar, kdot, err);
+    k_rowblock_sum<float, 4><<<grid, p.threads, 0, st>>>(
+        static_cast<const float*>(x), src_ids, n_pages, rows, cols, B, p.nb, p.bps, p.block0,
+        p.block0 + p.n_blocks, p.by_page, blocksum, qbar, kdot, err);
   }
   return check_launch("rowblock_sum");
+}
+
+RowsumPlan rowsum_plan_range(int rows, int cols, int B, wa_dtype dt, int block0, int n_blocks) {
+  RowsumPlan p = rowsum_plan(1, n_blocks * B, cols, B, dt);
+  p.nb = (rows + B - 1) / B;
+  p.block0 = block0;
+  p.n_blocks = n_blocks;
+  p.n_split = (n_blocks + p.bps - 1) / p.bps;
+  return p;
+}
+
+// kdot[c][b] = qbar . page_index[cand[c]][b][:]  (one CTA per (block, candidate page))
+__global__ void __launch_bounds__(128)
+k_index_dot(const double* __restrict__ page_index, const int32_t* __restrict__ cand, int n_pages,
+            int nbp, int cols, const double* __restrict__ qbar, double* __restrict__ kdot,
+            uint32_t* err) {
+  __shared__ double red[32];
+  const int b = blockIdx.x, c = blockIdx.y;
+  int page = cand[c];
+  if (page < 0 || page >= n_pages) {
+    if (threadIdx.x == 0) atomicOr(err, WA_DEVERR_PAGE_ID);
+    page = 0;
+  }
+  const double* row = page_index + (static_cast<size_t>(page) * nbp + b) * cols;
+  double acc = 0.0;
+  for (int e = threadIdx.x; e < cols; e += blockDim.x) acc += row[e] * qbar[e];
+  acc = block_sum(acc, red);
+  if (threadIdx.x == 0) kdot[static_cast<size_t>(c) * nbp + b] = acc;
+}
+
+wa_status launch_index_dot(const double* page_index, const int32_t* cand, int n_c, int n_pages,
+                           int nbp, int cols, const double* qbar, double* kdot, uint32_t* err,
+                           cudaStream_t st) {
+  k_index_dot<<<dim3(nbp, n_c), 128, 0, st>>>(page_index, cand, n_pages, nbp, cols, qbar, kdot, err);
+  return check_launch("index_dot");
 }
 
 wa_status launch_qmeans(const double* qsum, int n_qb, int Nq, int B, int cols, double* qbar,

@@ -186,7 +186,9 @@ PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, 
   w.qbar = c.take<double>(cols);
   w.q_blockmean = c.take<double>(static_cast<size_t>(n_qb) * cols);
   w.k_blocksum = k_blocks ? c.take<double>(static_cast<size_t>(n_c) * ceil_div(T_p, B) * cols) : nullptr;
-  w.kdot = c.take<double>(static_cast<size_t>(n_c) * w.kp.n_split * w.kp.n_cc);
+  const size_t per_page = static_cast<size_t>(w.kp.n_split) * w.kp.n_cc;
+  const size_t nbp = static_cast<size_t>(ceil_div(T_p, B));
+  w.kdot = c.take<double>(static_cast<size_t>(n_c) * (per_page > nbp ? per_page : nbp));
   return w;
 }
 
@@ -195,13 +197,19 @@ PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, 
 wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int d,
                          const void* k_pool, int n_pool_pages, int T_p, const int32_t* cand,
                          int n_c, int K_p, int B, wa_dtype dt, double* alpha, int32_t* sel,
-                         int32_t* sel_pos, cudaStream_t st) {
+                         int32_t* sel_pos, cudaStream_t st, const double* page_index = nullptr) {
   const int cols = H * d;
   uint32_t* err = errw();
   if (!err) return set_error(WA_ERR_CUDA, "no device error word (is a CUDA device present?)");
   WA_TRY(launch_rowblock_sum(q, dt, nullptr, 1, 1, Nq, cols, B, w.q_blocksum, nullptr, nullptr, w.qp,
                              err, st));
   WA_TRY(launch_qmeans(w.q_blocksum, ceil_div(Nq, B), Nq, B, cols, w.qbar, w.q_blockmean, st));
+  if (page_index) {
+    // the page index already holds the candidate pages' block sums
+    const int nbp = T_p / B;
+    WA_TRY(launch_index_dot(page_index, cand, n_c, n_pool_pages, nbp, cols, w.qbar, w.kdot, err, st));
+    return launch_alpha_topk(w.kdot, nbp, n_c, T_p, H, d, K_p, cand, alpha, sel, sel_pos, st);
+  }
   WA_TRY(launch_rowblock_sum(k_pool, dt, cand, n_c, n_pool_pages, T_p, cols, B, w.k_blocksum, w.qbar,
                              w.kdot, w.kp, err, st));
   return launch_alpha_topk(w.kdot, w.kp.n_split * w.kp.n_cc, n_c, T_p, H, d, K_p, cand, alpha, sel,
@@ -298,6 +306,59 @@ wa_status wa_gather_pages(const void* k_pool, const void* v_pool, int n_pool_pag
 }
 
 // ------------------------------------------------------------------ S3
+// ------------------------------------------------------------------ pool
+wa_status wa_pool_index(const void* k_pool, int n_pool_pages, int T_p, int H, int d, int B,
+                        wa_dtype dtype, const int32_t* pages, int n_pages, double* page_index,
+                        void* stream) {
+  WA_REQUIRE(k_pool && pages && page_index, "NULL pointer");
+  WA_REQUIRE(n_pool_pages >= 1 && T_p >= 1 && n_pages >= 1, "sizes must be >= 1");
+  WA_TRY(check_shape(H, d, B, dtype));
+  if (T_p % B != 0) return set_error(WA_ERR_UNSUPPORTED, "the page index needs T_p %% B == 0");
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  const int cols = H * d;
+  RowsumPlan p = rowsum_plan(n_pages, T_p, cols, B, dtype);
+  p.by_page = 1;
+  return launch_rowblock_sum(k_pool, dtype, pages, n_pages, n_pool_pages, T_p, cols, B, page_index,
+                             nullptr, nullptr, p, err, static_cast<cudaStream_t>(stream));
+}
+
+wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, int H, int d,
+                         wa_dtype dtype, const void* k_new, const void* v_new, int n_tokens,
+                         long long token_offset, double* page_index, int B, void* stream) {
+  WA_REQUIRE(k_pool && v_pool && k_new && v_new, "NULL pointer");
+  WA_REQUIRE(n_pool_pages >= 1 && T_p >= 1 && n_tokens >= 1, "sizes must be >= 1");
+  WA_REQUIRE(dtype == WA_F32 || dtype == WA_BF16, "bad dtype");
+  WA_REQUIRE(H >= 1 && d >= 1, "sizes must be >= 1");
+  const long long rows = static_cast<long long>(n_pool_pages) * T_p;
+  WA_REQUIRE(rows < (1LL << 31), "pool too large");
+  WA_REQUIRE(token_offset >= 0 && token_offset + n_tokens <= rows,
+             "rows [%lld, %lld) fall outside the pool's %lld rows", token_offset,
+             token_offset + n_tokens, rows);
+  if (page_index) {
+    WA_TRY(check_shape(H, d, B, dtype));
+    if (T_p % B != 0) return set_error(WA_ERR_UNSUPPORTED, "the page index needs T_p %% B == 0");
+  }
+  const size_t row_bytes = static_cast<size_t>(H) * d * elem_size(dtype);
+  if (row_bytes % 16 != 0 || !aligned16(k_pool) || !aligned16(v_pool) || !aligned16(k_new) ||
+      !aligned16(v_new))
+    return set_error(WA_ERR_UNSUPPORTED, "pool append needs 16-byte aligned rows");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t off = static_cast<size_t>(token_offset) * row_bytes;
+  const size_t n16 = static_cast<size_t>(n_tokens) * row_bytes / 16;
+  WA_TRY(launch_copy16(k_new, static_cast<char*>(k_pool) + off, n16, st));
+  WA_TRY(launch_copy16(v_new, static_cast<char*>(v_pool) + off, n16, st));
+  if (!page_index) return WA_OK;
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  const int b_first = static_cast<int>(token_offset / B);
+  const int b_last = static_cast<int>((token_offset + n_tokens - 1) / B);
+  const int cols = H * d;
+  RowsumPlan p = rowsum_plan_range(static_cast<int>(rows), cols, B, dtype, b_first, b_last - b_first + 1);
+  return launch_rowblock_sum(k_pool, dtype, nullptr, 1, 1, static_cast<int>(rows), cols, B, page_index,
+                             nullptr, nullptr, p, err, st);
+}
+
 namespace wa_detail {
 struct BlockSelectWs {
   double* qsum;
@@ -499,6 +560,8 @@ wa_status validate_step(const wa_step_args* a) {
   WA_REQUIRE(ceil_div(static_cast<int>(L), a->B) <= 8192, "at most 8192 key blocks");
   if (a->fused_gather && a->T_p % a->B != 0)
     return set_error(WA_ERR_UNSUPPORTED, "fused gather needs T_p %% B == 0");
+  if (a->page_index && (!a->fused_gather || a->T_p % a->B != 0))
+    return set_error(WA_ERR_UNSUPPORTED, "the page index needs fused_gather and T_p %% B == 0");
   WA_REQUIRE(static_cast<long long>(a->n_pool_pages) * a->T_p < (1LL << 31), "pool too large");
   return WA_OK;
 }
@@ -580,7 +643,7 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
   double* alpha = a->alpha_out ? a->alpha_out : w.alpha;
   int32_t* sel = a->sel_out ? a->sel_out : w.sel;
   WA_TRY(run_page_score(w.ps, a->q, a->Nq, a->H, a->d, a->k_pool, a->n_pool_pages, a->T_p, w.cand,
-                        a->n_c, a->K_p, a->B, a->dtype, alpha, sel, w.sel_pos, st));
+                        a->n_c, a->K_p, a->B, a->dtype, alpha, sel, w.sel_pos, st, a->page_index));
 
   mark(1);
   // S2: page table (fused) or explicit gather
@@ -591,9 +654,14 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
   if (a->fused_gather) {
     rs.k = a->k_pool; rs.v = a->v_pool; rs.page_ids = sel; rs.page_rows = a->T_p;
     rs.n_pages = a->n_pool_pages; rs.L = L;
-    km.data = w.ps.k_blocksum;
-    km.page_pos = w.sel_pos;
     km.nbp = a->T_p / a->B;
+    if (a->page_index) {
+      km.data = a->page_index;   // indexed by pool page id
+      km.page_pos = sel;
+    } else {
+      km.data = w.ps.k_blocksum; // indexed by candidate position
+      km.page_pos = w.sel_pos;
+    }
   } else {
     const size_t page_bytes = static_cast<size_t>(a->T_p) * cols * elem_size(a->dtype);
     WA_TRY(launch_gather(a->k_pool, a->v_pool, a->n_pool_pages, page_bytes, sel, a->K_p, w.k_act,

@@ -41,11 +41,20 @@ wa_status launch_prompt_select(const float* e_cur, const float* e_chunks, int n_
 struct RowsumPlan {
   int threads = 0;   // threads per CTA (V columns each)
   int n_cc = 1;      // column chunks
-  int nb = 0;        // blocks per source
+  int nb = 0;        // blocks per source (also the source stride of blocksum)
   int bps = 1;       // blocks per CTA
   int n_split = 1;   // CTAs per source and column chunk
+  int block0 = 0;    // first block summed
+  int n_blocks = 0;  // blocks summed (from block0)
+  int by_page = 0;   // blocksum indexed by pool page id instead of source position
 };
 RowsumPlan rowsum_plan(int n_src, int rows, int cols, int B, wa_dtype dt);
+// Plan over blocks [block0, block0 + n_blocks) of one source of `rows` rows.
+RowsumPlan rowsum_plan_range(int rows, int cols, int B, wa_dtype dt, int block0, int n_blocks);
+// kdot[c][b] = qbar . page_index[cand[c]][b] (page scores from the page index).
+wa_status launch_index_dot(const double* page_index, const int32_t* cand, int n_c, int n_pages,
+                           int nbp, int cols, const double* qbar, double* kdot, uint32_t* err,
+                           cudaStream_t st);
 wa_status launch_rowblock_sum(const void* x, wa_dtype dt, const int32_t* src_ids, int n_src,
                               int n_pages, int rows, int cols, int B, double* blocksum,
                               const double* qbar, double* kdot, const RowsumPlan& p, uint32_t* err,
@@ -83,6 +92,9 @@ wa_status launch_block_select(const double* q_blockmean, int Nq, int H, int d, i
 wa_status launch_gather(const void* k_pool, const void* v_pool, int n_pages, size_t page_bytes,
                         const int32_t* sel, int K_p, void* k_act, void* v_act, uint32_t* err,
                         cudaStream_t st);
+
+// dst[0..n16) = src[0..n16) in 16-byte units.
+wa_status launch_copy16(const void* src, void* dst, size_t n16, cudaStream_t st);
 
 // ---------------------------------------------------------------- fp32 SIMT path
 wa_status launch_simt_project(const float* x, const int32_t* page_ids, int page_rows, int n_pages,

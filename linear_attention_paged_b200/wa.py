@@ -51,6 +51,7 @@ class StepArgs(ctypes.Structure):
         ("chunk_out", P), ("alpha_out", P), ("sel_out", P), ("blk_mask_out", P),
         ("k_til_out", P), ("v_til_out", P),
         ("stage_events", P),
+        ("page_index", P),
     ]
 
 
@@ -73,6 +74,9 @@ _SIGS = {
     "wa_hsa_attention_workspace_size": (c_size_t, [c_int] * 7),
     "wa_hsa_attention": (c_int, [P, c_int, c_int, c_int, P, P, c_int, c_int, P, P, P, c_int, P,
                                  c_int, P, P, P, P, c_size_t, P]),
+    "wa_pool_index": (c_int, [P, c_int, c_int, c_int, c_int, c_int, c_int, P, c_int, P, P]),
+    "wa_pool_append": (c_int, [P, P, c_int, c_int, c_int, c_int, c_int, P, P, c_int, ctypes.c_longlong,
+                               P, c_int, P]),
     "wa_hsa_step_workspace_size": (c_size_t, [ctypes.POINTER(StepArgs)]),
     "wa_hsa_step": (c_int, [ctypes.POINTER(StepArgs), P, c_size_t, P]),
 }
@@ -180,6 +184,29 @@ def wa_gather_pages(k_pool, v_pool, sel, stream=None):
     return k_act, v_act
 
 
+# --------------------------------------------------------------------- pool
+def wa_pool_index(k_pool, pages, B: int = 64, page_index=None, stream=None):
+    """Float64 block sums [P][T_p/B][H][d] of the given pool pages (others untouched)."""
+    _need_cuda(k_pool, pages, page_index)
+    P_, T_p, H, d = k_pool.shape
+    if page_index is None:
+        page_index = torch.zeros((P_, T_p // B, H, d), dtype=torch.float64, device=k_pool.device)
+    _check("wa_pool_index", lib.wa_pool_index(_p(k_pool), P_, T_p, H, d, B, dtype_code(k_pool),
+                                              _p(pages), pages.numel(), _p(page_index),
+                                              _stream(stream)))
+    return page_index
+
+
+def wa_pool_append(k_pool, v_pool, k_new, v_new, token_offset: int, page_index=None, B: int = 64,
+                   stream=None):
+    """Write new K/V rows into the pool's flat token space (and refresh the index)."""
+    _need_cuda(k_pool, v_pool, k_new, v_new, page_index)
+    P_, T_p, H, d = k_pool.shape
+    _check("wa_pool_append", lib.wa_pool_append(
+        _p(k_pool), _p(v_pool), P_, T_p, H, d, dtype_code(k_pool), _p(k_new), _p(v_new),
+        k_new.shape[0], int(token_offset), _p(page_index), B, _stream(stream)))
+
+
 # --------------------------------------------------------------------- S3
 def wa_block_select(q, tau, B: int = 64, k_act=None, k_blockmean=None, L: Optional[int] = None,
                     stream=None):
@@ -257,7 +284,7 @@ class HSAStep:
 
     def __init__(self, q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 4,
                  B: int = 64, e_cur=None, e_chunks=None, fused_gather: bool = True,
-                 keep_intermediates: bool = False, out=None):
+                 keep_intermediates: bool = False, out=None, page_index=None):
         _need_cuda(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, e_cur, e_chunks)
         Nq, H, d = q.shape
         P_, T_p = k_pool.shape[0], k_pool.shape[1]
@@ -282,6 +309,8 @@ class HSAStep:
         a.e_k, a.e_v, a.tau, a.gate = _p(e_k), _p(e_v), _p(tau), _p(gate)
         a.dtype, a.fused_gather = dtype_code(q), int(bool(fused_gather))
         a.out = _p(self.out)
+        a.page_index = _p(page_index)
+        self._keep.append(page_index)
         self.inter = {}
         if keep_intermediates:
             self.inter = dict(
@@ -314,10 +343,10 @@ class HSAStep:
 
 def wa_hsa_step(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 4, B: int = 64,
                 e_cur=None, e_chunks=None, fused_gather: bool = True, keep_intermediates: bool = False,
-                stream=None):
+                stream=None, page_index=None):
     """One HSA decode step; returns ``out`` (and the intermediates when asked)."""
     st = HSAStep(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p, B, e_cur, e_chunks,
-                 fused_gather, keep_intermediates)
+                 fused_gather, keep_intermediates, page_index=page_index)
     out = st(stream)
     return (out, st.inter) if keep_intermediates else out
 

@@ -271,3 +271,102 @@ def test_full_size_stress_step(wa):
     cfg = W.C2
     samples = [(0, 0), (4, cfg.n_qb - 1), (7, 20), (11, 50)]
     _full_size_step(wa, cfg, samples)
+
+
+# ---------------------------------------------------------------- page pool
+def test_pool_index_and_append(wa):
+    cfg = SMALL_BF16
+    inp = inputs(cfg)
+    P_, T_p = cfg.n_pool_pages, cfg.T_p
+    pages = torch.arange(P_, dtype=torch.int32, device="cuda")
+    idx = wa.wa_pool_index(inp["k_pool"], pages, cfg.B)
+    for p in range(P_):
+        ref = O.block_means(inp["k_pool"][p], cfg.B) * cfg.B
+        np.testing.assert_allclose(to64(idx[p]), ref, rtol=1e-12, atol=1e-12)
+    # append 700 rows across the boundary of pages 2 and 3
+    g = torch.Generator(device="cuda").manual_seed(9)
+    n, off = 700, 2 * T_p + 900
+    k_new = torch.randn((n, cfg.H, cfg.d), generator=g, device="cuda").to(torch.bfloat16)
+    v_new = torch.randn((n, cfg.H, cfg.d), generator=g, device="cuda").to(torch.bfloat16)
+    k_before = inp["k_pool"].clone()
+    wa.wa_pool_append(inp["k_pool"], inp["v_pool"], k_new, v_new, off, page_index=idx, B=cfg.B)
+    torch.cuda.synchronize()
+    flat_k = inp["k_pool"].view(P_ * T_p, cfg.H, cfg.d)
+    flat_v = inp["v_pool"].view(P_ * T_p, cfg.H, cfg.d)
+    assert torch.equal(flat_k[off:off + n], k_new) and torch.equal(flat_v[off:off + n], v_new)
+    untouched = torch.ones(P_ * T_p, dtype=torch.bool)
+    untouched[off:off + n] = False
+    assert torch.equal(flat_k[untouched.cuda()], k_before.view(P_ * T_p, cfg.H, cfg.d)[untouched.cuda()])
+    for p in (2, 3):
+        ref = O.block_means(inp["k_pool"][p], cfg.B) * cfg.B
+        np.testing.assert_allclose(to64(idx[p]), ref, rtol=1e-12, atol=1e-12)
+    check_device_ok(wa)
+
+
+@pytest.mark.parametrize("cfg", [SMALL_BF16, SMALL_BF16_D64], ids=lambda c: c.name)
+def test_hsa_step_with_page_index(wa, cfg):
+    inp = inputs(cfg)
+    pages = torch.arange(cfg.n_pool_pages, dtype=torch.int32, device="cuda")
+    idx = wa.wa_pool_index(inp["k_pool"], pages, cfg.B)
+    out, inter = wa.wa_hsa_step(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"],
+                                inp["e_v"], inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B,
+                                keep_intermediates=True, page_index=idx)
+    res = O.hsa_step(inp, cfg.B, cfg.K_p)
+    np.testing.assert_allclose(to64(inter["alpha"]), res["alpha"], rtol=1e-9, atol=1e-13)
+    if res["page_margin"] >= 1e-5:
+        assert inter["sel"].cpu().tolist() == res["sel"]
+    compare_selection(mask_to_sets(inter["blk_mask"], cfg.n_kb), res["kept"], res["block_margin"],
+                      f"{cfg.name} masks (page index)")
+    assert_close(out, res["o"], "bf16", f"{cfg.name} step O (page index)")
+    check_device_ok(wa)
+
+
+def test_full_size_long_history_step(wa):
+    """120-page pool (1.5 M tokens, 9.2 GB of K+V); prompt-level retrieval picks the chunk."""
+    cfg = W.C3
+    samples = [(0, 0), (11, cfg.n_qb - 1), (6, 40)]
+    _full_size_step(wa, cfg, samples)
+
+
+def test_denoise_stack_procedure(wa):
+    """The full denoise-stack procedure at one-layer shapes: steps with fresh queries,
+    new chunks' KV appended to the pool between chunks with the page index kept
+    current, checked against the oracle on the first and last steps."""
+    cfg = W.C1.with_(name="c4_layer", n_chunks=2, seed=41)   # 16-page pool: 8 history + 8 for appends
+    inp = W.make_inputs(cfg, device="cuda", gen_device="cuda")
+    P_ = cfg.n_pool_pages
+    hist = inp["chunk_pages"][0:1]                            # the candidate chunk stays the history
+    idx = wa.wa_pool_index(inp["k_pool"], torch.arange(P_, dtype=torch.int32, device="cuda"), cfg.B)
+    g = torch.Generator(device="cuda").manual_seed(77)
+    fill = cfg.n_c * cfg.T_p
+    n_chunks, n_steps = 3, 2
+    checked = []
+    for chunk in range(n_chunks):
+        for s in range(n_steps):
+            q = (torch.randn((cfg.Nq, cfg.H, cfg.d), generator=g, device="cuda") / cfg.d ** 0.5).to(torch.bfloat16)
+            gate = torch.randn((cfg.Nq, cfg.H), generator=g, device="cuda")
+            out, inter = wa.wa_hsa_step(q, inp["k_pool"], inp["v_pool"], hist, inp["e_k"], inp["e_v"],
+                                        inp["tau"].cuda(), gate, cfg.K_p, cfg.B, keep_intermediates=True,
+                                        page_index=idx)
+            if (chunk, s) in ((0, 0), (n_chunks - 1, n_steps - 1)):
+                checked.append((q.clone(), gate.clone(), out.clone(), inter["sel"].cpu().tolist()))
+        # the chunk's own KV (3 frames) goes into the pool after its denoising steps
+        k_new = (torch.randn((cfg.Nq, cfg.H, cfg.d), generator=g, device="cuda") / cfg.d ** 0.5).to(torch.bfloat16)
+        v_new = (torch.randn((cfg.Nq, cfg.H, cfg.d), generator=g, device="cuda") / cfg.d ** 0.5).to(torch.bfloat16)
+        wa.wa_pool_append(inp["k_pool"], inp["v_pool"], k_new, v_new, fill, page_index=idx, B=cfg.B)
+        fill += cfg.Nq
+    torch.cuda.synchronize()
+    # the index of the appended pages matches the keys now in the pool
+    for p in (cfg.n_c, cfg.n_c + 1):
+        ref = O.block_means(inp["k_pool"][p], cfg.B) * cfg.B
+        np.testing.assert_allclose(to64(idx[p]), ref, rtol=1e-12, atol=1e-12)
+    for k, (q, gate, out, sel) in enumerate(checked):
+        step_inp = dict(inp, q=q, gate=gate, cand=hist[0].cpu())
+        step_inp.pop("e_cur", None)
+        res = O.hsa_step(step_inp, cfg.B, cfg.K_p, rows_of_blocks=[(0, 0), (7, cfg.n_qb - 1)])
+        if res["page_margin"] >= 1e-5:
+            assert sel == res["sel"]
+        for (h, i), blk in res["blocks"].items():
+            r0, r1 = i * cfg.B, min(cfg.Nq, (i + 1) * cfg.B)
+            assert_close(out[r0:r1, h], blk["o"], "bf16", f"denoise stack step {k}: O[h={h}, block {i}]")
+    check_device_ok(wa)
