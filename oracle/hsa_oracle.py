@@ -178,7 +178,8 @@ def block_scores(q, k_act, B: int) -> np.ndarray:
     qb = block_means(q, B)                 # [n_qb][H][d]
     kb = block_means(k_act, B)             # [n_kb][H][d]
     d = qb.shape[2]
-    return np.einsum("ihd,jhd->hij", qb, kb) / math.sqrt(d)
+    # per head: [n_qb][d] @ [d][n_kb]
+    return np.stack([qb[:, h, :] @ kb[:, h, :].T for h in range(qb.shape[1])]) / math.sqrt(d)
 
 
 def block_select(q, k_act, tau, B: int, scores: Optional[np.ndarray] = None):
@@ -204,8 +205,10 @@ def linear_project(k_act, v_act, e_k, e_v):
     V = f64(v_act)
     EK = f64(e_k)
     EV = f64(e_v)
-    kt = np.einsum("lr,lhd->rhd", EK, K)
-    vt = np.einsum("lr,lhd->rhd", EV, V)
+    # sum over l of E[l][c] * X[l][h][:], as one [r][L] @ [L][H*d] product
+    L, H, d = K.shape
+    kt = (EK.T @ K.reshape(L, H * d)).reshape(-1, H, d)
+    vt = (EV.T @ V.reshape(L, H * d)).reshape(-1, H, d)
     return kt, vt
 
 
