@@ -12,19 +12,31 @@
 // MMA wants M = 128, so a tile is a pair of query blocks of the same head (rows
 // 0-63 and 64-127) that walks the union of their two key-block sets, each half
 // masking the blocks it did not select.  Pairs are chosen to overlap as much as
-// possible (k_pair_heads).  A pair's key list is split in two work items when it
-// is long enough, so that the work items fill whole waves of CTAs; the two
-// partial results (unnormalised O, running max m, sum l per row) are merged by
-// k_combine, which also applies the gate.  Items run longest first.
+// possible (k_pair_heads).  When the pairs fill fewer than two waves of CTAs, a
+// pair's key list is split in two work items whose partial results (unnormalised
+// O, running max m, sum l per row) k_combine merges before applying the gate.
+// Items run longest first.
 //
-// CTA = 256 threads, two CTAs per SM: warp 0 loads Q and the K blocks, warp 2 the
-// V blocks (TMA, 128-byte swizzle, straight from the pool pages through the page
-// table, each through its own 2-slot ring: a K slot frees as soon as its S = Q K^T
-// MMA completes, a V slot when its O += P V MMA completes); warp 1 owns TMEM and
-// issues tcgen05.mma; warps 4-7 run the online softmax with one thread per TMEM
-// lane (query row), write P back as bf16 into the S buffer, rescale O in TMEM only
-// when the running max grows by more than 2^8, and run the epilogue.  One CTA's
-// softmax overlaps the other CTA's MMAs.  Every wait is bounded in time.
+// CTA = 384 threads, one CTA per SM.  The item's key blocks are listed once in
+// shared memory; an iteration takes two consecutive blocks of the list (128 keys),
+// so S = Q K^T is one M=128, N=128 MMA chain (N=64 chains run at about two thirds of
+// the tensor rate: their operand reads from shared memory dominate).  Roles:
+//   warp 0  loads Q and the K blocks, warp 2 the V blocks (TMA, 128-byte swizzle,
+//           straight from the pool pages through a page table staged in shared
+//           memory) into rings of 128-key slots (3 for K, 2 for V);
+//   warp 1  owns TMEM (two 128-column S/P buffers, two O accumulators) and issues
+//           the S MMAs; warp 3 issues the P V MMAs.  An MMA's issue blocks behind
+//           the one executing, so one issuer waiting for the softmax would idle the
+//           tensor pipe; with two, S of iteration t+1 runs while P V of t waits.
+//           S_t reuses the buffer of iteration t-2 once that iteration's P V MMAs
+//           have completed;
+//   warps 4-7 / 8-11  two softmax groups, one per block of the iteration (S columns
+//           0-63 / 64-127), one thread per TMEM lane (query row), each with its own
+//           running max, sum and O accumulator, merged in the epilogue.  P goes
+//           back into the S buffer as bf16; O is rescaled in TMEM only when the
+//           running max grows by more than 2^8; a quarter of the exponentials run
+//           on the FMA pipe (exp2_poly) to unload the MUFU unit.
+// Every wait is bounded in time.
 #include <cuda.h>
 #include <cuda_bf16.h>
 
@@ -41,13 +53,21 @@ using namespace sm100;
 
 constexpr int kBM = 128;          // query rows per tile (two 64-row blocks)
 constexpr int kBN = 64;           // keys per block
-constexpr int kRing = 2;          // slots of the K ring and of the V ring
-constexpr int kThreads = 256;
-constexpr uint32_t kTmemCols = 256;
-constexpr int kColS = 0;          // two S/P buffers at columns 0 and 64
-constexpr int kColO = 128;        // O accumulator at columns 128 .. 128+d
+constexpr int kIterKeys = 128;    // keys per iteration: two blocks of the tile's list
+constexpr int kRingK = 3;         // 128-key slots of the K ring
+constexpr int kRingV = 2;         // 128-key slots of the V ring
+constexpr int kThreads = 384;     // warps 0-3: loads and MMA; 4-7 and 8-11: softmax
+constexpr uint32_t kTmemCols = 512;
+constexpr int kColS = 0;          // two 128-column S/P buffers at columns 0 and 128
+constexpr int kColO = 256;        // O accumulators: group g at columns 256 + g*d
 constexpr int kMaxW = 256;        // up to 8192 key blocks
-constexpr int kSplitMin = 8;      // pairs with at least this many key blocks are split in two
+constexpr int kMaxList = kMaxW * 32;
+constexpr int kMaxPages = 64;     // page-table entries staged in shared memory
+
+// Key-list entries (16 bits): block index in bits 0-12, bit 13 / bit 14 set when
+// the tile's first / second query block kept the block; kNoBlock pads an odd list.
+constexpr uint32_t kSel0 = 1u << 13, kSel1 = 1u << 14;
+constexpr uint32_t kNoBlock = 0xFFFFu;
 
 // item.y values
 constexpr int kWhole = -1;        // the whole key list; writes the final output
@@ -57,22 +77,27 @@ template <int D>
 struct Cfg {
   static constexpr int kPanels = D / 64;                 // 128-byte column panels
   static constexpr int kQBytes = kBM * D * 2;
-  static constexpr int kKVBytes = kBN * D * 2;
-  static constexpr int kSmem = kQBytes + 2 * kRing * kKVBytes + 1024;  // + alignment slack
-  static constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kBN, false, false);
+  static constexpr int kBlockBytes = kBN * D * 2;         // one 64-key block of K or V
+  static constexpr int kSlotBytes = 2 * kBlockBytes;      // a 128-key slot
+  static constexpr int kPanelBytes = kIterKeys * 128;     // one panel of a slot: 128 rows x 128 B
+  static constexpr int kSmem = kQBytes + (kRingK + kRingV) * kSlotBytes + 1024;  // + alignment slack
+  static constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kIterKeys, false, false);
   static constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, false, true);
 };
 
 struct Shared {
   uint64_t q_full;
-  uint64_t k_full[kRing], k_empty[kRing];
-  uint64_t v_full[kRing], v_empty[kRing];
+  uint64_t k_full[kRingK], k_empty[kRingK];
+  uint64_t v_full[kRingV], v_empty[kRingV];
   uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_done[2];   // completion of O += P_u V_u, by the parity of u
+  uint64_t p_full[2][2];  // [S buffer][softmax group], one arrival per softmax warp
+  uint64_t o_done[2];     // completion of O_g += P_u V_u (both groups), by the parity of u
   uint32_t tmem_base;
   int abort_flag;
-  uint32_t mask[2][kMaxW];
+  int scan[8];
+  int page_row0[kMaxPages];  // first pool row of each page of the key sequence
+  float xch[2][2][kBM];   // epilogue exchange of (m, l) between the two groups
+  uint16_t list[kMaxList + 2];  // the item's key blocks, two per iteration
 };
 
 // Bounded wait that also gives up when another role has aborted.
@@ -93,46 +118,86 @@ __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared&
   }
 }
 
-// Walks key blocks [k0, k1) of a tile's list in ascending block order: the list is
-// the union of the two masks (mode 1) or every block (mode 0).
-struct BlockIter {
-  const uint32_t* a;
-  const uint32_t* b;
-  int W, n_kb, w, all, pos, k1;
-  uint32_t bits;
-  __device__ int next_raw() {
-    if (all) { ++w; return w < n_kb ? w : -1; }
-    while (bits == 0u) {
-      if (++w >= W) return -1;
-      bits = a[w] | b[w];
-    }
-    const int j = w * 32 + __ffs(bits) - 1;
-    bits &= bits - 1u;
-    return j;
-  }
-  __device__ void init(const uint32_t* a_, const uint32_t* b_, int W_, int n_kb_, int all_, int k0_,
-                       int k1_) {
-    a = a_; b = b_; W = W_; n_kb = n_kb_; all = all_; w = -1; bits = 0u; pos = 0; k1 = k1_;
-    for (; pos < k0_; ++pos) next_raw();
-  }
-  __device__ int next() {
-    if (pos >= k1) return -1;
-    ++pos;
-    return next_raw();
-  }
-};
-
 __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
 
-__device__ __forceinline__ int key_row(const RowSource& rs, int bpp, int j, uint32_t* err) {
-  if (!rs.page_ids) return j * kBN;
-  int pg = rs.page_ids[j / bpp];
+// 2^y for a pair on the FMA pipe, to take part of the exponentials off the MUFU
+// unit (16 results per clock per SM, the softmax's narrowest pipe): y = j + f with
+// j = round(y) (adding 1.5 * 2^23 leaves j in the low mantissa bits) and f in
+// [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted for minimum relative error
+// (7.5e-5, far below bf16's 2^-9 for P), and 2^j is added into the exponent field.
+// y is clamped at -125 so the exponent never underflows; inputs are finite.
+__device__ __forceinline__ float2 exp2_poly(float2 y) {
+  y.x = fmaxf(y.x, -125.f);
+  y.y = fmaxf(y.y, -125.f);
+  const float2 shifter = make_float2(12582912.f, 12582912.f);
+  const float2 t = __fadd2_rn(y, shifter);
+  const float2 jf = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
+  const float2 f = __ffma2_rn(jf, make_float2(-1.f, -1.f), y);
+  float2 q = __ffma2_rn(make_float2(0.05517222f, 0.05517222f), f, make_float2(0.24261115f, 0.24261115f));
+  q = __ffma2_rn(q, f, make_float2(0.69326085f, 0.69326085f));
+  q = __ffma2_rn(q, f, make_float2(0.99992806f, 0.99992806f));
+  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
+                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
+}
+
+// One softmax pass over a 64-column half row held in r: p = 2^(s * scale_log2 - m)
+// packed to bf16 pairs in pk, the sum of p in lsum and (kMax) the raw row maximum.
+// kPoly routes one pair in four through exp2_poly (full blocks only: masked
+// columns hold -inf).
+template <bool kMax, bool kPoly>
+__device__ __forceinline__ void softmax_pass(const uint32_t (&r)[64], float2 sc2, float2 nm2,
+                                             uint32_t (&pk)[32], float& lsum, float& mraw) {
+  float2 acc2[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) acc2[e] = make_float2(0.f, 0.f);
+  float mx8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx8[e] = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const float2 x = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
+    if (kMax) mx8[e & 7] = max3f(mx8[e & 7], x.x, x.y);
+    const float2 y = __ffma2_rn(x, sc2, nm2);
+    const float2 pp = (kPoly && (e & 3) == 3) ? exp2_poly(y) : make_float2(ex2(y.x), ex2(y.y));
+    acc2[e & 3] = __fadd2_rn(acc2[e & 3], pp);
+    pk[e] = pack_bf16x2(pp.x, pp.y);
+  }
+  const float2 a01 = __fadd2_rn(acc2[0], acc2[1]), a23 = __fadd2_rn(acc2[2], acc2[3]);
+  const float2 a03 = __fadd2_rn(a01, a23);
+  lsum = a03.x + a03.y;
+  if (kMax)
+    mraw = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+}
+
+__device__ __forceinline__ float rowmax64(const uint32_t (&r)[64]) {
+  float mx8[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(__uint_as_float(r[e]), __uint_as_float(r[8 + e]));
+#pragma unroll
+  for (int c = 16; c < 64; c += 16)
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      mx8[e] = max3f(mx8[e], __uint_as_float(r[c + e]), __uint_as_float(r[c + 8 + e]));
+  return max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]), fmaxf(mx8[6], mx8[7]));
+}
+
+__device__ __forceinline__ int page_row0(const RowSource& rs, int i, uint32_t* err) {
+  int pg = rs.page_ids[i];
   if (pg < 0 || pg >= rs.n_pages) { atomicOr(err, WA_DEVERR_PAGE_ID); pg = 0; }
-  return pg * rs.page_rows + (j % bpp) * kBN;
+  return pg * rs.page_rows;
+}
+
+// First pool row of key block j: contiguous keys, or through the page table (staged
+// in shared memory when it is short, so the loads never wait on global memory).
+__device__ __forceinline__ int key_row(const RowSource& rs, const int* staged, int bpp, int j,
+                                       uint32_t* err) {
+  if (!rs.page_ids) return j * kBN;
+  const int i = j / bpp;
+  return (staged ? staged[i] : page_row0(rs, i, err)) + (j - i * bpp) * kBN;
 }
 
 struct Partials {
@@ -140,8 +205,16 @@ struct Partials {
   float* ml;   // [slots][128][2]  running max (log2 units) and sum
 };
 
+// One CTA per SM.  An iteration covers two consecutive blocks (ja, jb) of the
+// tile's key list: S = Q K^T is one N=128 MMA chain (full tensor rate; N=64 chains
+// are bound by their shared-memory operand reads), K and V of the two blocks sit in
+// one 128-key slot of their rings (the second half unused when the list is odd).
+// Softmax group 0 (warps 4-7) owns the blocks at even list positions (S columns
+// 0-63), group 1 (warps 8-11) those at odd positions (columns 64-127): each keeps
+// its own running max and sum and its own O accumulator, so the groups never
+// synchronise inside the loop; the epilogue merges the two (O, m, l) states.
 template <int D>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
 k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, int mode, int Nq, int H, int Lk,
                  RowSource rs, const uint32_t* __restrict__ blk_mask, int W, int n_qb,
@@ -174,29 +247,60 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   uint8_t* tiles = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* Qs = tiles;
-  auto Ks = [&](int s) { return tiles + C::kQBytes + s * C::kKVBytes; };
-  auto Vs = [&](int s) { return tiles + C::kQBytes + (kRing + s) * C::kKVBytes; };
+  auto Ks = [&](int s) { return tiles + C::kQBytes + s * C::kSlotBytes; };
+  auto Vs = [&](int s) { return tiles + C::kQBytes + (kRingK + s) * C::kSlotBytes; };
 
   if (tid == 0) {
     mbar_init(&sh.q_full, 1);
-    for (int s = 0; s < kRing; ++s) {
-      mbar_init(&sh.k_full[s], 1); mbar_init(&sh.k_empty[s], 1);
-      mbar_init(&sh.v_full[s], 1); mbar_init(&sh.v_empty[s], 1);
+    for (int s = 0; s < kRingK; ++s) { mbar_init(&sh.k_full[s], 1); mbar_init(&sh.k_empty[s], 1); }
+    for (int s = 0; s < kRingV; ++s) { mbar_init(&sh.v_full[s], 1); mbar_init(&sh.v_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sh.s_full[b], 1);
+      mbar_init(&sh.p_full[b][0], 4);
+      mbar_init(&sh.p_full[b][1], 4);
+      mbar_init(&sh.o_done[b], 1);
     }
-    for (int b = 0; b < 2; ++b) { mbar_init(&sh.s_full[b], 1); mbar_init(&sh.p_full[b], 128); }
-    mbar_init(&sh.o_done[0], 1);
-    mbar_init(&sh.o_done[1], 1);
     sh.abort_flag = 0;
     fence_mbar_init();
   }
-  if (mode == 1) {
-    const uint32_t* ma = blk_mask + (static_cast<size_t>(h) * n_qb + i0) * W;
-    const uint32_t* mb = i1 >= 0 ? blk_mask + (static_cast<size_t>(h) * n_qb + i1) * W : nullptr;
-    for (int w = tid; w < W; w += kThreads) {
-      sh.mask[0][w] = ma[w];
-      sh.mask[1][w] = mb ? mb[w] : 0u;
+  // The item's key blocks, positions [k0, k1) of the tile's list, with the
+  // selection bits of both query blocks: one scan over the mask words (at most
+  // kMaxW, one per thread).
+  const int n_blk = k1 - k0;
+  if (mode == 0) {
+    for (int q = tid; q < n_blk; q += kThreads)
+      sh.list[q] = static_cast<uint16_t>((k0 + q) | kSel0 | kSel1);
+  } else {
+    uint32_t ma = 0u, mb = 0u;
+    if (tid < W) {
+      ma = blk_mask[(static_cast<size_t>(h) * n_qb + i0) * W + tid];
+      if (i1 >= 0) mb = blk_mask[(static_cast<size_t>(h) * n_qb + i1) * W + tid];
+    }
+    const uint32_t un = ma | mb;
+    const int c = __popc(un);
+    int incl = c;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31 && warp < 8) sh.scan[warp] = incl;
+    __syncthreads();
+    if (tid < W) {
+      int pos = incl - c;
+      for (int w = 0; w < warp; ++w) pos += sh.scan[w];
+      for (uint32_t bits = un; bits != 0u; bits &= bits - 1u, ++pos) {
+        if (pos < k0 || pos >= k1) continue;
+        const int b = __ffs(bits) - 1;
+        sh.list[pos - k0] = static_cast<uint16_t>((tid * 32 + b) | (((ma >> b) & 1u) ? kSel0 : 0u) |
+                                                  (((mb >> b) & 1u) ? kSel1 : 0u));
+      }
     }
   }
+  if (tid == 0) sh.list[n_blk] = static_cast<uint16_t>(kNoBlock);
+  const int n_ids = rs.page_ids ? (Lk + rs.page_rows - 1) / rs.page_rows : 0;
+  const int* staged = (n_ids > 0 && n_ids <= kMaxPages) ? sh.page_row0 : nullptr;
+  if (staged && tid < n_ids) sh.page_row0[tid] = page_row0(rs, tid, err);
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, kTmemCols);
     tmem_relinquish();
@@ -205,242 +309,260 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sh.tmem_base;
-  const int n_blk = k1 - k0;
+  const int n_it = (n_blk + 1) / 2;
+  const uint32_t* list2 = reinterpret_cast<const uint32_t*>(sh.list);  // entries 2t, 2t+1
+  const bool odd_tail = (n_blk & 1) != 0;   // the last iteration holds one block
   const int bpp = rs.page_ids ? rs.page_rows / kBN : 0;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ Q + K producer
+  if (warp == 0 || warp == 2) {
+    // ------------------------------------------------------------ producers:
+    // warp 0 loads Q and the K blocks, warp 2 the V blocks
     if (lane == 0) {
-      prefetch_tmap(&tmQ);
-      prefetch_tmap(&tmK);
-      mbar_arrive_expect_tx(&sh.q_full, C::kQBytes);
-      const int y1 = i1 >= 0 ? i1 * 64 : Nq;  // out of range -> zero fill
-      for (int p = 0; p < C::kPanels; ++p) {
-        tma_load_2d(Qs + p * (kBM * 128), &tmQ, &sh.q_full, h * D + p * 64, i0 * 64);
-        tma_load_2d(Qs + p * (kBM * 128) + 64 * 128, &tmQ, &sh.q_full, h * D + p * 64, y1);
+      const bool isK = warp == 0;
+      const CUtensorMap* tm = isK ? &tmK : &tmV;
+      prefetch_tmap(tm);
+      if (isK) {
+        prefetch_tmap(&tmQ);
+        mbar_arrive_expect_tx(&sh.q_full, C::kQBytes);
+        const int y1 = i1 >= 0 ? i1 * 64 : Nq;  // out of range -> zero fill
+        for (int p = 0; p < C::kPanels; ++p) {
+          tma_load_2d(Qs + p * (kBM * 128), &tmQ, &sh.q_full, h * D + p * 64, i0 * 64);
+          tma_load_2d(Qs + p * (kBM * 128) + 64 * 128, &tmQ, &sh.q_full, h * D + p * 64, y1);
+        }
       }
-      BlockIter it;
-      it.init(sh.mask[0], sh.mask[1], W, n_kb, mode == 0, k0, k1);
-      int t = 0;
-      for (int j = it.next(); j >= 0; j = it.next(), ++t) {
-        const int s = t % kRing;
-        if (!wait_bar(&sh.k_empty[s], ((t / kRing) & 1) ^ 1, sh, err)) break;
-        const int row = key_row(rs, bpp, j, err);
-        mbar_arrive_expect_tx(&sh.k_full[s], C::kKVBytes);
+      const int ring = isK ? kRingK : kRingV;
+      for (int t = 0; t < n_it; ++t) {
+        const int s = t % ring;
+        uint64_t* empty = isK ? &sh.k_empty[s] : &sh.v_empty[s];
+        uint64_t* full = isK ? &sh.k_full[s] : &sh.v_full[s];
+        if (!wait_bar(empty, ((t / ring) & 1) ^ 1, sh, err)) break;
+        const uint32_t wrd = list2[t];
+        const int ja = static_cast<int>(wrd & 0x1FFFu);
+        const int jb = (wrd >> 16) == kNoBlock ? -1 : static_cast<int>((wrd >> 16) & 0x1FFFu);
+        uint8_t* dst = isK ? Ks(s) : Vs(s);
+        mbar_arrive_expect_tx(full, (jb >= 0 ? 2 : 1) * C::kBlockBytes);
+        const int ra = key_row(rs, staged, bpp, ja, err);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_2d(Ks(s) + p * (kBN * 128), &tmK, &sh.k_full[s], h * D + p * 64, row);
-      }
-    }
-  } else if (warp == 2) {
-    // ------------------------------------------------------------ V producer
-    if (lane == 0) {
-      prefetch_tmap(&tmV);
-      BlockIter it;
-      it.init(sh.mask[0], sh.mask[1], W, n_kb, mode == 0, k0, k1);
-      int t = 0;
-      for (int j = it.next(); j >= 0; j = it.next(), ++t) {
-        const int s = t % kRing;
-        if (!wait_bar(&sh.v_empty[s], ((t / kRing) & 1) ^ 1, sh, err)) break;
-        const int row = key_row(rs, bpp, j, err);
-        mbar_arrive_expect_tx(&sh.v_full[s], C::kKVBytes);
-        for (int p = 0; p < C::kPanels; ++p)
-          tma_load_2d(Vs(s) + p * (kBN * 128), &tmV, &sh.v_full[s], h * D + p * 64, row);
+          tma_load_2d(dst + p * C::kPanelBytes, tm, full, h * D + p * 64, ra);
+        if (jb >= 0) {
+          const int rb = key_row(rs, staged, bpp, jb, err);
+          for (int p = 0; p < C::kPanels; ++p)
+            tma_load_2d(dst + p * C::kPanelBytes + kBN * 128, tm, full, h * D + p * 64, rb);
+        }
       }
     }
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+    // ------------------------------------------------------------ S issuer
     if (lane == 0) {
       bool ok = wait_bar(&sh.q_full, 0, sh, err);
       tc_fence_after();
       const uint32_t q_base = smem_u32(Qs);
-      for (int t = 0; ok && t <= n_blk; ++t) {
-        if (t < n_blk) {
-          // S_t = Q K_t^T into S buffer t % 2 (its previous P was consumed by PV_{t-2},
-          // issued earlier by this thread)
-          const int s = t % kRing;
-          if (!wait_bar(&sh.k_full[s], (t / kRing) & 1, sh, err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t k_base = smem_u32(Ks(s));
-          const int sb = t & 1;
+      for (int t = 0; ok && t < n_it; ++t) {
+        // S_t = Q K_t^T (N = 128) into S buffer t % 2, once the P V MMAs of iteration
+        // t-2 (issued by the other issuer) have read that buffer's P
+        const int s = t % kRingK, sb = t & 1;
+        if (!wait_bar(&sh.k_full[s], (t / kRingK) & 1, sh, err)) break;
+        if (t >= 2 && !wait_bar(&sh.o_done[sb], ((t - 2) >> 1) & 1, sh, err)) break;
+        tc_fence_after();
+        const uint32_t k_base = smem_u32(Ks(s));
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t adesc = smem_desc_sw128(q_base + (k >> 2) * (kBM * 128) + (k & 3) * 32, 16, 1024);
-            const uint64_t bdesc = smem_desc_sw128(k_base + (k >> 2) * (kBN * 128) + (k & 3) * 32, 16, 1024);
-            mma_ss(tbase + kColS + sb * 64, adesc, bdesc, C::kIdescS, k > 0 ? 1u : 0u);
-          }
-          mma_commit(&sh.k_empty[s]);
-          mma_commit(&sh.s_full[sb]);
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t adesc = smem_desc_sw128(q_base + (k >> 2) * (kBM * 128) + (k & 3) * 32, 16, 1024);
+          const uint64_t bdesc = smem_desc_sw128(k_base + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
+          mma_ss(tbase + kColS + sb * kIterKeys, adesc, bdesc, C::kIdescS, k > 0 ? 1u : 0u);
         }
-        if (t > 0) {
-          // O += P_u V_u, P read from TMEM
-          const int u = t - 1, su = u & 1, vs = u % kRing;
-          if (!wait_bar(&sh.p_full[su], (u >> 1) & 1, sh, err)) { ok = false; break; }
-          if (!wait_bar(&sh.v_full[vs], (u / kRing) & 1, sh, err)) { ok = false; break; }
+        mma_commit(&sh.k_empty[s]);
+        mma_commit(&sh.s_full[sb]);
+      }
+    }
+  } else if (warp == 3) {
+    // ------------------------------------------------------------ P V issuer:
+    // O_g += P_g V_g for each group's block of iteration u, P read from TMEM.  A
+    // second issuing thread, so that S MMAs keep the tensor pipe busy while this one
+    // waits for the softmax (an MMA's issue blocks behind the one executing).
+    if (lane == 0) {
+      for (int u = 0; u < n_it; ++u) {
+        const int su = u & 1, vs = u % kRingV;
+        if (!wait_bar(&sh.v_full[vs], (u / kRingV) & 1, sh, err)) break;
+        const int n_grp = (u == n_it - 1 && odd_tail) ? 1 : 2;
+        bool ok = true;
+        for (int g = 0; g < 2; ++g) {
+          if (!wait_bar(&sh.p_full[su][g], (u >> 1) & 1, sh, err)) { ok = false; break; }
+          if (g >= n_grp) break;
           tc_fence_after();
-          const uint32_t v_base = smem_u32(Vs(vs));
+          const uint32_t v_base = smem_u32(Vs(vs)) + g * (kBN * 128);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
-            const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, 64 * 128, 1024);
-            mma_ts(tbase + kColO, tbase + kColS + su * 64 + kk * 8, bdesc, C::kIdescO,
-                   (u > 0 || kk > 0) ? 1u : 0u);
+            const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, C::kPanelBytes, 1024);
+            mma_ts(tbase + kColO + g * D, tbase + kColS + su * kIterKeys + g * kBN + kk * 8, bdesc,
+                   C::kIdescO, (u > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&sh.v_empty[vs]);
-          mma_commit(&sh.o_done[u & 1]);
         }
+        if (!ok) break;
+        mma_commit(&sh.v_empty[vs]);
+        mma_commit(&sh.o_done[su]);
       }
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------ softmax + epilogue
-    const int q4 = warp - 4;
+    const int g = (warp - 4) >> 2;                  // softmax group
+    const int q4 = warp & 3;                        // TMEM lane quarter of this warp
     const int row = q4 * 32 + lane;                 // TMEM lane = tile row
     const uint32_t lane_base = static_cast<uint32_t>(q4 * 32) << 16;
+    const uint32_t o_col = kColO + g * D;
     const int half = row >> 6;
     const int ib = half ? i1 : i0;
     const int qrow = ib * 64 + (row & 63);
     const bool row_valid = ib >= 0 && qrow < Nq;
-    const uint32_t* mymask = sh.mask[half];
+    const uint32_t sel_bit = half ? kSel1 : kSel0;   // the same for the whole warp
     const float scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(D));
+    const float2 sc2 = make_float2(scale_log2, scale_log2);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    BlockIter it;
-    it.init(sh.mask[0], sh.mask[1], W, n_kb, mode == 0, k0, k1);
+    // one arrival per warp once all its lanes' TMEM stores are complete
+    auto release_p = [&](int sb) {
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.p_full[sb][g]);
+    };
     int t = 0;
-    for (int j = it.next(); j >= 0; j = it.next(), ++t) {
+    for (; t < n_it; ++t) {
+      const uint32_t e = (list2[t] >> (16 * g)) & 0xFFFFu;
       const int sb = t & 1;
       if (!__all_sync(0xffffffffu, wait_bar(&sh.s_full[sb], (t >> 1) & 1, sh, err))) { ok = false; break; }
+      const uint32_t s_addr = tbase + lane_base + kColS + sb * kIterKeys + g * kBN;
+      if (e == kNoBlock) {         // group 1 in an odd list's last iteration: no block
+        release_p(sb);
+        continue;
+      }
+      if (!(e & sel_bit)) {
+        // this warp's query block did not keep the block: P = 0, state unchanged
+        uint32_t z[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) z[c] = 0u;
+        tmem_st32(s_addr, z);
+        tmem_wait_st();
+        release_p(sb);
+        continue;
+      }
       tc_fence_after();
       uint32_t r[64];
-      tmem_ld32(tbase + lane_base + kColS + sb * 64, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
-      tmem_ld32(tbase + lane_base + kColS + sb * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
+      tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
+      tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       tmem_wait_ld();
-      const bool sel = mode == 0 || ((mymask[j >> 5] >> (j & 31)) & 1u);
-      const int valid = min(kBN, Lk - j * kBN);
-      if (!sel || valid < kBN) {
-        // a block this half did not select, or the ragged last block: mask columns
+      const int valid = min(kBN, Lk - static_cast<int>(e & 0x1FFFu) * kBN);
+      const bool ragged = valid < kBN;   // the key sequence's last, partial block
+      if (ragged) {
 #pragma unroll
         for (int c = 0; c < 64; ++c)
-          if (!sel || c >= valid) r[c] = __float_as_uint(-INFINITY);
+          if (c >= valid) r[c] = __float_as_uint(-INFINITY);
       }
-      // row max of the raw scores: eight independent chains of 3-input maxima
-      float mx8[8];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) mx8[e] = fmaxf(__uint_as_float(r[e]), __uint_as_float(r[8 + e]));
-#pragma unroll
-      for (int c = 16; c < 64; c += 16)
-#pragma unroll
-        for (int e = 0; e < 8; ++e)
-          mx8[e] = max3f(mx8[e], __uint_as_float(r[c + e]), __uint_as_float(r[c + 8 + e]));
-      const float mraw = max3f(max3f(mx8[0], mx8[1], mx8[2]), max3f(mx8[3], mx8[4], mx8[5]),
-                               fmaxf(mx8[6], mx8[7]));
-      const float mx = mraw * scale_log2;   // scale_log2 > 0: the max commutes with it
+      // A row's first kept block sets its reference max before any exponential;
+      // afterwards the pass runs with the current (possibly stale) max and finds the
+      // new one alongside, and is redone only if the max grew by more than 2^8.
+      if (__any_sync(0xffffffffu, m_run == -INFINITY)) {
+        const float m0 = rowmax64(r) * scale_log2;   // scale_log2 > 0: max commutes
+        if (m_run == -INFINITY) m_run = m0;
+      }
+      uint32_t pk[32];
+      float lsum, mraw;
+      float2 nm2 = make_float2(-m_run, -m_run);
+      if (ragged) softmax_pass<true, false>(r, sc2, nm2, pk, lsum, mraw);
+      else softmax_pass<true, true>(r, sc2, nm2, pk, lsum, mraw);
+      const float mx = mraw * scale_log2;
       float factor = 1.f;
-      bool resc = false;
-      if (m_run == -INFINITY) {
-        m_run = mx;                        // no mass yet: O holds zeros for this row
-      } else if (mx > m_run + 8.f) {       // keep a stale max unless it grows by > 2^8
+      const bool resc = mx > m_run + 8.f;
+      if (resc) {
         factor = ex2(m_run - mx);
         m_run = mx;
-        resc = true;
+        nm2 = make_float2(-m_run, -m_run);
+        softmax_pass<false, false>(r, sc2, nm2, pk, lsum, mraw);
       }
-      const float neg_m = (m_run == -INFINITY) ? 0.f : -m_run;
-      // p = 2^(s * log2(e)/sqrt(d) - m) on column pairs (paired fp32 FMA and add),
-      // summed in four two-lane chains, packed to bf16 pairs
-      const float2 sc2 = make_float2(scale_log2, scale_log2);
-      const float2 nm2 = make_float2(neg_m, neg_m);
-      float2 acc2[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc2[e] = make_float2(0.f, 0.f);
-#pragma unroll
-      for (int c = 0; c < 64; c += 32) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float2 x = make_float2(__uint_as_float(r[c + 2 * e]), __uint_as_float(r[c + 2 * e + 1]));
-          const float2 y = __ffma2_rn(x, sc2, nm2);
-          const float2 pp = make_float2(ex2(y.x), ex2(y.y));
-          acc2[e & 3] = __fadd2_rn(acc2[e & 3], pp);
-          pk[e] = pack_bf16x2(pp.x, pp.y);
-        }
-        tmem_st16(tbase + lane_base + kColS + sb * 64 + c / 2, pk);
-      }
-      const float2 a01 = __fadd2_rn(acc2[0], acc2[1]), a23 = __fadd2_rn(acc2[2], acc2[3]);
-      const float2 a03 = __fadd2_rn(a01, a23);
-      const float sum = a03.x + a03.y;
-      l_run = l_run * factor + sum;
+      l_run = l_run * factor + lsum;
+      tmem_st32(s_addr, pk);
       tmem_wait_st();
       if (__any_sync(0xffffffffu, resc)) {
-        // O may be rescaled only once PV_{t-1} has landed in it.  MMAs complete in
-        // issue order and S_{t-1} (already waited for) was issued after PV_{t-3},
-        // so on the barrier of PV_{t-1}'s parity at most PV_{t-1} is outstanding and
-        // this parity wait is unambiguous although iterations without a rescale
-        // skip it; S_t (waited for) also implies PV_{t-2} has landed.
+        // O_g may be rescaled only once the P V MMAs of iteration t-1 have landed.
+        // S_t (waited for) was issued after those of iteration t-2 had completed and
+        // iteration t+1's need P_{t+1}, so on the barrier of t-1's parity at most
+        // iteration t-1 is outstanding: the parity wait is unambiguous although
+        // iterations without a rescale skip it.
         const int u = t - 1;
         if (!__all_sync(0xffffffffu, wait_bar(&sh.o_done[u & 1], (u >> 1) & 1, sh, err))) { ok = false; break; }
         tc_fence_after();
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
-          tmem_ld32(tbase + lane_base + kColO + c0, o);
+          tmem_ld32(tbase + lane_base + o_col + c0, o);
           tmem_wait_ld();
 #pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * factor);
-          tmem_st32(tbase + lane_base + kColO + c0, o);
+          for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * factor);
+          tmem_st32(tbase + lane_base + o_col + c0, o);
         }
         tmem_wait_st();
       }
-      tc_fence_before();
-      mbar_arrive(&sh.p_full[sb]);
+      release_p(sb);
     }
-    // the last two PVs may both be outstanding: one wait on each parity's barrier
+    // the last two iterations' P V MMAs may both be outstanding: one wait on each
+    // parity's barrier
     if (ok && t > 0) ok = __all_sync(0xffffffffu, wait_bar(&sh.o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, sh, err));
     if (ok && t > 1) ok = __all_sync(0xffffffffu, wait_bar(&sh.o_done[(t - 2) & 1], ((t - 2) >> 1) & 1, sh, err));
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
-    const bool have_o = ok && t > 0;
+    // merge the groups' states: M = max(m_0, m_1), w_g = 2^(m_g - M); each group then
+    // writes half of the columns of  w_0 O_0 + w_1 O_1  and  l = w_0 l_0 + w_1 l_1
+    sh.xch[0][g][row] = m_run;
+    sh.xch[1][g][row] = l_run;
+    asm volatile("bar.sync 1, 256;" ::: "memory");
+    const float m_o = sh.xch[0][g ^ 1][row], l_o = sh.xch[1][g ^ 1][row];
+    const float m0 = g ? m_o : m_run, m1 = g ? m_run : m_o;
+    const float l0 = g ? l_o : l_run, l1 = g ? l_run : l_o;
+    const float M = fmaxf(m0, m1);
+    const float w0 = (m0 == -INFINITY) ? 0.f : ex2(m0 - M);
+    const float w1 = (m1 == -INFINITY) ? 0.f : ex2(m1 - M);
+    const float l_tot = w0 * l0 + w1 * l1;
+    // O_1 exists only if the item has at least two blocks
+    const bool have0 = ok && n_blk >= 1, have1 = ok && n_blk >= 2;
+    auto merged = [&](int c0, float (&v)[32]) {
+      uint32_t a[32], b[32];
+      if (have0) tmem_ld32(tbase + lane_base + kColO + c0, a);
+      if (have1) tmem_ld32(tbase + lane_base + kColO + D + c0, b);
+      if (have0 || have1) tmem_wait_ld();
+#pragma unroll
+      for (int e = 0; e < 32; ++e)
+        v[e] = (have0 ? w0 * __uint_as_float(a[e]) : 0.f) + (have1 ? w1 * __uint_as_float(b[e]) : 0.f);
+    };
+    const int cbeg = g * (D / 2), cend = cbeg + D / 2;
     if (kind >= 0) {
       // one half of a split key list: hand the unnormalised state to k_combine
       float* po = part.o + (static_cast<size_t>(slot) * kBM + row) * D;
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        if (have_o) {
-          tmem_ld32(tbase + lane_base + kColO + c0, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
+      for (int c0 = cbeg; c0 < cend; c0 += 32) {
+        float v[32];
+        merged(c0, v);
         float4* p4 = reinterpret_cast<float4*>(po + c0);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
-          p4[e] = make_float4(__uint_as_float(o[4 * e]), __uint_as_float(o[4 * e + 1]),
-                              __uint_as_float(o[4 * e + 2]), __uint_as_float(o[4 * e + 3]));
+        for (int e = 0; e < 8; ++e) p4[e] = make_float4(v[4 * e], v[4 * e + 1], v[4 * e + 2], v[4 * e + 3]);
       }
-      *reinterpret_cast<float2*>(part.ml + (static_cast<size_t>(slot) * kBM + row) * 2) =
-          make_float2(m_run, l_run);
+      if (g == 0)
+        *reinterpret_cast<float2*>(part.ml + (static_cast<size_t>(slot) * kBM + row) * 2) =
+            make_float2(M, l_tot);
     } else {
-      const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+      const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
       float sg = 0.f;
       size_t obase = 0;
       if (row_valid) {
-        const float g = gate[static_cast<size_t>(qrow) * H + h];
-        sg = 1.f / (1.f + expf(-g));
+        const float gt = gate[static_cast<size_t>(qrow) * H + h];
+        sg = 1.f / (1.f + expf(-gt));
         obase = static_cast<size_t>(qrow) * H * D + static_cast<size_t>(h) * D;
       }
 #pragma unroll
-      for (int c0 = 0; c0 < D; c0 += 32) {
-        uint32_t o[32];
-        if (have_o) {
-          tmem_ld32(tbase + lane_base + kColO + c0, o);
-          tmem_wait_ld();
-        } else {
-#pragma unroll
-          for (int e = 0; e < 32; ++e) o[e] = 0u;
-        }
-        if (!row_valid) continue;
+      for (int c0 = cbeg; c0 < cend; c0 += 32) {
         float v[32];
+        merged(c0, v);
+        if (!row_valid) continue;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(o[e]) * inv;
+        for (int e = 0; e < 32; ++e) v[e] *= inv;
         if (o_branch) {
           float4* ob = reinterpret_cast<float4*>(o_branch + obase + c0);
 #pragma unroll
@@ -482,12 +604,12 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 // covers 4 rows x 512 contiguous bytes), all its loads issued up front.
 template <int D>
 __global__ void __launch_bounds__(2 * D)
-k_combine(const int4* __restrict__ pairs, Partials part, int Nq, int H,
+k_combine(const int4* __restrict__ pairs, Partials part, int Nq, int H, int split_min,
           const float* __restrict__ gate, const float* __restrict__ lin_ws,
           __nv_bfloat16* __restrict__ out, float* __restrict__ o_branch) {
   constexpr int kSeg = D / 16;                 // 16-column segments per row
   const int4 pr = pairs[blockIdx.x];
-  if (pr.w < kSplitMin) return;                // written whole by the attention kernel
+  if (pr.w < split_min) return;                // written whole by the attention kernel
   const int row = blockIdx.y * 32 + threadIdx.x / kSeg;
   const int c0 = (threadIdx.x % kSeg) * 16;
   const int half = row >> 6;
@@ -620,7 +742,8 @@ k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W, int4* __restric
 constexpr int kLenBins = 1024;
 
 __global__ void __launch_bounds__(1024)
-k_make_items(const int4* __restrict__ pairs, int n_pairs, int shift, int4* __restrict__ items) {
+k_make_items(const int4* __restrict__ pairs, int n_pairs, int shift, int split_min,
+             int4* __restrict__ items) {
   __shared__ int hist[kLenBins];
   __shared__ int base[kLenBins];
   __shared__ int wsum[32];
@@ -629,7 +752,7 @@ k_make_items(const int4* __restrict__ pairs, int n_pairs, int shift, int4* __res
   auto bin_of = [&](int len) { return kLenBins - 1 - min(kLenBins - 1, len >> shift); };  // long first
   for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
     const int cnt = pairs[p].w;
-    if (cnt >= kSplitMin) {
+    if (cnt >= split_min) {
       atomicAdd(&hist[bin_of(cnt / 2)], 1);
       atomicAdd(&hist[bin_of(cnt - cnt / 2)], 1);
     } else {
@@ -655,7 +778,7 @@ k_make_items(const int4* __restrict__ pairs, int n_pairs, int shift, int4* __res
   __syncthreads();
   for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
     const int cnt = pairs[p].w;
-    if (cnt >= kSplitMin) {
+    if (cnt >= split_min) {
       const int hlf = cnt / 2;
       items[atomicAdd(&base[bin_of(hlf)], 1)] = make_int4(p, 0, 0, hlf);
       items[atomicAdd(&base[bin_of(cnt - hlf)], 1)] = make_int4(p, 1, hlf, cnt);
@@ -732,6 +855,20 @@ struct SparseLayout {
   int4* items;
   Partials part;
 };
+// Key lists are split in two (and merged by k_combine) only when the pairs fill
+// fewer than two waves of one CTA per SM: with more, the longest-first order
+// already balances the SMs and a split only adds partial-state traffic.
+int split_min_for(int n_pairs) {
+  static int n_sm = 0;
+  if (n_sm == 0) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n_sm < 1)
+      n_sm = 148;
+  }
+  return n_pairs >= 2 * n_sm ? INT_MAX : 8;
+}
+
 SparseLayout sparse_layout(void* scratch, int Nq, int H, int d, int B, int L) {
   SparseLayout s;
   s.n_qb = (Nq + B - 1) / B;
@@ -759,7 +896,7 @@ wa_status launch_attn_worklist(int Nq, int H, int d, int B, int L, const uint32_
   k_pair_heads<<<H, 256, 0, st>>>(blk_mask, s.n_qb, s.W, s.pairs);
   int shift = 0;
   while ((s.n_kb >> shift) >= kLenBins) ++shift;
-  k_make_items<<<1, 1024, 0, st>>>(s.pairs, s.n_pairs, shift, s.items);
+  k_make_items<<<1, 1024, 0, st>>>(s.pairs, s.n_pairs, shift, split_min_for(s.n_pairs), s.items);
   return check_launch("attention work list");
 }
 
@@ -775,15 +912,16 @@ wa_status launch_attn_sparse(const void* q, int Nq, int H, int d, RowSource rs, 
   if (e != WA_OK) return e;
   const int grid = 2 * s.n_pairs;
   float* lin_rw = const_cast<float*>(lin_ws);
+  const int split_min = split_min_for(s.n_pairs);
   if (d == 128) {
     launch_attn_kernel<128>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
                             s.part, gate, lin_rw, out, o_sp, err);
-    k_combine<128><<<dim3(s.n_pairs, kBM / 32), 2 * 128, 0, st>>>(s.pairs, s.part, Nq, H, gate, lin_ws,
+    k_combine<128><<<dim3(s.n_pairs, kBM / 32), 2 * 128, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate, lin_ws,
                                                                   static_cast<__nv_bfloat16*>(out), o_sp);
   } else {
     launch_attn_kernel<64>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
                            s.part, gate, lin_rw, out, o_sp, err);
-    k_combine<64><<<dim3(s.n_pairs, kBM / 32), 2 * 64, 0, st>>>(s.pairs, s.part, Nq, H, gate, lin_ws,
+    k_combine<64><<<dim3(s.n_pairs, kBM / 32), 2 * 64, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate, lin_ws,
                                                                 static_cast<__nv_bfloat16*>(out), o_sp);
   }
   return check_launch("sparse attention");
