@@ -26,8 +26,8 @@
  *  - `dtype` (WA_F32 or WA_BF16) applies to q, k/v, e_k/e_v, k_til/v_til and out.
  *    Scores, page/block means and every quantity that decides an index (page or
  *    block selection) are computed in float64; attention accumulates in float32.
- *  - Supported shapes: d in {64, 128}; B = 64; for WA_BF16 also r % 64 == 0 and
- *    r <= 256.  Others return WA_ERR_UNSUPPORTED.
+ *  - Supported shapes: d in {64, 128}; B = 64; for WA_BF16 also r in {128, 256}
+ *    (the projection's tensor-core tile height).  Others return WA_ERR_UNSUPPORTED.
  *  - Errors: every call validates its scalar arguments on the host and returns a
  *    wa_status; no C++ exception crosses the ABI.  `wa_last_error()` returns a
  *    message for the calling thread's last failure.  Index arguments that live in
