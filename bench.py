@@ -46,6 +46,8 @@ sys.path.insert(0, ROOT)
 import numpy as np  # noqa: E402
 import torch  # noqa: E402
 
+from linear_attention_paged_b200 import replicas  # noqa: E402
+
 METRIC = "HSA ms/chunk-layer & attention frames/s; % of BF16 tensor / HBM roofline"
 FRAMES_PER_CHUNK = 3
 CHUNK_LAYERS_PER_CHUNK = 30 * 4
@@ -184,7 +186,8 @@ def cores():
 
 
 def frames_per_s(ms_per_chunk_layer, n=1):
-    return n * FRAMES_PER_CHUNK / (CHUNK_LAYERS_PER_CHUNK * ms_per_chunk_layer / 1000.0)
+    """Whole-job frames/s of n replicas whose slowest takes ms_per_chunk_layer per step."""
+    return replicas.job_throughput(FRAMES_PER_CHUNK / CHUNK_LAYERS_PER_CHUNK, n, ms_per_chunk_layer / 1000.0)
 
 
 # ----------------------------------------------------------------------------- reference arm
@@ -237,14 +240,13 @@ def run_ours(args, rank, world, local_rank):
     from linear_attention_paged_b200 import build as wb
     if rank == 0:
         wb.build()
-    if world > 1:
-        torch.distributed.barrier()
+    replicas.barrier(world)
     from linear_attention_paged_b200 import wa, workloads as W
 
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     base = W.C1 if args.heads is None else W.C1.with_(name=f"c1_layer_bf16_h{args.heads}", H=args.heads)
-    cfg = base.with_(seed=base.seed + 1000 * rank)     # each rank: its own layer
+    cfg = base.with_(seed=replicas.rank_seed(base.seed, rank))   # each rank: its own layer
     inp = W.make_inputs(cfg, device="cuda", gen_device="cuda")
     tau = inp["tau"].cuda()
     stream = torch.cuda.current_stream()
@@ -275,8 +277,7 @@ def run_ours(args, rank, world, local_rank):
 
     clk = ClockSampler(local_rank)
     clk.start()
-    if world > 1:
-        torch.distributed.barrier()
+    replicas.barrier(world)
     torch.cuda.synchronize()
     t_start = torch.cuda.Event(enable_timing=True)
     t_end = torch.cuda.Event(enable_timing=True)
@@ -286,15 +287,11 @@ def run_ours(args, rank, world, local_rank):
         step()
     t_end.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    replicas.barrier(world)
     clocks = clk.stop()
     step.args.stage_events = None
     elapsed = t_start.elapsed_time(t_end)
-    el = torch.tensor([elapsed], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(el, op=torch.distributed.ReduceOp.MAX)
-    elapsed_max = float(el.item())
+    elapsed_max = replicas.max_over_ranks(elapsed, world, dev)
     ms_step = elapsed_max / args.steps
 
     stage_ms = {}
@@ -318,8 +315,7 @@ def run_ours(args, rank, world, local_rank):
         step()
         o_host.copy_(step.out, non_blocking=True)
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    replicas.barrier(world)
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
     e0.record(stream)
@@ -330,10 +326,7 @@ def run_ours(args, rank, world, local_rank):
         o_host.copy_(step.out, non_blocking=True)
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_el = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(e2e_el, op=torch.distributed.ReduceOp.MAX)
-    e2e_ms = float(e2e_el.item()) / max(e2e_steps, 1)
+    e2e_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev) / max(e2e_steps, 1)
     h2d = q_host.numel() * q_host.element_size() + g_host.numel() * g_host.element_size()
     d2h = o_host.numel() * o_host.element_size()
 
@@ -392,8 +385,7 @@ def run_c4(args, rank, world, local_rank):
     from linear_attention_paged_b200 import build as wb
     if rank == 0:
         wb.build()
-    if world > 1:
-        torch.distributed.barrier()
+    replicas.barrier(world)
     from linear_attention_paged_b200 import wa, workloads as W
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -402,7 +394,7 @@ def run_c4(args, rank, world, local_rank):
     base = W.C1.with_(name="c4_layer", n_chunks=2)
     layers = []
     for l in range(n_layers):
-        cfg = base.with_(seed=4000 + 1000 * rank + l)
+        cfg = base.with_(seed=replicas.rank_seed(4000 + l, rank))
         inp = W.make_inputs(cfg, device="cuda", gen_device="cuda")
         P_ = cfg.n_pool_pages
         hist = inp["chunk_pages"][0:1].contiguous()
@@ -448,8 +440,7 @@ def run_c4(args, rank, world, local_rank):
         raise RuntimeError(f"device error flags 0x{flags:x}")
     clk = ClockSampler(local_rank)
     clk.start()
-    if world > 1:
-        torch.distributed.barrier()
+    replicas.barrier(world)
     torch.cuda.synchronize()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
@@ -457,13 +448,9 @@ def run_c4(args, rank, world, local_rank):
     run(n_chunks, fill0)              # rewrites the pool tail from the same offset
     e1.record(stream)
     torch.cuda.synchronize()
-    if world > 1:
-        torch.distributed.barrier()
+    replicas.barrier(world)
     clocks = clk.stop()
-    el = torch.tensor([e0.elapsed_time(e1)], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(el, op=torch.distributed.ReduceOp.MAX)
-    total_ms = float(el.item())
+    total_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
     frames = world * FRAMES_PER_CHUNK * n_chunks
     if rank == 0:
         n_step_calls = n_chunks * n_steps * n_layers
@@ -507,23 +494,18 @@ def main():
     ap.add_argument("--layers", type=int, default=30, help="c4: layers")
     ap.add_argument("--chunks", type=int, default=20, help="c4: chunks")
     args = ap.parse_args()
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    rank, world, local_rank = replicas.env_ranks()
     if args.impl == "reference":
         return run_reference(args, rank, world)
     if world > 1:
-        import datetime
         torch.cuda.set_device(local_rank)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local_rank))
+        replicas.init(world, "nccl", 120.0, device=torch.device("cuda", local_rank))
     try:
         if args.config == "c4":
             return run_c4(args, rank, world, local_rank)
         return run_ours(args, rank, world, local_rank)
     finally:
-        if world > 1:
-            torch.distributed.destroy_process_group()
+        replicas.shutdown(world)
 
 
 if __name__ == "__main__":
