@@ -52,7 +52,10 @@ class HSAConfig:
     tau_const: Optional[float] = None
     n_chunks: int = 1        # chunks in the pool (C3: 15); each chunk has n_c pages
     prompt_dim: int = 0      # prompt embedding dimension (C3: 4096)
-    hot_beta_scale: float = 3.0   # C2: hot-block shift, in units of sigma_k*sqrt(d)
+    # C2: hot-block shift, in units of sigma_k*sqrt(d).  3 ("+3 sigma") left every
+    # head's kept fraction between 36 % and 97 %; 7 spreads the per-head means from
+    # 0.8 % to 90 %, the intended 1 % -> 100 % range.
+    hot_beta_scale: float = 7.0
 
     @property
     def L(self) -> int:
