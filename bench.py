@@ -49,6 +49,9 @@ import torch  # noqa: E402
 from linear_attention_paged_b200 import replicas  # noqa: E402
 
 METRIC = "HSA ms/chunk-layer & attention frames/s; % of BF16 tensor / HBM roofline"
+# DRAM bytes per launch of the sparse-branch attention kernel per head, from one ncu
+# capture of the 6-head C1 launch (360.1 MB / 6); set to None when the kernel changes
+ATTN_DRAM_BYTES_PER_HEAD = 360.1e6 / 6
 FRAMES_PER_CHUNK = 3
 CHUNK_LAYERS_PER_CHUNK = 30 * 4
 # stage -> (start event, end event) of the events wa_hsa_step records; the
@@ -349,7 +352,11 @@ def run_ours(args, rank, world, local_rank):
                              "larger than the 126 MB L2",
                        "parallelism": f"replicas x{world} (one layer per rank, no collective)"},
             "roofline": {"bound": "tensor", "achieved": achieved_t, "peak": peak_t, "unit": "TFLOP/s",
-                         "frac": achieved_t / peak_t, "traffic": None,
+                         "frac": achieved_t / peak_t,
+                         "traffic": ATTN_DRAM_BYTES_PER_HEAD * cfg.H,
+                         "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the "
+                                           "6-head launch (profiles/k_umma_attention_sparse_h6.md), "
+                                           "scaled by heads",
                          "kernel": "k_umma_attention (sparse branch + gate)",
                          "flops_per_launch": flops, "kept_fraction": kept_frac,
                          "peak_source": f"bf16_tflops_sustained, of {peak_src}",
