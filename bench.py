@@ -353,7 +353,8 @@ def run_ours(args, rank, world, local_rank):
                        "parallelism": f"replicas x{world} (one layer per rank, no collective)"},
             "roofline": {"bound": "tensor", "achieved": achieved_t, "peak": peak_t, "unit": "TFLOP/s",
                          "frac": achieved_t / peak_t,
-                         "traffic": ATTN_DRAM_BYTES_PER_HEAD * cfg.H,
+                         "traffic": (ATTN_DRAM_BYTES_PER_HEAD * cfg.H
+                                     if ATTN_DRAM_BYTES_PER_HEAD is not None else None),
                          "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the "
                                            "6-head launch (profiles/k_umma_attention_sparse_h6.md), "
                                            "scaled by heads",
