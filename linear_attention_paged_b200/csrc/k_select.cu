@@ -263,18 +263,22 @@ k_block_scores(const double* __restrict__ qmean, KeyMeans km, int n_qb, int n_kb
   double* kc = sm_scores + 32 * d;           // [32][d+1]
   const int j0 = blockIdx.x * 32, i0 = blockIdx.y * 32, h = blockIdx.z;
   const int cols = H * d;
-  for (int e = threadIdx.x; e < 32 * d; e += blockDim.x) {
-    const int rr = e / d, c = e - rr * d;
+  // a warp per row: the row's source (through the page position when the key means
+  // come from the candidate pass) is resolved once, the d values load coalesced
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int rr = warp; rr < 32; rr += blockDim.x >> 5) {
     const int j = j0 + rr, i = i0 + rr;
-    double v = 0.0;
+    const double* ksrc = nullptr;
     if (j < n_kb) {
       size_t row = j;
       if (km.page_pos) row = static_cast<size_t>(km.page_pos[j / km.nbp]) * km.nbp + j % km.nbp;
-      v = km.data[row * cols + h * d + c];
-      if (km.is_sum) v /= static_cast<double>(min(km.L, (j + 1) * B) - j * B);
+      ksrc = km.data + row * cols + h * d;
     }
-    kc[rr * (d + 1) + c] = v;
-    qs[e] = i < n_qb ? qmean[static_cast<size_t>(i) * cols + h * d + c] : 0.0;
+    const double* qsrc = i < n_qb ? qmean + static_cast<size_t>(i) * cols + h * d : nullptr;
+    for (int c = lane; c < d; c += 32) {
+      kc[rr * (d + 1) + c] = ksrc ? ksrc[c] : 0.0;
+      qs[rr * d + c] = qsrc ? qsrc[c] : 0.0;
+    }
   }
   __syncthreads();
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
@@ -288,15 +292,20 @@ k_block_scores(const double* __restrict__ qmean, KeyMeans km, int n_qb, int n_kb
     const double x0 = q0[c], x1 = q1[c], y0 = k0[c], y1 = k1[c];
     a00 += x0 * y0; a01 += x0 * y1; a10 += x1 * y0; a11 += x1 * y1;
   }
+  // key block sums become means here: q . (sum / n) / sqrt(d) = (q . sum) / (n sqrt(d))
   const double sqrt_d = sqrt(static_cast<double>(d));
   const double acc[2][2] = {{a00, a01}, {a10, a11}};
 #pragma unroll
-  for (int u = 0; u < 2; ++u)
+  for (int v = 0; v < 2; ++v) {
+    const int j = j0 + tx + 16 * v;
+    if (j >= n_kb) continue;
+    const double den = km.is_sum ? static_cast<double>(min(km.L, (j + 1) * B) - j * B) * sqrt_d : sqrt_d;
 #pragma unroll
-    for (int v = 0; v < 2; ++v) {
-      const int i = i0 + ty + 16 * u, j = j0 + tx + 16 * v;
-      if (i < n_qb && j < n_kb) scores[(static_cast<size_t>(h) * n_qb + i) * n_kb + j] = acc[u][v] / sqrt_d;
+    for (int u = 0; u < 2; ++u) {
+      const int i = i0 + ty + 16 * u;
+      if (i < n_qb) scores[(static_cast<size_t>(h) * n_qb + i) * n_kb + j] = acc[u][v] / den;
     }
+  }
 }
 
 // ------------------------------------------------------------------ S3 choice

@@ -34,8 +34,7 @@
 //           0-63 / 64-127), one thread per TMEM lane (query row), each with its own
 //           running max, sum and O accumulator, merged in the epilogue.  P goes
 //           back into the S buffer as bf16; O is rescaled in TMEM only when the
-//           running max grows by more than 2^8; a quarter of the exponentials run
-//           on the FMA pipe (exp2_poly) to unload the MUFU unit.
+//           running max grows by more than 2^8.
 // Every wait is bounded in time.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -124,31 +123,9 @@ __device__ __forceinline__ float ex2(float x) {
   return y;
 }
 
-// 2^y for a pair on the FMA pipe, to take part of the exponentials off the MUFU
-// unit (16 results per clock per SM, the softmax's narrowest pipe): y = j + f with
-// j = round(y) (adding 1.5 * 2^23 leaves j in the low mantissa bits) and f in
-// [-1/2, 1/2]; 2^f is a degree-3 polynomial fitted for minimum relative error
-// (7.5e-5, far below bf16's 2^-9 for P), and 2^j is added into the exponent field.
-// y is clamped at -125 so the exponent never underflows; inputs are finite.
-__device__ __forceinline__ float2 exp2_poly(float2 y) {
-  y.x = fmaxf(y.x, -125.f);
-  y.y = fmaxf(y.y, -125.f);
-  const float2 shifter = make_float2(12582912.f, 12582912.f);
-  const float2 t = __fadd2_rn(y, shifter);
-  const float2 jf = __fadd2_rn(t, make_float2(-12582912.f, -12582912.f));
-  const float2 f = __ffma2_rn(jf, make_float2(-1.f, -1.f), y);
-  float2 q = __ffma2_rn(make_float2(0.05517222f, 0.05517222f), f, make_float2(0.24261115f, 0.24261115f));
-  q = __ffma2_rn(q, f, make_float2(0.69326085f, 0.69326085f));
-  q = __ffma2_rn(q, f, make_float2(0.99992806f, 0.99992806f));
-  return make_float2(__int_as_float(__float_as_int(q.x) + (__float_as_int(t.x) << 23)),
-                     __int_as_float(__float_as_int(q.y) + (__float_as_int(t.y) << 23)));
-}
-
 // One softmax pass over a 64-column half row held in r: p = 2^(s * scale_log2 - m)
 // packed to bf16 pairs in pk, the sum of p in lsum and (kMax) the raw row maximum.
-// kPoly routes one pair in four through exp2_poly (full blocks only: masked
-// columns hold -inf).
-template <bool kMax, bool kPoly>
+template <bool kMax>
 __device__ __forceinline__ void softmax_pass(const uint32_t (&r)[64], float2 sc2, float2 nm2,
                                              uint32_t (&pk)[32], float& lsum, float& mraw) {
   float2 acc2[4];
@@ -162,7 +139,7 @@ __device__ __forceinline__ void softmax_pass(const uint32_t (&r)[64], float2 sc2
     const float2 x = make_float2(__uint_as_float(r[2 * e]), __uint_as_float(r[2 * e + 1]));
     if (kMax) mx8[e & 7] = max3f(mx8[e & 7], x.x, x.y);
     const float2 y = __ffma2_rn(x, sc2, nm2);
-    const float2 pp = (kPoly && (e & 3) == 3) ? exp2_poly(y) : make_float2(ex2(y.x), ex2(y.y));
+    const float2 pp = make_float2(ex2(y.x), ex2(y.y));
     acc2[e & 3] = __fadd2_rn(acc2[e & 3], pp);
     pk[e] = pack_bf16x2(pp.x, pp.y);
   }
@@ -467,8 +444,7 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       uint32_t pk[32];
       float lsum, mraw;
       float2 nm2 = make_float2(-m_run, -m_run);
-      if (ragged) softmax_pass<true, false>(r, sc2, nm2, pk, lsum, mraw);
-      else softmax_pass<true, true>(r, sc2, nm2, pk, lsum, mraw);
+      softmax_pass<true>(r, sc2, nm2, pk, lsum, mraw);
       const float mx = mraw * scale_log2;
       float factor = 1.f;
       const bool resc = mx > m_run + 8.f;
@@ -476,7 +452,7 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         factor = ex2(m_run - mx);
         m_run = mx;
         nm2 = make_float2(-m_run, -m_run);
-        softmax_pass<false, false>(r, sc2, nm2, pk, lsum, mraw);
+        softmax_pass<false>(r, sc2, nm2, pk, lsum, mraw);
       }
       l_run = l_run * factor + lsum;
       tmem_st32(s_addr, pk);
@@ -660,7 +636,9 @@ k_combine(const int4* __restrict__ pairs, Partials part, int Nq, int H, int spli
 constexpr int kMaxPairTable = 128;
 constexpr int kMaxPairMaskWords = 3072;   // staged masks of one head (n_qb * W words)
 
-__global__ void __launch_bounds__(256)
+constexpr int kPairThreads = 1024;
+
+__global__ void __launch_bounds__(kPairThreads)
 k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W, int4* __restrict__ pairs) {
   __shared__ uint16_t dist[kMaxPairTable * kMaxPairTable];
   __shared__ uint32_t ms[kMaxPairMaskWords];
@@ -668,6 +646,7 @@ k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W, int4* __restric
   __shared__ int nn[kMaxPairTable];
   __shared__ int progress;
   const int h = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, n_warps = blockDim.x >> 5;
   const int n_pairs = (n_qb + 1) / 2;
   const uint32_t* mh = mask + static_cast<size_t>(h) * n_qb * W;
   const bool staged = n_qb * W <= kMaxPairMaskWords;
@@ -687,25 +666,35 @@ k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W, int4* __restric
     }
     return;
   }
-  for (int e = threadIdx.x; e < n_qb * n_qb; e += blockDim.x) {
-    const int a = e / n_qb, b = e - a * n_qb;
+  // symmetric-difference distances, each unordered pair once
+  const int n_tri = n_qb * (n_qb - 1) / 2;
+  for (int e = threadIdx.x; e < n_tri; e += blockDim.x) {
+    // e -> (a, b), a < b, row-major over the strict upper triangle
+    int a = static_cast<int>((2 * n_qb - 1 - sqrtf(static_cast<float>((2 * n_qb - 1) * (2 * n_qb - 1) - 8 * e))) * 0.5f);
+    if (a < 0) a = 0;
+    while (a > 0 && a * (2 * n_qb - a - 1) / 2 > e) --a;
+    while ((a + 1) * (2 * n_qb - a - 2) / 2 <= e) ++a;
+    const int b = e - a * (2 * n_qb - a - 1) / 2 + a + 1;
     int c = 0;
-    if (a != b)
-      for (int w = 0; w < W; ++w) c += __popc(m[a * W + w] ^ m[b * W + w]);
-    dist[e] = static_cast<uint16_t>(min(c, 65535));
+    for (int w = 0; w < W; ++w) c += __popc(m[a * W + w] ^ m[b * W + w]);
+    const uint16_t dv = static_cast<uint16_t>(min(c, 65535));
+    dist[a * n_qb + b] = dv;
+    dist[b * n_qb + a] = dv;
   }
   for (int a = threadIdx.x; a < n_qb; a += blockDim.x) partner[a] = -2;   // -2: unpaired
   __syncthreads();
+  // rounds of mutual nearest neighbours among the unpaired blocks; a warp finds the
+  // nearest of one block (ties: the lower index)
   for (int round = 0; round < n_qb; ++round) {
-    for (int a = threadIdx.x; a < n_qb; a += blockDim.x) {
-      int best = INT_MAX, bi = -1;
+    for (int a = warp; a < n_qb; a += n_warps) {
+      unsigned long long best = ~0ull;            // (distance << 32) | index
       if (partner[a] == -2)
-        for (int b = 0; b < n_qb; ++b) {
-          if (b == a || partner[b] != -2) continue;
-          const int dv = dist[a * n_qb + b];
-          if (dv < best) { best = dv; bi = b; }   // increasing b: ties keep the lower index
-        }
-      nn[a] = bi;
+        for (int b = lane; b < n_qb; b += 32)
+          if (b != a && partner[b] == -2)
+            best = min(best, (static_cast<unsigned long long>(dist[a * n_qb + b]) << 32) | b);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
+      if (lane == 0) nn[a] = best == ~0ull ? -1 : static_cast<int>(best & 0xffffffffu);
     }
     if (threadIdx.x == 0) progress = 0;
     __syncthreads();
@@ -893,7 +882,7 @@ wa_status launch_attn_worklist(int Nq, int H, int d, int B, int L, const uint32_
   if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
   SparseLayout s = sparse_layout(scratch, Nq, H, d, B, L);
   if (s.W > kMaxW) return set_error(WA_ERR_UNSUPPORTED, "too many key blocks (max %d)", kMaxW * 32);
-  k_pair_heads<<<H, 256, 0, st>>>(blk_mask, s.n_qb, s.W, s.pairs);
+  k_pair_heads<<<H, kPairThreads, 0, st>>>(blk_mask, s.n_qb, s.W, s.pairs);
   int shift = 0;
   while ((s.n_kb >> shift) >= kLenBins) ++shift;
   k_make_items<<<1, 1024, 0, st>>>(s.pairs, s.n_pairs, shift, split_min_for(s.n_pairs), s.items);
