@@ -21,6 +21,8 @@ Each function follows one step of the method as the WorldAttention pages state i
      linear_attention      K~ = E_K^T K, V~ = E_V^T V (Linformer projection)
   S5 sparse_attention   -- §3.3 "Sparse branch"; Appendix A.1.3 block-sparse attention
   S6 gate_fuse          -- §3.3 "Gated fusion of two branches" (sigmoid gate)
+     gate_fuse2            the same section's two-gate form O_lin (.) G_lin + O_sp (.) G_sp
+                           with G = sigmoid of a logit per (token, head)
 
 Readings where the pages are silent (each one is listed in the design notes):
   * Q-bar in the page score is per head; the per-head scores are averaged over heads,
@@ -274,6 +276,12 @@ def gate_fuse(o_sp, o_lin, g) -> np.ndarray:
     return G * f64(o_sp) + (1.0 - G) * f64(o_lin)
 
 
+def gate_fuse2(o_sp, o_lin, g_sp, g_lin) -> np.ndarray:
+    """O = sigmoid(g_sp) * O_sp + sigmoid(g_lin) * O_lin: one sigmoid gate per branch,
+    each per (token, head) (the two-gate form of the gated fusion)."""
+    return sigmoid(f64(g_sp))[..., None] * f64(o_sp) + sigmoid(f64(g_lin))[..., None] * f64(o_lin)
+
+
 # ----------------------------------------------------------------------------- step
 def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tuple]] = None) -> dict:
     """The whole decode step S0..S6 on one input dict (see the workload module).
@@ -305,11 +313,12 @@ def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tupl
     Q = f64(inp["q"])
     Nq, H, d = Q.shape
     g = f64(inp["gate"])
+    g_lin = f64(inp["gate_lin"]) if inp.get("gate_lin") is not None else None
     if rows_of_blocks is None:
         o_sp = sparse_attention(Q, k_act, v_act, kept, B)
         o_lin = linear_attention(Q, kt, vt)
         res["o_sp"], res["o_lin"] = o_sp, o_lin
-        res["o"] = gate_fuse(o_sp, o_lin, g)
+        res["o"] = gate_fuse(o_sp, o_lin, g) if g_lin is None else gate_fuse2(o_sp, o_lin, g, g_lin)
     else:
         outs = {}
         for (h, i) in rows_of_blocks:
@@ -317,6 +326,7 @@ def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tupl
             osp = sparse_attention_block(Q, k_act, v_act, h, i, kept[h][i], B)
             olin = linear_attention(Q[r0:r1, h:h + 1, :], kt[:, h:h + 1, :], vt[:, h:h + 1, :])[:, 0, :]
             G = sigmoid(g[r0:r1, h])[:, None]
-            outs[(h, i)] = dict(o_sp=osp, o_lin=olin, o=G * osp + (1.0 - G) * olin)
+            Gl = (1.0 - G) if g_lin is None else sigmoid(g_lin[r0:r1, h])[:, None]
+            outs[(h, i)] = dict(o_sp=osp, o_lin=olin, o=G * osp + Gl * olin)
         res["blocks"] = outs
     return res

@@ -299,6 +299,43 @@ def test_gate_limits():
     np.testing.assert_allclose(O.sigmoid(g) + O.sigmoid(-g), 1.0, rtol=1e-15)
 
 
+def test_two_gate_fusion_pins():
+    """Two sigmoid gates, one per branch: limits per gate, the zero point, the one-gate
+    form as the special case g_lin = -g_sp, and per-(token, head) independence."""
+    r = rng(16)
+    a = r.normal(size=(4, 2, 3)); b = r.normal(size=(4, 2, 3))
+    big = np.full((4, 2), 60.0)
+    np.testing.assert_allclose(O.gate_fuse2(a, b, big, -big), a, atol=1e-20)
+    np.testing.assert_allclose(O.gate_fuse2(a, b, -big, big), b, atol=1e-20)
+    np.testing.assert_allclose(O.gate_fuse2(a, b, big, big), a + b, rtol=1e-15)
+    np.testing.assert_allclose(O.gate_fuse2(a, b, -big, -big), 0.0, atol=1e-20)
+    np.testing.assert_allclose(O.gate_fuse2(a, b, np.zeros((4, 2)), np.zeros((4, 2))), 0.5 * (a + b),
+                               rtol=1e-15)
+    g = r.normal(size=(4, 2))
+    np.testing.assert_allclose(O.gate_fuse2(a, b, g, -g), O.gate_fuse(a, b, g), rtol=1e-14)
+    # changing one (token, head) gate changes only that (token, head) row
+    g2 = r.normal(size=(4, 2)); gl = r.normal(size=(4, 2))
+    base = O.gate_fuse2(a, b, g2, gl)
+    gl_mod = gl.copy(); gl_mod[1, 0] += 1.0
+    mod = O.gate_fuse2(a, b, g2, gl_mod)
+    changed = np.any(mod != base, axis=2)
+    assert changed[1, 0] and changed.sum() == 1
+
+
+def test_step_two_gates_matches_recombined_branches():
+    cfg = W.C0.with_(T_p=64, Nq=72)
+    inp = W.make_inputs(cfg)
+    inp["gate_lin"] = torch.from_numpy(rng(17).normal(size=(cfg.Nq, cfg.H))).float()
+    res = O.hsa_step(inp, cfg.B, cfg.K_p)
+    expect = O.gate_fuse2(res["o_sp"], res["o_lin"], inp["gate"].double().numpy(),
+                          inp["gate_lin"].double().numpy())
+    np.testing.assert_array_equal(res["o"], expect)
+    inp_one = dict(inp); inp_one["gate_lin"] = -inp["gate"]
+    res_one = O.hsa_step(inp_one, cfg.B, cfg.K_p)
+    np.testing.assert_allclose(res_one["o"], O.gate_fuse(res["o_sp"], res["o_lin"], inp["gate"]),
+                               rtol=1e-13, atol=1e-15)
+
+
 # ----------------------------------------------------------------------------- step
 def test_step_composes_pinned_parts_on_tiny_workload():
     cfg = W.C0.with_(T_p=64, Nq=72)
