@@ -40,6 +40,13 @@
 #include <stddef.h>
 #include <stdint.h>
 
+/* Symbols of the C ABI; libwa is built with hidden visibility for everything else. */
+#if defined(__GNUC__)
+#define WA_API __attribute__((visibility("default")))
+#else
+#define WA_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -61,15 +68,15 @@ typedef enum wa_dtype { WA_F32 = 0, WA_BF16 = 1 } wa_dtype;
 #define WA_DEVERR_TIMEOUT   0x4u  /* a bounded wait inside a kernel gave up         */
 
 /* Message describing the calling thread's most recent failure ("" if none). */
-const char* wa_last_error(void);
+WA_API const char* wa_last_error(void);
 
 /* Library version string. */
-const char* wa_version(void);
+WA_API const char* wa_version(void);
 
 /* Synchronise `stream`, read and clear the current device's error word.
  * *flags (may be NULL) receives the WA_DEVERR_* bits.  Returns WA_ERR_DEVICE when
  * any bit was set, WA_OK otherwise. */
-wa_status wa_device_error(void* stream, uint32_t* flags);
+WA_API wa_status wa_device_error(void* stream, uint32_t* flags);
 
 /* ---------------------------------------------------------------------------
  * S0 -- prompt-level retrieval (WorldAttention §3.2, "Stage 1: prompt-level
@@ -80,7 +87,7 @@ wa_status wa_device_error(void* stream, uint32_t* flags);
  *   chunk_out[1] int32          the chosen chunk; -1 and WA_DEVERR_ZERO_NORM when a
  *                               norm is zero
  * Computed in float64.  INVALID_ARG: NULL pointer, n_chunks < 1, D < 1. */
-wa_status wa_prompt_select(const float* e_cur, const float* e_chunks, int n_chunks, int D,
+WA_API wa_status wa_prompt_select(const float* e_cur, const float* e_chunks, int n_chunks, int D,
                            int32_t* chunk_out, void* stream);
 
 /* ---------------------------------------------------------------------------
@@ -100,8 +107,8 @@ wa_status wa_prompt_select(const float* e_cur, const float* e_chunks, int n_chun
  *                                        T_p % B == 0
  * One HBM pass over q and the candidate pages.  INVALID_ARG: K_p > n_c, sizes < 1,
  * NULL required pointer.  A candidate id outside the pool sets WA_DEVERR_PAGE_ID. */
-size_t wa_page_score_workspace_size(int Nq, int H, int d, int n_c, int T_p, int B);
-wa_status wa_page_score(const void* q, int Nq, int H, int d,
+WA_API size_t wa_page_score_workspace_size(int Nq, int H, int d, int n_c, int T_p, int B);
+WA_API wa_status wa_page_score(const void* q, int Nq, int H, int d,
                         const void* k_pool, int n_pool_pages, int T_p,
                         const int32_t* cand_pages, int n_c, int K_p, int B, wa_dtype dtype,
                         double* alpha, int32_t* sel, double* k_blockmean,
@@ -113,7 +120,7 @@ wa_status wa_page_score(const void* q, int Nq, int H, int d,
  * V_active): k_act[s*T_p + t] = k_pool[sel[s]][t], likewise for V.  A bit-exact
  * copy.  A page id outside the pool sets WA_DEVERR_PAGE_ID and that page is
  * skipped. */
-wa_status wa_gather_pages(const void* k_pool, const void* v_pool, int n_pool_pages, int T_p,
+WA_API wa_status wa_gather_pages(const void* k_pool, const void* v_pool, int n_pool_pages, int T_p,
                           int H, int d, const int32_t* sel, int K_p, wa_dtype dtype,
                           void* k_act, void* v_act, void* stream);
 
@@ -133,10 +140,10 @@ wa_status wa_gather_pages(const void* k_pool, const void* v_pool, int n_pool_pag
  *   (a chunk may span page boundaries); when page_index is non-NULL, also refresh
  *   the index entries of every block the write touches (a block's entry is exact
  *   once all its rows are written).  INVALID_ARG: rows outside the pool. */
-wa_status wa_pool_index(const void* k_pool, int n_pool_pages, int T_p, int H, int d, int B,
+WA_API wa_status wa_pool_index(const void* k_pool, int n_pool_pages, int T_p, int H, int d, int B,
                         wa_dtype dtype, const int32_t* pages, int n_pages, double* page_index,
                         void* stream);
-wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, int H, int d,
+WA_API wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, int H, int d,
                          wa_dtype dtype, const void* k_new, const void* v_new, int n_tokens,
                          long long token_offset, double* page_index, int B, void* stream);
 
@@ -157,8 +164,8 @@ wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, 
  *   blk_cnt     [H][n_qb] int32 (out, nullable)       number of kept blocks
  *   blk_mask    [H][n_qb][W] uint32 (out, nullable)   bit j of word j/32 = kept
  * INVALID_ARG: both or neither key sources, NULL q/tau, n_kb > 8192. */
-size_t wa_block_select_workspace_size(int Nq, int H, int d, int L, int B);
-wa_status wa_block_select(const void* q, int Nq, int H, int d,
+WA_API size_t wa_block_select_workspace_size(int Nq, int H, int d, int L, int B);
+WA_API wa_status wa_block_select(const void* q, int Nq, int H, int d,
                           const void* k_act, const double* k_blockmean, int L, int B,
                           wa_dtype dtype, const float* tau,
                           int32_t* blk_idx, int32_t* blk_cnt, uint32_t* blk_mask,
@@ -171,8 +178,8 @@ wa_status wa_block_select(const void* q, int Nq, int H, int d,
  * E is shared by all heads.  Accumulates in float32 (bf16 inputs on tcgen05
  * tensor cores with split-L and an ordered reduction); the result is rounded to
  * dtype. */
-size_t wa_linear_project_workspace_size(int L, int H, int d, int r, wa_dtype dtype);
-wa_status wa_linear_project(const void* k_act, const void* v_act, const void* e_k,
+WA_API size_t wa_linear_project_workspace_size(int L, int H, int d, int r, wa_dtype dtype);
+WA_API wa_status wa_linear_project(const void* k_act, const void* v_act, const void* e_k,
                             const void* e_v, int L, int H, int d, int r, wa_dtype dtype,
                             void* k_til, void* v_til, void* ws, size_t ws_bytes,
                             void* stream);
@@ -202,7 +209,7 @@ wa_status wa_linear_project(const void* k_act, const void* v_act, const void* e_
  *     32 MiB) are rejected with WA_ERR_UNSUPPORTED and a message; larger problems use
  *     fewer splits of L, down to one.
  *   - dtype must be WA_BF16, d in {64, 128}, r in {128, 256}, H*d % 64 == 0. */
-wa_status wa_linear_project_noalloc(const void* k_act, const void* v_act, const void* e_k,
+WA_API wa_status wa_linear_project_noalloc(const void* k_act, const void* v_act, const void* e_k,
                                     const void* e_v, int L, int H, int d, int r, wa_dtype dtype,
                                     void* k_til, void* v_til, void* stream);
 
@@ -222,14 +229,31 @@ wa_status wa_linear_project_noalloc(const void* k_act, const void* v_act, const 
  *                                  the gate, for identity checks
  * A (head, query block) whose mask is empty gets O_sp = 0.  Masked key rows of a
  * ragged last block never enter a softmax. */
-size_t wa_hsa_attention_workspace_size(int Nq, int H, int d, int L, int B, int r, wa_dtype dtype);
-wa_status wa_hsa_attention(const void* q, int Nq, int H, int d,
+WA_API size_t wa_hsa_attention_workspace_size(int Nq, int H, int d, int L, int B, int r, wa_dtype dtype);
+WA_API wa_status wa_hsa_attention(const void* q, int Nq, int H, int d,
                            const void* k_act, const void* v_act, int L, int B,
                            const uint32_t* blk_mask,
                            const void* k_til, const void* v_til, int r,
                            const float* gate, wa_dtype dtype,
                            void* out, float* o_sp, float* o_lin,
                            void* ws, size_t ws_bytes, void* stream);
+
+/* The same with two independent gates, one per branch (WorldAttention §3.3, "Gated
+ * fusion of two branches": sigmoid gates modulate both branches per token and head;
+ * the section's formula O_lin ⊙ G_lin + O_sp ⊙ G_sp with G = sigmoid of the gate
+ * logits):
+ *   out[n][h] = sigmoid(gate_sp[n][h]) * O_sp[n][h] + sigmoid(gate_lin[n][h]) * O_lin[n][h]
+ *   gate_sp, gate_lin [Nq][H] float32 (gate_lin must not be NULL); the logits are
+ * inputs (the projection G = XW that makes them belongs to the model).  With
+ * gate_lin = -gate_sp this is wa_hsa_attention.  Same workspace, errors and
+ * layouts as wa_hsa_attention. */
+WA_API wa_status wa_hsa_attention_gated2(const void* q, int Nq, int H, int d,
+                                  const void* k_act, const void* v_act, int L, int B,
+                                  const uint32_t* blk_mask,
+                                  const void* k_til, const void* v_til, int r,
+                                  const float* gate_sp, const float* gate_lin, wa_dtype dtype,
+                                  void* out, float* o_sp, float* o_lin,
+                                  void* ws, size_t ws_bytes, void* stream);
 
 /* ---------------------------------------------------------------------------
  * The whole decode step (WorldAttention §3.2 + §3.3; summary steps 2-6):
@@ -276,6 +300,10 @@ typedef struct wa_step_args {
      block sums kept current by the caller; with it S1 and S3 read the index instead
      of re-reducing the candidate pages (needs fused_gather and T_p % B == 0) */
   const double* page_index;
+  /* optional second gate, [Nq][H] float32: with it the step fuses the branches as
+     sigmoid(gate) * O_sp + sigmoid(gate_lin) * O_lin (see wa_hsa_attention_gated2);
+     NULL keeps sigmoid(gate) * O_sp + (1 - sigmoid(gate)) * O_lin */
+  const float* gate_lin;
 } wa_step_args;
 
 /* Stage boundaries recorded into wa_step_args.stage_events:
@@ -286,8 +314,8 @@ typedef struct wa_step_args {
  * joins before event 6, so events 4 and 5 are recorded on that stream. */
 #define WA_STEP_EVENTS 8
 
-size_t wa_hsa_step_workspace_size(const wa_step_args* a);
-wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* stream);
+WA_API size_t wa_hsa_step_workspace_size(const wa_step_args* a);
+WA_API wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */

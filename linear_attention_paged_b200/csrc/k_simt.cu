@@ -47,8 +47,8 @@ template <int D>
 __global__ void __launch_bounds__(128)
 k_simt_attention(int mode, const float* __restrict__ q, int Nq, int H, RowSource rs, int B,
                  const uint32_t* __restrict__ mask, int W, const float* __restrict__ gate,
-                 float* __restrict__ lin_ws, float* __restrict__ out, float* __restrict__ o_branch,
-                 uint32_t* err) {
+                 float lin_sign, float* __restrict__ lin_ws, float* __restrict__ out,
+                 float* __restrict__ o_branch, uint32_t* err) {
   extern __shared__ float sm[];
   float* Ks = sm;                 // [kTile][D]
   float* Vs = sm + kTile * D;     // [kTile][D]
@@ -119,14 +119,16 @@ k_simt_attention(int mode, const float* __restrict__ q, int Nq, int H, RowSource
   if (bad && threadIdx.x == 0) atomicOr(err, WA_DEVERR_PAGE_ID);
   if (!valid) return;
   const float inv = l > 0.f ? 1.0f / l : 0.f;
+  // mode 1: sigmoid(g); mode 0: the linear branch's weight sigmoid(lin_sign * x), with
+  // x = g, lin_sign = -1 (1 - sigmoid(g)) or x = g_lin, lin_sign = +1 (two gates)
   const float g = gate[static_cast<size_t>(row) * H + h];
-  const float sg = 1.0f / (1.0f + expf(-g));
+  const float sg = 1.0f / (1.0f + expf(mode == 0 ? -lin_sign * g : -g));
   const size_t o = static_cast<size_t>(row) * cols + h * D;
 #pragma unroll
   for (int c = 0; c < D; ++c) {
     const float v = acc[c] * inv;
     if (o_branch) o_branch[o + c] = v;
-    if (mode == 0) lin_ws[o + c] = (1.0f - sg) * v;
+    if (mode == 0) lin_ws[o + c] = sg * v;
     else out[o + c] = sg * v + lin_ws[o + c];
   }
 }
@@ -148,20 +150,22 @@ wa_status launch_simt_project(const float* x, const int32_t* page_ids, int page_
 
 wa_status launch_simt_attention(int mode, const float* q, int Nq, int H, int d, RowSource rs,
                                 int B, const uint32_t* blk_mask, int W, const float* gate,
-                                float* lin_ws, float* out, float* o_branch, uint32_t* err,
-                                cudaStream_t st) {
+                                const float* gate_lin, float* lin_ws, float* out, float* o_branch,
+                                uint32_t* err, cudaStream_t st) {
+  const float* gx = (mode == 0 && gate_lin) ? gate_lin : gate;
+  const float lin_sign = gate_lin ? 1.f : -1.f;
   const int n_qb = (Nq + B - 1) / B;
   dim3 grid(n_qb, H);
   const size_t smem = 2 * static_cast<size_t>(kTile) * d * sizeof(float);
   if (B > 128) return set_error(WA_ERR_UNSUPPORTED, "fp32 attention needs B <= 128");
   if (d == 64) {
     cudaFuncSetAttribute(k_simt_attention<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_simt_attention<64><<<grid, 128, smem, st>>>(mode, q, Nq, H, rs, B, blk_mask, W, gate, lin_ws,
-                                                  out, o_branch, err);
+    k_simt_attention<64><<<grid, 128, smem, st>>>(mode, q, Nq, H, rs, B, blk_mask, W, gx, lin_sign,
+                                                  lin_ws, out, o_branch, err);
   } else if (d == 128) {
     cudaFuncSetAttribute(k_simt_attention<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    k_simt_attention<128><<<grid, 128, smem, st>>>(mode, q, Nq, H, rs, B, blk_mask, W, gate,
-                                                   lin_ws, out, o_branch, err);
+    k_simt_attention<128><<<grid, 128, smem, st>>>(mode, q, Nq, H, rs, B, blk_mask, W, gx,
+                                                   lin_sign, lin_ws, out, o_branch, err);
   } else {
     return set_error(WA_ERR_UNSUPPORTED, "fp32 attention supports d in {64,128}");
   }

@@ -196,7 +196,7 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
                  const __grid_constant__ CUtensorMap tmV, int mode, int Nq, int H, int Lk,
                  RowSource rs, const uint32_t* __restrict__ blk_mask, int W, int n_qb,
                  const int4* __restrict__ pairs, const int4* __restrict__ items, Partials part,
-                 const float* __restrict__ gate, float* __restrict__ lin_ws,
+                 const float* __restrict__ gate, float lin_sign, float* __restrict__ lin_ws,
                  __nv_bfloat16* __restrict__ out, float* __restrict__ o_branch, uint32_t* err) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_dyn[];
@@ -525,11 +525,13 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
             make_float2(M, l_tot);
     } else {
       const float inv = l_tot > 0.f ? 1.f / l_tot : 0.f;
+      // mode 1: sg = sigmoid(g); mode 0: the linear branch's weight sigmoid(lin_sign * x)
+      // (x = g and lin_sign = -1 for 1 - sigmoid(g); x = g_lin and +1 for two gates)
       float sg = 0.f;
       size_t obase = 0;
       if (row_valid) {
         const float gt = gate[static_cast<size_t>(qrow) * H + h];
-        sg = 1.f / (1.f + expf(-gt));
+        sg = 1.f / (1.f + expf(mode == 0 ? -lin_sign * gt : -gt));
         obase = static_cast<size_t>(qrow) * H * D + static_cast<size_t>(h) * D;
       }
 #pragma unroll
@@ -546,7 +548,7 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         }
         if (mode == 0) {
           float4* lw = reinterpret_cast<float4*>(lin_ws + obase + c0);
-          const float a = 1.f - sg;
+          const float a = sg;
 #pragma unroll
           for (int e = 0; e < 8; ++e)
             lw[e] = make_float4(a * v[4 * e], a * v[4 * e + 1], a * v[4 * e + 2], a * v[4 * e + 3]);
@@ -795,12 +797,12 @@ template <int D>
 void launch_attn_kernel(int grid, cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& tk,
                         const CUtensorMap& tv, int mode, int Nq, int H, RowSource rs,
                         const uint32_t* blk_mask, int W, int n_qb, const int4* pairs,
-                        const int4* items, Partials part, const float* gate, float* lin_ws,
-                        void* out, float* o_branch, uint32_t* err) {
+                        const int4* items, Partials part, const float* gate, float lin_sign,
+                        float* lin_ws, void* out, float* o_branch, uint32_t* err) {
   const int smem = Cfg<D>::kSmem;
   cudaFuncSetAttribute(k_umma_attention<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   k_umma_attention<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, mode, Nq, H, rs.L, rs, blk_mask, W,
-                                                     n_qb, pairs, items, part, gate, lin_ws,
+                                                     n_qb, pairs, items, part, gate, lin_sign, lin_ws,
                                                      static_cast<__nv_bfloat16*>(out), o_branch, err);
 }
 
@@ -818,8 +820,8 @@ wa_status make_maps(const void* q, int Nq, int H, int d, const RowSource& rs, CU
 }  // namespace
 
 wa_status launch_linear_attention(const void* q, int Nq, int H, int d, RowSource lin, int B,
-                                  const float* gate, float* lin_ws, float* o_lin, uint32_t* err,
-                                  cudaStream_t st) {
+                                  const float* gate, const float* gate_lin, float* lin_ws,
+                                  float* o_lin, uint32_t* err, cudaStream_t st) {
   if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
   if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs d in {64,128}");
   alignas(64) CUtensorMap tq, tk, tv;
@@ -830,10 +832,12 @@ wa_status launch_linear_attention(const void* q, int Nq, int H, int d, RowSource
   Partials none{nullptr, nullptr};
   if (d == 128)
     launch_attn_kernel<128>(grid, st, tq, tk, tv, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
-                            none, gate, lin_ws, nullptr, o_lin, err);
+                            none, gate_lin ? gate_lin : gate, gate_lin ? 1.f : -1.f, lin_ws, nullptr,
+                            o_lin, err);
   else
     launch_attn_kernel<64>(grid, st, tq, tk, tv, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
-                           none, gate, lin_ws, nullptr, o_lin, err);
+                           none, gate_lin ? gate_lin : gate, gate_lin ? 1.f : -1.f, lin_ws, nullptr,
+                           o_lin, err);
   return check_launch("linear attention");
 }
 
@@ -904,12 +908,12 @@ wa_status launch_attn_sparse(const void* q, int Nq, int H, int d, RowSource rs, 
   const int split_min = split_min_for(s.n_pairs);
   if (d == 128) {
     launch_attn_kernel<128>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
-                            s.part, gate, lin_rw, out, o_sp, err);
+                            s.part, gate, 0.f, lin_rw, out, o_sp, err);
     k_combine<128><<<dim3(s.n_pairs, kBM / 32), 2 * 128, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate, lin_ws,
                                                                   static_cast<__nv_bfloat16*>(out), o_sp);
   } else {
     launch_attn_kernel<64>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
-                           s.part, gate, lin_rw, out, o_sp, err);
+                           s.part, gate, 0.f, lin_rw, out, o_sp, err);
     k_combine<64><<<dim3(s.n_pairs, kBM / 32), 2 * 64, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate, lin_ws,
                                                                 static_cast<__nv_bfloat16*>(out), o_sp);
   }

@@ -360,6 +360,7 @@ wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, 
 }
 
 namespace wa_detail {
+namespace {  // internal linkage: nothing here is exported from libwa
 struct BlockSelectWs {
   double* qsum;
   double* qbar;
@@ -381,6 +382,7 @@ BlockSelectWs carve_block_select(Carver& c, int Nq, int H, int d, int L, int B, 
   w.scores = reinterpret_cast<double*>(c.take<char>(block_scores_bytes(H, n_qb, n_kb)));
   return w;
 }
+}  // namespace
 }  // namespace wa_detail
 
 size_t wa_block_select_workspace_size(int Nq, int H, int d, int L, int B) {
@@ -465,10 +467,11 @@ size_t wa_hsa_attention_workspace_size(int Nq, int H, int d, int L, int B, int r
 }
 
 namespace wa_detail {
+namespace {  // internal linkage: nothing here is exported from libwa
 wa_status run_attention(const void* q, int Nq, int H, int d, RowSource rs, int B,
                         const uint32_t* blk_mask, const void* k_til, const void* v_til, int r,
-                        const float* gate, wa_dtype dtype, void* out, float* o_sp, float* o_lin,
-                        float* lin_ws, void* scratch, cudaStream_t st,
+                        const float* gate, const float* gate_lin, wa_dtype dtype, void* out,
+                        float* o_sp, float* o_lin, float* lin_ws, void* scratch, cudaStream_t st,
                         void* const* events = nullptr) {
   auto mark = [&](int k) {
     if (events && events[k]) cudaEventRecord(static_cast<cudaEvent_t>(events[k]), st);
@@ -481,17 +484,17 @@ wa_status run_attention(const void* q, int Nq, int H, int d, RowSource rs, int B
   RowSource lin;
   lin.k = k_til; lin.v = v_til; lin.page_rows = r; lin.n_pages = 1; lin.L = r;
   if (dtype == WA_BF16) {
-    WA_TRY(launch_linear_attention(q, Nq, H, d, lin, B, gate, lin_ws, o_lin, err, st));
+    WA_TRY(launch_linear_attention(q, Nq, H, d, lin, B, gate, gate_lin, lin_ws, o_lin, err, st));
     mark(5);
     return launch_sparse_attention(q, Nq, H, d, rs, B, blk_mask, gate, lin_ws, out, o_sp, scratch,
                                    err, st, events);
   }
   WA_TRY(launch_simt_attention(0, static_cast<const float*>(q), Nq, H, d, lin, B, nullptr, 0, gate,
-                               lin_ws, nullptr, o_lin, err, st));
+                               gate_lin, lin_ws, nullptr, o_lin, err, st));
   mark(5);
   mark(6);
   return launch_simt_attention(1, static_cast<const float*>(q), Nq, H, d, rs, B, blk_mask, W, gate,
-                               lin_ws, static_cast<float*>(out), o_sp, err, st);
+                               nullptr, lin_ws, static_cast<float*>(out), o_sp, err, st);
 }
 
 wa_status check_rank(int r, wa_dtype dt) {
@@ -500,13 +503,16 @@ wa_status check_rank(int r, wa_dtype dt) {
   if (dt == WA_F32 && (r > 4096)) return set_error(WA_ERR_UNSUPPORTED, "r too large");
   return WA_OK;
 }
+}  // namespace
 }  // namespace wa_detail
 using namespace wa_detail;
 
-wa_status wa_hsa_attention(const void* q, int Nq, int H, int d, const void* k_act, const void* v_act,
-                           int L, int B, const uint32_t* blk_mask, const void* k_til,
-                           const void* v_til, int r, const float* gate, wa_dtype dtype, void* out,
-                           float* o_sp, float* o_lin, void* ws, size_t ws_bytes, void* stream) {
+namespace wa_detail {
+namespace {  // internal linkage: nothing here is exported from libwa
+wa_status hsa_attention(const void* q, int Nq, int H, int d, const void* k_act, const void* v_act,
+                        int L, int B, const uint32_t* blk_mask, const void* k_til, const void* v_til,
+                        int r, const float* gate, const float* gate_lin, wa_dtype dtype, void* out,
+                        float* o_sp, float* o_lin, void* ws, size_t ws_bytes, void* stream) {
   WA_REQUIRE(q && k_act && v_act && blk_mask && k_til && v_til && gate && out, "NULL pointer");
   WA_REQUIRE(Nq >= 1 && L >= 1 && r >= 1, "sizes must be >= 1");
   WA_TRY(check_shape(H, d, B, dtype));
@@ -518,12 +524,33 @@ wa_status wa_hsa_attention(const void* q, int Nq, int H, int d, const void* k_ac
   void* scratch = dtype == WA_BF16 ? c.take<char>(sparse_attn_ws_bytes(H, Nq, d, B)) : nullptr;
   RowSource rs;
   rs.k = k_act; rs.v = v_act; rs.page_rows = L; rs.n_pages = 1; rs.L = L;
-  return run_attention(q, Nq, H, d, rs, B, blk_mask, k_til, v_til, r, gate, dtype, out, o_sp, o_lin,
-                       lin_ws, scratch, static_cast<cudaStream_t>(stream));
+  return run_attention(q, Nq, H, d, rs, B, blk_mask, k_til, v_til, r, gate, gate_lin, dtype, out, o_sp,
+                       o_lin, lin_ws, scratch, static_cast<cudaStream_t>(stream));
+}
+}  // namespace
+}  // namespace wa_detail
+
+wa_status wa_hsa_attention(const void* q, int Nq, int H, int d, const void* k_act, const void* v_act,
+                           int L, int B, const uint32_t* blk_mask, const void* k_til,
+                           const void* v_til, int r, const float* gate, wa_dtype dtype, void* out,
+                           float* o_sp, float* o_lin, void* ws, size_t ws_bytes, void* stream) {
+  return hsa_attention(q, Nq, H, d, k_act, v_act, L, B, blk_mask, k_til, v_til, r, gate, nullptr,
+                       dtype, out, o_sp, o_lin, ws, ws_bytes, stream);
+}
+
+wa_status wa_hsa_attention_gated2(const void* q, int Nq, int H, int d, const void* k_act,
+                                  const void* v_act, int L, int B, const uint32_t* blk_mask,
+                                  const void* k_til, const void* v_til, int r, const float* gate_sp,
+                                  const float* gate_lin, wa_dtype dtype, void* out, float* o_sp,
+                                  float* o_lin, void* ws, size_t ws_bytes, void* stream) {
+  WA_REQUIRE(gate_lin, "NULL pointer");
+  return hsa_attention(q, Nq, H, d, k_act, v_act, L, B, blk_mask, k_til, v_til, r, gate_sp, gate_lin,
+                       dtype, out, o_sp, o_lin, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ step
 namespace wa_detail {
+namespace {  // internal linkage: nothing here is exported from libwa
 struct StepWs {
   int32_t* chunk;
   int32_t* cand;       // candidate page ids copied from chunk_pages row
@@ -602,6 +629,7 @@ __global__ void k_pick_chunk(const int32_t* chunk_pages, int n_c, const int32_t*
   if (m < 0 || m >= n_chunks) m = 0;
   for (int j = threadIdx.x; j < n_c; j += blockDim.x) cand[j] = chunk_pages[static_cast<size_t>(m) * n_c + j];
 }
+}  // namespace
 }  // namespace wa_detail
 using namespace wa_detail;
 
@@ -693,8 +721,8 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
     WA_TRY(launch_umma_project(rs.k, rs.v, rs, a->e_k, a->e_v, L, a->H, a->d, a->r, kt, vt, w.proj,
                                err, side->stream));
     mark_side(4);
-    WA_TRY(launch_linear_attention(a->q, a->Nq, a->H, a->d, lin, a->B, a->gate, w.lin, nullptr, err,
-                                   side->stream));
+    WA_TRY(launch_linear_attention(a->q, a->Nq, a->H, a->d, lin, a->B, a->gate, a->gate_lin, w.lin,
+                                   nullptr, err, side->stream));
     mark_side(5);
     cudaEventRecord(side->join, side->stream);
     // S3: block selection
@@ -718,8 +746,8 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
                                rs.n_pages, static_cast<const float*>(a->e_v), L, cols, a->r,
                                static_cast<float*>(vt), err, st));
     mark(4);
-    WA_TRY(run_attention(a->q, a->Nq, a->H, a->d, rs, a->B, mask, kt, vt, a->r, a->gate, a->dtype,
-                         a->out, nullptr, nullptr, w.lin, w.attn, st, a->stage_events));
+    WA_TRY(run_attention(a->q, a->Nq, a->H, a->d, rs, a->B, mask, kt, vt, a->r, a->gate, a->gate_lin,
+                         a->dtype, a->out, nullptr, nullptr, w.lin, w.attn, st, a->stage_events));
   }
   mark(7);
   return WA_OK;

@@ -100,12 +100,13 @@ wa_status launch_copy16(const void* src, void* dst, size_t n16, cudaStream_t st)
 wa_status launch_simt_project(const float* x, const int32_t* page_ids, int page_rows, int n_pages,
                               const float* e, int L, int cols, int r, float* out,
                               uint32_t* err, cudaStream_t st);
-// mode 0: linear branch over (k_til, v_til), writes lin_ws = (1-sigmoid(g))*O_lin
+// mode 0: linear branch over (k_til, v_til), writes lin_ws = w * O_lin with
+//         w = 1 - sigmoid(g), or sigmoid(g_lin) when gate_lin is given (two gates)
 // mode 1: sparse branch over blk_mask, writes out = sigmoid(g)*O_sp + lin_ws
 wa_status launch_simt_attention(int mode, const float* q, int Nq, int H, int d, RowSource rs,
                                 int B, const uint32_t* blk_mask, int W, const float* gate,
-                                float* lin_ws, float* out, float* o_branch, uint32_t* err,
-                                cudaStream_t st);
+                                const float* gate_lin, float* lin_ws, float* out, float* o_branch,
+                                uint32_t* err, cudaStream_t st);
 
 // ---------------------------------------------------------------- bf16 tcgen05 path
 size_t umma_project_ws_bytes(int L, int H, int d, int r);
@@ -114,10 +115,11 @@ wa_status launch_umma_project(const void* k, const void* v, RowSource rs, const 
                               void* v_til, void* ws, uint32_t* err, cudaStream_t st);
 
 // Linear branch on tcgen05 (keys = k_til/v_til [r][H][d], every block): writes
-//   lin_ws[n][h][:] = (1 - sigmoid(g)) * O_lin (fp32) and o_lin (nullable).
+//   lin_ws[n][h][:] = w * O_lin (fp32) and o_lin (nullable), with w = 1 - sigmoid(g),
+//   or sigmoid(g_lin) when gate_lin is given (two independent gates).
 wa_status launch_linear_attention(const void* q, int Nq, int H, int d, RowSource lin, int B,
-                                  const float* gate, float* lin_ws, float* o_lin, uint32_t* err,
-                                  cudaStream_t st);
+                                  const float* gate, const float* gate_lin, float* lin_ws,
+                                  float* o_lin, uint32_t* err, cudaStream_t st);
 // Sparse branch on tcgen05 over the kept blocks of blk_mask, fused with the gate:
 //   out = bf16(sigmoid(g) * O_sp + lin_ws), o_sp (nullable) = O_sp in fp32.
 // `scratch` holds the work list and the split partials (sparse_attn_ws_bytes).

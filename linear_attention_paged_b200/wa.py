@@ -52,6 +52,7 @@ class StepArgs(ctypes.Structure):
         ("k_til_out", P), ("v_til_out", P),
         ("stage_events", P),
         ("page_index", P),
+        ("gate_lin", P),
     ]
 
 
@@ -74,6 +75,8 @@ _SIGS = {
     "wa_hsa_attention_workspace_size": (c_size_t, [c_int] * 7),
     "wa_hsa_attention": (c_int, [P, c_int, c_int, c_int, P, P, c_int, c_int, P, P, P, c_int, P,
                                  c_int, P, P, P, P, c_size_t, P]),
+    "wa_hsa_attention_gated2": (c_int, [P, c_int, c_int, c_int, P, P, c_int, c_int, P, P, P, c_int,
+                                        P, P, c_int, P, P, P, P, c_size_t, P]),
     "wa_pool_index": (c_int, [P, c_int, c_int, c_int, c_int, c_int, c_int, P, c_int, P, P]),
     "wa_pool_append": (c_int, [P, P, c_int, c_int, c_int, c_int, c_int, P, P, c_int, ctypes.c_longlong,
                                P, c_int, P]),
@@ -89,7 +92,7 @@ for _name, (_res, _args) in _SIGS.items():
 def header_functions() -> list:
     """Names of the functions declared in include/wa.h."""
     txt = open(HEADER_PATH).read()
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\*?\s+\**(wa_\w+)\s*\(", txt, re.M)))
+    return sorted(set(re.findall(r"^\s*(?:WA_API\s+)?(?:const\s+)?\w+\*?\s+\**(wa_\w+)\s*\(", txt, re.M)))
 
 
 def last_error() -> str:
@@ -260,8 +263,10 @@ def wa_linear_project_noalloc(k_act, v_act, e_k, e_v, stream=None):
 
 # --------------------------------------------------------------------- S4b+S5+S6
 def wa_hsa_attention(q, k_act, v_act, blk_mask, k_til, v_til, gate, B: int = 64,
-                     want_branches: bool = False, stream=None):
-    _need_cuda(q, k_act, v_act, blk_mask, k_til, v_til, gate)
+                     want_branches: bool = False, stream=None, gate_lin=None):
+    """out = sigmoid(gate) O_sp + (1 - sigmoid(gate)) O_lin, or with ``gate_lin``
+    sigmoid(gate) O_sp + sigmoid(gate_lin) O_lin (wa_hsa_attention_gated2)."""
+    _need_cuda(q, k_act, v_act, blk_mask, k_til, v_til, gate, gate_lin)
     Nq, H, d = q.shape
     L = k_act.shape[0]
     r = k_til.shape[0]
@@ -271,9 +276,15 @@ def wa_hsa_attention(q, k_act, v_act, blk_mask, k_til, v_til, gate, B: int = 64,
     o_lin = torch.empty(q.shape, dtype=torch.float32, device=q.device) if want_branches else None
     nbytes = lib.wa_hsa_attention_workspace_size(Nq, H, d, L, B, r, dt)
     ws = workspace(nbytes, q.device)
-    _check("wa_hsa_attention", lib.wa_hsa_attention(
-        _p(q), Nq, H, d, _p(k_act), _p(v_act), L, B, _p(blk_mask), _p(k_til), _p(v_til), r,
-        _p(gate), dt, _p(out), _p(o_sp), _p(o_lin), _p(ws), nbytes, _stream(stream)))
+    if gate_lin is None:
+        _check("wa_hsa_attention", lib.wa_hsa_attention(
+            _p(q), Nq, H, d, _p(k_act), _p(v_act), L, B, _p(blk_mask), _p(k_til), _p(v_til), r,
+            _p(gate), dt, _p(out), _p(o_sp), _p(o_lin), _p(ws), nbytes, _stream(stream)))
+    else:
+        _check("wa_hsa_attention_gated2", lib.wa_hsa_attention_gated2(
+            _p(q), Nq, H, d, _p(k_act), _p(v_act), L, B, _p(blk_mask), _p(k_til), _p(v_til), r,
+            _p(gate), _p(gate_lin), dt, _p(out), _p(o_sp), _p(o_lin), _p(ws), nbytes,
+            _stream(stream)))
     return (out, o_sp, o_lin) if want_branches else out
 
 
@@ -284,8 +295,8 @@ class HSAStep:
 
     def __init__(self, q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 4,
                  B: int = 64, e_cur=None, e_chunks=None, fused_gather: bool = True,
-                 keep_intermediates: bool = False, out=None, page_index=None):
-        _need_cuda(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, e_cur, e_chunks)
+                 keep_intermediates: bool = False, out=None, page_index=None, gate_lin=None):
+        _need_cuda(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, e_cur, e_chunks, gate_lin)
         Nq, H, d = q.shape
         P_, T_p = k_pool.shape[0], k_pool.shape[1]
         if chunk_pages.dim() == 1:
@@ -310,7 +321,8 @@ class HSAStep:
         a.dtype, a.fused_gather = dtype_code(q), int(bool(fused_gather))
         a.out = _p(self.out)
         a.page_index = _p(page_index)
-        self._keep.append(page_index)
+        a.gate_lin = _p(gate_lin)
+        self._keep += [page_index, gate_lin]
         self.inter = {}
         if keep_intermediates:
             self.inter = dict(
@@ -343,10 +355,10 @@ class HSAStep:
 
 def wa_hsa_step(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 4, B: int = 64,
                 e_cur=None, e_chunks=None, fused_gather: bool = True, keep_intermediates: bool = False,
-                stream=None, page_index=None):
+                stream=None, page_index=None, gate_lin=None):
     """One HSA decode step; returns ``out`` (and the intermediates when asked)."""
     st = HSAStep(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p, B, e_cur, e_chunks,
-                 fused_gather, keep_intermediates, page_index=page_index)
+                 fused_gather, keep_intermediates, page_index=page_index, gate_lin=gate_lin)
     out = st(stream)
     return (out, st.inter) if keep_intermediates else out
 

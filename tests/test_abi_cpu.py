@@ -21,6 +21,9 @@ def test_exports_every_declared_function():
     exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
     missing = [f for f in declared if f not in exported]
     assert not missing, f"declared but not exported: {missing}"
+    # and nothing else: internal helpers and kernels stay hidden
+    extra = sorted(e for e in exported if e not in declared)
+    assert not extra, f"exported but not declared in wa.h: {extra[:8]}"
     for f in declared:
         assert hasattr(wa.lib, f)
 
@@ -89,6 +92,13 @@ def test_attention_and_projection_validation():
     assert call(d=32) == wa.WA_ERR_UNSUPPORTED
     g = wa.lib.wa_linear_project
     assert g(FAKE, FAKE, FAKE, None, 2048, 1, 64, 32, wa.WA_F32, FAKE, FAKE, None, 0, None) == wa.WA_ERR_INVALID_ARG
+    f2 = wa.lib.wa_hsa_attention_gated2
+
+    def call2(gl):
+        a = ok
+        return f2(a["q"], a["Nq"], a["H"], a["d"], a["k"], a["v"], a["L"], a["B"], a["m"], a["kt"],
+                  a["vt"], a["r"], a["g"], gl, a["dt"], a["out"], None, None, FAKE, 1 << 40, None)
+    assert call2(None) == wa.WA_ERR_INVALID_ARG         # the second gate is required here
 
 
 def _step_args(**kw):

@@ -217,7 +217,52 @@ def test_hsa_attention_identities(wa):
     check_device_ok(wa)
 
 
+@pytest.mark.parametrize("cfg", [SMALL_BF16, SMALL_BF16_D64, SMALL_F32], ids=lambda c: c.name)
+def test_hsa_attention_two_gates(wa, cfg):
+    """sigmoid(g_sp) O_sp + sigmoid(g_lin) O_lin against the oracle's two-gate fusion;
+    g_lin = -g_sp reproduces the one-gate entry point."""
+    inp = inputs(cfg)
+    sel = [int(x) for x in inp["cand"][: cfg.K_p].cpu()]
+    k_act = O.gather_pages(inp["k_pool"], sel)
+    v_act = O.gather_pages(inp["v_pool"], sel)
+    kept, margin = O.block_select(inp["q"], k_act, inp["tau"], cfg.B)
+    _, _, mask = wa.wa_block_select(inp["q"], inp["tau"].cuda(), cfg.B, k_act=k_act)
+    compare_selection(mask_to_sets(mask, cfg.n_kb), kept, margin, f"{cfg.name} masks")
+    kt, vt = O.linear_project(k_act, v_act, inp["e_k"], inp["e_v"])
+    kt_in = torch.from_numpy(kt).to(cfg.torch_dtype).cuda()
+    vt_in = torch.from_numpy(vt).to(cfg.torch_dtype).cuda()
+    g_lin = torch.randn(inp["gate"].shape, generator=torch.Generator().manual_seed(cfg.seed + 5)).cuda()
+    out, o_sp, o_lin = wa.wa_hsa_attention(inp["q"], k_act, v_act, mask, kt_in, vt_in, inp["gate"],
+                                           cfg.B, want_branches=True, gate_lin=g_lin)
+    ref_sp = O.sparse_attention(inp["q"], k_act, v_act, kept, cfg.B)
+    ref_lin = O.linear_attention(inp["q"], kt_in, vt_in)
+    assert_close(o_lin, ref_lin, dkey(cfg), f"{cfg.name} O_lin")
+    assert_close(o_sp, ref_sp, dkey(cfg), f"{cfg.name} O_sp")
+    assert_close(out, O.gate_fuse2(ref_sp, ref_lin, inp["gate"], g_lin), dkey(cfg), f"{cfg.name} O (two gates)")
+    one = wa.wa_hsa_attention(inp["q"], k_act, v_act, mask, kt_in, vt_in, inp["gate"], cfg.B)
+    neg = wa.wa_hsa_attention(inp["q"], k_act, v_act, mask, kt_in, vt_in, inp["gate"], cfg.B,
+                              gate_lin=-inp["gate"])
+    assert torch.equal(neg, one), f"{cfg.name}: g_lin = -g must reproduce the one-gate output exactly"
+    check_device_ok(wa)
+
+
 # ---------------------------------------------------------------- whole step
+@pytest.mark.parametrize("cfg", [SMALL_BF16, SMALL_F32], ids=lambda c: c.name)
+def test_hsa_step_two_gates(wa, cfg):
+    inp = inputs(cfg)
+    g_lin = torch.randn(inp["gate"].shape, generator=torch.Generator().manual_seed(cfg.seed + 6)).cuda()
+    out, inter = wa.wa_hsa_step(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"],
+                                inp["e_v"], inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B,
+                                keep_intermediates=True, gate_lin=g_lin)
+    inp_o = dict(inp)
+    inp_o["gate_lin"] = g_lin.cpu()
+    res = O.hsa_step(inp_o, cfg.B, cfg.K_p)
+    compare_selection(mask_to_sets(inter["blk_mask"], cfg.n_kb), res["kept"], res["block_margin"],
+                      f"{cfg.name} step masks")
+    assert_close(out, res["o"], dkey(cfg), f"{cfg.name} step O (two gates)")
+    check_device_ok(wa)
+
+
 @pytest.mark.parametrize("fused", [True, False], ids=["fused", "gathered"])
 @pytest.mark.parametrize("cfg", [W.C0, SMALL_BF16, SMALL_BF16_D64, SMALL_F32], ids=lambda c: c.name)
 def test_hsa_step_small(wa, cfg, fused):
