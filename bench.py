@@ -51,7 +51,7 @@ from linear_attention_paged_b200 import replicas  # noqa: E402
 METRIC = "HSA ms/chunk-layer & attention frames/s; % of BF16 tensor / HBM roofline"
 # DRAM bytes per launch of the sparse-branch attention kernel per head, from one ncu
 # capture of the 6-head C1 launch (360.1 MB / 6); set to None when the kernel changes
-ATTN_DRAM_BYTES_PER_HEAD = None   # the last capture predates the current kernel
+ATTN_DRAM_BYTES_PER_HEAD = 356.9e6 / 6
 FRAMES_PER_CHUNK = 3
 CHUNK_LAYERS_PER_CHUNK = 30 * 4
 # stage -> (start event, end event) of the events wa_hsa_step records; the
@@ -333,6 +333,25 @@ def run_ours(args, rank, world, local_rank):
     h2d = q_host.numel() * q_host.element_size() + g_host.numel() * g_host.element_size()
     d2h = o_host.numel() * o_host.element_size()
 
+    # S2 on its own: the gather of the selected pages that the fused step avoids
+    # (non-fused path), K and V read once and written once
+    sel = step.inter["sel"]
+    ka = torch.empty((cfg.L, cfg.H, cfg.d), dtype=inp["k_pool"].dtype, device=dev)
+    va = torch.empty_like(ka)
+    for _ in range(3):
+        wa.wa_gather_pages(inp["k_pool"], inp["v_pool"], sel, out=(ka, va))
+    n_g = 20
+    gs, ge = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    gs.record(stream)
+    for _ in range(n_g):
+        wa.wa_gather_pages(inp["k_pool"], inp["v_pool"], sel, out=(ka, va))
+    ge.record(stream)
+    torch.cuda.synchronize()
+    gather_ms = gs.elapsed_time(ge) / n_g
+    gather_bytes = 2 * 2 * ka.numel() * ka.element_size()
+    gather_gbs = gather_bytes / (gather_ms * 1e-3) / 1e9
+    del ka, va
+
     line = None
     if rank == 0:
         cpu = None
@@ -365,6 +384,10 @@ def run_ours(args, rank, world, local_rank):
             "hbm_page_scoring": {"achieved": hbm_achieved, "peak": float(peaks["hbm_gbs"]),
                                  "unit": "GB/s", "frac": hbm_achieved / float(peaks["hbm_gbs"]),
                                  "bytes_per_launch": page_bytes},
+            "hbm_gather": {"kernel": "k_gather (non-fused S2)", "achieved": gather_gbs,
+                           "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                           "frac": gather_gbs / float(peaks["hbm_gbs"]), "bytes_per_launch": gather_bytes,
+                           "ms_per_launch": gather_ms},
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "e2e": ({"value": frames_per_s(e2e_ms, world), "unit": "frames/s", "ms_per_step": e2e_ms,
                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps}

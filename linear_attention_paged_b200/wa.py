@@ -175,12 +175,20 @@ def wa_page_score(q, k_pool, cand_pages, K_p: int, B: int = 64, want_blockmean: 
 
 
 # --------------------------------------------------------------------- S2
-def wa_gather_pages(k_pool, v_pool, sel, stream=None):
+def wa_gather_pages(k_pool, v_pool, sel, stream=None, out=None):
+    """K_active, V_active = the selected pool pages, concatenated in `sel` order
+    (``out``: optional preallocated (k_act, v_act))."""
     _need_cuda(k_pool, v_pool, sel)
     P_, T_p, H, d = k_pool.shape
     K_p = sel.numel()
-    k_act = torch.empty((K_p * T_p, H, d), dtype=k_pool.dtype, device=k_pool.device)
-    v_act = torch.empty_like(k_act)
+    if out is None:
+        k_act = torch.empty((K_p * T_p, H, d), dtype=k_pool.dtype, device=k_pool.device)
+        v_act = torch.empty_like(k_act)
+    else:
+        k_act, v_act = out
+        _need_cuda(k_act, v_act)
+        assert k_act.shape == (K_p * T_p, H, d) and v_act.shape == k_act.shape
+        assert k_act.dtype == k_pool.dtype and v_act.dtype == k_pool.dtype
     _check("wa_gather_pages", lib.wa_gather_pages(
         _p(k_pool), _p(v_pool), P_, T_p, H, d, _p(sel), K_p, dtype_code(k_pool), _p(k_act),
         _p(v_act), _stream(stream)))
