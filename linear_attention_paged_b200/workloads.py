@@ -56,6 +56,8 @@ class HSAConfig:
     # head's kept fraction between 36 % and 97 %; 7 spreads the per-head means from
     # 0.8 % to 90 %, the intended 1 % -> 100 % range.
     hot_beta_scale: float = 7.0
+    # the current chunk's own K and V ([Nq][H][d]) join the sparse branch's keys
+    intra: bool = False
 
     @property
     def L(self) -> int:
@@ -189,6 +191,12 @@ def make_inputs(cfg: HSAConfig, device: str = "cpu", gen_device: Optional[str] =
     if cfg.n_chunks > 1:
         out["e_cur"] = randn(cfg.prompt_dim).to(device)
         out["e_chunks"] = randn(cfg.n_chunks, cfg.prompt_dim).to(device)
+    if cfg.intra:
+        # the current chunk's own keys and values, drawn last so that every other
+        # input keeps its bits: N(0,1) (gauss) or N(0,1)/sqrt(d), no page offset
+        sc = 1.0 if cfg.recipe == "gauss" else inv_sqrt_d
+        out["k_cur"] = (randn(Nq, H, d) * sc).to(dt).to(device)
+        out["v_cur"] = (randn(Nq, H, d) * sc).to(dt).to(device)
     out["chunk_pages"] = torch.arange(P, dtype=torch.int32).reshape(cfg.n_chunks, cfg.n_c).to(device)
     out["cand"] = out["chunk_pages"][0].clone()
 

@@ -287,7 +287,14 @@ def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tupl
     """The whole decode step S0..S6 on one input dict (see the workload module).
 
     With ``rows_of_blocks`` = [(h, i), ...] only those (head, query block) outputs are
-    computed (the selection is still computed for every row); otherwise all of O."""
+    computed (the selection is still computed for every row); otherwise all of O.
+
+    With ``k_cur``/``v_cur`` in the input (the current chunk's own keys and values,
+    [Nq][H][d]), the sparse branch's key sequence is the retrieved history followed by
+    the current chunk (main text §3.3, "Inter- and intra-chunk sparse granularity":
+    the sparse branch attends to both, in blocks of the same kernel); block selection
+    runs over all blocks of that sequence jointly, and the linear branch stays over
+    the history, whose positions E indexes."""
     res: dict = {}
     if "e_cur" in inp:
         m = prompt_select(inp["e_cur"], inp["e_chunks"])
@@ -306,7 +313,11 @@ def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tupl
     k_act = gather_pages(k_pool, sel)
     v_act = gather_pages(v_pool, sel)
     res["k_act"], res["v_act"] = k_act, v_act
-    kept, margin = block_select(inp["q"], k_act, inp["tau"], B)
+    k_sp, v_sp = k_act, v_act
+    if inp.get("k_cur") is not None:
+        k_sp = np.concatenate([f64(k_act), f64(inp["k_cur"])], axis=0)
+        v_sp = np.concatenate([f64(v_act), f64(inp["v_cur"])], axis=0)
+    kept, margin = block_select(inp["q"], k_sp, inp["tau"], B)
     res["kept"], res["block_margin"] = kept, margin
     kt, vt = linear_project(k_act, v_act, inp["e_k"], inp["e_v"])
     res["k_til"], res["v_til"] = kt, vt
@@ -315,7 +326,7 @@ def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tupl
     g = f64(inp["gate"])
     g_lin = f64(inp["gate_lin"]) if inp.get("gate_lin") is not None else None
     if rows_of_blocks is None:
-        o_sp = sparse_attention(Q, k_act, v_act, kept, B)
+        o_sp = sparse_attention(Q, k_sp, v_sp, kept, B)
         o_lin = linear_attention(Q, kt, vt)
         res["o_sp"], res["o_lin"] = o_sp, o_lin
         res["o"] = gate_fuse(o_sp, o_lin, g) if g_lin is None else gate_fuse2(o_sp, o_lin, g, g_lin)
@@ -323,7 +334,7 @@ def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tupl
         outs = {}
         for (h, i) in rows_of_blocks:
             r0, r1 = i * B, min(Nq, (i + 1) * B)
-            osp = sparse_attention_block(Q, k_act, v_act, h, i, kept[h][i], B)
+            osp = sparse_attention_block(Q, k_sp, v_sp, h, i, kept[h][i], B)
             olin = linear_attention(Q[r0:r1, h:h + 1, :], kt[:, h:h + 1, :], vt[:, h:h + 1, :])[:, 0, :]
             G = sigmoid(g[r0:r1, h])[:, None]
             Gl = (1.0 - G) if g_lin is None else sigmoid(g_lin[r0:r1, h])[:, None]

@@ -322,6 +322,51 @@ def test_two_gate_fusion_pins():
     assert changed[1, 0] and changed.sum() == 1
 
 
+def _intra_cfg(**kw):
+    # ragged query tail (Nq % B = 8): the current chunk's last key block has 8 rows
+    return W.C0.with_(T_p=64, Nq=72, intra=True, **kw)
+
+
+def test_intra_keys_tau_one_is_dense_attention_over_history_and_chunk():
+    """tau = 1 keeps every block, so the sparse branch is textbook attention over
+    the retrieved history followed by the current chunk's own keys."""
+    cfg = _intra_cfg(tau_const=1.0)
+    inp = W.make_inputs(cfg)
+    res = O.hsa_step(inp, cfg.B, cfg.K_p)
+    k_all = np.concatenate([O.f64(res["k_act"]), O.f64(inp["k_cur"])])
+    v_all = np.concatenate([O.f64(res["v_act"]), O.f64(inp["v_cur"])])
+    n_all = -(-k_all.shape[0] // cfg.B)
+    assert all(len(row) == n_all for row in res["kept"][0])
+    q = O.f64(inp["q"])[:, 0, :]
+    np.testing.assert_allclose(res["o_sp"][:, 0, :], sdpa(q, k_all[:, 0, :], v_all[:, 0, :]),
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_intra_keys_hot_chunk_blocks_are_selected_and_linear_branch_ignores_them():
+    """Current-chunk keys pushed toward the mean query carry almost all pooled mass:
+    a low tau keeps only chunk blocks, including the 8-row tail pooled over its valid
+    rows; the linear branch (over the history) does not change."""
+    cfg = _intra_cfg(tau_const=0.5)
+    inp = W.make_inputs(cfg)
+    # a common query direction u for every query block, and chunk keys along u
+    u = torch.from_numpy(rng(18).normal(size=(cfg.H, cfg.d))).float()
+    u = u / u.norm(dim=-1, keepdim=True)
+    inp["q"] = inp["q"] + 3.0 * u[None]
+    inp["k_cur"] = inp["k_cur"] + 40.0 * u[None]
+    res = O.hsa_step(inp, cfg.B, cfg.K_p)
+    n_hist = cfg.L // cfg.B
+    n_all = n_hist + -(-cfg.Nq // cfg.B)
+    for row in res["kept"][0]:
+        assert row and all(n_hist <= j < n_all for j in row)
+    base = dict(inp); base.pop("k_cur"); base.pop("v_cur")
+    res0 = O.hsa_step(base, cfg.B, cfg.K_p)
+    np.testing.assert_array_equal(res["o_lin"], res0["o_lin"])
+    # the tail block's pooled mean uses its 8 valid rows
+    kb = O.block_means(np.concatenate([O.f64(res["k_act"]), O.f64(inp["k_cur"])]), cfg.B)
+    tail = O.f64(inp["k_cur"])[64:72].mean(axis=0)
+    np.testing.assert_allclose(kb[n_all - 1], tail, rtol=1e-15, atol=1e-15)
+
+
 def test_step_two_gates_matches_recombined_branches():
     cfg = W.C0.with_(T_p=64, Nq=72)
     inp = W.make_inputs(cfg)
