@@ -71,9 +71,11 @@ def load_peaks():
 
 
 def workload_desc(cfg):
+    intra = (f"; sparse branch also over the chunk's own {cfg.Nq} keys (intra-chunk keys)"
+             if cfg.intra else "")
     return (f"{cfg.name}: one HSA decode step (chunk-layer), H={cfg.H}, d={cfg.d}, T_p={cfg.T_p} "
             f"(8 frames x 1560 tokens), n_c={cfg.n_c} candidate pages, Nq={cfg.Nq}, K_p={cfg.K_p} "
-            f"-> L={cfg.L}, B={cfg.B}, r={cfg.r}, tau_h=0.80+0.15h/11, bf16")
+            f"-> L={cfg.L}, B={cfg.B}, r={cfg.r}, tau_h=0.80+0.15h/11, bf16{intra}")
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -228,15 +230,20 @@ def selected_flops(mask, cfg):
     m = mask.cpu().numpy().astype(np.uint32)
     H, n_qb, W_ = m.shape
     bq = np.array([min(cfg.Nq, (i + 1) * cfg.B) - i * cfg.B for i in range(n_qb)], dtype=np.float64)
-    bk = np.array([min(cfg.L, (j + 1) * cfg.B) - j * cfg.B for j in range(cfg.n_kb)], dtype=np.float64)
+    # key blocks: the history, then (intra-chunk keys) the chunk's own Nq rows
+    bk = [min(cfg.L, (j + 1) * cfg.B) - j * cfg.B for j in range(cfg.n_kb)]
+    if cfg.intra:
+        bk += [min(cfg.Nq, (j + 1) * cfg.B) - j * cfg.B for j in range(-(-cfg.Nq // cfg.B))]
+    bk = np.array(bk, dtype=np.float64)
+    n_kb = len(bk)
     total = 0.0
     kept = 0
     for h in range(H):
         for i in range(n_qb):
-            bits = np.unpackbits(m[h, i].view(np.uint8), bitorder="little")[:cfg.n_kb].astype(bool)
+            bits = np.unpackbits(m[h, i].view(np.uint8), bitorder="little")[:n_kb].astype(bool)
             kept += int(bits.sum())
             total += 4.0 * bq[i] * float(bk[bits].sum()) * cfg.d
-    return total, kept / float(H * n_qb * cfg.n_kb)
+    return total, kept / float(H * n_qb * n_kb)
 
 
 def run_ours(args, rank, world, local_rank):
@@ -249,13 +256,16 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     base = W.C1 if args.heads is None else W.C1.with_(name=f"c1_layer_bf16_h{args.heads}", H=args.heads)
+    if args.intra:
+        base = base.with_(name=base.name + "_intra", intra=True)
     cfg = base.with_(seed=replicas.rank_seed(base.seed, rank))   # each rank: its own layer
     inp = W.make_inputs(cfg, device="cuda", gen_device="cuda")
     tau = inp["tau"].cuda()
     stream = torch.cuda.current_stream()
 
     step = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"], inp["e_v"],
-                      tau, inp["gate"], cfg.K_p, cfg.B, fused_gather=True, keep_intermediates=True)
+                      tau, inp["gate"], cfg.K_p, cfg.B, fused_gather=True, keep_intermediates=True,
+                      k_cur=inp.get("k_cur"), v_cur=inp.get("v_cur"))
     step()
     torch.cuda.synchronize()
     flags = wa.wa_device_error()
@@ -523,6 +533,8 @@ def main():
     ap.add_argument("--config", choices=["c1", "c4"], default="c1",
                     help="c1: one-layer step (default); c4: the full denoise stack")
     ap.add_argument("--layers", type=int, default=30, help="c4: layers")
+    ap.add_argument("--intra", action="store_true",
+                    help="c1: add the chunk's own keys to the sparse branch (intra-chunk keys)")
     ap.add_argument("--chunks", type=int, default=20, help="c4: chunks")
     args = ap.parse_args()
     rank, world, local_rank = replicas.env_ranks()

@@ -304,6 +304,14 @@ typedef struct wa_step_args {
      sigmoid(gate) * O_sp + sigmoid(gate_lin) * O_lin (see wa_hsa_attention_gated2);
      NULL keeps sigmoid(gate) * O_sp + (1 - sigmoid(gate)) * O_lin */
   const float* gate_lin;
+  /* optional intra-chunk keys (main text §3.3, "Inter- and intra-chunk sparse
+     granularity"): the current chunk's own keys and values, [Nq][H][d] in the step's
+     dtype, both or neither.  With them the sparse branch's key sequence is the
+     retrieved history followed by these Nq rows, block selection (S3) runs over all
+     its blocks jointly, and blk_mask_out covers ceil((K_p*T_p + Nq)/B) blocks; the
+     linear branch stays over the history.  Needs K_p*T_p % B == 0. */
+  const void* k_cur;
+  const void* v_cur;
 } wa_step_args;
 
 /* Stage boundaries recorded into wa_step_args.stage_events:

@@ -270,9 +270,13 @@ k_block_scores(const double* __restrict__ qmean, KeyMeans km, int n_qb, int n_kb
     const int j = j0 + rr, i = i0 + rr;
     const double* ksrc = nullptr;
     if (j < n_kb) {
-      size_t row = j;
-      if (km.page_pos) row = static_cast<size_t>(km.page_pos[j / km.nbp]) * km.nbp + j % km.nbp;
-      ksrc = km.data + row * cols + h * d;
+      if (km.data2 && j >= km.n_kb1) {
+        ksrc = km.data2 + static_cast<size_t>(j - km.n_kb1) * cols + h * d;
+      } else {
+        size_t row = j;
+        if (km.page_pos) row = static_cast<size_t>(km.page_pos[j / km.nbp]) * km.nbp + j % km.nbp;
+        ksrc = km.data + row * cols + h * d;
+      }
     }
     const double* qsrc = i < n_qb ? qmean + static_cast<size_t>(i) * cols + h * d : nullptr;
     for (int c = lane; c < d; c += 32) {
@@ -299,7 +303,13 @@ k_block_scores(const double* __restrict__ qmean, KeyMeans km, int n_qb, int n_kb
   for (int v = 0; v < 2; ++v) {
     const int j = j0 + tx + 16 * v;
     if (j >= n_kb) continue;
-    const double den = km.is_sum ? static_cast<double>(min(km.L, (j + 1) * B) - j * B) * sqrt_d : sqrt_d;
+    double den = sqrt_d;
+    if (km.data2 && j >= km.n_kb1) {
+      const int jj = j - km.n_kb1;
+      den = static_cast<double>(min(km.L2, (jj + 1) * B) - jj * B) * sqrt_d;
+    } else if (km.is_sum) {
+      den = static_cast<double>(min(km.L, (j + 1) * B) - j * B) * sqrt_d;
+    }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
       const int i = i0 + ty + 16 * u;

@@ -54,7 +54,7 @@ k_simt_attention(int mode, const float* __restrict__ q, int Nq, int H, RowSource
   float* Vs = sm + kTile * D;     // [kTile][D]
   const int h = blockIdx.y, i = blockIdx.x;
   const int n_qb = (Nq + B - 1) / B;
-  const int L = rs.L;
+  const int L = rs.L + rs.L2;      // the second segment (if any) follows the first
   const int n_kb = (L + B - 1) / B;
   const float* kb = static_cast<const float*>(rs.k);
   const float* vb = static_cast<const float*>(rs.v);
@@ -84,8 +84,15 @@ k_simt_attention(int mode, const float* __restrict__ q, int Nq, int H, RowSource
       __syncthreads();
       for (int e = threadIdx.x; e < cnt * D; e += blockDim.x) {
         const int t = e / D, c = e % D;
+        const int l = t0 + t;
+        if (rs.k2 && l >= rs.L) {
+          const size_t r2 = static_cast<size_t>(l - rs.L) * cols + h * D + c;
+          Ks[t * D + c] = static_cast<const float*>(rs.k2)[r2];
+          Vs[t * D + c] = static_cast<const float*>(rs.v2)[r2];
+          continue;
+        }
         bool ok;
-        const long long r = row_of(rs, t0 + t, B, ok);
+        const long long r = row_of(rs, l, B, ok);
         bad |= !ok;
         Ks[t * D + c] = kb[r * cols + h * D + c];
         Vs[t * D + c] = vb[r * cols + h * D + c];

@@ -193,7 +193,8 @@ struct Partials {
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
 k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                 const __grid_constant__ CUtensorMap tmV, int mode, int Nq, int H, int Lk,
+                 const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
+                 const __grid_constant__ CUtensorMap tmV2, int mode, int Nq, int H, int Lk,
                  RowSource rs, const uint32_t* __restrict__ blk_mask, int W, int n_qb,
                  const int4* __restrict__ pairs, const int4* __restrict__ items, Partials part,
                  const float* __restrict__ gate, float lin_sign, float* __restrict__ lin_ws,
@@ -275,7 +276,8 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     }
   }
   if (tid == 0) sh.list[n_blk] = static_cast<uint16_t>(kNoBlock);
-  const int n_ids = rs.page_ids ? (Lk + rs.page_rows - 1) / rs.page_rows : 0;
+  // page-table entries cover the first segment only (rs.L rows)
+  const int n_ids = rs.page_ids ? (rs.L + rs.page_rows - 1) / rs.page_rows : 0;
   const int* staged = (n_ids > 0 && n_ids <= kMaxPages) ? sh.page_row0 : nullptr;
   if (staged && tid < n_ids) sh.page_row0[tid] = page_row0(rs, tid, err);
   if (warp == 1) {
@@ -297,7 +299,10 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (lane == 0) {
       const bool isK = warp == 0;
       const CUtensorMap* tm = isK ? &tmK : &tmV;
+      const CUtensorMap* tm2 = isK ? &tmK2 : &tmV2;   // the chunk's own keys (second segment)
+      const int n_kb1 = rs.k2 ? rs.L / kBN : INT_MAX;
       prefetch_tmap(tm);
+      if (rs.k2) prefetch_tmap(tm2);
       if (isK) {
         prefetch_tmap(&tmQ);
         mbar_arrive_expect_tx(&sh.q_full, C::kQBytes);
@@ -318,13 +323,15 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         const int jb = (wrd >> 16) == kNoBlock ? -1 : static_cast<int>((wrd >> 16) & 0x1FFFu);
         uint8_t* dst = isK ? Ks(s) : Vs(s);
         mbar_arrive_expect_tx(full, (jb >= 0 ? 2 : 1) * C::kBlockBytes);
-        const int ra = key_row(rs, staged, bpp, ja, err);
+        const bool a2 = ja >= n_kb1;
+        const int ra = a2 ? (ja - n_kb1) * kBN : key_row(rs, staged, bpp, ja, err);
         for (int p = 0; p < C::kPanels; ++p)
-          tma_load_2d(dst + p * C::kPanelBytes, tm, full, h * D + p * 64, ra);
+          tma_load_2d(dst + p * C::kPanelBytes, a2 ? tm2 : tm, full, h * D + p * 64, ra);
         if (jb >= 0) {
-          const int rb = key_row(rs, staged, bpp, jb, err);
+          const bool b2 = jb >= n_kb1;
+          const int rb = b2 ? (jb - n_kb1) * kBN : key_row(rs, staged, bpp, jb, err);
           for (int p = 0; p < C::kPanels; ++p)
-            tma_load_2d(dst + p * C::kPanelBytes + kBN * 128, tm, full, h * D + p * 64, rb);
+            tma_load_2d(dst + p * C::kPanelBytes + kBN * 128, b2 ? tm2 : tm, full, h * D + p * 64, rb);
         }
       }
     }
@@ -795,26 +802,39 @@ bool make_tmap_bf16_2d(void* tmap, const void* base, uint64_t inner, uint64_t ou
 namespace {
 template <int D>
 void launch_attn_kernel(int grid, cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& tk,
-                        const CUtensorMap& tv, int mode, int Nq, int H, RowSource rs,
+                        const CUtensorMap& tv, const CUtensorMap& tk2, const CUtensorMap& tv2,
+                        int mode, int Nq, int H, RowSource rs,
                         const uint32_t* blk_mask, int W, int n_qb, const int4* pairs,
                         const int4* items, Partials part, const float* gate, float lin_sign,
                         float* lin_ws, void* out, float* o_branch, uint32_t* err) {
   const int smem = Cfg<D>::kSmem;
   cudaFuncSetAttribute(k_umma_attention<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  k_umma_attention<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, mode, Nq, H, rs.L, rs, blk_mask, W,
+  k_umma_attention<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, tk2, tv2, mode, Nq, H, rs.L + rs.L2, rs,
+                                                     blk_mask, W,
                                                      n_qb, pairs, items, part, gate, lin_sign, lin_ws,
                                                      static_cast<__nv_bfloat16*>(out), o_branch, err);
 }
 
+// Q, the keys/values of the first segment (pool pages or a contiguous buffer) and,
+// when the row source has one, of the second (tk2/tv2 repeat tk/tv otherwise).
 wa_status make_maps(const void* q, int Nq, int H, int d, const RowSource& rs, CUtensorMap* tq,
-                    CUtensorMap* tk, CUtensorMap* tv) {
+                    CUtensorMap* tk, CUtensorMap* tv, CUtensorMap* tk2, CUtensorMap* tv2) {
   const int cols = H * d;
   const uint64_t key_rows = rs.page_ids ? static_cast<uint64_t>(rs.n_pages) * rs.page_rows
                                         : static_cast<uint64_t>(rs.L);
-  if (!make_tmap_bf16_2d(tq, q, cols, Nq, static_cast<uint64_t>(cols) * 2, 64, 64) ||
-      !make_tmap_bf16_2d(tk, rs.k, cols, key_rows, static_cast<uint64_t>(cols) * 2, 64, 64) ||
-      !make_tmap_bf16_2d(tv, rs.v, cols, key_rows, static_cast<uint64_t>(cols) * 2, 64, 64))
+  const uint64_t rb = static_cast<uint64_t>(cols) * 2;
+  if (!make_tmap_bf16_2d(tq, q, cols, Nq, rb, 64, 64) ||
+      !make_tmap_bf16_2d(tk, rs.k, cols, key_rows, rb, 64, 64) ||
+      !make_tmap_bf16_2d(tv, rs.v, cols, key_rows, rb, 64, 64))
     return set_error(WA_ERR_CUDA, "cuTensorMapEncodeTiled failed for the attention operands");
+  if (rs.k2) {
+    if (!make_tmap_bf16_2d(tk2, rs.k2, cols, rs.L2, rb, 64, 64) ||
+        !make_tmap_bf16_2d(tv2, rs.v2, cols, rs.L2, rb, 64, 64))
+      return set_error(WA_ERR_CUDA, "cuTensorMapEncodeTiled failed for the chunk's keys");
+  } else {
+    *tk2 = *tk;
+    *tv2 = *tv;
+  }
   return WA_OK;
 }
 }  // namespace
@@ -824,18 +844,18 @@ wa_status launch_linear_attention(const void* q, int Nq, int H, int d, RowSource
                                   float* o_lin, uint32_t* err, cudaStream_t st) {
   if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
   if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs d in {64,128}");
-  alignas(64) CUtensorMap tq, tk, tv;
-  wa_status s = make_maps(q, Nq, H, d, lin, &tq, &tk, &tv);
+  alignas(64) CUtensorMap tq, tk, tv, tk2, tv2;
+  wa_status s = make_maps(q, Nq, H, d, lin, &tq, &tk, &tv, &tk2, &tv2);
   if (s != WA_OK) return s;
   const int n_qb = (Nq + B - 1) / B;
   const int grid = H * ((n_qb + 1) / 2);
   Partials none{nullptr, nullptr};
   if (d == 128)
-    launch_attn_kernel<128>(grid, st, tq, tk, tv, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
+    launch_attn_kernel<128>(grid, st, tq, tk, tv, tk2, tv2, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
                             none, gate_lin ? gate_lin : gate, gate_lin ? 1.f : -1.f, lin_ws, nullptr,
                             o_lin, err);
   else
-    launch_attn_kernel<64>(grid, st, tq, tk, tv, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
+    launch_attn_kernel<64>(grid, st, tq, tk, tv, tk2, tv2, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
                            none, gate_lin ? gate_lin : gate, gate_lin ? 1.f : -1.f, lin_ws, nullptr,
                            o_lin, err);
   return check_launch("linear attention");
@@ -898,21 +918,23 @@ wa_status launch_attn_sparse(const void* q, int Nq, int H, int d, RowSource rs, 
                              void* out, float* o_sp, void* scratch, uint32_t* err, cudaStream_t st) {
   if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
   if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs d in {64,128}");
-  SparseLayout s = sparse_layout(scratch, Nq, H, d, B, rs.L);
+  if (rs.k2 && rs.L % kBN != 0)
+    return set_error(WA_ERR_UNSUPPORTED, "a second key segment needs the first to fill whole blocks");
+  SparseLayout s = sparse_layout(scratch, Nq, H, d, B, rs.L + rs.L2);
   if (s.W > kMaxW) return set_error(WA_ERR_UNSUPPORTED, "too many key blocks (max %d)", kMaxW * 32);
-  alignas(64) CUtensorMap tq, tk, tv;
-  wa_status e = make_maps(q, Nq, H, d, rs, &tq, &tk, &tv);
+  alignas(64) CUtensorMap tq, tk, tv, tk2, tv2;
+  wa_status e = make_maps(q, Nq, H, d, rs, &tq, &tk, &tv, &tk2, &tv2);
   if (e != WA_OK) return e;
   const int grid = 2 * s.n_pairs;
   float* lin_rw = const_cast<float*>(lin_ws);
   const int split_min = split_min_for(s.n_pairs);
   if (d == 128) {
-    launch_attn_kernel<128>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
+    launch_attn_kernel<128>(grid, st, tq, tk, tv, tk2, tv2, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
                             s.part, gate, 0.f, lin_rw, out, o_sp, err);
     k_combine<128><<<dim3(s.n_pairs, kBM / 32), 2 * 128, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate, lin_ws,
                                                                   static_cast<__nv_bfloat16*>(out), o_sp);
   } else {
-    launch_attn_kernel<64>(grid, st, tq, tk, tv, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
+    launch_attn_kernel<64>(grid, st, tq, tk, tv, tk2, tv2, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
                            s.part, gate, 0.f, lin_rw, out, o_sp, err);
     k_combine<64><<<dim3(s.n_pairs, kBM / 32), 2 * 64, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate, lin_ws,
                                                                 static_cast<__nv_bfloat16*>(out), o_sp);
@@ -924,7 +946,7 @@ wa_status launch_sparse_attention(const void* q, int Nq, int H, int d, RowSource
                                   const uint32_t* blk_mask, const float* gate, const float* lin_ws,
                                   void* out, float* o_sp, void* scratch, uint32_t* err,
                                   cudaStream_t st, void* const* events) {
-  wa_status e = launch_attn_worklist(Nq, H, d, B, rs.L, blk_mask, scratch, st);
+  wa_status e = launch_attn_worklist(Nq, H, d, B, rs.L + rs.L2, blk_mask, scratch, st);
   if (e != WA_OK) return e;
   if (events && events[6]) cudaEventRecord(static_cast<cudaEvent_t>(events[6]), st);
   return launch_attn_sparse(q, Nq, H, d, rs, B, blk_mask, gate, lin_ws, out, o_sp, scratch, err, st);

@@ -568,6 +568,7 @@ struct StepWs {
   void* v_act;
   double* ksum;     // non-fused: block sums of the gathered keys
   double* scores;   // float64 pooled block scores
+  double* cur_sum;  // block sums of the current chunk's keys (intra-chunk keys)
 };
 
 wa_status validate_step(const wa_step_args* a) {
@@ -590,14 +591,26 @@ wa_status validate_step(const wa_step_args* a) {
   if (a->page_index && (!a->fused_gather || a->T_p % a->B != 0))
     return set_error(WA_ERR_UNSUPPORTED, "the page index needs fused_gather and T_p %% B == 0");
   WA_REQUIRE(static_cast<long long>(a->n_pool_pages) * a->T_p < (1LL << 31), "pool too large");
+  WA_REQUIRE(!a->k_cur == !a->v_cur, "k_cur and v_cur are given together");
+  if (a->k_cur) {
+    if (L % a->B != 0)
+      return set_error(WA_ERR_UNSUPPORTED, "the chunk's keys need K_p*T_p %% B == 0");
+    WA_REQUIRE(ceil_div(static_cast<int>(L) + a->Nq, a->B) <= 8192, "at most 8192 key blocks");
+  }
   return WA_OK;
+}
+
+// key blocks of the sparse branch: the history, then (intra-chunk keys) the chunk's own
+int sparse_key_rows(const wa_step_args* a) {
+  return a->K_p * a->T_p + (a->k_cur ? a->Nq : 0);
 }
 
 StepWs carve_step(Carver& c, const wa_step_args* a) {
   StepWs w{};
   const int cols = a->H * a->d;
   const int L = a->K_p * a->T_p;
-  const int n_qb = ceil_div(a->Nq, a->B), n_kb = ceil_div(L, a->B), W = ceil_div(n_kb, 32);
+  const int n_qb = ceil_div(a->Nq, a->B), n_kb = ceil_div(sparse_key_rows(a), a->B),
+            W = ceil_div(n_kb, 32);
   const size_t es = elem_size(a->dtype);
   w.chunk = c.take<int32_t>(1);
   w.cand = c.take<int32_t>(a->n_c);
@@ -618,8 +631,9 @@ StepWs carve_step(Carver& c, const wa_step_args* a) {
     w.k_act = c.take<char>(static_cast<size_t>(L) * cols * es);
     w.v_act = c.take<char>(static_cast<size_t>(L) * cols * es);
     // k block sums of the gathered buffer for selection
-    w.ksum = c.take<double>(static_cast<size_t>(n_kb) * cols);
+    w.ksum = c.take<double>(static_cast<size_t>(ceil_div(L, a->B)) * cols);
   }
+  if (a->k_cur) w.cur_sum = c.take<double>(static_cast<size_t>(ceil_div(a->Nq, a->B)) * cols);
   return w;
 }
 
@@ -656,7 +670,7 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
   mark(0);
   const int cols = a->H * a->d;
   const int L = a->K_p * a->T_p;
-  const int n_qb = ceil_div(a->Nq, a->B), n_kb = ceil_div(L, a->B), W = ceil_div(n_kb, 32);
+  const int n_kb = ceil_div(sparse_key_rows(a), a->B);
 
   // S0: candidate chunk
   int32_t* chunk = a->chunk_out ? a->chunk_out : w.chunk;
@@ -699,6 +713,13 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
                                nullptr, rowsum_plan(1, L, cols, a->B, a->dtype), err, st));
     km.data = w.ksum;
   }
+  if (a->k_cur) {
+    // intra-chunk keys: the chunk's own K/V follow the history in the sparse branch
+    rs.k2 = a->k_cur; rs.v2 = a->v_cur; rs.L2 = a->Nq;
+    WA_TRY(launch_rowblock_sum(a->k_cur, a->dtype, nullptr, 1, 1, a->Nq, cols, a->B, w.cur_sum,
+                               nullptr, nullptr, rowsum_plan(1, a->Nq, cols, a->B, a->dtype), err, st));
+    km.data2 = w.cur_sum; km.n_kb1 = L / a->B; km.L2 = a->Nq;
+  }
 
   mark(2);
   uint32_t* mask = a->blk_mask_out ? a->blk_mask_out : w.mask;
@@ -729,7 +750,7 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
     WA_TRY(launch_block_select(w.ps.q_blockmean, a->Nq, a->H, a->d, a->B, km, n_kb, a->tau, w.scores,
                                nullptr, nullptr, mask, st));
     mark(3);
-    WA_TRY(launch_attn_worklist(a->Nq, a->H, a->d, a->B, L, mask, w.attn, st));
+    WA_TRY(launch_attn_worklist(a->Nq, a->H, a->d, a->B, sparse_key_rows(a), mask, w.attn, st));
     cudaStreamWaitEvent(st, side->join, 0);
     mark(6);
     // S5 + S6

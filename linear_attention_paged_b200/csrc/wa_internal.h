@@ -21,6 +21,12 @@ struct RowSource {
   int page_rows = 0;                  // T_p (paged) or L (contiguous)
   int n_pages = 1;                    // pool pages addressable from k / v
   int L = 0;                          // rows of the active sequence
+  // optional second segment (the current chunk's own keys and values): rows
+  // [L, L + L2) of the key sequence, contiguous [L2][H][d]; L is then a multiple of
+  // the block size, so no block straddles the two segments
+  const void* k2 = nullptr;
+  const void* v2 = nullptr;
+  int L2 = 0;
 };
 
 // Status of an internal launch: WA_OK or WA_ERR_CUDA with a message set.
@@ -79,6 +85,11 @@ struct KeyMeans {
   int nbp = 0;                    // blocks per page (when page_pos != nullptr)
   int is_sum = 0;                 // data holds sums: divide by the block's row count
   int L = 0;                      // rows of the key sequence (for ragged counts)
+  // optional second segment: blocks j >= n_kb1 read fp64 sums data2[j - n_kb1],
+  // over L2 rows
+  const double* data2 = nullptr;
+  int n_kb1 = 0;
+  int L2 = 0;
 };
 // S3: float64 pooled block scores into `scores` [H][n_qb][n_kb], then per (head,
 // query block) the shortest descending prefix reaching tau_h.

@@ -53,6 +53,7 @@ class StepArgs(ctypes.Structure):
         ("stage_events", P),
         ("page_index", P),
         ("gate_lin", P),
+        ("k_cur", P), ("v_cur", P),
     ]
 
 
@@ -303,8 +304,10 @@ class HSAStep:
 
     def __init__(self, q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 4,
                  B: int = 64, e_cur=None, e_chunks=None, fused_gather: bool = True,
-                 keep_intermediates: bool = False, out=None, page_index=None, gate_lin=None):
-        _need_cuda(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, e_cur, e_chunks, gate_lin)
+                 keep_intermediates: bool = False, out=None, page_index=None, gate_lin=None,
+                 k_cur=None, v_cur=None):
+        _need_cuda(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, e_cur, e_chunks, gate_lin,
+                   k_cur, v_cur)
         Nq, H, d = q.shape
         P_, T_p = k_pool.shape[0], k_pool.shape[1]
         if chunk_pages.dim() == 1:
@@ -312,7 +315,7 @@ class HSAStep:
         n_chunks, n_c = chunk_pages.shape
         r = e_k.shape[1]
         L = K_p * T_p
-        n_qb, n_kb = -(-Nq // B), -(-L // B)
+        n_qb, n_kb = -(-Nq // B), -(-(L + (Nq if k_cur is not None else 0)) // B)
         W = -(-n_kb // 32)
         dev = q.device
         self.out = out if out is not None else torch.empty_like(q)
@@ -330,7 +333,8 @@ class HSAStep:
         a.out = _p(self.out)
         a.page_index = _p(page_index)
         a.gate_lin = _p(gate_lin)
-        self._keep += [page_index, gate_lin]
+        a.k_cur, a.v_cur = _p(k_cur), _p(v_cur)
+        self._keep += [page_index, gate_lin, k_cur, v_cur]
         self.inter = {}
         if keep_intermediates:
             self.inter = dict(
@@ -363,10 +367,11 @@ class HSAStep:
 
 def wa_hsa_step(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 4, B: int = 64,
                 e_cur=None, e_chunks=None, fused_gather: bool = True, keep_intermediates: bool = False,
-                stream=None, page_index=None, gate_lin=None):
+                stream=None, page_index=None, gate_lin=None, k_cur=None, v_cur=None):
     """One HSA decode step; returns ``out`` (and the intermediates when asked)."""
     st = HSAStep(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p, B, e_cur, e_chunks,
-                 fused_gather, keep_intermediates, page_index=page_index, gate_lin=gate_lin)
+                 fused_gather, keep_intermediates, page_index=page_index, gate_lin=gate_lin,
+                 k_cur=k_cur, v_cur=v_cur)
     out = st(stream)
     return (out, st.inter) if keep_intermediates else out
 

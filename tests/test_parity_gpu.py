@@ -280,12 +280,18 @@ def test_hsa_step_small(wa, cfg, fused):
     check_device_ok(wa)
 
 
+def sparse_blocks(cfg):
+    """Key blocks of the sparse branch: the history, plus the chunk's own with intra keys."""
+    return -(-(cfg.L + (cfg.Nq if cfg.intra else 0)) // cfg.B)
+
+
 def _full_size_step(wa, cfg, samples, gen_device="cuda"):
     inp = W.make_inputs(cfg, device="cuda", gen_device=gen_device)
     e_cur = inp.get("e_cur")
     step = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"], inp["e_v"],
                       inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B, e_cur=e_cur,
-                      e_chunks=inp.get("e_chunks"), fused_gather=True, keep_intermediates=True)
+                      e_chunks=inp.get("e_chunks"), fused_gather=True, keep_intermediates=True,
+                      k_cur=inp.get("k_cur"), v_cur=inp.get("v_cur"))
     out = step()
     torch.cuda.synchronize()
     res = O.hsa_step(inp, cfg.B, cfg.K_p, rows_of_blocks=samples)
@@ -294,9 +300,10 @@ def _full_size_step(wa, cfg, samples, gen_device="cuda"):
     np.testing.assert_allclose(to64(step.inter["alpha"]), res["alpha"], rtol=1e-9, atol=1e-13)
     if res["page_margin"] >= 1e-5:
         assert step.inter["sel"].cpu().tolist() == res["sel"]
-    compare_selection(mask_to_sets(step.inter["blk_mask"], cfg.n_kb), res["kept"], res["block_margin"],
+    n_kb = sparse_blocks(cfg)
+    compare_selection(mask_to_sets(step.inter["blk_mask"], n_kb), res["kept"], res["block_margin"],
                       f"{cfg.name} masks")
-    print(f"[info] {cfg.name} kept fraction per head: {np.round(kept_fraction(res['kept'], cfg.n_kb), 3)}")
+    print(f"[info] {cfg.name} kept fraction per head: {np.round(kept_fraction(res['kept'], n_kb), 3)}")
     assert_close(step.inter["k_til"], res["k_til"], "bf16", f"{cfg.name} K~")
     assert_close(step.inter["v_til"], res["v_til"], "bf16", f"{cfg.name} V~")
     for (h, i), blk in res["blocks"].items():
@@ -310,6 +317,34 @@ def test_full_size_layer_step(wa):
     n_qb = cfg.n_qb
     samples = [(0, 0), (11, n_qb - 1), (5, 37), (3, n_qb - 2), (8, 12), (11, 0)]
     _full_size_step(wa, cfg, samples)
+
+
+def test_full_size_layer_step_intra_keys(wa):
+    """C1 with the current chunk's own K/V in the sparse branch (780 + 74 key blocks,
+    the last one 8 rows)."""
+    cfg = W.C1.with_(name="c1_intra", intra=True)
+    samples = [(0, 0), (11, cfg.n_qb - 1), (4, 30), (9, 60)]
+    _full_size_step(wa, cfg, samples)
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "gathered"])
+@pytest.mark.parametrize("cfg", [SMALL_BF16, SMALL_BF16_D64, SMALL_F32], ids=lambda c: c.name)
+def test_hsa_step_intra_keys_small(wa, cfg, fused):
+    cfg = cfg.with_(intra=True)
+    inp = inputs(cfg)
+    out, inter = wa.wa_hsa_step(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"],
+                                inp["e_v"], inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B,
+                                fused_gather=fused, keep_intermediates=True, k_cur=inp["k_cur"],
+                                v_cur=inp["v_cur"])
+    res = O.hsa_step(inp, cfg.B, cfg.K_p)
+    n_kb = sparse_blocks(cfg)
+    assert inter["blk_mask"].shape[-1] == -(-n_kb // 32)
+    compare_selection(mask_to_sets(inter["blk_mask"], n_kb), res["kept"], res["block_margin"],
+                      f"{cfg.name} intra masks")
+    chunk_kept = sum(1 for h in res["kept"] for row in h for j in row if j >= cfg.L // cfg.B)
+    assert chunk_kept > 0, "no chunk block kept: the case would not test the second segment"
+    assert_close(out, res["o"], dkey(cfg), f"{cfg.name} step O with intra keys ({'fused' if fused else 'gathered'})")
+    check_device_ok(wa)
 
 
 def test_full_size_stress_step(wa):
