@@ -275,7 +275,7 @@ def run_ours(args, rank, world, local_rank):
     # per step: pick_chunk, Q row sums, query means, candidate-page row sums, alpha/top-k,
     # block scores, block choice, pairing, work items, sparse attention, combine on the
     # caller's stream; projection, split reduction, linear branch on the side stream
-    launches_per_step = 14
+    launches_per_step = 14 + (1 if cfg.intra else 0)   # + block sums of the chunk's keys
 
     n_ev = 8  # WA_STEP_EVENTS
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
@@ -383,7 +383,7 @@ def run_ours(args, rank, world, local_rank):
             "roofline": {"bound": "tensor", "achieved": achieved_t, "peak": peak_t, "unit": "TFLOP/s",
                          "frac": achieved_t / peak_t,
                          "traffic": (ATTN_DRAM_BYTES_PER_HEAD * cfg.H
-                                     if ATTN_DRAM_BYTES_PER_HEAD is not None else None),
+                                     if ATTN_DRAM_BYTES_PER_HEAD is not None and not cfg.intra else None),
                          "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of the "
                                            "6-head launch (profiles/k_umma_attention_sparse_h6.md), "
                                            "scaled by heads",
