@@ -314,6 +314,57 @@ typedef struct wa_step_args {
   const void* v_cur;
 } wa_step_args;
 
+/* ---------------------------------------------------------------------------
+ * L1 <-> L2 page tiering (WorldAttention §3.2, "Hierarchical KV Cache": pages that
+ * are not active leave GPU memory for CPU DRAM by LRU and return on demand; pages
+ * predicted to be needed are prefetched asynchronously).
+ *
+ * A tier owns no memory.  The caller gives
+ *   slot_k, slot_v  device pool of n_slots page slots, [n_slots][page_bytes] each
+ *                   (the L1 tier; a step uses it as its k_pool / v_pool)
+ *   host_k, host_v  pinned host memory (cudaHostAlloc) holding every page,
+ *                   [n_pages][page_bytes] each (the L2 tier)
+ * and keeps all four alive until wa_tier_destroy.  With all four NULL the tier only
+ * keeps the books (page -> slot map, LRU order, dirty bits, statistics), with no
+ * copies.  One caller stream should be used for a tier's ensure / release / flush
+ * calls and for the kernels that read its slots.
+ *
+ *   wa_tier_ensure    makes `pages` resident and writes their slots to slots_out
+ *                     (host array of n).  Misses are filled in order on `stream`:
+ *                     a free slot if any, else the least recently handed-out slot
+ *                     not in this request; a dirty victim is first written back to
+ *                     its host page.  A page whose prefetch is in flight makes
+ *                     `stream` wait for it.  More distinct pages than slots is
+ *                     WA_ERR_INVALID_ARG.
+ *   wa_tier_release   the work that reads every slot handed out so far has been
+ *                     enqueued on `stream`: those slots may now be evicted by
+ *                     prefetches (which wait on this point of `stream`).
+ *   wa_tier_prefetch  loads the non-resident `pages` on the tier's own stream into
+ *                     free slots or released LRU slots; a hint: it stops when no
+ *                     slot qualifies.  *issued (nullable) = pages started.
+ *   wa_tier_mark_dirty  the resident `page` was written on the device (an appended
+ *                     chunk): it is written back when evicted or flushed.
+ *   wa_tier_flush     writes every dirty resident page back on `stream`.
+ *   wa_tier_slot_of   the slot of `page`, or -1.
+ * Errors: WA_ERR_INVALID_ARG (bad ids, sizes, NULL), WA_ERR_CUDA (a copy or event
+ * call failed). */
+typedef struct wa_tier wa_tier;
+typedef struct wa_tier_stats {
+  long long hits, misses, prefetch_hits, prefetches, evictions, writebacks;
+  long long bytes_h2d, bytes_d2h;
+} wa_tier_stats;
+WA_API wa_status wa_tier_create(int n_pages, int n_slots, size_t page_bytes, void* host_k,
+                                void* host_v, void* slot_k, void* slot_v, wa_tier** out);
+WA_API wa_status wa_tier_destroy(wa_tier* t);
+WA_API wa_status wa_tier_ensure(wa_tier* t, const int32_t* pages, int n, int32_t* slots_out,
+                                void* stream);
+WA_API wa_status wa_tier_release(wa_tier* t, void* stream);
+WA_API wa_status wa_tier_prefetch(wa_tier* t, const int32_t* pages, int n, int* issued);
+WA_API wa_status wa_tier_mark_dirty(wa_tier* t, int32_t page);
+WA_API wa_status wa_tier_flush(wa_tier* t, void* stream);
+WA_API wa_status wa_tier_slot_of(wa_tier* t, int32_t page, int32_t* slot);
+WA_API wa_status wa_tier_get_stats(wa_tier* t, wa_tier_stats* out);
+
 /* Stage boundaries recorded into wa_step_args.stage_events:
  *   0 start | 1 after S0+S1 (page retrieval) | 2 after S2 (gather; = 1 when fused)
  *   3 after S3 (block selection) | 4 after S4a (projection) | 5 after S4b (linear

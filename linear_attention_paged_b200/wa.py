@@ -83,6 +83,15 @@ _SIGS = {
                                P, c_int, P]),
     "wa_hsa_step_workspace_size": (c_size_t, [ctypes.POINTER(StepArgs)]),
     "wa_hsa_step": (c_int, [ctypes.POINTER(StepArgs), P, c_size_t, P]),
+    "wa_tier_create": (c_int, [c_int, c_int, c_size_t, P, P, P, P, P]),
+    "wa_tier_destroy": (c_int, [P]),
+    "wa_tier_ensure": (c_int, [P, P, c_int, P, P]),
+    "wa_tier_release": (c_int, [P, P]),
+    "wa_tier_prefetch": (c_int, [P, P, c_int, P]),
+    "wa_tier_mark_dirty": (c_int, [P, c_int]),
+    "wa_tier_flush": (c_int, [P, P]),
+    "wa_tier_slot_of": (c_int, [P, c_int, P]),
+    "wa_tier_get_stats": (c_int, [P, P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -381,3 +390,87 @@ def wa_device_error(stream=None) -> int:
     flags = ctypes.c_uint32(0)
     lib.wa_device_error(_stream(stream), ctypes.byref(flags))
     return int(flags.value)
+
+
+# --------------------------------------------------------------------- L1 <-> L2 tiering
+class TierStats(ctypes.Structure):
+    """Mirror of ``wa_tier_stats``."""
+    _fields_ = [(n, ctypes.c_longlong) for n in
+                ("hits", "misses", "prefetch_hits", "prefetches", "evictions", "writebacks",
+                 "bytes_h2d", "bytes_d2h")]
+
+
+class Tier:
+    """A page tier over a device slot pool and pinned host pages (see wa_tier_* in
+    include/wa.h).  ``host_k``/``host_v`` are pinned CPU tensors [n_pages][...] and
+    ``slot_k``/``slot_v`` device tensors [n_slots][...] of the same page shape; with
+    none of them the tier only keeps the books (``n_pages``, ``n_slots`` given)."""
+
+    def __init__(self, host_k=None, host_v=None, slot_k=None, slot_v=None, n_pages=None,
+                 n_slots=None, page_bytes=None):
+        bufs = (host_k, host_v, slot_k, slot_v)
+        self.books = all(b is None for b in bufs)
+        if self.books:
+            self._keep = ()
+            ptrs = (None,) * 4
+        else:
+            assert host_k.is_pinned() and host_v.is_pinned()
+            _need_cuda(slot_k, slot_v)
+            n_pages, n_slots = host_k.shape[0], slot_k.shape[0]
+            page_bytes = host_k[0].numel() * host_k.element_size()
+            assert slot_k[0].numel() * slot_k.element_size() == page_bytes
+            for b in bufs:
+                assert b.is_contiguous()
+            self._keep = bufs
+            ptrs = tuple(_p(b) for b in bufs)
+        self.n_pages, self.n_slots = n_pages, n_slots
+        h = ctypes.c_void_p()
+        _check("wa_tier_create", lib.wa_tier_create(n_pages, n_slots, page_bytes or 1, *ptrs,
+                                                    ctypes.byref(h)))
+        self.h = h
+
+    def _st(self, stream):
+        return None if self.books else _stream(stream)
+
+    def ensure(self, pages, stream=None):
+        ids = (ctypes.c_int32 * len(pages))(*[int(p) for p in pages])
+        out = (ctypes.c_int32 * len(pages))()
+        st = self._st(stream)
+        _check("wa_tier_ensure", lib.wa_tier_ensure(self.h, ids, len(pages), out, st))
+        return list(out)
+
+    def release(self, stream=None):
+        _check("wa_tier_release", lib.wa_tier_release(self.h, self._st(stream)))
+
+    def prefetch(self, pages) -> int:
+        ids = (ctypes.c_int32 * len(pages))(*[int(p) for p in pages])
+        n = ctypes.c_int(0)
+        _check("wa_tier_prefetch", lib.wa_tier_prefetch(self.h, ids, len(pages), ctypes.byref(n)))
+        return int(n.value)
+
+    def mark_dirty(self, page: int):
+        _check("wa_tier_mark_dirty", lib.wa_tier_mark_dirty(self.h, int(page)))
+
+    def flush(self, stream=None):
+        _check("wa_tier_flush", lib.wa_tier_flush(self.h, self._st(stream)))
+
+    def slot_of(self, page: int) -> int:
+        s = ctypes.c_int32(0)
+        _check("wa_tier_slot_of", lib.wa_tier_slot_of(self.h, int(page), ctypes.byref(s)))
+        return int(s.value)
+
+    def stats(self) -> dict:
+        st = TierStats()
+        _check("wa_tier_get_stats", lib.wa_tier_get_stats(self.h, ctypes.byref(st)))
+        return {n: int(getattr(st, n)) for n, _ in TierStats._fields_}
+
+    def close(self):
+        if getattr(self, "h", None):
+            lib.wa_tier_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
