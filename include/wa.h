@@ -315,6 +315,30 @@ typedef struct wa_step_args {
 } wa_step_args;
 
 /* ---------------------------------------------------------------------------
+ * A decode-step pipeline over host buffers (no counterpart in the pages: serving
+ * plumbing).  Each submit uploads q and the gate logits from host memory, runs
+ * wa_hsa_step and downloads out, on three streams so that step k+1's upload and step
+ * k-1's download overlap step k.  Two device sets of (q, gate, out) alternate: set 0
+ * is a->q / a->gate / a->out, set 1 is q1 / gate1 / out1 (same shapes).  Every
+ * other field of *a (pool, E, tau, optional inputs) is copied once and used by every
+ * step; ws (wa_hsa_step_workspace_size(a) bytes) is shared by the steps, which run in
+ * order on `stream`.  Host buffers should be pinned for the copies to be
+ * asynchronous; inputs must stay unchanged and outputs unread until wa_pipe_sync (or
+ * work ordered after wa_pipe_end on `stream`).
+ *   wa_pipe_begin   later copies wait for everything enqueued on `stream` so far
+ *   wa_pipe_end     `stream` waits for every copy submitted so far
+ *   wa_pipe_sync    waits on the host for everything submitted */
+typedef struct wa_pipe wa_pipe;
+WA_API wa_status wa_pipe_create(const wa_step_args* a, void* q1, const float* gate1, void* out1,
+                                void* ws, size_t ws_bytes, void* stream, wa_pipe** out);
+WA_API wa_status wa_pipe_destroy(wa_pipe* p);
+WA_API wa_status wa_pipe_begin(wa_pipe* p);
+WA_API wa_status wa_pipe_submit(wa_pipe* p, const void* q_host, const float* gate_host,
+                                void* out_host);
+WA_API wa_status wa_pipe_end(wa_pipe* p);
+WA_API wa_status wa_pipe_sync(wa_pipe* p);
+
+/* ---------------------------------------------------------------------------
  * L1 <-> L2 page tiering (WorldAttention §3.2, "Hierarchical KV Cache": pages that
  * are not active leave GPU memory for CPU DRAM by LRU and return on demand; pages
  * predicted to be needed are prefetched asynchronously).

@@ -83,6 +83,12 @@ _SIGS = {
                                P, c_int, P]),
     "wa_hsa_step_workspace_size": (c_size_t, [ctypes.POINTER(StepArgs)]),
     "wa_hsa_step": (c_int, [ctypes.POINTER(StepArgs), P, c_size_t, P]),
+    "wa_pipe_create": (c_int, [ctypes.POINTER(StepArgs), P, P, P, P, c_size_t, P, P]),
+    "wa_pipe_destroy": (c_int, [P]),
+    "wa_pipe_begin": (c_int, [P]),
+    "wa_pipe_submit": (c_int, [P, P, P, P]),
+    "wa_pipe_end": (c_int, [P]),
+    "wa_pipe_sync": (c_int, [P]),
     "wa_tier_create": (c_int, [c_int, c_int, c_size_t, P, P, P, P, P]),
     "wa_tier_destroy": (c_int, [P]),
     "wa_tier_ensure": (c_int, [P, P, c_int, P, P]),
@@ -467,6 +473,51 @@ class Tier:
     def close(self):
         if getattr(self, "h", None):
             lib.wa_tier_destroy(self.h)
+            self.h = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+# --------------------------------------------------------------------- host-buffer pipeline
+class HSAPipeline:
+    """Steps over host buffers with uploads and downloads overlapping the compute
+    (wa_pipe_* in include/wa.h).  Built on a prepared HSAStep, whose q, gate and out
+    are the first device set; the second set is allocated here."""
+
+    def __init__(self, step: "HSAStep", q, gate, stream=None):
+        self.step = step
+        self.q1, self.g1 = torch.empty_like(q), torch.empty_like(gate)
+        self.o1 = torch.empty_like(step.out)
+        self.stream = stream if stream is not None else torch.cuda.current_stream()
+        h = ctypes.c_void_p()
+        _check("wa_pipe_create", lib.wa_pipe_create(ctypes.byref(step.args), _p(self.q1), _p(self.g1),
+                                                    _p(self.o1), _p(step.ws), step.nbytes,
+                                                    _stream(self.stream), ctypes.byref(h)))
+        self.h = h
+
+    def begin(self):
+        _check("wa_pipe_begin", lib.wa_pipe_begin(self.h))
+
+    def submit(self, q_host, gate_host, out_host):
+        for t in (q_host, gate_host, out_host):
+            assert t.device.type == "cpu" and t.is_contiguous()
+        _check("wa_pipe_submit", lib.wa_pipe_submit(self.h, ctypes.c_void_p(q_host.data_ptr()),
+                                                    ctypes.c_void_p(gate_host.data_ptr()),
+                                                    ctypes.c_void_p(out_host.data_ptr())))
+
+    def end(self):
+        _check("wa_pipe_end", lib.wa_pipe_end(self.h))
+
+    def sync(self):
+        _check("wa_pipe_sync", lib.wa_pipe_sync(self.h))
+
+    def close(self):
+        if getattr(self, "h", None):
+            lib.wa_pipe_destroy(self.h)
             self.h = None
 
     def __del__(self):

@@ -96,3 +96,32 @@ def test_step_over_the_slot_pool_matches_the_full_pool(wa):
         assert torch.equal(full, via), f"chunk {chunk}: step over the slot pool differs"
     assert wa.wa_device_error() == 0
     t.close()
+
+
+def test_pipeline_over_host_buffers_matches_direct_steps(wa):
+    """Steps submitted through the host-buffer pipeline (double-buffered device sets,
+    overlapped copies) give the same bits as direct steps on the same inputs."""
+    cfg = W.HSAConfig("pipe_small", H=2, d=128, T_p=1280, n_c=6, Nq=520, K_p=3, B=64, r=128,
+                      dtype="bf16", seed=33, recipe="offset")
+    inp = W.make_inputs(cfg, device="cuda")
+    tau = inp["tau"].cuda()
+    step = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"], inp["e_v"],
+                      tau, inp["gate"], cfg.K_p, cfg.B)
+    g = torch.Generator().manual_seed(4)
+    n = 5
+    qs = [(torch.randn(inp["q"].shape, generator=g) / cfg.d ** 0.5).to(torch.bfloat16).pin_memory()
+          for _ in range(n)]
+    gs = [torch.randn(inp["gate"].shape, generator=g).pin_memory() for _ in range(n)]
+    outs = [torch.empty(inp["q"].shape, dtype=torch.bfloat16).pin_memory() for _ in range(n)]
+    pipe = wa.HSAPipeline(step, inp["q"], inp["gate"])
+    pipe.begin()
+    for k in range(n):
+        pipe.submit(qs[k], gs[k], outs[k])
+    pipe.end()
+    pipe.sync()
+    pipe.close()
+    for k in range(n):
+        ref = wa.wa_hsa_step(qs[k].cuda(), inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"],
+                             inp["e_v"], tau, gs[k].cuda(), cfg.K_p, cfg.B)
+        assert torch.equal(outs[k], ref.cpu()), f"pipelined step {k} differs"
+    assert wa.wa_device_error() == 0
