@@ -507,7 +507,7 @@ k_index_dot(const double* __restrict__ page_index, const int32_t* __restrict__ c
             uint32_t* err) {
   __shared__ double red[32];
   const int b = blockIdx.x, c = blockIdx.y;
-  int page = cand[c];
+  int page = cand ? cand[c] : c;   // no cand: rows are indexed by candidate position
   if (page < 0 || page >= n_pages) {
     if (threadIdx.x == 0) atomicOr(err, WA_DEVERR_PAGE_ID);
     page = 0;

@@ -201,6 +201,26 @@ wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int
   const int cols = H * d;
   uint32_t* err = errw();
   if (!err) return set_error(WA_ERR_CUDA, "no device error word (is a CUDA device present?)");
+  if (!page_index && w.k_blocksum) {
+    // The candidate pages' block sums are kept for selection anyway, so the page
+    // scores come from them after the pass; the query pass and query means then run
+    // on the side stream during the (larger) candidate pass instead of before it.
+    SideStream* side = nullptr;
+    WA_TRY(side_stream(&side));
+    cudaEventRecord(side->fork, st);
+    cudaStreamWaitEvent(side->stream, side->fork, 0);
+    WA_TRY(launch_rowblock_sum(q, dt, nullptr, 1, 1, Nq, cols, B, w.q_blocksum, nullptr, nullptr, w.qp,
+                               err, side->stream));
+    WA_TRY(launch_qmeans(w.q_blocksum, ceil_div(Nq, B), Nq, B, cols, w.qbar, w.q_blockmean,
+                         side->stream));
+    cudaEventRecord(side->join, side->stream);
+    WA_TRY(launch_rowblock_sum(k_pool, dt, cand, n_c, n_pool_pages, T_p, cols, B, w.k_blocksum,
+                               nullptr, nullptr, w.kp, err, st));
+    cudaStreamWaitEvent(st, side->join, 0);
+    const int nbp = ceil_div(T_p, B);
+    WA_TRY(launch_index_dot(w.k_blocksum, nullptr, n_c, n_c, nbp, cols, w.qbar, w.kdot, err, st));
+    return launch_alpha_topk(w.kdot, nbp, n_c, T_p, H, d, K_p, cand, alpha, sel, sel_pos, st);
+  }
   WA_TRY(launch_rowblock_sum(q, dt, nullptr, 1, 1, Nq, cols, B, w.q_blocksum, nullptr, nullptr, w.qp,
                              err, st));
   WA_TRY(launch_qmeans(w.q_blocksum, ceil_div(Nq, B), Nq, B, cols, w.qbar, w.q_blockmean, st));

@@ -57,7 +57,8 @@ struct RowsumPlan {
 RowsumPlan rowsum_plan(int n_src, int rows, int cols, int B, wa_dtype dt);
 // Plan over blocks [block0, block0 + n_blocks) of one source of `rows` rows.
 RowsumPlan rowsum_plan_range(int rows, int cols, int B, wa_dtype dt, int block0, int n_blocks);
-// kdot[c][b] = qbar . page_index[cand[c]][b] (page scores from the page index).
+// kdot[c][b] = qbar . page_index[cand[c]][b] (page scores from the page index);
+// cand == nullptr reads row c (block sums indexed by candidate position).
 wa_status launch_index_dot(const double* page_index, const int32_t* cand, int n_c, int n_pages,
                            int nbp, int cols, const double* qbar, double* kdot, uint32_t* err,
                            cudaStream_t st);
