@@ -272,10 +272,11 @@ def run_ours(args, rank, world, local_rank):
     if flags:
         raise RuntimeError(f"device error flags 0x{flags:x}")
     flops, kept_frac = selected_flops(step.inter["blk_mask"], cfg)
-    # per step: pick_chunk, Q row sums, query means, candidate-page row sums, alpha/top-k,
-    # block scores, block choice, pairing, work items, sparse attention, combine on the
-    # caller's stream; projection, split reduction, linear branch on the side stream
-    launches_per_step = 14 + (1 if cfg.intra else 0)   # + block sums of the chunk's keys
+    # per step: pick_chunk, candidate-page row sums, page-score dots, alpha/top-k, block
+    # scores, block choice, pairing, work items, sparse attention, combine on the
+    # caller's stream; query row sums and means, then projection, split reduction and
+    # linear branch on the side stream
+    launches_per_step = 15 + (1 if cfg.intra else 0)   # + block sums of the chunk's keys
 
     n_ev = 8  # WA_STEP_EVENTS
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]

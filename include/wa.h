@@ -314,6 +314,17 @@ typedef struct wa_step_args {
   const void* v_cur;
 } wa_step_args;
 
+/* Stage boundaries recorded into wa_step_args.stage_events:
+ *   0 start | 1 after S0+S1 (page retrieval) | 2 after S2 (gather; = 1 when fused)
+ *   3 after S3 (block selection) | 4 after S4a (projection) | 5 after S4b (linear
+ *   branch) | 6 after the work list | 7 after S5+S6 (sparse branch + gate).
+ * With bf16 inputs S4a and S4b run on a second stream that forks after event 2 and
+ * joins before event 6, so events 4 and 5 are recorded on that stream. */
+#define WA_STEP_EVENTS 8
+
+WA_API size_t wa_hsa_step_workspace_size(const wa_step_args* a);
+WA_API wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------
  * A decode-step pipeline over host buffers (no counterpart in the pages: serving
  * plumbing).  Each submit uploads q and the gate logits from host memory, runs
@@ -388,17 +399,6 @@ WA_API wa_status wa_tier_mark_dirty(wa_tier* t, int32_t page);
 WA_API wa_status wa_tier_flush(wa_tier* t, void* stream);
 WA_API wa_status wa_tier_slot_of(wa_tier* t, int32_t page, int32_t* slot);
 WA_API wa_status wa_tier_get_stats(wa_tier* t, wa_tier_stats* out);
-
-/* Stage boundaries recorded into wa_step_args.stage_events:
- *   0 start | 1 after S0+S1 (page retrieval) | 2 after S2 (gather; = 1 when fused)
- *   3 after S3 (block selection) | 4 after S4a (projection) | 5 after S4b (linear
- *   branch) | 6 after the work list | 7 after S5+S6 (sparse branch + gate).
- * With bf16 inputs S4a and S4b run on a second stream that forks after event 2 and
- * joins before event 6, so events 4 and 5 are recorded on that stream. */
-#define WA_STEP_EVENTS 8
-
-WA_API size_t wa_hsa_step_workspace_size(const wa_step_args* a);
-WA_API wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* stream);
 
 #ifdef __cplusplus
 }  /* extern "C" */
