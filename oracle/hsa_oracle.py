@@ -11,12 +11,12 @@ Each function follows one step of the method as the WorldAttention pages state i
 
   S0 prompt_select      -- §3.2 "Stage 1: prompt-level retrieval" (cosine top-1 chunk)
   S1 page_scores /      -- §3.2 "Stage 2: page-level retrieval", the alpha_{m,j} equation
-     select_pages          and "top-K_p pages"
-  S2 gather_pages       -- §3.2 "Active KV construction"; summary step (4) "concatenate
-                           the selected pages into K_active, V_active"
+     select_pages          and the top-K_p choice of pages
+  S2 gather_pages       -- §3.2 "Active KV construction"; summary step (4): the chosen
+                           pages joined into K_active, V_active
   S3 block_select       -- §3.3 "Head-level sparsity adaptation" (minimal block set whose
-                           cumulative mass reaches tau_h); summary step (5) "block pooling
-                           coarse selection"
+                           cumulative mass reaches tau_h); summary step (5), coarse
+                           selection over pooled blocks
   S4 linear_project /   -- §3.3 "Linear branch", the O_lin equation with
      linear_attention      K~ = E_K^T K, V~ = E_V^T V (Linformer projection)
   S5 sparse_attention   -- §3.3 "Sparse branch"; Appendix A.1.3 block-sparse attention
@@ -29,13 +29,14 @@ Readings where the pages are silent (each one is listed in the design notes):
     giving one page set per layer (one shared 49,920-token active buffer).
   * The chosen pages are concatenated in ascending candidate position.
   * Ties in any ranking go to the lower index.
-  * "exceeds tau_h" is read as ">= tau_h"; tau_h >= 1 keeps every block, and so does a
-    row whose cumulative mass never reaches tau_h.
+  * The mass condition is read as ">= tau_h"; tau_h >= 1 keeps every block, and so
+    does a row whose cumulative mass never reaches tau_h.
   * Block pooling is the mean over the valid rows of a block; a block's score is
     q-bar . k-bar / sqrt(d); the mass is the softmax of one (head, query block) row.
   * E_K, E_V are shared by all heads, shape [L][r]; no extra scaling.
-  * Keys of both branches are the retrieved history only; no causal mask.
-  * O = sigmoid(g) * O_sp + (1 - sigmoid(g)) * O_lin, per token and head.
+  * Keys of both branches are the retrieved history; with k_cur/v_cur the sparse
+    branch also takes the current chunk's own keys (after the history); no causal mask.
+  * O = sigmoid(g) * O_sp + (1 - sigmoid(g)) * O_lin, per token and head (or two gates).
 """
 from __future__ import annotations
 
