@@ -149,11 +149,13 @@ def oracle_sample(inp, cfg, n_blocks=2, head_frac=1, l_slices=8, seed=0):
     t = {}
     t0 = time.perf_counter()
     cand = [int(x) for x in inp["cand"]]
-    k_cand = np.stack([O.f64(inp["k_pool"][p]) for p in cand])
+    # page scores over 1/l_slices of every candidate page's rows: same cost per row
+    Ts = cfg.T_p // l_slices
+    k_cand = np.stack([O.f64(inp["k_pool"][p][:Ts]) for p in cand])
     alpha = O.page_scores(inp["q"], k_cand)
     sel = [cand[j] for j in O.select_pages(alpha, cfg.K_p)]
     del k_cand
-    t["page_retrieval"] = time.perf_counter() - t0
+    t["page_retrieval"] = (time.perf_counter() - t0) * l_slices
     t0 = time.perf_counter()
     k_act = O.gather_pages(inp["k_pool"], sel)
     v_act = O.gather_pages(inp["v_pool"], sel)
@@ -176,7 +178,8 @@ def oracle_sample(inp, cfg, n_blocks=2, head_frac=1, l_slices=8, seed=0):
         O.linear_attention(O.f64(inp["q"][r0:r1, h:h + 1]), kt[:, h:h + 1], vt[:, h:h + 1])
     t["attention"] = (time.perf_counter() - t0) / n_blocks * cfg.H * cfg.n_qb
     total = sum(t.values())
-    desc = (f"fp64 numpy oracle on a bounded sample of one step: page scores in full, block "
+    desc = (f"fp64 numpy oracle on a bounded sample of one step: page scores on T_p/{l_slices} rows "
+            f"of each candidate page (x{l_slices}), block "
             f"selection for 1 of {cfg.H} heads (x{cfg.H}), projection on L/{l_slices} (x{l_slices}), "
             f"both branches for {n_blocks} of {cfg.H * cfg.n_qb} (head, query block) pairs "
             f"(x{cfg.H * cfg.n_qb // n_blocks}); per-step time extrapolated")
