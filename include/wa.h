@@ -338,7 +338,8 @@ WA_API wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, v
  * work ordered after wa_pipe_end on `stream`).
  *   wa_pipe_begin   later copies wait for everything enqueued on `stream` so far
  *   wa_pipe_end     `stream` waits for every copy submitted so far
- *   wa_pipe_sync    waits on the host for everything submitted */
+ *   wa_pipe_sync    waits on the host for everything submitted
+ * A pipeline is driven from one host thread at a time (it keeps no lock). */
 typedef struct wa_pipe wa_pipe;
 WA_API wa_status wa_pipe_create(const wa_step_args* a, void* q1, const float* gate1, void* out1,
                                 void* ws, size_t ws_bytes, void* stream, wa_pipe** out);
@@ -381,8 +382,9 @@ WA_API wa_status wa_pipe_sync(wa_pipe* p);
  *                     chunk): it is written back when evicted or flushed.
  *   wa_tier_flush     writes every dirty resident page back on `stream`.
  *   wa_tier_slot_of   the slot of `page`, or -1.
- * Errors: WA_ERR_INVALID_ARG (bad ids, sizes, NULL), WA_ERR_CUDA (a copy or event
- * call failed). */
+ * The calls of one tier may come from several host threads (an internal lock
+ * orders them).  Errors: WA_ERR_INVALID_ARG (bad ids, sizes, NULL), WA_ERR_CUDA (a
+ * copy or event call failed). */
 typedef struct wa_tier wa_tier;
 typedef struct wa_tier_stats {
   long long hits, misses, prefetch_hits, prefetches, evictions, writebacks;
