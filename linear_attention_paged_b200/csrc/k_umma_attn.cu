@@ -21,20 +21,19 @@
 // shared memory; an iteration takes two consecutive blocks of the list (128 keys),
 // so S = Q K^T is one M=128, N=128 MMA chain (N=64 chains run at about two thirds of
 // the tensor rate: their operand reads from shared memory dominate).  Roles:
-//   warp 0  loads Q and the K blocks, warp 2 the V blocks (TMA, 128-byte swizzle,
+//   warp 0  loads the K blocks, warp 2 the V blocks (TMA, 128-byte swizzle,
 //           straight from the pool pages through a page table staged in shared
-//           memory) into rings of 128-key slots (3 for K, 2 for V);
-//   warp 1  owns TMEM (two 128-column S/P buffers, two O accumulators) and issues
-//           the S MMAs; warp 3 issues the P V MMAs.  An MMA's issue blocks behind
-//           the one executing, so one issuer waiting for the softmax would idle the
-//           tensor pipe; with two, S of iteration t+1 runs while P V of t waits.
-//           S_t reuses the buffer of iteration t-2 once that iteration's P V MMAs
-//           have completed;
+//           memory) into rings of 128-key slots (3 each);
+//   warp 1  owns TMEM and issues the S MMAs with Q as the TMEM operand (the softmax
+//           warps write the tile's Q rows into TMEM once), so an S MMA reads only K
+//           from shared memory; warp 3 issues the P V MMAs.  TMEM holds one S
+//           buffer, one P buffer, Q and two O accumulators.  S_{t+1} is issued as soon
+//           as the softmax has loaded S_t into registers, so it runs during the
+//           softmax of iteration t; P_t is stored once the P V MMAs of t-1 are done;
 //   warps 4-7 / 8-11  two softmax groups, one per block of the iteration (S columns
 //           0-63 / 64-127), one thread per TMEM lane (query row), each with its own
-//           running max, sum and O accumulator, merged in the epilogue.  P goes
-//           back into the S buffer as bf16; O is rescaled in TMEM only when the
-//           running max grows by more than 2^8.
+//           running max, sum and O accumulator, merged in the epilogue.  O is
+//           rescaled in TMEM only when the running max grows by more than 2^8.
 // Every wait is bounded in time.
 #include <cuda.h>
 #include <cuda_bf16.h>
@@ -54,10 +53,12 @@ constexpr int kBM = 128;          // query rows per tile (two 64-row blocks)
 constexpr int kBN = 64;           // keys per block
 constexpr int kIterKeys = 128;    // keys per iteration: two blocks of the tile's list
 constexpr int kRingK = 3;         // 128-key slots of the K ring
-constexpr int kRingV = 2;         // 128-key slots of the V ring
+constexpr int kRingV = 3;         // 128-key slots of the V ring
 constexpr int kThreads = 384;     // warps 0-3: loads and MMA; 4-7 and 8-11: softmax
 constexpr uint32_t kTmemCols = 512;
-constexpr int kColS = 0;          // two 128-column S/P buffers at columns 0 and 128
+constexpr int kColS = 0;          // the S buffer: 128 fp32 columns
+constexpr int kColP = 128;        // P (bf16 pairs): group g at columns 128 + 32g
+constexpr int kColQ = 192;        // Q (bf16 pairs): d/2 columns
 constexpr int kColO = 256;        // O accumulators: group g at columns 256 + g*d
 constexpr int kMaxW = 256;        // up to 8192 key blocks
 constexpr int kMaxList = kMaxW * 32;
@@ -75,22 +76,23 @@ constexpr int kEmpty = -2;        // placeholder: nothing to do
 template <int D>
 struct Cfg {
   static constexpr int kPanels = D / 64;                 // 128-byte column panels
-  static constexpr int kQBytes = kBM * D * 2;
   static constexpr int kBlockBytes = kBN * D * 2;         // one 64-key block of K or V
   static constexpr int kSlotBytes = 2 * kBlockBytes;      // a 128-key slot
   static constexpr int kPanelBytes = kIterKeys * 128;     // one panel of a slot: 128 rows x 128 B
-  static constexpr int kSmem = kQBytes + (kRingK + kRingV) * kSlotBytes + 1024;  // + alignment slack
+  static constexpr int kSmem = (kRingK + kRingV) * kSlotBytes + 1024;  // + alignment slack
   static constexpr uint32_t kIdescS = idesc_bf16_f32(kBM, kIterKeys, false, false);
   static constexpr uint32_t kIdescO = idesc_bf16_f32(kBM, D, false, true);
+  static constexpr int kQWarps = 4 * (D / 64);            // softmax warps that write Q to TMEM
 };
 
 struct Shared {
-  uint64_t q_full;
+  uint64_t q_full;        // Q rows in TMEM (one arrival per writing softmax warp)
   uint64_t k_full[kRingK], k_empty[kRingK];
   uint64_t v_full[kRingV], v_empty[kRingV];
-  uint64_t s_full[2];
-  uint64_t p_full[2][2];  // [S buffer][softmax group], one arrival per softmax warp
-  uint64_t o_done[2];     // completion of O_g += P_u V_u (both groups), by the parity of u
+  uint64_t s_full;        // S_t computed
+  uint64_t s_free;        // S_t loaded by all eight softmax warps
+  uint64_t p_full[2];     // P_t of group g stored, one arrival per warp of the group
+  uint64_t o_done;        // O_g += P_t V_t complete (both groups)
   uint32_t tmem_base;
   int abort_flag;
   int scan[8];
@@ -192,7 +194,7 @@ struct Partials {
 // synchronise inside the loop; the epilogue merges the two (O, m, l) states.
 template <int D>
 __global__ void __launch_bounds__(kThreads, 1)
-k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmK2,
                  const __grid_constant__ CUtensorMap tmV2, int mode, int Nq, int H, int Lk,
                  RowSource rs, const uint32_t* __restrict__ blk_mask, int W, int n_qb,
@@ -224,20 +226,18 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
   }
   uint8_t* tiles = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_dyn) + 1023) & ~static_cast<uintptr_t>(1023));
-  uint8_t* Qs = tiles;
-  auto Ks = [&](int s) { return tiles + C::kQBytes + s * C::kSlotBytes; };
-  auto Vs = [&](int s) { return tiles + C::kQBytes + (kRingK + s) * C::kSlotBytes; };
+  auto Ks = [&](int s) { return tiles + s * C::kSlotBytes; };
+  auto Vs = [&](int s) { return tiles + (kRingK + s) * C::kSlotBytes; };
 
   if (tid == 0) {
-    mbar_init(&sh.q_full, 1);
+    mbar_init(&sh.q_full, C::kQWarps);
     for (int s = 0; s < kRingK; ++s) { mbar_init(&sh.k_full[s], 1); mbar_init(&sh.k_empty[s], 1); }
     for (int s = 0; s < kRingV; ++s) { mbar_init(&sh.v_full[s], 1); mbar_init(&sh.v_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&sh.s_full[b], 1);
-      mbar_init(&sh.p_full[b][0], 4);
-      mbar_init(&sh.p_full[b][1], 4);
-      mbar_init(&sh.o_done[b], 1);
-    }
+    mbar_init(&sh.s_full, 1);
+    mbar_init(&sh.s_free, 8);
+    mbar_init(&sh.p_full[0], 4);
+    mbar_init(&sh.p_full[1], 4);
+    mbar_init(&sh.o_done, 1);
     sh.abort_flag = 0;
     fence_mbar_init();
   }
@@ -295,7 +295,7 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
 
   if (warp == 0 || warp == 2) {
     // ------------------------------------------------------------ producers:
-    // warp 0 loads Q and the K blocks, warp 2 the V blocks
+    // warp 0 loads the K blocks, warp 2 the V blocks
     if (lane == 0) {
       const bool isK = warp == 0;
       const CUtensorMap* tm = isK ? &tmK : &tmV;
@@ -303,15 +303,6 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       const int n_kb1 = rs.k2 ? rs.L / kBN : INT_MAX;
       prefetch_tmap(tm);
       if (rs.k2) prefetch_tmap(tm2);
-      if (isK) {
-        prefetch_tmap(&tmQ);
-        mbar_arrive_expect_tx(&sh.q_full, C::kQBytes);
-        const int y1 = i1 >= 0 ? i1 * 64 : Nq;  // out of range -> zero fill
-        for (int p = 0; p < C::kPanels; ++p) {
-          tma_load_2d(Qs + p * (kBM * 128), &tmQ, &sh.q_full, h * D + p * 64, i0 * 64);
-          tma_load_2d(Qs + p * (kBM * 128) + 64 * 128, &tmQ, &sh.q_full, h * D + p * 64, y1);
-        }
-      }
       const int ring = isK ? kRingK : kRingV;
       for (int t = 0; t < n_it; ++t) {
         const int s = t % ring;
@@ -340,23 +331,21 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     if (lane == 0) {
       bool ok = wait_bar(&sh.q_full, 0, sh, err);
       tc_fence_after();
-      const uint32_t q_base = smem_u32(Qs);
       for (int t = 0; ok && t < n_it; ++t) {
-        // S_t = Q K_t^T (N = 128) into S buffer t % 2, once the P V MMAs of iteration
-        // t-2 (issued by the other issuer) have read that buffer's P
-        const int s = t % kRingK, sb = t & 1;
+        // S_t = Q K_t^T (N = 128, Q from TMEM) once all softmax warps hold S_{t-1}
+        // in registers
+        const int s = t % kRingK;
         if (!wait_bar(&sh.k_full[s], (t / kRingK) & 1, sh, err)) break;
-        if (t >= 2 && !wait_bar(&sh.o_done[sb], ((t - 2) >> 1) & 1, sh, err)) break;
+        if (t >= 1 && !wait_bar(&sh.s_free, (t - 1) & 1, sh, err)) break;
         tc_fence_after();
         const uint32_t k_base = smem_u32(Ks(s));
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
-          const uint64_t adesc = smem_desc_sw128(q_base + (k >> 2) * (kBM * 128) + (k & 3) * 32, 16, 1024);
           const uint64_t bdesc = smem_desc_sw128(k_base + (k >> 2) * C::kPanelBytes + (k & 3) * 32, 16, 1024);
-          mma_ss(tbase + kColS + sb * kIterKeys, adesc, bdesc, C::kIdescS, k > 0 ? 1u : 0u);
+          mma_ts(tbase + kColS, tbase + kColQ + k * 8, bdesc, C::kIdescS, k > 0 ? 1u : 0u);
         }
         mma_commit(&sh.k_empty[s]);
-        mma_commit(&sh.s_full[sb]);
+        mma_commit(&sh.s_full);
       }
     }
   } else if (warp == 3) {
@@ -366,25 +355,25 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     // waits for the softmax (an MMA's issue blocks behind the one executing).
     if (lane == 0) {
       for (int u = 0; u < n_it; ++u) {
-        const int su = u & 1, vs = u % kRingV;
+        const int vs = u % kRingV;
         if (!wait_bar(&sh.v_full[vs], (u / kRingV) & 1, sh, err)) break;
+        // group 1 has no block in an odd list's last iteration
         const int n_grp = (u == n_it - 1 && odd_tail) ? 1 : 2;
         bool ok = true;
-        for (int g = 0; g < 2; ++g) {
-          if (!wait_bar(&sh.p_full[su][g], (u >> 1) & 1, sh, err)) { ok = false; break; }
-          if (g >= n_grp) break;
+        for (int g = 0; g < n_grp; ++g) {
+          if (!wait_bar(&sh.p_full[g], u & 1, sh, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t v_base = smem_u32(Vs(vs)) + g * (kBN * 128);
 #pragma unroll
           for (int kk = 0; kk < kBN / 16; ++kk) {
             const uint64_t bdesc = smem_desc_sw128(v_base + kk * 2048, C::kPanelBytes, 1024);
-            mma_ts(tbase + kColO + g * D, tbase + kColS + su * kIterKeys + g * kBN + kk * 8, bdesc,
+            mma_ts(tbase + kColO + g * D, tbase + kColP + g * (kBN / 2) + kk * 8, bdesc,
                    C::kIdescO, (u > 0 || kk > 0) ? 1u : 0u);
           }
         }
         if (!ok) break;
         mma_commit(&sh.v_empty[vs]);
-        mma_commit(&sh.o_done[su]);
+        mma_commit(&sh.o_done);
       }
     }
   } else if (warp >= 4) {
@@ -403,30 +392,61 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
     const float2 sc2 = make_float2(scale_log2, scale_log2);
     float m_run = -INFINITY, l_run = 0.f;
     bool ok = true;
-    // one arrival per warp once all its lanes' TMEM stores are complete
-    auto release_p = [&](int sb) {
+    // one arrival per warp once all its lanes' TMEM accesses are complete
+    auto arrive_warp = [&](uint64_t* bar) {
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.p_full[sb][g]);
+      if (lane == 0) mbar_arrive(bar);
     };
+    // Wait until the P V MMAs of iteration t-1 are done: P_t may then overwrite
+    // P_{t-1} and O_g is stable for a rescale.  Every softmax warp waits once per
+    // iteration, and P V of t needs this warp's P_t, so at this wait the barrier has
+    // completed t-1 or t phases: its parity is unambiguous.
+    auto wait_pv = [&](int t) -> bool {
+      if (t == 0) return true;
+      const bool w = __all_sync(0xffffffffu, wait_bar(&sh.o_done, (t - 1) & 1, sh, err));
+      tc_fence_after();
+      return w;
+    };
+    // The tile's Q rows into TMEM as bf16 pairs (the S MMA's A operand): one thread
+    // per row, 64 elements per group; rows past Nq or of a missing second block are 0.
+    if (g < D / 64) {
+      uint32_t qv[32];
+      if (row_valid) {
+        const uint4* src =
+            reinterpret_cast<const uint4*>(q + (static_cast<size_t>(qrow) * H + h) * D + g * 64);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          const uint4 x = src[e];
+          qv[4 * e] = x.x; qv[4 * e + 1] = x.y; qv[4 * e + 2] = x.z; qv[4 * e + 3] = x.w;
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 32; ++c) qv[c] = 0u;
+      }
+      tmem_st32(tbase + lane_base + kColQ + g * 32, qv);
+      tmem_wait_st();
+      arrive_warp(&sh.q_full);
+    }
+    const uint32_t s_addr = tbase + lane_base + kColS + g * kBN;
+    const uint32_t p_addr = tbase + lane_base + kColP + g * (kBN / 2);
     int t = 0;
     for (; t < n_it; ++t) {
       const uint32_t e = (list2[t] >> (16 * g)) & 0xFFFFu;
-      const int sb = t & 1;
-      if (!__all_sync(0xffffffffu, wait_bar(&sh.s_full[sb], (t >> 1) & 1, sh, err))) { ok = false; break; }
-      const uint32_t s_addr = tbase + lane_base + kColS + sb * kIterKeys + g * kBN;
-      if (e == kNoBlock) {         // group 1 in an odd list's last iteration: no block
-        release_p(sb);
-        continue;
-      }
-      if (!(e & sel_bit)) {
-        // this warp's query block did not keep the block: P = 0, state unchanged
-        uint32_t z[32];
+      if (!__all_sync(0xffffffffu, wait_bar(&sh.s_full, t & 1, sh, err))) { ok = false; break; }
+      if (e == kNoBlock || !(e & sel_bit)) {
+        // no block (group 1 in an odd list's last iteration), or this warp's query
+        // block did not keep it: S is not read, P = 0, the state is unchanged
+        arrive_warp(&sh.s_free);
+        if (!wait_pv(t)) { ok = false; break; }
+        if (e != kNoBlock) {
+          uint32_t z[32];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) z[c] = 0u;
-        tmem_st32(s_addr, z);
-        tmem_wait_st();
-        release_p(sb);
+          for (int c = 0; c < 32; ++c) z[c] = 0u;
+          tmem_st32(p_addr, z);
+          tmem_wait_st();
+          arrive_warp(&sh.p_full[g]);
+        }
         continue;
       }
       tc_fence_after();
@@ -434,6 +454,7 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
       tmem_ld32(s_addr, *reinterpret_cast<uint32_t(*)[32]>(&r[0]));
       tmem_ld32(s_addr + 32, *reinterpret_cast<uint32_t(*)[32]>(&r[32]));
       tmem_wait_ld();
+      arrive_warp(&sh.s_free);   // S_{t+1} may now overwrite the buffer
       const int valid = min(kBN, Lk - static_cast<int>(e & 0x1FFFu) * kBN);
       const bool ragged = valid < kBN;   // the key sequence's last, partial block
       if (ragged) {
@@ -462,17 +483,8 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
         softmax_pass<false>(r, sc2, nm2, pk, lsum, mraw);
       }
       l_run = l_run * factor + lsum;
-      tmem_st32(s_addr, pk);
-      tmem_wait_st();
+      if (!wait_pv(t)) { ok = false; break; }
       if (__any_sync(0xffffffffu, resc)) {
-        // O_g may be rescaled only once the P V MMAs of iteration t-1 have landed.
-        // S_t (waited for) was issued after those of iteration t-2 had completed and
-        // iteration t+1's need P_{t+1}, so on the barrier of t-1's parity at most
-        // iteration t-1 is outstanding: the parity wait is unambiguous although
-        // iterations without a rescale skip it.
-        const int u = t - 1;
-        if (!__all_sync(0xffffffffu, wait_bar(&sh.o_done[u & 1], (u >> 1) & 1, sh, err))) { ok = false; break; }
-        tc_fence_after();
 #pragma unroll
         for (int c0 = 0; c0 < D; c0 += 32) {
           uint32_t o[32];
@@ -482,14 +494,13 @@ k_umma_attention(const __grid_constant__ CUtensorMap tmQ, const __grid_constant_
           for (int q = 0; q < 32; ++q) o[q] = __float_as_uint(__uint_as_float(o[q]) * factor);
           tmem_st32(tbase + lane_base + o_col + c0, o);
         }
-        tmem_wait_st();
       }
-      release_p(sb);
+      tmem_st32(p_addr, pk);
+      tmem_wait_st();
+      arrive_warp(&sh.p_full[g]);
     }
-    // the last two iterations' P V MMAs may both be outstanding: one wait on each
-    // parity's barrier
-    if (ok && t > 0) ok = __all_sync(0xffffffffu, wait_bar(&sh.o_done[(t - 1) & 1], ((t - 1) >> 1) & 1, sh, err));
-    if (ok && t > 1) ok = __all_sync(0xffffffffu, wait_bar(&sh.o_done[(t - 2) & 1], ((t - 2) >> 1) & 1, sh, err));
+    // the last iteration's P V MMAs
+    if (ok && t > 0) ok = wait_pv(t);
     ok = __all_sync(0xffffffffu, ok);
     tc_fence_after();
     // merge the groups' states: M = max(m_0, m_1), w_g = 2^(m_g - M); each group then
@@ -801,7 +812,7 @@ bool make_tmap_bf16_2d(void* tmap, const void* base, uint64_t inner, uint64_t ou
 
 namespace {
 template <int D>
-void launch_attn_kernel(int grid, cudaStream_t st, const CUtensorMap& tq, const CUtensorMap& tk,
+void launch_attn_kernel(int grid, cudaStream_t st, const void* q, const CUtensorMap& tk,
                         const CUtensorMap& tv, const CUtensorMap& tk2, const CUtensorMap& tv2,
                         int mode, int Nq, int H, RowSource rs,
                         const uint32_t* blk_mask, int W, int n_qb, const int4* pairs,
@@ -809,22 +820,21 @@ void launch_attn_kernel(int grid, cudaStream_t st, const CUtensorMap& tq, const 
                         float* lin_ws, void* out, float* o_branch, uint32_t* err) {
   const int smem = Cfg<D>::kSmem;
   cudaFuncSetAttribute(k_umma_attention<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  k_umma_attention<D><<<grid, kThreads, smem, st>>>(tq, tk, tv, tk2, tv2, mode, Nq, H, rs.L + rs.L2, rs,
+  k_umma_attention<D><<<grid, kThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(q), tk, tv, tk2, tv2, mode, Nq, H, rs.L + rs.L2, rs,
                                                      blk_mask, W,
                                                      n_qb, pairs, items, part, gate, lin_sign, lin_ws,
                                                      static_cast<__nv_bfloat16*>(out), o_branch, err);
 }
 
-// Q, the keys/values of the first segment (pool pages or a contiguous buffer) and,
+// The keys/values of the first segment (pool pages or a contiguous buffer) and,
 // when the row source has one, of the second (tk2/tv2 repeat tk/tv otherwise).
-wa_status make_maps(const void* q, int Nq, int H, int d, const RowSource& rs, CUtensorMap* tq,
-                    CUtensorMap* tk, CUtensorMap* tv, CUtensorMap* tk2, CUtensorMap* tv2) {
+wa_status make_maps(int H, int d, const RowSource& rs, CUtensorMap* tk, CUtensorMap* tv,
+                    CUtensorMap* tk2, CUtensorMap* tv2) {
   const int cols = H * d;
   const uint64_t key_rows = rs.page_ids ? static_cast<uint64_t>(rs.n_pages) * rs.page_rows
                                         : static_cast<uint64_t>(rs.L);
   const uint64_t rb = static_cast<uint64_t>(cols) * 2;
-  if (!make_tmap_bf16_2d(tq, q, cols, Nq, rb, 64, 64) ||
-      !make_tmap_bf16_2d(tk, rs.k, cols, key_rows, rb, 64, 64) ||
+  if (!make_tmap_bf16_2d(tk, rs.k, cols, key_rows, rb, 64, 64) ||
       !make_tmap_bf16_2d(tv, rs.v, cols, key_rows, rb, 64, 64))
     return set_error(WA_ERR_CUDA, "cuTensorMapEncodeTiled failed for the attention operands");
   if (rs.k2) {
@@ -844,18 +854,18 @@ wa_status launch_linear_attention(const void* q, int Nq, int H, int d, RowSource
                                   float* o_lin, uint32_t* err, cudaStream_t st) {
   if (B != kBN) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs B == 64");
   if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "bf16 attention needs d in {64,128}");
-  alignas(64) CUtensorMap tq, tk, tv, tk2, tv2;
-  wa_status s = make_maps(q, Nq, H, d, lin, &tq, &tk, &tv, &tk2, &tv2);
+  alignas(64) CUtensorMap tk, tv, tk2, tv2;
+  wa_status s = make_maps(H, d, lin, &tk, &tv, &tk2, &tv2);
   if (s != WA_OK) return s;
   const int n_qb = (Nq + B - 1) / B;
   const int grid = H * ((n_qb + 1) / 2);
   Partials none{nullptr, nullptr};
   if (d == 128)
-    launch_attn_kernel<128>(grid, st, tq, tk, tv, tk2, tv2, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
+    launch_attn_kernel<128>(grid, st, q, tk, tv, tk2, tv2, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
                             none, gate_lin ? gate_lin : gate, gate_lin ? 1.f : -1.f, lin_ws, nullptr,
                             o_lin, err);
   else
-    launch_attn_kernel<64>(grid, st, tq, tk, tv, tk2, tv2, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
+    launch_attn_kernel<64>(grid, st, q, tk, tv, tk2, tv2, 0, Nq, H, lin, nullptr, 0, n_qb, nullptr, nullptr,
                            none, gate_lin ? gate_lin : gate, gate_lin ? 1.f : -1.f, lin_ws, nullptr,
                            o_lin, err);
   return check_launch("linear attention");
@@ -922,19 +932,19 @@ wa_status launch_attn_sparse(const void* q, int Nq, int H, int d, RowSource rs, 
     return set_error(WA_ERR_UNSUPPORTED, "a second key segment needs the first to fill whole blocks");
   SparseLayout s = sparse_layout(scratch, Nq, H, d, B, rs.L + rs.L2);
   if (s.W > kMaxW) return set_error(WA_ERR_UNSUPPORTED, "too many key blocks (max %d)", kMaxW * 32);
-  alignas(64) CUtensorMap tq, tk, tv, tk2, tv2;
-  wa_status e = make_maps(q, Nq, H, d, rs, &tq, &tk, &tv, &tk2, &tv2);
+  alignas(64) CUtensorMap tk, tv, tk2, tv2;
+  wa_status e = make_maps(H, d, rs, &tk, &tv, &tk2, &tv2);
   if (e != WA_OK) return e;
   const int grid = 2 * s.n_pairs;
   float* lin_rw = const_cast<float*>(lin_ws);
   const int split_min = split_min_for(s.n_pairs);
   if (d == 128) {
-    launch_attn_kernel<128>(grid, st, tq, tk, tv, tk2, tv2, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
+    launch_attn_kernel<128>(grid, st, q, tk, tv, tk2, tv2, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
                             s.part, gate, 0.f, lin_rw, out, o_sp, err);
     k_combine<128><<<dim3(s.n_pairs, kBM / 32), 2 * 128, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate, lin_ws,
                                                                   static_cast<__nv_bfloat16*>(out), o_sp);
   } else {
-    launch_attn_kernel<64>(grid, st, tq, tk, tv, tk2, tv2, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
+    launch_attn_kernel<64>(grid, st, q, tk, tv, tk2, tv2, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
                            s.part, gate, 0.f, lin_rw, out, o_sp, err);
     k_combine<64><<<dim3(s.n_pairs, kBM / 32), 2 * 64, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate, lin_ws,
                                                                 static_cast<__nv_bfloat16*>(out), o_sp);
