@@ -19,8 +19,8 @@
 //
 // CTA = 384 threads, one CTA per SM.  The item's key blocks are listed once in
 // shared memory; an iteration takes two consecutive blocks of the list (128 keys),
-// so S = Q K^T is one M=128, N=128 MMA chain (N=64 chains run at about two thirds of
-// the tensor rate: their operand reads from shared memory dominate).  Roles:
+// so S = Q K^T is one M=128, N=128 MMA chain (with both operands in shared memory,
+// N=64 chains ran at about two thirds of the tensor rate).  Roles:
 //   warp 0  loads the K blocks, warp 2 the V blocks (TMA, 128-byte swizzle,
 //           straight from the pool pages through a page table staged in shared
 //           memory) into rings of 128-key slots (3 each);
@@ -185,9 +185,9 @@ struct Partials {
 };
 
 // One CTA per SM.  An iteration covers two consecutive blocks (ja, jb) of the
-// tile's key list: S = Q K^T is one N=128 MMA chain (full tensor rate; N=64 chains
-// are bound by their shared-memory operand reads), K and V of the two blocks sit in
-// one 128-key slot of their rings (the second half unused when the list is odd).
+// tile's key list: S = Q K^T is one N=128 MMA chain with Q read from TMEM; K and V
+// of the two blocks sit in one 128-key slot of their rings (the second half unused
+// when the list is odd).
 // Softmax group 0 (warps 4-7) owns the blocks at even list positions (S columns
 // 0-63), group 1 (warps 8-11) those at odd positions (columns 64-127): each keeps
 // its own running max and sum and its own O accumulator, so the groups never
