@@ -365,6 +365,25 @@ def run_ours(args, rank, world, local_rank):
     gather_ms = gs.elapsed_time(ge) / n_g
     gather_bytes = 2 * 2 * ka.numel() * ka.element_size()
     gather_gbs = gather_bytes / (gather_ms * 1e-3) / 1e9
+    # cube-tile token order: the active keys (K_p pages) re-ordered page by page into
+    # (8, 2, 4) cubes of an 8-frame 30 x 52 latent page, one row gather over L rows
+    perm_ms = perm_gbs = perm_bytes = None
+    if cfg.T_p == W.PAGE_FRAMES * 30 * 52:
+        pp = wa.wa_cube_order(W.PAGE_FRAMES, 30, 52, 8, 2, 4).long()
+        perm = torch.cat([pp + s_ * cfg.T_p for s_ in range(cfg.K_p)]).to(torch.int32).to(dev)
+        kc = torch.empty_like(ka)
+        for _ in range(3):
+            wa.wa_permute_rows(ka, perm, out=kc)
+        ps, pe = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ps.record(stream)
+        for _ in range(n_g):
+            wa.wa_permute_rows(ka, perm, out=kc)
+        pe.record(stream)
+        torch.cuda.synchronize()
+        perm_ms = ps.elapsed_time(pe) / n_g
+        perm_bytes = 2 * ka.numel() * ka.element_size() + perm.numel() * 4
+        perm_gbs = perm_bytes / (perm_ms * 1e-3) / 1e9
+        del kc
     del ka, va
 
     line = None
@@ -403,6 +422,10 @@ def run_ours(args, rank, world, local_rank):
                            "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                            "frac": gather_gbs / float(peaks["hbm_gbs"]), "bytes_per_launch": gather_bytes,
                            "ms_per_launch": gather_ms},
+            "hbm_cube_permute": ({"kernel": "k_permute_rows (cube-tile token order of the active keys)",
+                                  "achieved": perm_gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                                  "frac": perm_gbs / float(peaks["hbm_gbs"]), "bytes_per_launch": perm_bytes,
+                                  "ms_per_launch": perm_ms} if perm_ms else None),
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "e2e": ({"value": frames_per_s(e2e_ms, world), "unit": "frames/s", "ms_per_step": e2e_ms,
                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,

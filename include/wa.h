@@ -66,6 +66,7 @@ typedef enum wa_dtype { WA_F32 = 0, WA_BF16 = 1 } wa_dtype;
 #define WA_DEVERR_PAGE_ID   0x1u  /* a page id outside [0, n_pool_pages)            */
 #define WA_DEVERR_ZERO_NORM 0x2u  /* a zero-norm prompt embedding in prompt select  */
 #define WA_DEVERR_TIMEOUT   0x4u  /* a bounded wait inside a kernel gave up         */
+#define WA_DEVERR_ROW_ID    0x8u  /* a row index outside [0, n_rows) in wa_permute_rows */
 
 /* Message describing the calling thread's most recent failure ("" if none). */
 WA_API const char* wa_last_error(void);
@@ -146,6 +147,37 @@ WA_API wa_status wa_pool_index(const void* k_pool, int n_pool_pages, int T_p, in
 WA_API wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, int H, int d,
                          wa_dtype dtype, const void* k_new, const void* v_new, int n_tokens,
                          long long token_offset, double* page_index, int B, void* stream);
+
+/* ---------------------------------------------------------------------------
+ * Token order: 3-D cube tiles (WorldAttention Appendix A.1.3, "Block Sparse
+ * Attention": the flattened token sequence is re-indexed so that every contiguous
+ * group of B tokens is one (C_t, C_h, C_w) cube of the video volume, so that a
+ * selected or skipped block is a spatio-temporal cube).  The pages lost the index
+ * formula; the reading implemented here: the tokens of a grid of T frames x H_l
+ * rows x W_l columns (raster index (t*H_l + h)*W_l + w) are ordered cube by cube,
+ * the cubes in raster order of their corners (t_c, h_c, w_c) and the tokens inside
+ * a cube in raster order.  Where a grid side is not a multiple of the cube side the
+ * last cube along it is cut short, so groups of C_t*C_h*C_w tokens are exact cubes
+ * only when C_t | T, C_h | H_l and C_w | W_l (an 8-frame page of 30 x 52 latents
+ * with (8, 2, 4) cubes: 195 cubes of 64 tokens, one per key block).  Attention over
+ * cube-ordered keys is the same computation; only the blocks that selection pools
+ * and keeps change.
+ *
+ * wa_cube_order: host function, no device work.  perm[n] (n in [0, T*H_l*W_l)) is
+ *   the raster index of the token at cube-order position n; perm is caller-owned
+ *   host memory of T*H_l*W_l int32.  INVALID_ARG: a size < 1, NULL perm, or more
+ *   than 2^31 - 1 tokens.
+ * wa_permute_rows: row permutation of [n_rows][row_bytes] device data on `stream`:
+ *     inverse == 0:  dst[n] = src[perm[n]]   (raster -> cube order with wa_cube_order's perm)
+ *     inverse != 0:  dst[perm[n]] = src[n]   (cube -> raster order)
+ *   perm: device int32 [n_rows], a permutation of [0, n_rows); src and dst must not
+ *   overlap; row_bytes a multiple of 16 and both pointers 16-byte aligned
+ *   (UNSUPPORTED otherwise).  A bit-exact copy.  An entry of perm outside
+ *   [0, n_rows) sets WA_DEVERR_ROW_ID and that row is skipped.  INVALID_ARG: NULL
+ *   pointer, n_rows < 1, row_bytes == 0. */
+WA_API wa_status wa_cube_order(int T, int H_l, int W_l, int C_t, int C_h, int C_w, int32_t* perm);
+WA_API wa_status wa_permute_rows(const void* src, void* dst, const int32_t* perm, int n_rows,
+                                 size_t row_bytes, int inverse, void* stream);
 
 /* ---------------------------------------------------------------------------
  * S3 -- head-adaptive block selection (WorldAttention §3.3, "Head-level sparsity

@@ -51,7 +51,49 @@ k_copy16(const uint4* __restrict__ src, uint4* __restrict__ dst, size_t n16) {
     st_stream(dst + i, ld_stream(src + i));
 }
 
+// Row permutation (cube-tile token order, WorldAttention Appendix A.1.3): one warp
+// per row, lanes striding over the row's 16-byte vectors with four loads in flight;
+// the warps stride over the rows.  inverse == 0 gathers dst[n] = src[perm[n]],
+// inverse != 0 scatters dst[perm[n]] = src[n].
+__global__ void __launch_bounds__(256)
+k_permute_rows(const uint4* __restrict__ src, uint4* __restrict__ dst,
+               const int32_t* __restrict__ perm, int n_rows, size_t n16, int inverse,
+               uint32_t* err) {
+  const int lane = threadIdx.x & 31;
+  const int n_warps = static_cast<int>((gridDim.x * blockDim.x) >> 5);
+  for (int n = static_cast<int>((blockIdx.x * blockDim.x + threadIdx.x) >> 5); n < n_rows;
+       n += n_warps) {
+    const int j = perm[n];
+    if (j < 0 || j >= n_rows) {
+      if (lane == 0) atomicOr(err, WA_DEVERR_ROW_ID);
+      continue;
+    }
+    const uint4* a = src + static_cast<size_t>(inverse ? n : j) * n16;
+    uint4* b = dst + static_cast<size_t>(inverse ? j : n) * n16;
+    size_t i = lane;
+    for (; i + 96 < n16; i += 128) {
+      const uint4 x0 = ld_stream(a + i), x1 = ld_stream(a + i + 32);
+      const uint4 x2 = ld_stream(a + i + 64), x3 = ld_stream(a + i + 96);
+      st_stream(b + i, x0);
+      st_stream(b + i + 32, x1);
+      st_stream(b + i + 64, x2);
+      st_stream(b + i + 96, x3);
+    }
+    for (; i < n16; i += 32) st_stream(b + i, ld_stream(a + i));
+  }
+}
+
 }  // namespace
+
+wa_status launch_permute_rows(const void* src, void* dst, const int32_t* perm, int n_rows,
+                              size_t row_bytes, int inverse, uint32_t* err, cudaStream_t st) {
+  size_t blocks = (static_cast<size_t>(n_rows) + 7) / 8;   // eight warps (rows) per CTA
+  if (blocks > 8 * 148) blocks = 8 * 148;
+  k_permute_rows<<<static_cast<unsigned>(blocks), 256, 0, st>>>(
+      static_cast<const uint4*>(src), static_cast<uint4*>(dst), perm, n_rows, row_bytes / 16,
+      inverse, err);
+  return check_launch("permute_rows");
+}
 
 wa_status launch_copy16(const void* src, void* dst, size_t n16, cudaStream_t st) {
   size_t blocks = (n16 + 1023) / 1024;

@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <climits>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -323,6 +325,49 @@ wa_status wa_gather_pages(const void* k_pool, const void* v_pool, int n_pool_pag
   if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
   return launch_gather(k_pool, v_pool, n_pool_pages, page_bytes, sel, K_p, k_act, v_act, err,
                        static_cast<cudaStream_t>(stream));
+}
+
+// ------------------------------------------------------------------ token order
+// Cube-tile order (Appendix A.1.3), in closed form: the cubes before cube (a, b, c)
+// hold a*C_t*H_l*W_l tokens (whole frame slabs), then ct*b*C_h*W_l (whole row bands
+// of slab a) and ct*ch*c*C_w (cubes to the left in band b), where ct and ch are the
+// (possibly cut short) extents of slab a and band b; inside the cube a token's
+// offset is raster over the cube's extents.
+wa_status wa_cube_order(int T, int H_l, int W_l, int C_t, int C_h, int C_w, int32_t* perm) {
+  WA_REQUIRE(perm, "NULL pointer");
+  WA_REQUIRE(T >= 1 && H_l >= 1 && W_l >= 1 && C_t >= 1 && C_h >= 1 && C_w >= 1,
+             "sizes must be >= 1");
+  const long long n = static_cast<long long>(T) * H_l * W_l;
+  WA_REQUIRE(n <= INT_MAX, "more than 2^31 - 1 tokens");
+  const long long plane = static_cast<long long>(H_l) * W_l;
+  for (int t = 0; t < T; ++t) {
+    const int a = t / C_t, ct = std::min(C_t, T - a * C_t);
+    for (int h = 0; h < H_l; ++h) {
+      const int b = h / C_h, ch = std::min(C_h, H_l - b * C_h);
+      for (int w = 0; w < W_l; ++w) {
+        const int c = w / C_w, cw = std::min(C_w, W_l - c * C_w);
+        const long long cube0 = static_cast<long long>(a) * C_t * plane +
+                                static_cast<long long>(ct) * b * C_h * W_l +
+                                static_cast<long long>(ct) * ch * c * C_w;
+        const long long local =
+            (static_cast<long long>(t - a * C_t) * ch + (h - b * C_h)) * cw + (w - c * C_w);
+        perm[cube0 + local] = static_cast<int32_t>(t * plane + static_cast<long long>(h) * W_l + w);
+      }
+    }
+  }
+  return WA_OK;
+}
+
+wa_status wa_permute_rows(const void* src, void* dst, const int32_t* perm, int n_rows,
+                          size_t row_bytes, int inverse, void* stream) {
+  WA_REQUIRE(src && dst && perm, "NULL pointer");
+  WA_REQUIRE(n_rows >= 1 && row_bytes >= 1, "sizes must be >= 1");
+  if (row_bytes % 16 != 0 || !aligned16(src) || !aligned16(dst))
+    return set_error(WA_ERR_UNSUPPORTED, "permute_rows needs 16-byte aligned rows");
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  return launch_permute_rows(src, dst, perm, n_rows, row_bytes, inverse, err,
+                             static_cast<cudaStream_t>(stream));
 }
 
 // ------------------------------------------------------------------ S3

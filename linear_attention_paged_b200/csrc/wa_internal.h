@@ -107,6 +107,8 @@ wa_status launch_gather(const void* k_pool, const void* v_pool, int n_pages, siz
 
 // dst[0..n16) = src[0..n16) in 16-byte units.
 wa_status launch_copy16(const void* src, void* dst, size_t n16, cudaStream_t st);
+wa_status launch_permute_rows(const void* src, void* dst, const int32_t* perm, int n_rows,
+                              size_t row_bytes, int inverse, uint32_t* err, cudaStream_t st);
 
 // ---------------------------------------------------------------- fp32 SIMT path
 wa_status launch_simt_project(const float* x, const int32_t* page_ids, int page_rows, int n_pages,

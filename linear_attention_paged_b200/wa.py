@@ -25,7 +25,7 @@ lib = ctypes.CDLL(LIB_PATH)
 
 WA_OK, WA_ERR_INVALID_ARG, WA_ERR_UNSUPPORTED, WA_ERR_CUDA, WA_ERR_DEVICE, WA_ERR_WORKSPACE = range(6)
 WA_F32, WA_BF16 = 0, 1
-DEVERR_PAGE_ID, DEVERR_ZERO_NORM, DEVERR_TIMEOUT = 1, 2, 4
+DEVERR_PAGE_ID, DEVERR_ZERO_NORM, DEVERR_TIMEOUT, DEVERR_ROW_ID = 1, 2, 4, 8
 
 c_void_p, c_int, c_size_t = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
 P = c_void_p
@@ -98,6 +98,8 @@ _SIGS = {
     "wa_tier_flush": (c_int, [P, P]),
     "wa_tier_slot_of": (c_int, [P, c_int, P]),
     "wa_tier_get_stats": (c_int, [P, P]),
+    "wa_cube_order": (c_int, [c_int] * 6 + [P]),
+    "wa_permute_rows": (c_int, [P, P, P, c_int, c_size_t, c_int, P]),
 }
 for _name, (_res, _args) in _SIGS.items():
     _f = getattr(lib, _name)
@@ -209,6 +211,31 @@ def wa_gather_pages(k_pool, v_pool, sel, stream=None, out=None):
         _p(k_pool), _p(v_pool), P_, T_p, H, d, _p(sel), K_p, dtype_code(k_pool), _p(k_act),
         _p(v_act), _stream(stream)))
     return k_act, v_act
+
+
+# --------------------------------------------------------------------- token order
+def wa_cube_order(T: int, H_l: int, W_l: int, C_t: int, C_h: int, C_w: int) -> torch.Tensor:
+    """Cube-tile token order (host, int32 CPU tensor): element n is the raster index
+    of the token at cube-order position n."""
+    perm = torch.empty(T * H_l * W_l, dtype=torch.int32)
+    _check("wa_cube_order", lib.wa_cube_order(T, H_l, W_l, C_t, C_h, C_w, _p(perm)))
+    return perm
+
+
+def wa_permute_rows(src, perm, inverse: bool = False, out=None, stream=None):
+    """Rows of ``src`` (first dimension) permuted on the device: out[n] = src[perm[n]],
+    or out[perm[n]] = src[n] with ``inverse``; ``perm`` a device int32 permutation."""
+    _need_cuda(src, perm)
+    assert perm.dtype == torch.int32 and perm.numel() == src.shape[0]
+    if out is None:
+        out = torch.empty_like(src)
+    else:
+        _need_cuda(out)
+        assert out.shape == src.shape and out.dtype == src.dtype
+    row_bytes = src[0].numel() * src.element_size()
+    _check("wa_permute_rows", lib.wa_permute_rows(
+        _p(src), _p(out), _p(perm), src.shape[0], row_bytes, 1 if inverse else 0, _stream(stream)))
+    return out
 
 
 # --------------------------------------------------------------------- pool

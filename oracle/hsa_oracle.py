@@ -23,6 +23,8 @@ Each function follows one step of the method as the WorldAttention pages state i
   S6 gate_fuse          -- §3.3 "Gated fusion of two branches" (sigmoid gate)
      gate_fuse2            the same section's two-gate form O_lin (.) G_lin + O_sp (.) G_sp
                            with G = sigmoid of a logit per (token, head)
+  cube_order            -- Appendix A.1.3: the token re-indexing under which every group
+                           of B consecutive tokens is one (C_t, C_h, C_w) cube
 
 Readings where the pages are silent (each one is listed in the design notes):
   * Q-bar in the page score is per head; the per-head scores are averaged over heads,
@@ -37,6 +39,9 @@ Readings where the pages are silent (each one is listed in the design notes):
   * Keys of both branches are the retrieved history; with k_cur/v_cur the sparse
     branch also takes the current chunk's own keys (after the history); no causal mask.
   * O = sigmoid(g) * O_sp + (1 - sigmoid(g)) * O_lin, per token and head (or two gates).
+  * Cube order (its formula is lost): cubes in raster order of their corners, tokens
+    in raster order inside a cube, the last cube along a side cut short when the side
+    is not a multiple of the cube side.
 """
 from __future__ import annotations
 
@@ -54,6 +59,24 @@ def f64(x) -> np.ndarray:
             x = x.float()
         x = x.numpy()
     return np.asarray(x, dtype=np.float64)
+
+
+# ----------------------------------------------------------------------------- token order
+def cube_order(T: int, H_l: int, W_l: int, C_t: int, C_h: int, C_w: int) -> list:
+    """Appendix A.1.3 (block-sparse attention): the flattened video tokens are
+    re-indexed so that each run of C_t*C_h*C_w consecutive tokens is one
+    (C_t, C_h, C_w) cube.  Returns perm with perm[n] = raster index (t*H_l + h)*W_l + w
+    of the token at position n: walk the cubes in raster order of their corners and,
+    inside each, the tokens in raster order (cubes at the far edges cut short)."""
+    perm = []
+    for t0 in range(0, T, C_t):
+        for h0 in range(0, H_l, C_h):
+            for w0 in range(0, W_l, C_w):
+                for t in range(t0, min(T, t0 + C_t)):
+                    for h in range(h0, min(H_l, h0 + C_h)):
+                        for w in range(w0, min(W_l, w0 + C_w)):
+                            perm.append((t * H_l + h) * W_l + w)
+    return perm
 
 
 # ----------------------------------------------------------------------------- S0

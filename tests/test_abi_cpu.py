@@ -137,3 +137,25 @@ def test_binding_has_no_fallback():
     # the header is bound to the shared object
     for name in wa.header_functions():
         assert getattr(wa.lib, name).__name__ == name
+
+
+def test_cube_order_matches_oracle():
+    # the library's closed form against the oracle's walk over the cubes (host only)
+    from oracle import hsa_oracle as O
+    shapes = [(2, 2, 4, 1, 2, 2), (1, 3, 3, 1, 2, 2), (8, 30, 52, 8, 2, 4), (3, 30, 52, 8, 2, 4),
+              (5, 7, 11, 2, 3, 4), (2, 10, 26, 8, 2, 4), (1, 1, 1, 4, 4, 4), (4, 9, 13, 4, 4, 4)]
+    for sh in shapes:
+        assert wa.wa_cube_order(*sh).tolist() == O.cube_order(*sh), sh
+
+
+def test_cube_order_and_permute_validation():
+    perm = (ctypes.c_int32 * 4)()
+    assert wa.lib.wa_cube_order(0, 2, 2, 1, 1, 1, perm) == wa.WA_ERR_INVALID_ARG
+    assert wa.lib.wa_cube_order(1, 2, 2, 1, 0, 1, perm) == wa.WA_ERR_INVALID_ARG
+    assert wa.lib.wa_cube_order(1, 2, 2, 1, 1, 1, None) == wa.WA_ERR_INVALID_ARG
+    assert wa.lib.wa_cube_order(65536, 65536, 2, 1, 1, 1, perm) == wa.WA_ERR_INVALID_ARG
+    f = wa.lib.wa_permute_rows
+    assert f(None, FAKE, FAKE, 4, 16, 0, None) == wa.WA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 0, 16, 0, None) == wa.WA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 4, 24, 0, None) == wa.WA_ERR_UNSUPPORTED     # rows of 16-byte multiples
+    assert f(FAKE, ctypes.c_void_p(4096 + 8), FAKE, 4, 16, 0, None) == wa.WA_ERR_UNSUPPORTED

@@ -420,3 +420,38 @@ def test_prompt_selected_chunk_drives_candidates():
     res = O.hsa_step(inp, cfg.B, cfg.K_p)
     assert res["chunk"] == 2
     assert set(res["sel"]) <= set(range(2 * cfg.n_c, 3 * cfg.n_c))
+
+
+# ---------------------------------------------------------------- token order (A.1.3)
+def test_cube_order_hand_examples():
+    # 2 frames of 2 x 4 tokens (raster ids 0-7 in frame 0, 8-15 in frame 1), cubes of
+    # (1, 2, 2): frame 0 left cube {0, 1, 4, 5}, right cube {2, 3, 6, 7}, then frame 1
+    assert O.cube_order(2, 2, 4, 1, 2, 2) == [0, 1, 4, 5, 2, 3, 6, 7, 8, 9, 12, 13, 10, 11, 14, 15]
+    # one 3 x 3 frame, (1, 2, 2) cubes cut short at the far edges:
+    # {0, 1, 3, 4}, {2, 5}, {6, 7}, {8}
+    assert O.cube_order(1, 3, 3, 1, 2, 2) == [0, 1, 3, 4, 2, 5, 6, 7, 8]
+    # one cube covering everything, a cube per token, and a cube per row are raster order
+    for cube in [(2, 3, 5), (1, 1, 1), (1, 1, 5)]:
+        assert O.cube_order(2, 3, 5, *cube) == list(range(30))
+
+
+@pytest.mark.parametrize("grid,cube", [((8, 10, 16), (8, 2, 4)), ((4, 6, 8), (2, 3, 4)),
+                                       ((8, 30, 52), (8, 2, 4))])
+def test_cube_order_groups_are_cubes(grid, cube):
+    T, Hl, Wl = grid
+    ct, ch, cw = cube
+    perm = O.cube_order(T, Hl, Wl, ct, ch, cw)
+    n = T * Hl * Wl
+    assert sorted(perm) == list(range(n))          # a permutation
+    Bc = ct * ch * cw
+    corners = []
+    for g in range(n // Bc):
+        pts = [divmod(divmod(x, Wl)[0], Hl) + (x % Wl,) for x in perm[g * Bc:(g + 1) * Bc]]
+        ts, hs, ws = zip(*pts)
+        t0, h0, w0 = min(ts), min(hs), min(ws)
+        # the group is exactly the cube with this corner, aligned to the cube grid
+        assert (t0 % ct, h0 % ch, w0 % cw) == (0, 0, 0)
+        assert set(pts) == {(t, h, w) for t in range(t0, t0 + ct) for h in range(h0, h0 + ch)
+                            for w in range(w0, w0 + cw)}
+        corners.append((t0, h0, w0))
+    assert corners == sorted(corners)              # cubes in raster order of their corners
