@@ -174,7 +174,7 @@ WA_API wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, in
  *   overlap; row_bytes a multiple of 16 and both pointers 16-byte aligned
  *   (UNSUPPORTED otherwise).  A bit-exact copy.  An entry of perm outside
  *   [0, n_rows) sets WA_DEVERR_ROW_ID and that row is skipped.  INVALID_ARG: NULL
- *   pointer, n_rows < 1, row_bytes == 0. */
+ *   pointer, n_rows < 1 or above 2^31 - 2^20, row_bytes == 0. */
 WA_API wa_status wa_cube_order(int T, int H_l, int W_l, int C_t, int C_h, int C_w, int32_t* perm);
 WA_API wa_status wa_permute_rows(const void* src, void* dst, const int32_t* perm, int n_rows,
                                  size_t row_bytes, int inverse, void* stream);

@@ -362,6 +362,7 @@ wa_status wa_permute_rows(const void* src, void* dst, const int32_t* perm, int n
                           size_t row_bytes, int inverse, void* stream) {
   WA_REQUIRE(src && dst && perm, "NULL pointer");
   WA_REQUIRE(n_rows >= 1 && row_bytes >= 1, "sizes must be >= 1");
+  WA_REQUIRE(n_rows <= INT_MAX - (1 << 20), "too many rows (at most 2^31 - 2^20)");
   if (row_bytes % 16 != 0 || !aligned16(src) || !aligned16(dst))
     return set_error(WA_ERR_UNSUPPORTED, "permute_rows needs 16-byte aligned rows");
   uint32_t* err = errw();

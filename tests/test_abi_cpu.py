@@ -157,5 +157,6 @@ def test_cube_order_and_permute_validation():
     f = wa.lib.wa_permute_rows
     assert f(None, FAKE, FAKE, 4, 16, 0, None) == wa.WA_ERR_INVALID_ARG
     assert f(FAKE, FAKE, FAKE, 0, 16, 0, None) == wa.WA_ERR_INVALID_ARG
+    assert f(FAKE, FAKE, FAKE, 2**31 - 1, 16, 0, None) == wa.WA_ERR_INVALID_ARG
     assert f(FAKE, FAKE, FAKE, 4, 24, 0, None) == wa.WA_ERR_UNSUPPORTED     # rows of 16-byte multiples
     assert f(FAKE, ctypes.c_void_p(4096 + 8), FAKE, 4, 16, 0, None) == wa.WA_ERR_UNSUPPORTED
