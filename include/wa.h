@@ -223,16 +223,22 @@ WA_API wa_status wa_linear_project(const void* k_act, const void* v_act, const v
  * Some callers cannot call cudaMalloc and have no workspace to hand over: code
  * that runs inside a host framework which owns every device allocation through
  * its own pool, or a real-time loop where an allocation (which can synchronise
- * the device) is not allowed.  This call computes exactly what wa_linear_project
- * computes for bf16 inputs, on the same tcgen05 kernels, but keeps its split-L
- * partial sums in a fixed 32 MiB array that the library holds as a file-scope
- * device variable: every GPU that loads libwa holds those 32 MiB until the
- * process exits.  It calls no cudaMalloc, cudaFree or other allocating routine.
+ * the device) is not allowed.  This call computes what wa_linear_project computes
+ * for bf16 inputs, on the same tcgen05 kernels, to within the order of the float32
+ * sums over L: when the scratch is the limit it uses fewer splits of L than the
+ * workspace entry point, and the partials are then added in a different grouping.
+ * It keeps its split-L partial sums in a fixed 32 MiB array that the library holds
+ * as a file-scope device variable: every GPU that loads libwa holds those 32 MiB
+ * until the process exits.  It calls no cudaMalloc, cudaFree or other allocating
+ * routine.
  *   - The caller still passes inputs and outputs (same layouts as
  *     wa_linear_project; contiguous k_act / v_act [L][H][d], e_k / e_v [L][r]).
  *   - The first call on a device looks the array's device address up
  *     (cudaGetSymbolAddress, once per device, with that device current); make that
- *     first call before any stream capture.
+ *     first call before any stream capture.  The address is kept for the life of
+ *     the process and belongs to the device's primary context: after a
+ *     cudaDeviceReset on that device it is stale, so do not call this entry point
+ *     on a device again once it has been reset.
  *   - All calls share the array, which keeps the last call's contents.  Each call
  *     writes every partial it later reads, so no earlier contents leak into a
  *     result; but calls that overlap on the GPU (two streams at once) race on it

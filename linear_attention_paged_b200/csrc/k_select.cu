@@ -366,7 +366,11 @@ k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int lg_np,
   const double th = static_cast<double>(tau[h]);
   int m = n_kb;
   if (th < 1.0) {
+    // every thread takes the maximum before thread 0 overwrites key[0] with its
+    // exponential below (without this barrier a warp running ahead changes the
+    // maximum that slower warps read, and the masses of their blocks come out wrong)
     const double smax = key[0];
+    __syncthreads();
     const int per = NP / kChooseThreads > 0 ? NP / kChooseThreads : 1;
     const int t0 = tid * per;
     // z_t = exp(s_t - max), kept in place of the sorted scores

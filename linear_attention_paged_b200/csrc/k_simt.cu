@@ -62,9 +62,7 @@ k_simt_attention(int mode, const float* __restrict__ q, int Nq, int H, RowSource
   const float scale = 1.0f / sqrtf(static_cast<float>(D));
   bool bad = false;
 
-  for (int rr = threadIdx.x; rr < B; rr += blockDim.x) {
-    // rows are processed in groups of blockDim.x; each thread owns one query row
-  }
+  // each thread owns one query row of the block
   const int row = i * B + threadIdx.x;
   const bool valid = threadIdx.x < B && row < Nq;
   float qr[D];

@@ -664,7 +664,6 @@ k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W, int4* __restric
   __shared__ uint32_t ms[kMaxPairMaskWords];
   __shared__ int partner[kMaxPairTable];
   __shared__ int nn[kMaxPairTable];
-  __shared__ int progress;
   const int h = blockIdx.x;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, n_warps = blockDim.x >> 5;
   const int n_pairs = (n_qb + 1) / 2;
@@ -716,14 +715,15 @@ k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W, int4* __restric
       for (int o = 16; o > 0; o >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, o));
       if (lane == 0) nn[a] = best == ~0ull ? -1 : static_cast<int>(best & 0xffffffffu);
     }
-    if (threadIdx.x == 0) progress = 0;
     __syncthreads();
+    int paired = 0;
     for (int a = threadIdx.x; a < n_qb; a += blockDim.x) {
       const int b = nn[a];
-      if (b > a && nn[b] == a) { partner[a] = b; partner[b] = a; progress = 1; }
+      if (b > a && nn[b] == a) { partner[a] = b; partner[b] = a; paired = 1; }
     }
-    __syncthreads();
-    if (!progress) break;
+    // barrier and vote in one: every thread sees the same answer, and no shared flag
+    // is reset while a slower thread may still be reading it
+    if (!__syncthreads_or(paired)) break;
   }
   // emit pairs in order of their first block (deterministic); a block left alone
   // (odd count) gets partner -1

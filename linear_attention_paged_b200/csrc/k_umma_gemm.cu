@@ -291,7 +291,9 @@ wa_status launch_umma_project(const void* k, const void* v, RowSource rs, const 
 // still passes its inputs and outputs.
 //
 // The array is kNoAllocScratchBytes (32 MiB) and is held by every GPU that loads
-// this library until the process exits.  All calls share it, so calls that
+// this library until the process exits.  Its device address is looked up once per
+// device and kept for the process: it belongs to the device's primary context and
+// goes stale if that device is reset.  All calls share it, so calls that
 // overlap on the GPU (for instance on two streams at once) race on it; callers
 // must order them.  Each call overwrites every partial it reads before reading
 // it, so the contents left by an earlier call never leak into a result.
@@ -341,17 +343,19 @@ extern "C" wa_status wa_linear_project_noalloc(const void* k_act, const void* v_
     return set_error(WA_ERR_UNSUPPORTED, "wa_linear_project_noalloc takes bf16 inputs only");
   if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "d must be 64 or 128");
   if (r != 128 && r != 256) return set_error(WA_ERR_UNSUPPORTED, "r must be 128 or 256");
-  const int cols = H * d;
+  // as many splits of L as the default launch uses, but no more than the static
+  // scratch holds (2 matrices x n_split x r x H*d floats); the product is formed in
+  // 64 bits, so no H wraps around to a size that would pass
+  const unsigned long long cols64 = static_cast<unsigned long long>(H) * d;
+  const unsigned long long per_split = 2ull * r * cols64 * sizeof(float);
+  if (per_split > kNoAllocScratchBytes)
+    return set_error(WA_ERR_UNSUPPORTED,
+                     "r*H*d = %llu needs %llu bytes of scratch per split; the static scratch holds %zu",
+                     static_cast<unsigned long long>(r) * cols64, per_split, kNoAllocScratchBytes);
+  const int cols = static_cast<int>(cols64);   // < 2^22 here
   const int tn = pick_tn(cols);
   if (tn == 0) return set_error(WA_ERR_UNSUPPORTED, "H*d must be a multiple of 64");
-  // as many splits of L as the default launch uses, but no more than the static
-  // scratch holds (2 matrices x n_split x r x H*d floats)
-  const size_t per_split = 2ull * r * cols * sizeof(float);
   const size_t fit = kNoAllocScratchBytes / per_split;
-  if (fit < 1)
-    return set_error(WA_ERR_UNSUPPORTED,
-                     "r*H*d = %zu needs %zu bytes of scratch per split; the static scratch holds %zu",
-                     static_cast<size_t>(r) * cols, per_split, kNoAllocScratchBytes);
   int n_split = pick_splits(L, r, cols);
   if (static_cast<size_t>(n_split) > fit) n_split = static_cast<int>(fit);
   float* part = nullptr;

@@ -153,7 +153,7 @@ wa_status check_shape(int H, int d, int B, wa_dtype dt) {
   if (d != 64 && d != 128) return set_error(WA_ERR_UNSUPPORTED, "d must be 64 or 128 (got %d)", d);
   if (B != 64) return set_error(WA_ERR_UNSUPPORTED, "B must be 64 (got %d)", B);
   const int vec = dt == WA_BF16 ? 8 : 4;
-  if ((H * d) / vec > 1024) return set_error(WA_ERR_UNSUPPORTED, "H*d too large");
+  if (static_cast<long long>(H) * d / vec > 1024) return set_error(WA_ERR_UNSUPPORTED, "H*d too large");
   return WA_OK;
 }
 

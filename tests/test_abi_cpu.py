@@ -160,3 +160,23 @@ def test_cube_order_and_permute_validation():
     assert f(FAKE, FAKE, FAKE, 2**31 - 1, 16, 0, None) == wa.WA_ERR_INVALID_ARG
     assert f(FAKE, FAKE, FAKE, 4, 24, 0, None) == wa.WA_ERR_UNSUPPORTED     # rows of 16-byte multiples
     assert f(FAKE, ctypes.c_void_p(4096 + 8), FAKE, 4, 16, 0, None) == wa.WA_ERR_UNSUPPORTED
+
+
+def test_noalloc_projection_host_rejections():
+    """wa_linear_project_noalloc rejects on the host, before any CUDA call: shapes whose
+    split partials exceed its fixed scratch, and an H so large that H*d would wrap
+    around in 32-bit arithmetic (2^25 + 1 heads of 128 -> 128 columns)."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("fake pointers are used only where no GPU can be reached")
+    f = wa.lib.wa_linear_project_noalloc
+    assert f(FAKE, FAKE, FAKE, FAKE, 1024, 257, 64, 256, wa.WA_BF16, FAKE, FAKE, None) == \
+        wa.WA_ERR_UNSUPPORTED
+    assert "scratch" in wa.last_error()
+    assert f(FAKE, FAKE, FAKE, FAKE, 1024, (1 << 25) + 1, 128, 128, wa.WA_BF16, FAKE, FAKE, None) == \
+        wa.WA_ERR_UNSUPPORTED
+    assert "scratch" in wa.last_error()
+    assert f(FAKE, FAKE, FAKE, FAKE, 1024, 12, 128, 256, wa.WA_F32, FAKE, FAKE, None) == \
+        wa.WA_ERR_UNSUPPORTED
+    assert f(None, FAKE, FAKE, FAKE, 1024, 12, 128, 256, wa.WA_BF16, FAKE, FAKE, None) == \
+        wa.WA_ERR_INVALID_ARG
