@@ -145,6 +145,22 @@ def dtype_code(t: torch.Tensor) -> int:
 
 _WS: dict = {}
 
+# Canary byte for the buffers this binding hands to the library (outputs and
+# workspaces), or None.  Tests set it (0xFF: NaN in every float and float64, -1 in
+# every int) so that a kernel which leaves part of an output or a workspace
+# unwritten, or reads scratch it did not write first, shows up as a wrong value.
+CANARY: Optional[int] = None
+
+
+def _fill(t: Optional[torch.Tensor]) -> Optional[torch.Tensor]:
+    if t is not None and CANARY is not None:
+        t.view(torch.uint8).fill_(CANARY)
+    return t
+
+
+def _empty(shape, dtype, device) -> torch.Tensor:
+    return _fill(torch.empty(shape, dtype=dtype, device=device))
+
 
 def workspace(nbytes: int, device=None) -> torch.Tensor:
     """Cached per-device scratch buffer of at least ``nbytes`` (256-byte aligned)."""
@@ -155,7 +171,7 @@ def workspace(nbytes: int, device=None) -> torch.Tensor:
         buf = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=dev)
         assert buf.data_ptr() % 256 == 0
         _WS[dev] = buf
-    return buf
+    return _fill(buf)
 
 
 def _need_cuda(*ts):
@@ -167,7 +183,7 @@ def _need_cuda(*ts):
 # --------------------------------------------------------------------- S0
 def wa_prompt_select(e_cur: torch.Tensor, e_chunks: torch.Tensor, stream=None) -> torch.Tensor:
     _need_cuda(e_cur, e_chunks)
-    out = torch.empty(1, dtype=torch.int32, device=e_cur.device)
+    out = _empty(1, torch.int32, e_cur.device)
     _check("wa_prompt_select", lib.wa_prompt_select(_p(e_cur), _p(e_chunks), e_chunks.shape[0],
                                                     e_chunks.shape[1], _p(out), _stream(stream)))
     return out
@@ -180,10 +196,9 @@ def wa_page_score(q, k_pool, cand_pages, K_p: int, B: int = 64, want_blockmean: 
     Nq, H, d = q.shape
     P_, T_p = k_pool.shape[0], k_pool.shape[1]
     n_c = cand_pages.numel()
-    alpha = torch.empty(n_c, dtype=torch.float64, device=q.device)
-    sel = torch.empty(K_p, dtype=torch.int32, device=q.device)
-    kbm = (torch.empty((n_c, T_p // B, H, d), dtype=torch.float64, device=q.device)
-           if want_blockmean else None)
+    alpha = _empty(n_c, torch.float64, q.device)
+    sel = _empty(K_p, torch.int32, q.device)
+    kbm = _empty((n_c, T_p // B, H, d), torch.float64, q.device) if want_blockmean else None
     nbytes = lib.wa_page_score_workspace_size(Nq, H, d, n_c, T_p, B)
     ws = workspace(nbytes, q.device)
     _check("wa_page_score", lib.wa_page_score(
@@ -200,8 +215,8 @@ def wa_gather_pages(k_pool, v_pool, sel, stream=None, out=None):
     P_, T_p, H, d = k_pool.shape
     K_p = sel.numel()
     if out is None:
-        k_act = torch.empty((K_p * T_p, H, d), dtype=k_pool.dtype, device=k_pool.device)
-        v_act = torch.empty_like(k_act)
+        k_act = _empty((K_p * T_p, H, d), k_pool.dtype, k_pool.device)
+        v_act = _empty((K_p * T_p, H, d), k_pool.dtype, k_pool.device)
     else:
         k_act, v_act = out
         _need_cuda(k_act, v_act)
@@ -228,7 +243,7 @@ def wa_permute_rows(src, perm, inverse: bool = False, out=None, stream=None):
     _need_cuda(src, perm)
     assert perm.dtype == torch.int32 and perm.numel() == src.shape[0]
     if out is None:
-        out = torch.empty_like(src)
+        out = _empty(src.shape, src.dtype, src.device)
     else:
         _need_cuda(out)
         assert out.shape == src.shape and out.dtype == src.dtype
@@ -270,9 +285,9 @@ def wa_block_select(q, tau, B: int = 64, k_act=None, k_blockmean=None, L: Option
         L = k_act.shape[0] if k_act is not None else k_blockmean.shape[0] * B
     n_qb, n_kb = -(-Nq // B), -(-L // B)
     W = -(-n_kb // 32)
-    idx = torch.empty((H, n_qb, n_kb), dtype=torch.int32, device=q.device)
-    cnt = torch.empty((H, n_qb), dtype=torch.int32, device=q.device)
-    mask = torch.empty((H, n_qb, W), dtype=torch.int32, device=q.device)
+    idx = _empty((H, n_qb, n_kb), torch.int32, q.device)
+    cnt = _empty((H, n_qb), torch.int32, q.device)
+    mask = _empty((H, n_qb, W), torch.int32, q.device)
     nbytes = lib.wa_block_select_workspace_size(Nq, H, d, L, B)
     ws = workspace(nbytes, q.device)
     _check("wa_block_select", lib.wa_block_select(
@@ -286,8 +301,8 @@ def wa_linear_project(k_act, v_act, e_k, e_v, stream=None):
     _need_cuda(k_act, v_act, e_k, e_v)
     L, H, d = k_act.shape
     r = e_k.shape[1]
-    k_til = torch.empty((r, H, d), dtype=k_act.dtype, device=k_act.device)
-    v_til = torch.empty_like(k_til)
+    k_til = _empty((r, H, d), k_act.dtype, k_act.device)
+    v_til = _empty((r, H, d), k_act.dtype, k_act.device)
     dt = dtype_code(k_act)
     nbytes = lib.wa_linear_project_workspace_size(L, H, d, r, dt)
     ws = workspace(nbytes, k_act.device)
@@ -304,8 +319,8 @@ def wa_linear_project_noalloc(k_act, v_act, e_k, e_v, stream=None):
     _need_cuda(k_act, v_act, e_k, e_v)
     L, H, d = k_act.shape
     r = e_k.shape[1]
-    k_til = torch.empty((r, H, d), dtype=k_act.dtype, device=k_act.device)
-    v_til = torch.empty_like(k_til)
+    k_til = _empty((r, H, d), k_act.dtype, k_act.device)
+    v_til = _empty((r, H, d), k_act.dtype, k_act.device)
     _check("wa_linear_project_noalloc", lib.wa_linear_project_noalloc(
         _p(k_act), _p(v_act), _p(e_k), _p(e_v), L, H, d, r, dtype_code(k_act), _p(k_til),
         _p(v_til), _stream(stream)))
@@ -322,9 +337,9 @@ def wa_hsa_attention(q, k_act, v_act, blk_mask, k_til, v_til, gate, B: int = 64,
     L = k_act.shape[0]
     r = k_til.shape[0]
     dt = dtype_code(q)
-    out = torch.empty_like(q)
-    o_sp = torch.empty(q.shape, dtype=torch.float32, device=q.device) if want_branches else None
-    o_lin = torch.empty(q.shape, dtype=torch.float32, device=q.device) if want_branches else None
+    out = _empty(q.shape, q.dtype, q.device)
+    o_sp = _empty(q.shape, torch.float32, q.device) if want_branches else None
+    o_lin = _empty(q.shape, torch.float32, q.device) if want_branches else None
     nbytes = lib.wa_hsa_attention_workspace_size(Nq, H, d, L, B, r, dt)
     ws = workspace(nbytes, q.device)
     if gate_lin is None:
@@ -360,7 +375,7 @@ class HSAStep:
         n_qb, n_kb = -(-Nq // B), -(-(L + (Nq if k_cur is not None else 0)) // B)
         W = -(-n_kb // 32)
         dev = q.device
-        self.out = out if out is not None else torch.empty_like(q)
+        self.out = out if out is not None else _empty(q.shape, q.dtype, q.device)
         self._keep = [q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, e_cur, e_chunks]
         a = StepArgs()
         a.e_cur, a.e_chunks = _p(e_cur), _p(e_chunks)
@@ -380,12 +395,12 @@ class HSAStep:
         self.inter = {}
         if keep_intermediates:
             self.inter = dict(
-                chunk=torch.empty(1, dtype=torch.int32, device=dev),
-                alpha=torch.empty(n_c, dtype=torch.float64, device=dev),
-                sel=torch.empty(K_p, dtype=torch.int32, device=dev),
-                blk_mask=torch.empty((H, n_qb, W), dtype=torch.int32, device=dev),
-                k_til=torch.empty((r, H, d), dtype=q.dtype, device=dev),
-                v_til=torch.empty((r, H, d), dtype=q.dtype, device=dev))
+                chunk=_empty(1, torch.int32, dev),
+                alpha=_empty(n_c, torch.float64, dev),
+                sel=_empty(K_p, torch.int32, dev),
+                blk_mask=_empty((H, n_qb, W), torch.int32, dev),
+                k_til=_empty((r, H, d), q.dtype, dev),
+                v_til=_empty((r, H, d), q.dtype, dev))
             a.chunk_out = _p(self.inter["chunk"])
             a.alpha_out = _p(self.inter["alpha"])
             a.sel_out = _p(self.inter["sel"])
@@ -398,7 +413,7 @@ class HSAStep:
             # a zero size means validation failed: surface the reason
             _check("wa_hsa_step_workspace_size", lib.wa_hsa_step(ctypes.byref(a), None, 0, None))
         self.nbytes = nbytes
-        self.ws = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+        self.ws = _empty(nbytes, torch.uint8, dev)
         assert self.ws.data_ptr() % 256 == 0
 
     def __call__(self, stream=None):

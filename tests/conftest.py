@@ -24,3 +24,22 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(autouse=True)
+def _canary_fill(request):
+    """GPU tests run with every output and workspace the binding allocates filled with
+    0xFF bytes first (NaN in floats, -1 in integers), so that a kernel which leaves part
+    of its output unwritten or reads scratch it never wrote fails the comparison."""
+    if "gpu" not in request.keywords:
+        yield
+        return
+    from linear_attention_paged_b200 import build
+    build.build()
+    from linear_attention_paged_b200 import wa
+    old = wa.CANARY
+    wa.CANARY = 0xFF
+    try:
+        yield
+    finally:
+        wa.CANARY = old

@@ -7,10 +7,13 @@ import torch
 # Tolerances against the float64 oracle: bf16 inputs -> max-abs 2e-2 and relative
 # Frobenius 5e-3; fp32 inputs -> 1e-4 for both.
 TOL = {"bf16": (2e-2, 5e-3), "f32": (1e-4, 1e-4)}
-# Index outputs must match bit for bit except where the oracle's own margin is
-# below this (a near tie that float rounding may decide either way); such rows are
-# counted and logged.
+# Rows whose oracle margin is below MARGIN are near ties: they are counted and
+# logged.  The GPU takes every index decision in float64 as the oracle does, from the
+# same input bits, so only a margin at the scale of float64 rounding of the sums
+# (below MARGIN_F64) may decide a row differently; every other row must match bit
+# for bit, near tie or not.
 MARGIN = 1e-5
+MARGIN_F64 = 1e-12
 
 
 def to64(x) -> np.ndarray:
@@ -51,7 +54,8 @@ def mask_to_sets(mask: torch.Tensor, n_kb: int):
 
 
 def compare_selection(gpu_sets, kept, margin, what: str):
-    """Rows must match exactly unless the oracle margin is below MARGIN."""
+    """Rows must match exactly unless the oracle margin is below MARGIN_F64; rows with
+    a margin below MARGIN (near ties) are counted and logged whether they match or not."""
     H = len(kept)
     n_rows = n_excused = 0
     bad = []
@@ -59,14 +63,14 @@ def compare_selection(gpu_sets, kept, margin, what: str):
         for i in range(len(kept[h])):
             n_rows += 1
             if gpu_sets[h][i] != kept[h][i]:
-                if margin[h][i] < MARGIN:
+                if margin[h][i] < MARGIN_F64:
                     n_excused += 1
                     print(f"[near-tie] {what}: head {h} block {i} margin {margin[h][i]:.2e}")
                 else:
                     bad.append((h, i, margin[h][i], len(gpu_sets[h][i]), len(kept[h][i])))
     n_near = int(sum(1 for h in range(H) for i in range(len(kept[h])) if margin[h][i] < MARGIN))
-    print(f"[parity] {what}: {n_rows} rows, {len(bad)} mismatches, {n_excused} excused near ties "
-          f"({n_near} rows with margin < {MARGIN:g})")
+    print(f"[parity] {what}: {n_rows} rows, {len(bad)} mismatches, {n_excused} excused "
+          f"(margin < {MARGIN_F64:g}); {n_near} near ties (margin < {MARGIN:g}) checked bit for bit")
     assert not bad, f"{what}: selection mismatches (h, i, margin, |gpu|, |oracle|): {bad[:5]}"
     return n_excused
 

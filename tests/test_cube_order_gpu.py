@@ -7,7 +7,7 @@ import torch
 
 from oracle import hsa_oracle as O
 from linear_attention_paged_b200 import workloads as W
-from tests.helpers import assert_close, compare_selection, mask_to_sets
+from tests.helpers import MARGIN_F64, assert_close, compare_selection, mask_to_sets
 
 pytestmark = pytest.mark.gpu
 
@@ -78,7 +78,7 @@ def test_hsa_step_on_cube_order(wa):
     ref_in["q"] = inp["q"].cpu()[oq]
     ref_in["gate"] = inp["gate"].cpu()[oq]
     res = O.hsa_step(ref_in, cfg.B, cfg.K_p)
-    if res["page_margin"] >= 1e-5:
+    if res["page_margin"] >= MARGIN_F64:
         assert inter["sel"].cpu().tolist() == res["sel"]
     compare_selection(mask_to_sets(inter["blk_mask"], cfg.n_kb), res["kept"], res["block_margin"],
                       "cube-order masks")

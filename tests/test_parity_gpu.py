@@ -11,7 +11,8 @@ import torch
 
 from oracle import hsa_oracle as O
 from linear_attention_paged_b200 import workloads as W
-from tests.helpers import (assert_close, compare_selection, mask_to_sets, kept_fraction, to64)
+from tests.helpers import (MARGIN_F64, assert_close, compare_selection, mask_to_sets, kept_fraction,
+                           to64)
 
 pytestmark = pytest.mark.gpu
 
@@ -81,7 +82,7 @@ def test_page_score_and_gather(wa, cfg):
     np.testing.assert_allclose(to64(alpha), a_ref, rtol=1e-10, atol=1e-13)
     margin = O.page_margin(a_ref, cfg.K_p)
     ref_sel = [int(inp["cand"][j]) for j in O.select_pages(a_ref, cfg.K_p)]
-    if margin >= 1e-5:
+    if margin >= MARGIN_F64:
         assert sel.cpu().tolist() == ref_sel
     # block means of every candidate page
     ref_bm = np.stack([O.block_means(k_cand[c], cfg.B) for c in range(cfg.n_c)])
@@ -271,7 +272,7 @@ def test_hsa_step_small(wa, cfg, fused):
                                 inp["e_v"], inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B,
                                 fused_gather=fused, keep_intermediates=True)
     res = O.hsa_step(inp, cfg.B, cfg.K_p)
-    if res["page_margin"] >= 1e-5:
+    if res["page_margin"] >= MARGIN_F64:
         assert inter["sel"].cpu().tolist() == res["sel"]
     compare_selection(mask_to_sets(inter["blk_mask"], cfg.n_kb), res["kept"], res["block_margin"],
                       f"{cfg.name} step masks")
@@ -298,7 +299,7 @@ def _full_size_step(wa, cfg, samples, gen_device="cuda"):
     if "chunk" in res:
         assert int(step.inter["chunk"].item()) == res["chunk"]
     np.testing.assert_allclose(to64(step.inter["alpha"]), res["alpha"], rtol=1e-9, atol=1e-13)
-    if res["page_margin"] >= 1e-5:
+    if res["page_margin"] >= MARGIN_F64:
         assert step.inter["sel"].cpu().tolist() == res["sel"]
     n_kb = sparse_blocks(cfg)
     compare_selection(mask_to_sets(step.inter["blk_mask"], n_kb), res["kept"], res["block_margin"],
@@ -347,6 +348,15 @@ def test_hsa_step_intra_keys_small(wa, cfg, fused):
     check_device_ok(wa)
 
 
+def test_full_size_narrow_projection_step(wa):
+    """Three heads of d=64 (H*d = 192, one 64-column projection tile) and r = 128 at the
+    one-layer page shapes: the smallest projection configuration, whose pipeline leaves
+    room on an SM for block-selection CTAs running beside it on the other stream."""
+    cfg = W.C1.with_(name="c1_narrow_proj", H=3, d=64, r=128, seed=43)
+    samples = [(0, 0), (2, cfg.n_qb - 1), (1, 36)]
+    _full_size_step(wa, cfg, samples)
+
+
 def test_full_size_stress_step(wa):
     cfg = W.C2
     samples = [(0, 0), (4, cfg.n_qb - 1), (7, 20), (11, 50)]
@@ -393,7 +403,7 @@ def test_hsa_step_with_page_index(wa, cfg):
                                 keep_intermediates=True, page_index=idx)
     res = O.hsa_step(inp, cfg.B, cfg.K_p)
     np.testing.assert_allclose(to64(inter["alpha"]), res["alpha"], rtol=1e-9, atol=1e-13)
-    if res["page_margin"] >= 1e-5:
+    if res["page_margin"] >= MARGIN_F64:
         assert inter["sel"].cpu().tolist() == res["sel"]
     compare_selection(mask_to_sets(inter["blk_mask"], cfg.n_kb), res["kept"], res["block_margin"],
                       f"{cfg.name} masks (page index)")
@@ -444,7 +454,7 @@ def test_denoise_stack_procedure(wa):
         step_inp = dict(inp, q=q, gate=gate, cand=hist[0].cpu())
         step_inp.pop("e_cur", None)
         res = O.hsa_step(step_inp, cfg.B, cfg.K_p, rows_of_blocks=[(0, 0), (7, cfg.n_qb - 1)])
-        if res["page_margin"] >= 1e-5:
+        if res["page_margin"] >= MARGIN_F64:
             assert sel == res["sel"]
         for (h, i), blk in res["blocks"].items():
             r0, r1 = i * cfg.B, min(cfg.Nq, (i + 1) * cfg.B)
