@@ -68,6 +68,23 @@ typedef enum wa_dtype { WA_F32 = 0, WA_BF16 = 1 } wa_dtype;
 #define WA_DEVERR_TIMEOUT   0x4u  /* a bounded wait inside a kernel gave up         */
 #define WA_DEVERR_ROW_ID    0x8u  /* a row index outside [0, n_rows) in wa_permute_rows */
 
+/* Bound of every mbarrier wait inside the kernels launched after this call, in
+ * nanoseconds of %globaltimer time (process-wide; 2 s by default).  A wait that runs
+ * out sets WA_DEVERR_TIMEOUT, makes the kernel's other roles stop, waits (within the
+ * same bound) for the loads and MMAs the kernel itself had issued, frees its TMEM
+ * and returns.  No counterpart in the paper: it is the runtime's failure detection.
+ * INVALID_ARG outside [1e3, 6e10]. */
+WA_API wa_status wa_set_wait_limit_ns(uint64_t limit_ns);
+WA_API uint64_t wa_get_wait_limit_ns(void);
+
+/* Failure-detection self-test (no counterpart in the paper).  Launches one CTA that
+ * waits, through the kernels' bounded wait limited to limit_ns, on an mbarrier that no
+ * thread ever arrives at.  The wait gives up: the kernel sets WA_DEVERR_TIMEOUT in the
+ * device error word (read it with wa_device_error) and returns, with no load or MMA
+ * in flight, so the context stays usable.  elapsed_ns (device, nullable) receives the
+ * %globaltimer time the wait took.  INVALID_ARG: limit_ns outside [1e3, 1e9]. */
+WA_API wa_status wa_check_bounded_wait(uint64_t limit_ns, uint64_t* elapsed_ns, void* stream);
+
 /* Message describing the calling thread's most recent failure ("" if none). */
 WA_API const char* wa_last_error(void);
 

@@ -93,6 +93,8 @@ struct Shared {
   uint64_t s_free;        // S_t loaded by all eight softmax warps
   uint64_t p_full[2];     // P_t of group g stored, one arrival per warp of the group
   uint64_t o_done;        // O_g += P_t V_t complete (both groups)
+  uint64_t drain[2];      // abort path: every MMA of issuer 0 (S) / 1 (P V) complete
+  uint64_t wait_ns;       // bound of every wait (wa_set_wait_limit_ns)
   uint32_t tmem_base;
   int abort_flag;
   int scan[8];
@@ -104,19 +106,9 @@ struct Shared {
 // Bounded wait that also gives up when another role has aborted.
 __device__ __forceinline__ bool wait_bar(uint64_t* bar, uint32_t parity, Shared& sh,
                                          uint32_t* err) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u) {
-      if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) return false;
-      if (globaltimer_ns() - t0 > 2000000000ull) {
-        atomicOr(err, WA_DEVERR_TIMEOUT);
-        *reinterpret_cast<volatile int*>(&sh.abort_flag) = 1;
-        return false;
-      }
-    }
-  }
+  const int r = mbar_wait_bounded(bar, parity, &sh.abort_flag, sh.wait_ns);
+  if (r == kWaitTimeout) atomicOr(err, WA_DEVERR_TIMEOUT);
+  return r == kWaitOk;
 }
 
 __device__ __forceinline__ float ex2(float x) {
@@ -200,7 +192,8 @@ k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CU
                  RowSource rs, const uint32_t* __restrict__ blk_mask, int W, int n_qb,
                  const int4* __restrict__ pairs, const int4* __restrict__ items, Partials part,
                  const float* __restrict__ gate, float lin_sign, float* __restrict__ lin_ws,
-                 __nv_bfloat16* __restrict__ out, float* __restrict__ o_branch, uint32_t* err) {
+                 __nv_bfloat16* __restrict__ out, float* __restrict__ o_branch, uint32_t* err,
+                 uint64_t wait_ns) {
   using C = Cfg<D>;
   extern __shared__ uint8_t smem_dyn[];
   __shared__ Shared sh;
@@ -238,6 +231,9 @@ k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CU
     mbar_init(&sh.p_full[0], 4);
     mbar_init(&sh.p_full[1], 4);
     mbar_init(&sh.o_done, 1);
+    mbar_init(&sh.drain[0], 1);
+    mbar_init(&sh.drain[1], 1);
+    sh.wait_ns = wait_ns;
     sh.abort_flag = 0;
     fence_mbar_init();
   }
@@ -292,6 +288,7 @@ k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CU
   const uint32_t* list2 = reinterpret_cast<const uint32_t*>(sh.list);  // entries 2t, 2t+1
   const bool odd_tail = (n_blk & 1) != 0;   // the last iteration holds one block
   const int bpp = rs.page_ids ? rs.page_rows / kBN : 0;
+  int issued = 0;   // producers: iterations whose loads were issued (for the abort drain)
 
   if (warp == 0 || warp == 2) {
     // ------------------------------------------------------------ producers:
@@ -324,6 +321,7 @@ k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CU
           for (int p = 0; p < C::kPanels; ++p)
             tma_load_2d(dst + p * C::kPanelBytes + kBN * 128, b2 ? tm2 : tm, full, h * D + p * 64, rb);
         }
+        issued = t + 1;
       }
     }
   } else if (warp == 1) {
@@ -588,6 +586,28 @@ k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CU
   }
   tc_fence_before();
   __syncthreads();
+  if (sh.abort_flag) {
+    // A role gave up: before TMEM is freed and the shared memory handed to another
+    // CTA, wait (bounded, whatever the flag says) for this CTA's own asynchronous
+    // work -- the loads each producer issued into its ring (at most the last `ring`
+    // can still be outstanding) and every MMA of both issuers (a commit to a drain
+    // barrier arrives once all of the issuing thread's earlier MMAs are complete).
+    int never = 0;
+    if ((warp == 0 || warp == 2) && lane == 0) {
+      const int ring = warp == 0 ? kRingK : kRingV;
+      for (int t = issued > ring ? issued - ring : 0; t < issued; ++t) {
+        uint64_t* full = warp == 0 ? &sh.k_full[t % ring] : &sh.v_full[t % ring];
+        if (mbar_wait_bounded(full, (t / ring) & 1, &never, sh.wait_ns) == kWaitTimeout)
+          atomicOr(err, WA_DEVERR_TIMEOUT);
+      }
+    } else if ((warp == 1 || warp == 3) && lane == 0) {
+      uint64_t* bar = &sh.drain[warp == 1 ? 0 : 1];
+      mma_commit(bar);
+      if (mbar_wait_bounded(bar, 0, &never, sh.wait_ns) == kWaitTimeout) atomicOr(err, WA_DEVERR_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, kTmemCols);
@@ -823,7 +843,8 @@ void launch_attn_kernel(int grid, cudaStream_t st, const void* q, const CUtensor
   k_umma_attention<D><<<grid, kThreads, smem, st>>>(static_cast<const __nv_bfloat16*>(q), tk, tv, tk2, tv2, mode, Nq, H, rs.L + rs.L2, rs,
                                                      blk_mask, W,
                                                      n_qb, pairs, items, part, gate, lin_sign, lin_ws,
-                                                     static_cast<__nv_bfloat16*>(out), o_branch, err);
+                                                     static_cast<__nv_bfloat16*>(out), o_branch, err,
+                                                     wait_limit_ns());
 }
 
 // The keys/values of the first segment (pool pages or a contiguous buffer) and,

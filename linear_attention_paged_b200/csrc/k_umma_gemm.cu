@@ -47,24 +47,16 @@ struct GShared {
   uint64_t full[8];
   uint64_t empty[8];
   uint64_t acc_full;
+  uint64_t drain;        // abort path: every MMA of the issuer complete
+  uint64_t wait_ns;      // bound of every wait (wa_set_wait_limit_ns)
   uint32_t tmem_base;
   int abort_flag;
 };
 
 __device__ __forceinline__ bool gwait(uint64_t* bar, uint32_t parity, GShared& sh, uint32_t* err) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u) {
-      if (*reinterpret_cast<volatile int*>(&sh.abort_flag)) return false;
-      if (globaltimer_ns() - t0 > 2000000000ull) {
-        atomicOr(err, WA_DEVERR_TIMEOUT);
-        *reinterpret_cast<volatile int*>(&sh.abort_flag) = 1;
-        return false;
-      }
-    }
-  }
+  const int r = mbar_wait_bounded(bar, parity, &sh.abort_flag, sh.wait_ns);
+  if (r == kWaitTimeout) atomicOr(err, WA_DEVERR_TIMEOUT);
+  return r == kWaitOk;
 }
 
 template <int NSUB, int TN>
@@ -72,7 +64,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_umma_project(const __grid_constant__ CUtensorMap tmEK, const __grid_constant__ CUtensorMap tmEV,
                const __grid_constant__ CUtensorMap tmXK, const __grid_constant__ CUtensorMap tmXV,
                RowSource rs, int L, int cols, int n_split, float* __restrict__ part,
-               uint32_t* err) {
+               uint32_t* err, uint64_t wait_ns) {
   using C = GCfg<NSUB, TN>;
   extern __shared__ uint8_t smem_dyn[];
   __shared__ GShared sh;
@@ -93,6 +85,8 @@ k_umma_project(const __grid_constant__ CUtensorMap tmEK, const __grid_constant__
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) { mbar_init(&sh.full[s], 1); mbar_init(&sh.empty[s], 1); }
     mbar_init(&sh.acc_full, 1);
+    mbar_init(&sh.drain, 1);
+    sh.wait_ns = wait_ns;
     sh.abort_flag = 0;
     fence_mbar_init();
   }
@@ -104,6 +98,7 @@ k_umma_project(const __grid_constant__ CUtensorMap tmEK, const __grid_constant__
   __syncthreads();
   tc_fence_after();
   const uint32_t tbase = sh.tmem_base;
+  int issued = 0;   // producer: stages whose loads were issued (for the abort drain)
 
   if (warp == 0) {
     if (lane == 0) {
@@ -125,6 +120,7 @@ k_umma_project(const __grid_constant__ CUtensorMap tmEK, const __grid_constant__
         for (int p = 0; p < C::kR / 64; ++p) tma_load_2d(As + p * 8192, tE, &sh.full[s], p * 64, l0);
         for (int p = 0; p < TN / 64; ++p)
           tma_load_2d(Bs + p * 8192, tX, &sh.full[s], nt * TN + p * 64, row);
+        issued = t + 1;
       }
     }
   } else if (warp == 1) {
@@ -178,6 +174,24 @@ k_umma_project(const __grid_constant__ CUtensorMap tmEK, const __grid_constant__
   }
   tc_fence_before();
   __syncthreads();
+  if (sh.abort_flag) {
+    // A role gave up: wait (bounded, whatever the flag says) for the loads the
+    // producer issued (at most the last kStages can be outstanding) and for every
+    // MMA of the issuer, before TMEM is freed and the shared memory reused.
+    int never = 0;
+    if (warp == 0 && lane == 0) {
+      for (int t = issued > C::kStages ? issued - C::kStages : 0; t < issued; ++t)
+        if (mbar_wait_bounded(&sh.full[t % C::kStages], (t / C::kStages) & 1, &never, sh.wait_ns) ==
+            kWaitTimeout)
+          atomicOr(err, WA_DEVERR_TIMEOUT);
+    } else if (warp == 1 && lane == 0) {
+      mma_commit(&sh.drain);
+      if (mbar_wait_bounded(&sh.drain, 0, &never, sh.wait_ns) == kWaitTimeout)
+        atomicOr(err, WA_DEVERR_TIMEOUT);
+    }
+    tc_fence_before();
+    __syncthreads();
+  }
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tbase, C::kTmem);
@@ -227,7 +241,7 @@ void launch_proj(dim3 grid, cudaStream_t st, const CUtensorMap& a, const CUtenso
   using C = GCfg<NSUB, TN>;
   cudaFuncSetAttribute(k_umma_project<NSUB, TN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   k_umma_project<NSUB, TN><<<grid, kThreads, C::kSmem, st>>>(a, b, c, d, rs, L, cols, n_split,
-                                                             part, err);
+                                                             part, err, wait_limit_ns());
 }
 
 }  // namespace

@@ -46,16 +46,26 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
   return t;
 }
-// Bounded wait: gives up (returns false, the caller records a timeout and
-// returns) once about `limit_ns` of wall time has passed, so that a protocol
-// error can never hang the GPU.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
-                                          uint64_t limit_ns = 2000000000ull) {
-  if (mbar_try_wait(bar, parity)) return true;
+// Bounded wait on the phase of `bar` with parity `parity`, shared by every kernel
+// that waits on an mbarrier.  Every 256 tries it looks at the CTA's abort flag
+// (raised by a role that gave up, so the others stop waiting too) and at the time
+// spent; once more than `limit_ns` of %globaltimer time has passed it raises the
+// flag itself and reports a timeout, so that a protocol error can never hang the
+// GPU.  The caller records the timeout in the device error word.
+enum WaitResult : int { kWaitOk = 0, kWaitAborted = 1, kWaitTimeout = 2 };
+__device__ __forceinline__ int mbar_wait_bounded(uint64_t* bar, uint32_t parity, int* abort_flag,
+                                                 uint64_t limit_ns) {
+  if (mbar_try_wait(bar, parity)) return kWaitOk;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((i & 255u) == 0u && globaltimer_ns() - t0 > limit_ns) return false;
+    if (mbar_try_wait(bar, parity)) return kWaitOk;
+    if ((i & 255u) == 0u) {
+      if (*reinterpret_cast<volatile int*>(abort_flag)) return kWaitAborted;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *reinterpret_cast<volatile int*>(abort_flag) = 1;
+        return kWaitTimeout;
+      }
+    }
   }
 }
 

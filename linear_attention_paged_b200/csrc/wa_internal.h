@@ -33,6 +33,9 @@ struct RowSource {
 wa_status set_error(wa_status s, const char* fmt, ...);
 wa_status check_launch(const char* what);
 uint32_t* device_error_word();  // current device's error word (device address)
+// Bound, in nanoseconds of %globaltimer time, of every mbarrier wait in the kernels
+// launched from now on (wa_set_wait_limit_ns; 2 s by default).
+uint64_t wait_limit_ns();
 
 // ---------------------------------------------------------------- selection
 // S0: cosine of every chunk embedding with the current one, argmax -> chunk_out.

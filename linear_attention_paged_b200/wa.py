@@ -98,6 +98,9 @@ _SIGS = {
     "wa_tier_flush": (c_int, [P, P]),
     "wa_tier_slot_of": (c_int, [P, c_int, P]),
     "wa_tier_get_stats": (c_int, [P, P]),
+    "wa_set_wait_limit_ns": (c_int, [ctypes.c_uint64]),
+    "wa_get_wait_limit_ns": (ctypes.c_uint64, []),
+    "wa_check_bounded_wait": (c_int, [ctypes.c_uint64, P, P]),
     "wa_cube_order": (c_int, [c_int] * 6 + [P]),
     "wa_permute_rows": (c_int, [P, P, P, c_int, c_size_t, c_int, P]),
 }
@@ -431,6 +434,23 @@ def wa_hsa_step(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 
                  k_cur=k_cur, v_cur=v_cur)
     out = st(stream)
     return (out, st.inter) if keep_intermediates else out
+
+
+def wa_set_wait_limit_ns(limit_ns: int) -> None:
+    """Bound of every mbarrier wait in the kernels launched from now on (ns)."""
+    _check("wa_set_wait_limit_ns", lib.wa_set_wait_limit_ns(int(limit_ns)))
+
+
+def wa_get_wait_limit_ns() -> int:
+    return int(lib.wa_get_wait_limit_ns())
+
+
+def wa_check_bounded_wait(limit_ns: int, stream=None) -> torch.Tensor:
+    """Run the bounded-wait self-test kernel (a wait nobody ends); returns a device
+    uint64 tensor (as int64) holding the time the wait took, in ns."""
+    el = _empty(1, torch.int64, torch.device("cuda", torch.cuda.current_device()))
+    _check("wa_check_bounded_wait", lib.wa_check_bounded_wait(int(limit_ns), _p(el), _stream(stream)))
+    return el
 
 
 def wa_device_error(stream=None) -> int:

@@ -180,3 +180,19 @@ def test_noalloc_projection_host_rejections():
         wa.WA_ERR_UNSUPPORTED
     assert f(None, FAKE, FAKE, FAKE, 1024, 12, 128, 256, wa.WA_BF16, FAKE, FAKE, None) == \
         wa.WA_ERR_INVALID_ARG
+
+
+def test_wait_limit_setting_and_selftest_validation():
+    """The bound of the kernels' mbarrier waits is a process-wide setting with a checked
+    range; the bounded-wait self-test rejects limits outside its range on the host."""
+    default = wa.wa_get_wait_limit_ns()
+    assert default == 2_000_000_000
+    for bad in (0, 999, 60_000_000_001):
+        assert wa.lib.wa_set_wait_limit_ns(bad) == wa.WA_ERR_INVALID_ARG
+    assert wa.wa_get_wait_limit_ns() == default
+    wa.wa_set_wait_limit_ns(5_000_000)
+    assert wa.wa_get_wait_limit_ns() == 5_000_000
+    wa.wa_set_wait_limit_ns(default)
+    for bad in (0, 999, 1_000_000_001):
+        assert wa.lib.wa_check_bounded_wait(bad, None, None) == wa.WA_ERR_INVALID_ARG
+        assert "limit" in wa.last_error()
