@@ -1,12 +1,11 @@
-// k_select.cu -- the index-producing steps of the HSA decode step:
+// k_select.cu -- the index-producing steps of the HSA decode step besides the page
+// scores (those, and the block sums every step starts from, are in k_blocksum.cu):
 //   S0 prompt-level retrieval (cosine top-1 chunk),
-//   S1 page-level retrieval (mean-query . mean-key page scores, top-K_p),
 //   S3 head-adaptive block selection (pooled block scores, minimal mass prefix).
-// WorldAttention §3.2 "Stage 1", "Stage 2"; §3.3 "Head-level sparsity adaptation".
+// WorldAttention §3.2 "Stage 1"; §3.3 "Head-level sparsity adaptation".
 //
 // Every quantity that decides an index is computed in float64, so the decision is
-// taken in the same precision as the float64 reference; the HBM passes read the
-// bf16/fp32 inputs once with 16-byte vector loads.
+// taken in the same precision as the float64 reference.
 #include <cuda_bf16.h>
 
 #include <cfloat>
@@ -23,37 +22,6 @@ __device__ __forceinline__ double warp_sum(double v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
   return v;
-}
-
-// Sum over a CTA of blockDim.x <= 1024 threads; result valid in every thread.
-__device__ double block_sum(double v, double* red /*[32]*/) {
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nw = (blockDim.x + 31) >> 5;
-  v = warp_sum(v);
-  __syncthreads();
-  if (lane == 0) red[warp] = v;
-  __syncthreads();
-  double t = 0.0;
-  for (int w = 0; w < nw; ++w) t += red[w];  // fixed order: deterministic
-  return t;
-}
-
-// 16-byte vectors of inputs, widened to double.
-__device__ __forceinline__ void load_raw(const float* p, uint4& r) {
-  r = __ldg(reinterpret_cast<const uint4*>(p));
-}
-__device__ __forceinline__ void widen(const float*, const uint4& r, double (&o)[4]) {
-  o[0] = __uint_as_float(r.x); o[1] = __uint_as_float(r.y);
-  o[2] = __uint_as_float(r.z); o[3] = __uint_as_float(r.w);
-}
-__device__ __forceinline__ void load_raw(const __nv_bfloat16* p, uint4& r) {
-  r = __ldg(reinterpret_cast<const uint4*>(p));
-}
-__device__ __forceinline__ double bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
-__device__ __forceinline__ double bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
-__device__ __forceinline__ void widen(const __nv_bfloat16*, const uint4& r, double (&o)[8]) {
-  o[0] = bf16_lo(r.x); o[1] = bf16_hi(r.x); o[2] = bf16_lo(r.y); o[3] = bf16_hi(r.y);
-  o[4] = bf16_lo(r.z); o[5] = bf16_hi(r.z); o[6] = bf16_lo(r.w); o[7] = bf16_hi(r.w);
 }
 
 // ------------------------------------------------------------------ S0
@@ -101,76 +69,6 @@ k_prompt_select(const float* __restrict__ e_cur, const float* __restrict__ e_chu
   }
 }
 
-// ------------------------------------------------------------------ S1 HBM pass
-// One CTA sums the B-row blocks [b0, b1) of one source (a pool page, or the buffer
-// itself) over one chunk of columns; thread t owns V consecutive columns.  Rows are
-// read with 16-byte loads, sixteen in flight per thread.  Optionally (qbar != null)
-// the CTA also forms the dot product of its running column sums with qbar, so the
-// page scores need only one scalar per CTA afterwards.
-template <typename T, int V>
-__global__ void __launch_bounds__(256)
-k_rowblock_sum(const T* __restrict__ x, const int32_t* __restrict__ src_ids, int n_pages,
-               int rows, int cols, int B, int nb, int bps, int block0, int nb_end, int bs_by_page,
-               double* __restrict__ blocksum, const double* __restrict__ qbar,
-               double* __restrict__ kdot, uint32_t* err) {
-  __shared__ double red[32];
-  const int s = blockIdx.y, split = blockIdx.x;
-  const int c0 = (blockIdx.z * blockDim.x + threadIdx.x) * V;
-  int page = src_ids ? src_ids[s] : s;
-  const bool ok = page >= 0 && page < n_pages;
-  if (!ok && threadIdx.x == 0) atomicOr(err, WA_DEVERR_PAGE_ID);
-  if (!ok) page = 0;
-  const T* base = x + static_cast<size_t>(page) * rows * cols + c0;
-  double part[V];
-#pragma unroll
-  for (int v = 0; v < V; ++v) part[v] = 0.0;
-  const int b0 = block0 + split * bps, b1 = min(nb_end, b0 + bps);
-  for (int b = b0; b < b1; ++b) {
-    const int r0 = b * B, r1 = min(rows, r0 + B);
-    double acc[V];
-#pragma unroll
-    for (int v = 0; v < V; ++v) acc[v] = 0.0;
-    if (ok) {
-      int r = r0;
-      for (; r + 16 <= r1; r += 16) {
-        uint4 raw[16];
-#pragma unroll
-        for (int u = 0; u < 16; ++u) load_raw(base + static_cast<size_t>(r + u) * cols, raw[u]);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-          double w[V];
-          widen(base, raw[u], w);
-#pragma unroll
-          for (int v = 0; v < V; ++v) acc[v] += w[v];
-        }
-      }
-      for (; r < r1; ++r) {
-        uint4 raw;
-        load_raw(base + static_cast<size_t>(r) * cols, raw);
-        double w[V];
-        widen(base, raw, w);
-#pragma unroll
-        for (int v = 0; v < V; ++v) acc[v] += w[v];
-      }
-    }
-    if (blocksum) {
-      double* o = blocksum + (static_cast<size_t>(bs_by_page ? page : s) * nb + b) * cols + c0;
-#pragma unroll
-      for (int v = 0; v < V; ++v) o[v] = acc[v];
-    }
-#pragma unroll
-    for (int v = 0; v < V; ++v) part[v] += acc[v];
-  }
-  if (qbar) {
-    double dot = 0.0;
-#pragma unroll
-    for (int v = 0; v < V; ++v) dot += part[v] * qbar[c0 + v];
-    dot = block_sum(dot, red);
-    if (threadIdx.x == 0)
-      kdot[(static_cast<size_t>(s) * gridDim.x + split) * gridDim.z + blockIdx.z] = dot;
-  }
-}
-
 // Qbar[col] = sum of all query rows / Nq; qmean[i][col] = block sum / rows of block i.
 // CTA = 32 columns x 8 row groups; group g sums blocks g, g+8, ...; the eight group
 // sums are added in a fixed order (deterministic).
@@ -195,51 +93,6 @@ k_qmeans(const double* __restrict__ qsum, int n_qb, int Nq, int B, int cols,
     double s = 0.0;
     for (int k = 0; k < 8; ++k) s += red[k][threadIdx.x];
     qbar[col] = s / Nq;
-  }
-}
-
-// ------------------------------------------------------------------ S1 scores
-// alpha[c] = (1/(H*sqrt(d))) * Qbar . Kbar_c, where Kbar_c = (sum of the page's rows)/T_p
-// and Qbar . (sum of rows) arrives as the per-CTA dot products of the K pass.  Then
-// the top-K_p pages (ties -> lower position), emitted in ascending position.
-__global__ void __launch_bounds__(256)
-k_alpha_topk(const double* __restrict__ kdot, int per_page, int n_c, int T_p, int H, int d,
-             int K_p, const int32_t* __restrict__ cand, double* __restrict__ alpha,
-             int32_t* __restrict__ sel, int32_t* __restrict__ sel_pos) {
-  extern __shared__ unsigned char chosen[];  // n_c bytes
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  for (int c = warp; c < n_c; c += nw) {
-    double t = 0.0;
-    for (int k = lane; k < per_page; k += 32) t += kdot[static_cast<size_t>(c) * per_page + k];
-    t = warp_sum(t);
-    if (lane == 0) alpha[c] = t / T_p / sqrt(static_cast<double>(d)) / H;
-  }
-  for (int j = threadIdx.x; j < n_c; j += blockDim.x) chosen[j] = 0;
-  __syncthreads();
-  if (warp != 0) return;
-  for (int s = 0; s < K_p; ++s) {
-    double best = -DBL_MAX;
-    int bi = INT_MAX;
-    for (int j = lane; j < n_c; j += 32) {
-      if (chosen[j]) continue;
-      const double a = alpha[j];
-      if (bi == INT_MAX || a > best) { best = a; bi = j; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != INT_MAX && (bi == INT_MAX || ob > best || (ob == best && oi < bi))) {
-        best = ob; bi = oi;
-      }
-    }
-    if (lane == 0 && bi != INT_MAX) chosen[bi] = 1;
-    __syncwarp();
-  }
-  if (lane == 0) {
-    int k = 0;
-    for (int j = 0; j < n_c && k < K_p; ++j)
-      if (chosen[j]) { sel[k] = cand[j]; if (sel_pos) sel_pos[k] = j; ++k; }
   }
 }
 
@@ -458,89 +311,10 @@ wa_status launch_prompt_select(const float* e_cur, const float* e_chunks, int n_
   return check_launch("prompt_select");
 }
 
-RowsumPlan rowsum_plan(int n_src, int rows, int cols, int B, wa_dtype dt) {
-  // 64-thread CTAs (V columns per thread) over one B-row block each: many small
-  // CTAs keep enough 16-byte loads in flight to cover HBM latency
-  RowsumPlan p;
-  const int V = dt == WA_BF16 ? 8 : 4;
-  const int threads_total = cols / V;
-  p.threads = threads_total;
-  p.n_cc = 1;
-  if (threads_total % 64 == 0) {
-    p.threads = 64;
-    p.n_cc = threads_total / 64;
-  }
-  p.nb = (rows + B - 1) / B;
-  p.n_blocks = p.nb;
-  const long long ctas = static_cast<long long>(n_src) * p.n_cc * p.nb;
-  p.bps = ctas > 32LL * 148 ? static_cast<int>((ctas + 32LL * 148 - 1) / (32LL * 148)) : 1;
-  p.n_split = (p.nb + p.bps - 1) / p.bps;
-  return p;
-}
-
-wa_status launch_rowblock_sum(const void* x, wa_dtype dt, const int32_t* src_ids, int n_src,
-                              int n_pages, int rows, int cols, int B, double* blocksum,
-                              const double* qbar, double* kdot, const RowsumPlan& p, uint32_t* err,
-                              cudaStream_t st) {
-  dim3 grid(p.n_split, n_src, p.n_cc);
-  if (dt == WA_BF16) {
-    k_rowblock_sum<__nv_bfloat16, 8><<<grid, p.threads, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), src_ids, n_pages, rows, cols, B, p.nb, p.bps,
-        p.block0, p.block0 + p.n_blocks, p.by_page, blocksum, qbar, kdot, err);
-  } else {
-    k_rowblock_sum<float, 4><<<grid, p.threads, 0, st>>>(
-        static_cast<const float*>(x), src_ids, n_pages, rows, cols, B, p.nb, p.bps, p.block0,
-        p.block0 + p.n_blocks, p.by_page, blocksum, qbar, kdot, err);
-  }
-  return check_launch("rowblock_sum");
-}
-
-RowsumPlan rowsum_plan_range(int rows, int cols, int B, wa_dtype dt, int block0, int n_blocks) {
-  RowsumPlan p = rowsum_plan(1, n_blocks * B, cols, B, dt);
-  p.nb = (rows + B - 1) / B;
-  p.block0 = block0;
-  p.n_blocks = n_blocks;
-  p.n_split = (n_blocks + p.bps - 1) / p.bps;
-  return p;
-}
-
-// kdot[c][b] = qbar . page_index[cand[c]][b][:]  (one CTA per (block, candidate page))
-__global__ void __launch_bounds__(128)
-k_index_dot(const double* __restrict__ page_index, const int32_t* __restrict__ cand, int n_pages,
-            int nbp, int cols, const double* __restrict__ qbar, double* __restrict__ kdot,
-            uint32_t* err) {
-  __shared__ double red[32];
-  const int b = blockIdx.x, c = blockIdx.y;
-  int page = cand ? cand[c] : c;   // no cand: rows are indexed by candidate position
-  if (page < 0 || page >= n_pages) {
-    if (threadIdx.x == 0) atomicOr(err, WA_DEVERR_PAGE_ID);
-    page = 0;
-  }
-  const double* row = page_index + (static_cast<size_t>(page) * nbp + b) * cols;
-  double acc = 0.0;
-  for (int e = threadIdx.x; e < cols; e += blockDim.x) acc += row[e] * qbar[e];
-  acc = block_sum(acc, red);
-  if (threadIdx.x == 0) kdot[static_cast<size_t>(c) * nbp + b] = acc;
-}
-
-wa_status launch_index_dot(const double* page_index, const int32_t* cand, int n_c, int n_pages,
-                           int nbp, int cols, const double* qbar, double* kdot, uint32_t* err,
-                           cudaStream_t st) {
-  k_index_dot<<<dim3(nbp, n_c), 128, 0, st>>>(page_index, cand, n_pages, nbp, cols, qbar, kdot, err);
-  return check_launch("index_dot");
-}
-
 wa_status launch_qmeans(const double* qsum, int n_qb, int Nq, int B, int cols, double* qbar,
                         double* qmean, cudaStream_t st) {
   k_qmeans<<<(cols + 31) / 32, dim3(32, 8), 0, st>>>(qsum, n_qb, Nq, B, cols, qbar, qmean);
   return check_launch("qmeans");
-}
-
-wa_status launch_alpha_topk(const double* kdot, int per_page, int n_c, int T_p, int H, int d,
-                            int K_p, const int32_t* cand, double* alpha, int32_t* sel,
-                            int32_t* sel_pos, cudaStream_t st) {
-  k_alpha_topk<<<1, 256, n_c, st>>>(kdot, per_page, n_c, T_p, H, d, K_p, cand, alpha, sel, sel_pos);
-  return check_launch("alpha_topk");
 }
 
 wa_status launch_scale_copy(const double* src, double* dst, size_t n, double scale,

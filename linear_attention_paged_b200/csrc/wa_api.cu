@@ -172,70 +172,59 @@ struct PageScoreWs {
   double* q_blocksum;   // [n_qb][cols]
   double* qbar;         // [cols]
   double* q_blockmean;  // [n_qb][cols]
-  double* k_blocksum;   // [n_c][nbp][cols] (nullable)
-  double* kdot;         // [n_c][k_split * k_cc]
-  RowsumPlan qp, kp;
+  double* k_blocksum;   // [n_c][nbp][cols] by candidate position (nullable: page index)
+  double* partial;      // partial dot products of the page scores
+  unsigned* counter;    // completion counter of the page-score kernel
 };
 
-PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks,
-                             wa_dtype dt) {
+PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks) {
   PageScoreWs w{};
   const int cols = H * d;
   const int n_qb = ceil_div(Nq, B);
-  w.qp = rowsum_plan(1, Nq, cols, B, dt);
-  w.kp = rowsum_plan(n_c, T_p, cols, B, dt);
   w.q_blocksum = c.take<double>(static_cast<size_t>(n_qb) * cols);
   w.qbar = c.take<double>(cols);
   w.q_blockmean = c.take<double>(static_cast<size_t>(n_qb) * cols);
   w.k_blocksum = k_blocks ? c.take<double>(static_cast<size_t>(n_c) * ceil_div(T_p, B) * cols) : nullptr;
-  const size_t per_page = static_cast<size_t>(w.kp.n_split) * w.kp.n_cc;
-  const size_t nbp = static_cast<size_t>(ceil_div(T_p, B));
-  w.kdot = c.take<double>(static_cast<size_t>(n_c) * (per_page > nbp ? per_page : nbp));
+  w.partial = c.take<double>(page_alpha_partial_count(cols, n_c));
+  w.counter = c.take<unsigned>(1);
   return w;
 }
 
-// Q pass (block sums), query means, then the K pass over the candidate pages with
-// the page-score dot products fused in, then alpha and the top-K_p pages.
+// One pass over the queries and the candidate pages (block sums, float64), then the
+// page scores and the top-K_p pages from those sums.  The candidate pages are row
+// *chunk (or row 0) of chunk_pages [n_chunks][n_c].  With a page index the pass reads
+// only the queries and the scores read the index's block sums of the candidates.
 wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int d,
-                         const void* k_pool, int n_pool_pages, int T_p, const int32_t* cand,
-                         int n_c, int K_p, int B, wa_dtype dt, double* alpha, int32_t* sel,
-                         int32_t* sel_pos, cudaStream_t st, const double* page_index = nullptr) {
+                         const void* k_pool, int n_pool_pages, int T_p, const int32_t* chunk_pages,
+                         const int32_t* chunk, int n_chunks, int n_c, int K_p, int B, wa_dtype dt,
+                         double* alpha, int32_t* sel, int32_t* sel_pos, cudaStream_t st,
+                         const double* page_index = nullptr) {
   const int cols = H * d;
   uint32_t* err = errw();
   if (!err) return set_error(WA_ERR_CUDA, "no device error word (is a CUDA device present?)");
-  if (!page_index && w.k_blocksum) {
-    // The candidate pages' block sums are kept for selection anyway, so the page
-    // scores come from them after the pass; the query pass and query means then run
-    // on the side stream during the (larger) candidate pass instead of before it.
-    SideStream* side = nullptr;
-    WA_TRY(side_stream(&side));
-    cudaEventRecord(side->fork, st);
-    cudaStreamWaitEvent(side->stream, side->fork, 0);
-    WA_TRY(launch_rowblock_sum(q, dt, nullptr, 1, 1, Nq, cols, B, w.q_blocksum, nullptr, nullptr, w.qp,
-                               err, side->stream));
-    WA_TRY(launch_qmeans(w.q_blocksum, ceil_div(Nq, B), Nq, B, cols, w.qbar, w.q_blockmean,
-                         side->stream));
-    cudaEventRecord(side->join, side->stream);
-    WA_TRY(launch_rowblock_sum(k_pool, dt, cand, n_c, n_pool_pages, T_p, cols, B, w.k_blocksum,
-                               nullptr, nullptr, w.kp, err, st));
-    cudaStreamWaitEvent(st, side->join, 0);
-    const int nbp = ceil_div(T_p, B);
-    WA_TRY(launch_index_dot(w.k_blocksum, nullptr, n_c, n_c, nbp, cols, w.qbar, w.kdot, err, st));
-    return launch_alpha_topk(w.kdot, nbp, n_c, T_p, H, d, K_p, cand, alpha, sel, sel_pos, st);
+  const int n_qb = ceil_div(Nq, B), nbp = ceil_div(T_p, B);
+  BlockSumSeg seg[2];
+  seg[0].x = q; seg[0].rows = Nq; seg[0].n_blocks = n_qb; seg[0].sums = w.q_blocksum; seg[0].nb_out = n_qb;
+  int n_segs = 1;
+  if (!page_index) {
+    BlockSumSeg& g = seg[1];
+    g.x = k_pool; g.ids = chunk_pages; g.chunk = chunk; g.id_rows = n_chunks; g.n_src = n_c;
+    g.n_pages = n_pool_pages; g.rows = T_p; g.n_blocks = nbp; g.sums = w.k_blocksum; g.nb_out = nbp;
+    n_segs = 2;
   }
-  WA_TRY(launch_rowblock_sum(q, dt, nullptr, 1, 1, Nq, cols, B, w.q_blocksum, nullptr, nullptr, w.qp,
-                             err, st));
-  WA_TRY(launch_qmeans(w.q_blocksum, ceil_div(Nq, B), Nq, B, cols, w.qbar, w.q_blockmean, st));
-  if (page_index) {
-    // the page index already holds the candidate pages' block sums
-    const int nbp = T_p / B;
-    WA_TRY(launch_index_dot(page_index, cand, n_c, n_pool_pages, nbp, cols, w.qbar, w.kdot, err, st));
-    return launch_alpha_topk(w.kdot, nbp, n_c, T_p, H, d, K_p, cand, alpha, sel, sel_pos, st);
-  }
-  WA_TRY(launch_rowblock_sum(k_pool, dt, cand, n_c, n_pool_pages, T_p, cols, B, w.k_blocksum, w.qbar,
-                             w.kdot, w.kp, err, st));
-  return launch_alpha_topk(w.kdot, w.kp.n_split * w.kp.n_cc, n_c, T_p, H, d, K_p, cand, alpha, sel,
-                           sel_pos, st);
+  WA_TRY(launch_block_sums(dt, cols, B, seg, n_segs, w.counter, err, st));
+  return launch_page_alpha(w.q_blocksum, n_qb, Nq, B, cols, page_index ? page_index : w.k_blocksum,
+                           page_index ? chunk_pages : nullptr, n_pool_pages, nbp, chunk_pages, chunk,
+                           n_chunks, n_c, T_p, H, d, K_p, w.qbar, w.q_blockmean, w.partial, w.counter,
+                           alpha, sel, sel_pos, err, st);
+}
+
+// Block sums of one contiguous buffer of `rows` rows (all its blocks).
+wa_status buffer_block_sums(const void* x, int rows, int cols, int B, wa_dtype dt, double* sums,
+                            uint32_t* err, cudaStream_t st) {
+  BlockSumSeg g;
+  g.x = x; g.rows = rows; g.n_blocks = ceil_div(rows, B); g.sums = sums; g.nb_out = g.n_blocks;
+  return launch_block_sums(dt, cols, B, &g, 1, nullptr, err, st);
 }
 
 }  // namespace wa_detail
@@ -277,12 +266,9 @@ wa_status wa_prompt_select(const float* e_cur, const float* e_chunks, int n_chun
 size_t wa_page_score_workspace_size(int Nq, int H, int d, int n_c, int T_p, int B) {
   if (Nq < 1 || H < 1 || d < 1 || n_c < 1 || T_p < 1 || B < 1) return 0;
   Carver c(nullptr);
-  carve_page_score(c, Nq, H, d, n_c, T_p, B, true, WA_BF16);
+  carve_page_score(c, Nq, H, d, n_c, T_p, B, true);
   c.take<int32_t>(n_c);
-  Carver c2(nullptr);
-  carve_page_score(c2, Nq, H, d, n_c, T_p, B, true, WA_F32);
-  c2.take<int32_t>(n_c);
-  return c.used > c2.used ? c.used : c2.used;
+  return c.used;
 }
 
 wa_status wa_page_score(const void* q, int Nq, int H, int d, const void* k_pool, int n_pool_pages,
@@ -299,10 +285,10 @@ wa_status wa_page_score(const void* q, int Nq, int H, int d, const void* k_pool,
   WA_TRY(check_ws(ws, ws_bytes, wa_page_score_workspace_size(Nq, H, d, n_c, T_p, B)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carver c(ws);
-  PageScoreWs w = carve_page_score(c, Nq, H, d, n_c, T_p, B, true, dtype);
+  PageScoreWs w = carve_page_score(c, Nq, H, d, n_c, T_p, B, true);
   int32_t* sel_pos = c.take<int32_t>(n_c);
-  WA_TRY(run_page_score(w, q, Nq, H, d, k_pool, n_pool_pages, T_p, cand_pages, n_c, K_p, B, dtype,
-                        alpha, sel, sel_pos, st));
+  WA_TRY(run_page_score(w, q, Nq, H, d, k_pool, n_pool_pages, T_p, cand_pages, nullptr, 1, n_c, K_p, B,
+                        dtype, alpha, sel, sel_pos, st));
   if (k_blockmean) {
     const size_t n = static_cast<size_t>(n_c) * (T_p / B) * H * d;
     WA_TRY(launch_scale_copy(w.k_blocksum, k_blockmean, n, 1.0 / B, st));
@@ -382,11 +368,10 @@ wa_status wa_pool_index(const void* k_pool, int n_pool_pages, int T_p, int H, in
   if (T_p % B != 0) return set_error(WA_ERR_UNSUPPORTED, "the page index needs T_p %% B == 0");
   uint32_t* err = errw();
   if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
-  const int cols = H * d;
-  RowsumPlan p = rowsum_plan(n_pages, T_p, cols, B, dtype);
-  p.by_page = 1;
-  return launch_rowblock_sum(k_pool, dtype, pages, n_pages, n_pool_pages, T_p, cols, B, page_index,
-                             nullptr, nullptr, p, err, static_cast<cudaStream_t>(stream));
+  BlockSumSeg g;
+  g.x = k_pool; g.ids = pages; g.n_src = n_pages; g.n_pages = n_pool_pages; g.rows = T_p;
+  g.n_blocks = T_p / B; g.sums = page_index; g.nb_out = T_p / B; g.by_page = 1;
+  return launch_block_sums(dtype, H * d, B, &g, 1, nullptr, err, static_cast<cudaStream_t>(stream));
 }
 
 wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, int H, int d,
@@ -419,10 +404,12 @@ wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, 
   if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
   const int b_first = static_cast<int>(token_offset / B);
   const int b_last = static_cast<int>((token_offset + n_tokens - 1) / B);
-  const int cols = H * d;
-  RowsumPlan p = rowsum_plan_range(static_cast<int>(rows), cols, B, dtype, b_first, b_last - b_first + 1);
-  return launch_rowblock_sum(k_pool, dtype, nullptr, 1, 1, static_cast<int>(rows), cols, B, page_index,
-                             nullptr, nullptr, p, err, st);
+  // the touched blocks of the pool's flat token space (T_p % B == 0: a block never
+  // straddles pages, and flat block b is block b % (T_p/B) of page b / (T_p/B))
+  BlockSumSeg g;
+  g.x = k_pool; g.rows = static_cast<int>(rows); g.block0 = b_first; g.n_blocks = b_last - b_first + 1;
+  g.sums = page_index; g.nb_out = static_cast<int>(rows / B);
+  return launch_block_sums(dtype, H * d, B, &g, 1, nullptr, err, st);
 }
 
 namespace wa_detail {
@@ -433,14 +420,12 @@ struct BlockSelectWs {
   double* qmean;
   double* ksum;
   double* scores;
-  RowsumPlan qp, kp;
 };
 BlockSelectWs carve_block_select(Carver& c, int Nq, int H, int d, int L, int B, wa_dtype dt) {
   BlockSelectWs w{};
   const int cols = H * d;
   const int n_qb = ceil_div(Nq, B), n_kb = ceil_div(L, B);
-  w.qp = rowsum_plan(1, Nq, cols, B, dt);
-  w.kp = rowsum_plan(1, L, cols, B, dt);
+  (void)dt;
   w.qsum = c.take<double>(static_cast<size_t>(n_qb) * cols);
   w.qbar = c.take<double>(cols);
   w.qmean = c.take<double>(static_cast<size_t>(n_qb) * cols);
@@ -476,14 +461,12 @@ wa_status wa_block_select(const void* q, int Nq, int H, int d, const void* k_act
   Carver c(ws);
   BlockSelectWs w = carve_block_select(c, Nq, H, d, L, B, dtype);
   const int cols = H * d;
-  WA_TRY(launch_rowblock_sum(q, dtype, nullptr, 1, 1, Nq, cols, B, w.qsum, nullptr, nullptr, w.qp,
-                             err, st));
+  WA_TRY(buffer_block_sums(q, Nq, cols, B, dtype, w.qsum, err, st));
   WA_TRY(launch_qmeans(w.qsum, ceil_div(Nq, B), Nq, B, cols, w.qbar, w.qmean, st));
   KeyMeans km;
   km.L = L;
   if (k_act) {
-    WA_TRY(launch_rowblock_sum(k_act, dtype, nullptr, 1, 1, L, cols, B, w.ksum, nullptr, nullptr,
-                               w.kp, err, st));
+    WA_TRY(buffer_block_sums(k_act, L, cols, B, dtype, w.ksum, err, st));
     km.data = w.ksum;
     km.is_sum = 1;
   } else {
@@ -619,7 +602,6 @@ namespace wa_detail {
 namespace {  // internal linkage: nothing here is exported from libwa
 struct StepWs {
   int32_t* chunk;
-  int32_t* cand;       // candidate page ids copied from chunk_pages row
   PageScoreWs ps;
   double* alpha;
   int32_t* sel;
@@ -679,10 +661,8 @@ StepWs carve_step(Carver& c, const wa_step_args* a) {
             W = ceil_div(n_kb, 32);
   const size_t es = elem_size(a->dtype);
   w.chunk = c.take<int32_t>(1);
-  w.cand = c.take<int32_t>(a->n_c);
-  // block sums of the candidate pages are only needed when selection reads them
-  w.ps = carve_page_score(c, a->Nq, a->H, a->d, a->n_c, a->T_p, a->B, a->fused_gather != 0,
-                          a->dtype);
+  // block sums of the candidate pages, unless the page index holds them
+  w.ps = carve_page_score(c, a->Nq, a->H, a->d, a->n_c, a->T_p, a->B, a->page_index == nullptr);
   w.alpha = c.take<double>(a->n_c);
   w.sel = c.take<int32_t>(a->K_p);
   w.sel_pos = c.take<int32_t>(a->K_p);
@@ -703,12 +683,6 @@ StepWs carve_step(Carver& c, const wa_step_args* a) {
   return w;
 }
 
-__global__ void k_pick_chunk(const int32_t* chunk_pages, int n_c, const int32_t* chunk,
-                             int n_chunks, int32_t* cand) {
-  int m = chunk ? *chunk : 0;
-  if (m < 0 || m >= n_chunks) m = 0;
-  for (int j = threadIdx.x; j < n_c; j += blockDim.x) cand[j] = chunk_pages[static_cast<size_t>(m) * n_c + j];
-}
 }  // namespace
 }  // namespace wa_detail
 using namespace wa_detail;
@@ -743,15 +717,17 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
   const int n_chunks = a->e_cur ? a->n_chunks : 1;
   if (a->e_cur)
     WA_TRY(launch_prompt_select(a->e_cur, a->e_chunks, a->n_chunks, a->D, chunk, err, st));
-  k_pick_chunk<<<1, 256, 0, st>>>(a->chunk_pages, a->n_c, a->e_cur ? chunk : nullptr, n_chunks, w.cand);
-  WA_TRY(check_launch("pick_chunk"));
-  if (!a->e_cur && a->chunk_out) cudaMemsetAsync(a->chunk_out, 0, sizeof(int32_t), st);
+  else if (a->chunk_out)
+    cudaMemsetAsync(a->chunk_out, 0, sizeof(int32_t), st);
 
-  // S1: page scores + top-K_p (+ the candidate pages' block sums, fused path)
+  // S1: page scores + top-K_p, and the block sums of the candidate pages (S3 reads
+  // them in place of a pass over the selected keys); the candidate pages are row
+  // `chunk` of chunk_pages (a chunk index of -1 from a zero-norm embedding reads row 0)
   double* alpha = a->alpha_out ? a->alpha_out : w.alpha;
   int32_t* sel = a->sel_out ? a->sel_out : w.sel;
-  WA_TRY(run_page_score(w.ps, a->q, a->Nq, a->H, a->d, a->k_pool, a->n_pool_pages, a->T_p, w.cand,
-                        a->n_c, a->K_p, a->B, a->dtype, alpha, sel, w.sel_pos, st, a->page_index));
+  WA_TRY(run_page_score(w.ps, a->q, a->Nq, a->H, a->d, a->k_pool, a->n_pool_pages, a->T_p,
+                        a->chunk_pages, a->e_cur ? chunk : nullptr, n_chunks, a->n_c, a->K_p, a->B,
+                        a->dtype, alpha, sel, w.sel_pos, st, a->page_index));
 
   mark(1);
   // S2: page table (fused) or explicit gather
@@ -775,15 +751,13 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
     WA_TRY(launch_gather(a->k_pool, a->v_pool, a->n_pool_pages, page_bytes, sel, a->K_p, w.k_act,
                          w.v_act, err, st));
     rs.k = w.k_act; rs.v = w.v_act; rs.page_rows = L; rs.n_pages = 1; rs.L = L;
-    WA_TRY(launch_rowblock_sum(w.k_act, a->dtype, nullptr, 1, 1, L, cols, a->B, w.ksum, nullptr,
-                               nullptr, rowsum_plan(1, L, cols, a->B, a->dtype), err, st));
+    WA_TRY(buffer_block_sums(w.k_act, L, cols, a->B, a->dtype, w.ksum, err, st));
     km.data = w.ksum;
   }
   if (a->k_cur) {
     // intra-chunk keys: the chunk's own K/V follow the history in the sparse branch
     rs.k2 = a->k_cur; rs.v2 = a->v_cur; rs.L2 = a->Nq;
-    WA_TRY(launch_rowblock_sum(a->k_cur, a->dtype, nullptr, 1, 1, a->Nq, cols, a->B, w.cur_sum,
-                               nullptr, nullptr, rowsum_plan(1, a->Nq, cols, a->B, a->dtype), err, st));
+    WA_TRY(buffer_block_sums(a->k_cur, a->Nq, cols, a->B, a->dtype, w.cur_sum, err, st));
     km.data2 = w.cur_sum; km.n_kb1 = L / a->B; km.L2 = a->Nq;
   }
 

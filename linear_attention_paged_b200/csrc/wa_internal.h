@@ -42,42 +42,48 @@ uint64_t wait_limit_ns();
 wa_status launch_prompt_select(const float* e_cur, const float* e_chunks, int n_chunks, int D,
                                int32_t* chunk_out, uint32_t* err, cudaStream_t st);
 
-// Row-block sums in float64 over B-row blocks of `n_src` sources of `rows` rows
-// each (a source is a pool page given by src_ids, or the buffer itself when
-// src_ids == nullptr), cols = H*d columns:
-//   blocksum[s][b][c]  (nullable)  sum of rows [b*B, min(rows,(b+1)*B)) of source s
-//   kdot[s][split][cc] (with qbar) dot product of qbar with the CTA's column sums
-struct RowsumPlan {
-  int threads = 0;   // threads per CTA (V columns each)
-  int n_cc = 1;      // column chunks
-  int nb = 0;        // blocks per source (also the source stride of blocksum)
-  int bps = 1;       // blocks per CTA
-  int n_split = 1;   // CTAs per source and column chunk
-  int block0 = 0;    // first block summed
-  int n_blocks = 0;  // blocks summed (from block0)
-  int by_page = 0;   // blocksum indexed by pool page id instead of source position
+// Float64 sums of B-row blocks, in one persistent pass fed by bulk copies (k_blocksum.cu).
+// A segment is `n_src` sources of `rows` rows of `cols` elements: the buffer x itself
+// (ids == nullptr, source s at row s * rows) or pool pages (source s is page
+// ids[row * n_src + s], row = *chunk or 0).  Blocks [block0, block0 + n_blocks) of every
+// source are summed (the last block of a source may be ragged) into
+//   sums[((by_page ? page : s) * nb_out + block) * cols + c].
+// Up to two segments per launch (e.g. the queries and the candidate pages).  With
+// `counter` the launch also zeroes that word for launch_page_alpha.
+struct BlockSumSeg {
+  const void* x = nullptr;
+  const int32_t* ids = nullptr;
+  const int32_t* chunk = nullptr;
+  int id_rows = 1;        // rows of ids; a chunk index outside [0, id_rows) reads row 0
+  int n_src = 1;
+  int n_pages = 1;
+  int rows = 0;
+  int block0 = 0;
+  int n_blocks = 0;
+  double* sums = nullptr;
+  int nb_out = 0;
+  int by_page = 0;
 };
-RowsumPlan rowsum_plan(int n_src, int rows, int cols, int B, wa_dtype dt);
-// Plan over blocks [block0, block0 + n_blocks) of one source of `rows` rows.
-RowsumPlan rowsum_plan_range(int rows, int cols, int B, wa_dtype dt, int block0, int n_blocks);
-// kdot[c][b] = qbar . page_index[cand[c]][b] (page scores from the page index);
-// cand == nullptr reads row c (block sums indexed by candidate position).
-wa_status launch_index_dot(const double* page_index, const int32_t* cand, int n_c, int n_pages,
-                           int nbp, int cols, const double* qbar, double* kdot, uint32_t* err,
-                           cudaStream_t st);
-wa_status launch_rowblock_sum(const void* x, wa_dtype dt, const int32_t* src_ids, int n_src,
-                              int n_pages, int rows, int cols, int B, double* blocksum,
-                              const double* qbar, double* kdot, const RowsumPlan& p, uint32_t* err,
-                              cudaStream_t st);
+wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* segs, int n_segs,
+                            unsigned* counter, uint32_t* err, cudaStream_t st);
+// Page scores from block sums: Qbar = sum of qsum rows / Nq (written to qbar, and the
+// query block means to qmean when non-null), column sums of each candidate page's
+// block sums (ksum rows of page kpage[row][j], or of position j when kpage is null),
+// alpha_j = Qbar . colsum_j / (T_p sqrt(d) H), then the top-K_p pages (sel: pool ids
+// from cand[row][.], or positions when cand is null; sel_pos: positions), ascending.
+// `partial` holds page_alpha_partial_count(cols, n_c) doubles; `counter` must be zero
+// (launch_block_sums zeroes it) and is left zero.
+size_t page_alpha_partial_count(int cols, int n_c);
+wa_status launch_page_alpha(const double* qsum, int n_qb, int Nq, int B, int cols, const double* ksum,
+                            const int32_t* kpage, int n_pages, int nbp, const int32_t* cand,
+                            const int32_t* chunk, int n_chunks, int n_c, int T_p, int H, int d,
+                            int K_p, double* qbar, double* qmean, double* partial, unsigned* counter,
+                            double* alpha, int32_t* sel, int32_t* sel_pos, uint32_t* err,
+                            cudaStream_t st);
+
 // qbar[c] = sum_i qsum[i][c] / Nq; qmean[i][c] (nullable) = qsum[i][c] / rows of block i.
 wa_status launch_qmeans(const double* qsum, int n_qb, int Nq, int B, int cols, double* qbar,
                         double* qmean, cudaStream_t st);
-// S1 tail: alpha[c] from the K pass's dot products (per_page scalars per page), then
-// top-K_p -> sel (pool ids) and sel_pos (candidate positions), ascending position.
-wa_status launch_alpha_topk(const double* kdot, int per_page, int n_c, int T_p, int H, int d,
-                            int K_p, const int32_t* cand, double* alpha, int32_t* sel,
-                            int32_t* sel_pos, cudaStream_t st);
-
 // dst[i] = src[i] * scale (float64).
 wa_status launch_scale_copy(const double* src, double* dst, size_t n, double scale,
                             cudaStream_t st);
