@@ -31,9 +31,12 @@ using namespace sm100;
 
 constexpr int kMaxSegs = 2;
 constexpr int kMaxStages = 16;
-constexpr int kRingBytes = 96 * 1024;     // shared-memory ring of one CTA (two CTAs per SM)
-constexpr int kCtasPerSm = 2;
-constexpr int kChunkBytesMax = 32 * 1024; // rows per bulk copy: at most this many bytes
+// Three CTAs per SM, each with a ring of three 24 KB stages at the one-layer shape
+// (a sweep over 2-6 CTAs per SM, 32-96 KB rings and 6-48 KB copies put this setting
+// first, at 4.9 TB/s on the 307 MB pass of eight candidate pages).
+constexpr int kRingBytes = 72 * 1024;     // shared-memory ring of one CTA
+constexpr int kCtasPerSm = 3;
+constexpr int kChunkBytesMax = 24 * 1024; // rows per bulk copy: at most this many bytes
 
 struct PassSeg {
   const char* x;            // rows of row_bytes bytes
@@ -61,7 +64,8 @@ struct PassArgs {
   int R;                    // rows per bulk copy (a power of two dividing B, or B)
   int S;                    // ring stages
   int G;                    // 16-byte groups per row = consumer threads
-  unsigned* counter;        // nullable: zeroed here for the page-score kernel that follows
+  unsigned* counter;        // nullable: n_counters words zeroed here for the page-score kernel
+  int n_counters;
   uint64_t wait_ns;
 };
 
@@ -133,7 +137,8 @@ k_block_sums(const __grid_constant__ PassArgs a, uint32_t* err) {
     }
     sh.abort_flag = 0;
     fence_mbar_init();
-    if (a.counter && blockIdx.x == 0) *a.counter = 0u;
+    if (a.counter && blockIdx.x == 0)
+      for (int i = 0; i < a.n_counters; ++i) a.counter[i] = 0u;
   }
   __syncthreads();
 
@@ -225,39 +230,72 @@ k_block_sums(const __grid_constant__ PassArgs a, uint32_t* err) {
 }
 
 // ------------------------------------------------------------------ page scores
-// CTA (column slice cs, candidate j): for its kAlphaCols columns, Qbar = (sum of the
-// query block sums) / Nq and the column sums of page j's block sums (kAlphaGroups row
-// groups, combined in order), then the partial dot product of the two.  CTAs of
-// j == 0 also write Qbar and the query block means.  The last CTA to finish adds the
-// partial dots of every page in slice order, forms alpha_j and takes the top-K_p
-// (ties -> lower position), emitted in ascending position.
+// Grid (column slice cs of kAlphaCols columns, role y).  y == 0: Qbar for the slice
+// (sum of the query block sums / Nq; also written out, with the query block means).
+// y = 1 + j * kAlphaSplits + p: the sum over blocks [p*nbp/S, (p+1)*nbp/S) of page j's
+// block sums for the slice (a column-sum part).  Each CTA's threads take the blocks in
+// kAlphaGroups strided groups, combined in order.  The last CTA of a slice forms the
+// slice's dot product of Qbar with every page's column sum (parts added in order);
+// the last slice to finish adds the slices in order, forms
+//   alpha_j = Qbar . colsum_j / (T_p sqrt(d) H)
+// and takes the top-K_p pages (ties -> lower position), emitted in ascending position.
 constexpr int kAlphaCols = 32;
 constexpr int kAlphaGroups = 8;
+constexpr int kAlphaSplits = 4;
 
 __global__ void __launch_bounds__(kAlphaCols * kAlphaGroups)
 k_page_alpha(const double* __restrict__ qsum, int n_qb, int Nq, int B, int cols,
              const double* __restrict__ ksum, const int32_t* __restrict__ kpage, int n_pages,
              int nbp, const int32_t* __restrict__ cand, const int32_t* __restrict__ chunk,
              int n_chunks, int n_c, int T_p, int H, int d, int K_p, double* __restrict__ qbar,
-             double* __restrict__ qmean, double* __restrict__ partial, unsigned* counter,
-             double* __restrict__ alpha, int32_t* __restrict__ sel, int32_t* __restrict__ sel_pos,
-             uint32_t* err) {
+             double* __restrict__ qmean, double* __restrict__ colpart, double* __restrict__ partial,
+             unsigned* counters, double* __restrict__ alpha, int32_t* __restrict__ sel,
+             int32_t* __restrict__ sel_pos, uint32_t* err) {
   __shared__ double red[kAlphaGroups][kAlphaCols];
-  __shared__ double qb[kAlphaCols];
   __shared__ bool last;
   extern __shared__ unsigned char chosen_sm[];   // [n_c], used by the last CTA
-  const int cs = blockIdx.x, j = blockIdx.y;
+  const int cs = blockIdx.x, y = blockIdx.y;
+  const int n_cs = gridDim.x;
   const int tx = threadIdx.x % kAlphaCols, gy = threadIdx.x / kAlphaCols;
   const int col = cs * kAlphaCols + tx;
   const bool cv = col < cols;
-  // Qbar for this column slice
+  const int lanei = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int row = chunk ? *chunk : 0;
+  if (row < 0 || row >= n_chunks) row = 0;
   double t = 0.0;
-  if (cv) {
-#pragma unroll 4
-    for (int i = gy; i < n_qb; i += kAlphaGroups) {
-      const double v = qsum[static_cast<size_t>(i) * cols + col];
-      t += v;
-      if (j == 0 && qmean) qmean[static_cast<size_t>(i) * cols + col] = v / (min(Nq, (i + 1) * B) - i * B);
+  if (y == 0) {
+    if (cv)
+      for (int i = gy; i < n_qb; i += kAlphaGroups) {
+        const double v = qsum[static_cast<size_t>(i) * cols + col];
+        t += v;
+        if (qmean) qmean[static_cast<size_t>(i) * cols + col] = v / (min(Nq, (i + 1) * B) - i * B);
+      }
+  } else {
+    const int j = (y - 1) / kAlphaSplits, p = (y - 1) % kAlphaSplits;
+    int page = j;
+    if (kpage) {
+      page = kpage[static_cast<size_t>(row) * n_c + j];
+      if (page < 0 || page >= n_pages) {
+        if (threadIdx.x == 0 && cs == 0 && p == 0) atomicOr(err, WA_DEVERR_PAGE_ID);
+        page = 0;
+      }
+    }
+    const int b0 = static_cast<int>(static_cast<long long>(p) * nbp / kAlphaSplits);
+    const int b1 = static_cast<int>(static_cast<long long>(p + 1) * nbp / kAlphaSplits);
+    const double* kp = ksum + static_cast<size_t>(page) * nbp * cols;
+    if (cv) {
+      // independent loads first (many in flight), then the adds in block order
+      constexpr int kBatch = 8;
+      for (int bb = b0 + gy; bb < b1; bb += kBatch * kAlphaGroups) {
+        double v[kBatch];
+#pragma unroll
+        for (int e = 0; e < kBatch; ++e) {
+          const int b = bb + e * kAlphaGroups;
+          v[e] = b < b1 ? kp[static_cast<size_t>(b) * cols + col] : 0.0;
+        }
+#pragma unroll
+        for (int e = 0; e < kBatch; ++e) t += v[e];
+      }
     }
   }
   red[gy][tx] = t;
@@ -265,60 +303,51 @@ k_page_alpha(const double* __restrict__ qsum, int n_qb, int Nq, int B, int cols,
   if (gy == 0) {
     double s = 0.0;
     for (int g = 0; g < kAlphaGroups; ++g) s += red[g][tx];
-    s /= Nq;
-    qb[tx] = s;
-    if (j == 0 && cv) qbar[col] = s;
+    if (y == 0) {
+      s /= Nq;
+      if (cv) qbar[col] = s;
+    }
+    // Qbar of the slice (y == 0) or a column-sum part, in [y][col]
+    colpart[static_cast<size_t>(y) * n_cs * kAlphaCols + col] = s;
   }
+  __threadfence();
   __syncthreads();
-  // column sums of page j
-  int row = chunk ? *chunk : 0;
-  if (row < 0 || row >= n_chunks) row = 0;
-  int page = j;
-  if (kpage) {
-    page = kpage[static_cast<size_t>(row) * n_c + j];
-    if (page < 0 || page >= n_pages) {
-      if (threadIdx.x == 0 && cs == 0) atomicOr(err, WA_DEVERR_PAGE_ID);
-      page = 0;
-    }
-  }
-  const double* kp = ksum + static_cast<size_t>(page) * nbp * cols;
-  t = 0.0;
-  if (cv) {
-#pragma unroll 4
-    for (int b = gy; b < nbp; b += kAlphaGroups) t += kp[static_cast<size_t>(b) * cols + col];
-  }
-  red[gy][tx] = t;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    double dot = 0.0;
-    for (int c = threadIdx.x; c < kAlphaCols; c += 32) {
-      double s = 0.0;
-      for (int g = 0; g < kAlphaGroups; ++g) s += red[g][c];
-      dot += (cs * kAlphaCols + c < cols) ? s * qb[c] : 0.0;
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    if (threadIdx.x == 0) {
-      partial[static_cast<size_t>(j) * gridDim.x + cs] = dot;
-      __threadfence();
-      last = atomicAdd(counter, 1u) == gridDim.x * gridDim.y - 1;
-    }
-  }
+  if (threadIdx.x == 0) last = atomicAdd(&counters[1 + cs], 1u) == gridDim.y - 1;
   __syncthreads();
   if (!last) return;
   __threadfence();
-  // the last CTA: alpha for every page, then the top-K_p
-  const int lanei = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  // the last CTA of the slice: the slice's dot product for every page
+  const double* qb = colpart + static_cast<size_t>(cs) * kAlphaCols;   // y == 0 row
+  for (int j = warp; j < n_c; j += nw) {
+    double dot = 0.0;
+    if (cs * kAlphaCols + lanei < cols) {
+      double c = 0.0;
+      for (int p = 0; p < kAlphaSplits; ++p)
+        c += __ldcg(colpart + static_cast<size_t>(1 + j * kAlphaSplits + p) * n_cs * kAlphaCols +
+                    cs * kAlphaCols + lanei);
+      dot = c * __ldcg(qb + lanei);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+    if (lanei == 0) partial[static_cast<size_t>(j) * n_cs + cs] = dot;
+  }
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) last = atomicAdd(&counters[0], 1u) == static_cast<unsigned>(n_cs) - 1;
+  __syncthreads();
+  if (!last) return;
+  __threadfence();
+  // the last slice: alpha for every page, then the top-K_p
   const double den = static_cast<double>(T_p) * sqrt(static_cast<double>(d)) * H;
   for (int c = warp; c < n_c; c += nw) {
-    if (lanei == 0) {
-      double s = 0.0;
-      const volatile double* pr = partial + static_cast<size_t>(c) * gridDim.x;
-      for (int k = 0; k < static_cast<int>(gridDim.x); ++k) s += pr[k];   // slice order
-      alpha[c] = s / den;
-    }
+    // lane l adds slices l, l + 32, ... in order, then a fixed butterfly
+    const double* pr = partial + static_cast<size_t>(c) * n_cs;
+    double s = 0.0;
+    for (int k = lanei; k < n_cs; k += 32) s += __ldcg(pr + k);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+    if (lanei == 0) alpha[c] = s / den;
   }
-  __syncthreads();
   unsigned char* chosen = chosen_sm;   // [n_c]
   for (int c = threadIdx.x; c < n_c; c += blockDim.x) chosen[c] = 0;
   __syncthreads();
@@ -350,7 +379,7 @@ k_page_alpha(const double* __restrict__ qsum, int n_qb, int Nq, int B, int cols,
         if (sel_pos) sel_pos[k] = c;
         ++k;
       }
-    *counter = 0u;
+    for (int i = 0; i <= n_cs; ++i) counters[i] = 0u;
   }
 }
 
@@ -368,7 +397,7 @@ int n_sm() {
 }  // namespace
 
 wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* segs, int n_segs,
-                            unsigned* counter, uint32_t* err, cudaStream_t st) {
+                            unsigned* counter, int n_counters, uint32_t* err, cudaStream_t st) {
   if (n_segs < 1 || n_segs > kMaxSegs) return set_error(WA_ERR_INVALID_ARG, "block sums: 1 or 2 segments");
   PassArgs a{};
   const int es = dt == WA_BF16 ? 2 : 4;
@@ -378,6 +407,7 @@ wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* seg
   a.B = B;
   a.n_segs = n_segs;
   a.counter = counter;
+  a.n_counters = n_counters;
   a.wait_ns = wait_limit_ns();
   long long total = 0;
   for (int i = 0; i < n_segs; ++i) {
@@ -427,20 +457,29 @@ wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* seg
   return check_launch("block_sums");
 }
 
-size_t page_alpha_partial_count(int cols, int n_c) {
-  return static_cast<size_t>((cols + kAlphaCols - 1) / kAlphaCols) * n_c;
+size_t page_alpha_scratch_doubles(int cols, int n_c) {
+  const size_t n_cs = (cols + kAlphaCols - 1) / kAlphaCols;
+  // column parts [1 + n_c * splits][n_cs * kAlphaCols] and slice dots [n_c][n_cs]
+  return (1 + static_cast<size_t>(n_c) * kAlphaSplits) * n_cs * kAlphaCols + static_cast<size_t>(n_c) * n_cs;
 }
+
+int page_alpha_counters(int cols) { return 1 + (cols + kAlphaCols - 1) / kAlphaCols; }
 
 wa_status launch_page_alpha(const double* qsum, int n_qb, int Nq, int B, int cols, const double* ksum,
                             const int32_t* kpage, int n_pages, int nbp, const int32_t* cand,
                             const int32_t* chunk, int n_chunks, int n_c, int T_p, int H, int d,
-                            int K_p, double* qbar, double* qmean, double* partial, unsigned* counter,
+                            int K_p, double* qbar, double* qmean, double* scratch, unsigned* counters,
                             double* alpha, int32_t* sel, int32_t* sel_pos, uint32_t* err,
                             cudaStream_t st) {
-  dim3 grid((cols + kAlphaCols - 1) / kAlphaCols, n_c);
+  const int n_cs = (cols + kAlphaCols - 1) / kAlphaCols;
+  const long long gy = 1 + static_cast<long long>(n_c) * kAlphaSplits;
+  if (gy > 65535) return set_error(WA_ERR_UNSUPPORTED, "page scores: too many candidate pages");
+  double* colpart = scratch;
+  double* partial = scratch + (1 + static_cast<size_t>(n_c) * kAlphaSplits) * n_cs * kAlphaCols;
+  dim3 grid(n_cs, static_cast<unsigned>(gy));
   k_page_alpha<<<grid, kAlphaCols * kAlphaGroups, n_c, st>>>(
       qsum, n_qb, Nq, B, cols, ksum, kpage, n_pages, nbp, cand, chunk, n_chunks, n_c, T_p, H, d, K_p,
-      qbar, qmean, partial, counter, alpha, sel, sel_pos, err);
+      qbar, qmean, colpart, partial, counters, alpha, sel, sel_pos, err);
   return check_launch("page_alpha");
 }
 

@@ -173,8 +173,8 @@ struct PageScoreWs {
   double* qbar;         // [cols]
   double* q_blockmean;  // [n_qb][cols]
   double* k_blocksum;   // [n_c][nbp][cols] by candidate position (nullable: page index)
-  double* partial;      // partial dot products of the page scores
-  unsigned* counter;    // completion counter of the page-score kernel
+  double* scratch;      // column-sum parts and partial dot products of the page scores
+  unsigned* counters;   // completion counters of the page-score kernel
 };
 
 PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks) {
@@ -185,8 +185,8 @@ PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, 
   w.qbar = c.take<double>(cols);
   w.q_blockmean = c.take<double>(static_cast<size_t>(n_qb) * cols);
   w.k_blocksum = k_blocks ? c.take<double>(static_cast<size_t>(n_c) * ceil_div(T_p, B) * cols) : nullptr;
-  w.partial = c.take<double>(page_alpha_partial_count(cols, n_c));
-  w.counter = c.take<unsigned>(1);
+  w.scratch = c.take<double>(page_alpha_scratch_doubles(cols, n_c));
+  w.counters = c.take<unsigned>(page_alpha_counters(cols));
   return w;
 }
 
@@ -212,10 +212,10 @@ wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int
     g.n_pages = n_pool_pages; g.rows = T_p; g.n_blocks = nbp; g.sums = w.k_blocksum; g.nb_out = nbp;
     n_segs = 2;
   }
-  WA_TRY(launch_block_sums(dt, cols, B, seg, n_segs, w.counter, err, st));
+  WA_TRY(launch_block_sums(dt, cols, B, seg, n_segs, w.counters, page_alpha_counters(cols), err, st));
   return launch_page_alpha(w.q_blocksum, n_qb, Nq, B, cols, page_index ? page_index : w.k_blocksum,
                            page_index ? chunk_pages : nullptr, n_pool_pages, nbp, chunk_pages, chunk,
-                           n_chunks, n_c, T_p, H, d, K_p, w.qbar, w.q_blockmean, w.partial, w.counter,
+                           n_chunks, n_c, T_p, H, d, K_p, w.qbar, w.q_blockmean, w.scratch, w.counters,
                            alpha, sel, sel_pos, err, st);
 }
 
@@ -224,7 +224,7 @@ wa_status buffer_block_sums(const void* x, int rows, int cols, int B, wa_dtype d
                             uint32_t* err, cudaStream_t st) {
   BlockSumSeg g;
   g.x = x; g.rows = rows; g.n_blocks = ceil_div(rows, B); g.sums = sums; g.nb_out = g.n_blocks;
-  return launch_block_sums(dt, cols, B, &g, 1, nullptr, err, st);
+  return launch_block_sums(dt, cols, B, &g, 1, nullptr, 0, err, st);
 }
 
 }  // namespace wa_detail
@@ -371,7 +371,7 @@ wa_status wa_pool_index(const void* k_pool, int n_pool_pages, int T_p, int H, in
   BlockSumSeg g;
   g.x = k_pool; g.ids = pages; g.n_src = n_pages; g.n_pages = n_pool_pages; g.rows = T_p;
   g.n_blocks = T_p / B; g.sums = page_index; g.nb_out = T_p / B; g.by_page = 1;
-  return launch_block_sums(dtype, H * d, B, &g, 1, nullptr, err, static_cast<cudaStream_t>(stream));
+  return launch_block_sums(dtype, H * d, B, &g, 1, nullptr, 0, err, static_cast<cudaStream_t>(stream));
 }
 
 wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, int H, int d,
@@ -409,7 +409,7 @@ wa_status wa_pool_append(void* k_pool, void* v_pool, int n_pool_pages, int T_p, 
   BlockSumSeg g;
   g.x = k_pool; g.rows = static_cast<int>(rows); g.block0 = b_first; g.n_blocks = b_last - b_first + 1;
   g.sums = page_index; g.nb_out = static_cast<int>(rows / B);
-  return launch_block_sums(dtype, H * d, B, &g, 1, nullptr, err, st);
+  return launch_block_sums(dtype, H * d, B, &g, 1, nullptr, 0, err, st);
 }
 
 namespace wa_detail {

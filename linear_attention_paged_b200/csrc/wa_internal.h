@@ -49,7 +49,7 @@ wa_status launch_prompt_select(const float* e_cur, const float* e_chunks, int n_
 // source are summed (the last block of a source may be ragged) into
 //   sums[((by_page ? page : s) * nb_out + block) * cols + c].
 // Up to two segments per launch (e.g. the queries and the candidate pages).  With
-// `counter` the launch also zeroes that word for launch_page_alpha.
+// `counter` the launch also zeroes n_counters words for launch_page_alpha.
 struct BlockSumSeg {
   const void* x = nullptr;
   const int32_t* ids = nullptr;
@@ -65,19 +65,21 @@ struct BlockSumSeg {
   int by_page = 0;
 };
 wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* segs, int n_segs,
-                            unsigned* counter, uint32_t* err, cudaStream_t st);
+                            unsigned* counter, int n_counters, uint32_t* err, cudaStream_t st);
 // Page scores from block sums: Qbar = sum of qsum rows / Nq (written to qbar, and the
 // query block means to qmean when non-null), column sums of each candidate page's
 // block sums (ksum rows of page kpage[row][j], or of position j when kpage is null),
 // alpha_j = Qbar . colsum_j / (T_p sqrt(d) H), then the top-K_p pages (sel: pool ids
 // from cand[row][.], or positions when cand is null; sel_pos: positions), ascending.
-// `partial` holds page_alpha_partial_count(cols, n_c) doubles; `counter` must be zero
-// (launch_block_sums zeroes it) and is left zero.
-size_t page_alpha_partial_count(int cols, int n_c);
+// `scratch` holds page_alpha_scratch_doubles(cols, n_c) doubles; the
+// page_alpha_counters(cols) words at `counters` must be zero (launch_block_sums zeroes
+// them) and are left zero.
+size_t page_alpha_scratch_doubles(int cols, int n_c);
+int page_alpha_counters(int cols);
 wa_status launch_page_alpha(const double* qsum, int n_qb, int Nq, int B, int cols, const double* ksum,
                             const int32_t* kpage, int n_pages, int nbp, const int32_t* cand,
                             const int32_t* chunk, int n_chunks, int n_c, int T_p, int H, int d,
-                            int K_p, double* qbar, double* qmean, double* partial, unsigned* counter,
+                            int K_p, double* qbar, double* qmean, double* scratch, unsigned* counters,
                             double* alpha, int32_t* sel, int32_t* sel_pos, uint32_t* err,
                             cudaStream_t st);
 
