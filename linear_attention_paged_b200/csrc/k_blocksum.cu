@@ -30,6 +30,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kMaxSegs = 2;
+constexpr int kMaxPagesFused = 4096;      // candidate pages of a pass with fused page scores
 constexpr int kMaxStages = 16;
 // Three CTAs per SM, each with a ring of three 24 KB stages at the one-layer shape
 // (a sweep over 2-6 CTAs per SM, 32-96 KB rings and 6-48 KB copies put this setting
@@ -67,12 +68,27 @@ struct PassArgs {
   unsigned* counter;        // nullable: n_counters words zeroed here for the page-score kernel
   int n_counters;
   uint64_t wait_ns;
+  // page scores fused into the pass (qbar != nullptr; one segment of candidate pages,
+  // one block per unit): each consumer warp adds the dot products of its columns of a
+  // block sum with qbar and writes one value per (unit, warp) to kdot; the last CTA to
+  // finish forms alpha and the top-K_p pages from them
+  const double* qbar;
+  double* kdot;             // [units][consumer warps]
+  unsigned* done;           // completion counter (zero at launch; left zero)
+  const int32_t* cand;      // [n_chunks][n_c] pool ids (row *chunk), for sel
+  const int32_t* chunk;
+  int n_chunks, n_c, nbp, K_p;
+  double alpha_den;         // T_p * sqrt(d) * H
+  double* alpha;
+  int32_t* sel;
+  int32_t* sel_pos;
 };
 
 struct PassShared {
   uint64_t full[kMaxStages];
   uint64_t empty[kMaxStages];
   int abort_flag;
+  int last;
 };
 
 // unit -> (segment, source position, block)
@@ -175,6 +191,9 @@ k_block_sums(const __grid_constant__ PassArgs a, uint32_t* err) {
   } else if (warp <= n_cons_warps) {
     const int grp = tid - 32;
     const bool active = grp < a.G;
+    double qb[V];   // this thread's columns of Qbar (fused page scores)
+#pragma unroll
+    for (int v = 0; v < V; ++v) qb[v] = (a.qbar && active) ? a.qbar[grp * V + v] : 0.0;
     int k = 0;
     bool alive = true;
     for (int u = blockIdx.x; u < a.total_units && alive; u += gridDim.x) {
@@ -217,6 +236,15 @@ k_block_sums(const __grid_constant__ PassArgs a, uint32_t* err) {
           for (int v = 0; v < V; ++v) out[v] = acc[v];
         }
       }
+      if (a.qbar) {
+        // this warp's part of Qbar . (block sum): columns in order, then a fixed butterfly
+        double dot = 0.0;
+#pragma unroll
+        for (int v = 0; v < V; ++v) dot += acc[v] * qb[v];
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+        if (lane == 0) a.kdot[static_cast<size_t>(u) * n_cons_warps + (warp - 1)] = dot;
+      }
     }
   }
   __syncthreads();
@@ -226,6 +254,59 @@ k_block_sums(const __grid_constant__ PassArgs a, uint32_t* err) {
     for (int k = issued > a.S ? issued - a.S : 0; k < issued; ++k)
       if (mbar_wait_bounded(&sh.full[k % a.S], (k / a.S) & 1, &never, a.wait_ns) == kWaitTimeout)
         atomicOr(err, WA_DEVERR_TIMEOUT);
+  }
+  // fused page scores: the last CTA to finish adds every page's (block, warp) dot
+  // products in order, forms alpha and takes the top-K_p pages (a CTA that gave up
+  // does not take part: the error word already reports the failure)
+  if (!a.qbar || sh.abort_flag) return;
+  __threadfence();
+  __syncthreads();
+  if (tid == 0) sh.last = atomicAdd(a.done, 1u) == gridDim.x - 1;
+  __syncthreads();
+  if (!sh.last) return;
+  __threadfence();
+  const int nw = blockDim.x >> 5;
+  const int per_page = a.nbp * n_cons_warps;
+  for (int c = warp; c < a.n_c; c += nw) {
+    const double* kd = a.kdot + static_cast<size_t>(c) * per_page;
+    double t = 0.0;
+    for (int e = lane; e < per_page; e += 32) t += __ldcg(kd + e);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+    if (lane == 0) a.alpha[c] = t / a.alpha_den;
+  }
+  unsigned char* chosen = smem_raw;   // the ring is idle now: n_c flags
+  for (int c = tid; c < a.n_c; c += blockDim.x) chosen[c] = 0;
+  __syncthreads();
+  if (warp != 0) return;
+  for (int k = 0; k < a.K_p; ++k) {
+    double best = -DBL_MAX;
+    int bi = INT_MAX;
+    for (int c = lane; c < a.n_c; c += 32) {
+      if (chosen[c]) continue;
+      const double v = const_cast<const volatile double*>(a.alpha)[c];
+      if (bi == INT_MAX || v > best) { best = v; bi = c; }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (oi != INT_MAX && (bi == INT_MAX || ob > best || (ob == best && oi < bi))) { best = ob; bi = oi; }
+    }
+    if (lane == 0 && bi != INT_MAX) chosen[bi] = 1;
+    __syncwarp();
+  }
+  if (lane == 0) {
+    int row = a.chunk ? *a.chunk : 0;
+    if (row < 0 || row >= a.n_chunks) row = 0;
+    int k = 0;
+    for (int c = 0; c < a.n_c && k < a.K_p; ++c)
+      if (chosen[c]) {
+        a.sel[k] = a.cand ? a.cand[static_cast<size_t>(row) * a.n_c + c] : c;
+        if (a.sel_pos) a.sel_pos[k] = c;
+        ++k;
+      }
+    *a.done = 0u;
   }
 }
 
@@ -396,10 +477,44 @@ int n_sm() {
 
 }  // namespace
 
+namespace {
+wa_status launch_pass(PassArgs& a, wa_dtype dt, int cols, int B, const BlockSumSeg* segs, int n_segs,
+                      unsigned* counter, int n_counters, uint32_t* err, cudaStream_t st);
+}
+
 wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* segs, int n_segs,
                             unsigned* counter, int n_counters, uint32_t* err, cudaStream_t st) {
-  if (n_segs < 1 || n_segs > kMaxSegs) return set_error(WA_ERR_INVALID_ARG, "block sums: 1 or 2 segments");
   PassArgs a{};
+  return launch_pass(a, dt, cols, B, segs, n_segs, counter, n_counters, err, st);
+}
+
+size_t fused_kdot_doubles(int cols, int B, int n_c, int T_p, wa_dtype dt) {
+  const int G = cols * (dt == WA_BF16 ? 2 : 4) / 16;
+  const size_t warps = (G + 31) / 32;
+  return static_cast<size_t>(n_c) * ((T_p + B - 1) / B) * warps;
+}
+
+wa_status launch_block_sums_scored(wa_dtype dt, int cols, int B, const BlockSumSeg& pages,
+                                   const double* qbar, double* kdot, unsigned* done,
+                                   int n_chunks, int T_p, int H, int d, int K_p, double* alpha,
+                                   int32_t* sel, int32_t* sel_pos, uint32_t* err, cudaStream_t st) {
+  if (pages.n_src > kMaxPagesFused)
+    return set_error(WA_ERR_UNSUPPORTED, "fused page scores: at most %d candidate pages", kMaxPagesFused);
+  if (pages.block0 != 0 || pages.by_page)
+    return set_error(WA_ERR_INVALID_ARG, "fused page scores: whole pages by position");
+  PassArgs a{};
+  a.qbar = qbar; a.kdot = kdot; a.done = done;
+  a.cand = pages.ids; a.chunk = pages.chunk; a.n_chunks = n_chunks < 1 ? 1 : n_chunks;
+  a.n_c = pages.n_src; a.nbp = pages.n_blocks; a.K_p = K_p;
+  a.alpha_den = static_cast<double>(T_p) * sqrt(static_cast<double>(d)) * H;
+  a.alpha = alpha; a.sel = sel; a.sel_pos = sel_pos;
+  return launch_pass(a, dt, cols, B, &pages, 1, nullptr, 0, err, st);
+}
+
+namespace {
+wa_status launch_pass(PassArgs& a, wa_dtype dt, int cols, int B, const BlockSumSeg* segs, int n_segs,
+                      unsigned* counter, int n_counters, uint32_t* err, cudaStream_t st) {
+  if (n_segs < 1 || n_segs > kMaxSegs) return set_error(WA_ERR_INVALID_ARG, "block sums: 1 or 2 segments");
   const int es = dt == WA_BF16 ? 2 : 4;
   a.cols = cols;
   a.row_bytes = cols * es;
@@ -456,6 +571,7 @@ wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* seg
   if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "block sums smem attr: %s", cudaGetErrorString(e));
   return check_launch("block_sums");
 }
+}  // namespace
 
 size_t page_alpha_scratch_doubles(int cols, int n_c) {
   const size_t n_cs = (cols + kAlphaCols - 1) / kAlphaCols;

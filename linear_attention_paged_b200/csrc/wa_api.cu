@@ -173,11 +173,13 @@ struct PageScoreWs {
   double* qbar;         // [cols]
   double* q_blockmean;  // [n_qb][cols]
   double* k_blocksum;   // [n_c][nbp][cols] by candidate position (nullable: page index)
-  double* scratch;      // column-sum parts and partial dot products of the page scores
-  unsigned* counters;   // completion counters of the page-score kernel
+  double* kdot;         // per (block, warp) page-score dot products of the candidate pass
+  double* scratch;      // page-score kernel scratch (page index path)
+  unsigned* counters;   // completion counters (zeroed by the query pass)
 };
 
-PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks) {
+PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks,
+                             wa_dtype dt) {
   PageScoreWs w{};
   const int cols = H * d;
   const int n_qb = ceil_div(Nq, B);
@@ -185,15 +187,18 @@ PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, 
   w.qbar = c.take<double>(cols);
   w.q_blockmean = c.take<double>(static_cast<size_t>(n_qb) * cols);
   w.k_blocksum = k_blocks ? c.take<double>(static_cast<size_t>(n_c) * ceil_div(T_p, B) * cols) : nullptr;
-  w.scratch = c.take<double>(page_alpha_scratch_doubles(cols, n_c));
+  w.kdot = k_blocks ? c.take<double>(fused_kdot_doubles(cols, B, n_c, T_p, dt)) : nullptr;
+  w.scratch = k_blocks ? nullptr : c.take<double>(page_alpha_scratch_doubles(cols, n_c));
   w.counters = c.take<unsigned>(page_alpha_counters(cols));
   return w;
 }
 
-// One pass over the queries and the candidate pages (block sums, float64), then the
-// page scores and the top-K_p pages from those sums.  The candidate pages are row
-// *chunk (or row 0) of chunk_pages [n_chunks][n_c].  With a page index the pass reads
-// only the queries and the scores read the index's block sums of the candidates.
+// S1.  The queries' block sums and their means first (Qbar, the query block means),
+// then one pass over the candidate pages that writes their block sums and forms the
+// page scores on the fly (each block's sum is dotted with Qbar while it is in
+// registers), the last CTA taking the top-K_p pages.  The candidate pages are row
+// *chunk (or row 0) of chunk_pages [n_chunks][n_c].  With a page index only the
+// queries are read, and the scores come from the index's block sums.
 wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int d,
                          const void* k_pool, int n_pool_pages, int T_p, const int32_t* chunk_pages,
                          const int32_t* chunk, int n_chunks, int n_c, int K_p, int B, wa_dtype dt,
@@ -203,20 +208,19 @@ wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int
   uint32_t* err = errw();
   if (!err) return set_error(WA_ERR_CUDA, "no device error word (is a CUDA device present?)");
   const int n_qb = ceil_div(Nq, B), nbp = ceil_div(T_p, B);
-  BlockSumSeg seg[2];
-  seg[0].x = q; seg[0].rows = Nq; seg[0].n_blocks = n_qb; seg[0].sums = w.q_blocksum; seg[0].nb_out = n_qb;
-  int n_segs = 1;
-  if (!page_index) {
-    BlockSumSeg& g = seg[1];
-    g.x = k_pool; g.ids = chunk_pages; g.chunk = chunk; g.id_rows = n_chunks; g.n_src = n_c;
-    g.n_pages = n_pool_pages; g.rows = T_p; g.n_blocks = nbp; g.sums = w.k_blocksum; g.nb_out = nbp;
-    n_segs = 2;
-  }
-  WA_TRY(launch_block_sums(dt, cols, B, seg, n_segs, w.counters, page_alpha_counters(cols), err, st));
-  return launch_page_alpha(w.q_blocksum, n_qb, Nq, B, cols, page_index ? page_index : w.k_blocksum,
-                           page_index ? chunk_pages : nullptr, n_pool_pages, nbp, chunk_pages, chunk,
-                           n_chunks, n_c, T_p, H, d, K_p, w.qbar, w.q_blockmean, w.scratch, w.counters,
-                           alpha, sel, sel_pos, err, st);
+  BlockSumSeg gq;
+  gq.x = q; gq.rows = Nq; gq.n_blocks = n_qb; gq.sums = w.q_blocksum; gq.nb_out = n_qb;
+  WA_TRY(launch_block_sums(dt, cols, B, &gq, 1, w.counters, page_alpha_counters(cols), err, st));
+  if (page_index)
+    return launch_page_alpha(w.q_blocksum, n_qb, Nq, B, cols, page_index, chunk_pages, n_pool_pages, nbp,
+                             chunk_pages, chunk, n_chunks, n_c, T_p, H, d, K_p, w.qbar, w.q_blockmean,
+                             w.scratch, w.counters, alpha, sel, sel_pos, err, st);
+  WA_TRY(launch_qmeans(w.q_blocksum, n_qb, Nq, B, cols, w.qbar, w.q_blockmean, st));
+  BlockSumSeg g;
+  g.x = k_pool; g.ids = chunk_pages; g.chunk = chunk; g.id_rows = n_chunks; g.n_src = n_c;
+  g.n_pages = n_pool_pages; g.rows = T_p; g.n_blocks = nbp; g.sums = w.k_blocksum; g.nb_out = nbp;
+  return launch_block_sums_scored(dt, cols, B, g, w.qbar, w.kdot, w.counters, n_chunks, T_p, H, d, K_p,
+                                  alpha, sel, sel_pos, err, st);
 }
 
 // Block sums of one contiguous buffer of `rows` rows (all its blocks).
@@ -266,7 +270,7 @@ wa_status wa_prompt_select(const float* e_cur, const float* e_chunks, int n_chun
 size_t wa_page_score_workspace_size(int Nq, int H, int d, int n_c, int T_p, int B) {
   if (Nq < 1 || H < 1 || d < 1 || n_c < 1 || T_p < 1 || B < 1) return 0;
   Carver c(nullptr);
-  carve_page_score(c, Nq, H, d, n_c, T_p, B, true);
+  carve_page_score(c, Nq, H, d, n_c, T_p, B, true, WA_F32);   // the larger of the two dtypes
   c.take<int32_t>(n_c);
   return c.used;
 }
@@ -285,7 +289,7 @@ wa_status wa_page_score(const void* q, int Nq, int H, int d, const void* k_pool,
   WA_TRY(check_ws(ws, ws_bytes, wa_page_score_workspace_size(Nq, H, d, n_c, T_p, B)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carver c(ws);
-  PageScoreWs w = carve_page_score(c, Nq, H, d, n_c, T_p, B, true);
+  PageScoreWs w = carve_page_score(c, Nq, H, d, n_c, T_p, B, true, WA_F32);
   int32_t* sel_pos = c.take<int32_t>(n_c);
   WA_TRY(run_page_score(w, q, Nq, H, d, k_pool, n_pool_pages, T_p, cand_pages, nullptr, 1, n_c, K_p, B,
                         dtype, alpha, sel, sel_pos, st));
@@ -662,7 +666,7 @@ StepWs carve_step(Carver& c, const wa_step_args* a) {
   const size_t es = elem_size(a->dtype);
   w.chunk = c.take<int32_t>(1);
   // block sums of the candidate pages, unless the page index holds them
-  w.ps = carve_page_score(c, a->Nq, a->H, a->d, a->n_c, a->T_p, a->B, a->page_index == nullptr);
+  w.ps = carve_page_score(c, a->Nq, a->H, a->d, a->n_c, a->T_p, a->B, a->page_index == nullptr, WA_F32);
   w.alpha = c.take<double>(a->n_c);
   w.sel = c.take<int32_t>(a->K_p);
   w.sel_pos = c.take<int32_t>(a->K_p);

@@ -66,6 +66,17 @@ struct BlockSumSeg {
 };
 wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* segs, int n_segs,
                             unsigned* counter, int n_counters, uint32_t* err, cudaStream_t st);
+// The same pass over whole candidate pages (one segment, sums by position) with the
+// page scores fused in: qbar [cols] must be ready; each consumer warp writes its dot
+// products with qbar to kdot (fused_kdot_doubles), and the last CTA forms
+// alpha_j = Qbar . colsum_j / (T_p sqrt(d) H) and the top-K_p pages (sel: pool ids of
+// row *chunk of pages.ids, sel_pos: positions), ascending.  *done must be zero
+// (launch_block_sums zeroes it) and is left zero.
+size_t fused_kdot_doubles(int cols, int B, int n_c, int T_p, wa_dtype dt);
+wa_status launch_block_sums_scored(wa_dtype dt, int cols, int B, const BlockSumSeg& pages,
+                                   const double* qbar, double* kdot, unsigned* done,
+                                   int n_chunks, int T_p, int H, int d, int K_p, double* alpha,
+                                   int32_t* sel, int32_t* sel_pos, uint32_t* err, cudaStream_t st);
 // Page scores from block sums: Qbar = sum of qsum rows / Nq (written to qbar, and the
 // query block means to qmean when non-null), column sums of each candidate page's
 // block sums (ksum rows of page kpage[row][j], or of position j when kpage is null),
