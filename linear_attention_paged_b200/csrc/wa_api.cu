@@ -173,13 +173,12 @@ struct PageScoreWs {
   double* qbar;         // [cols]
   double* q_blockmean;  // [n_qb][cols]
   double* k_blocksum;   // [n_c][nbp][cols] by candidate position (nullable: page index)
-  double* kdot;         // per (block, warp) page-score dot products of the candidate pass
+  double* kdot;         // page-score dot products per (candidate block, warp)
   double* scratch;      // page-score kernel scratch (page index path)
-  unsigned* counters;   // completion counters (zeroed by the query pass)
+  unsigned* counters;   // completion counters
 };
 
-PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks,
-                             wa_dtype dt) {
+PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks) {
   PageScoreWs w{};
   const int cols = H * d;
   const int n_qb = ceil_div(Nq, B);
@@ -187,18 +186,18 @@ PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, 
   w.qbar = c.take<double>(cols);
   w.q_blockmean = c.take<double>(static_cast<size_t>(n_qb) * cols);
   w.k_blocksum = k_blocks ? c.take<double>(static_cast<size_t>(n_c) * ceil_div(T_p, B) * cols) : nullptr;
-  w.kdot = k_blocks ? c.take<double>(fused_kdot_doubles(cols, B, n_c, T_p, dt)) : nullptr;
+  // sized for float32 rows, the larger per-row warp count of the two dtypes
+  w.kdot = k_blocks ? c.take<double>(page_retrieval_kdot_doubles(cols, n_c, T_p, B, WA_F32)) : nullptr;
   w.scratch = k_blocks ? nullptr : c.take<double>(page_alpha_scratch_doubles(cols, n_c));
-  w.counters = c.take<unsigned>(page_alpha_counters(cols));
+  w.counters = c.take<unsigned>(page_alpha_counters(cols) > 3 ? page_alpha_counters(cols) : 3);
   return w;
 }
 
-// S1.  The queries' block sums and their means first (Qbar, the query block means),
-// then one pass over the candidate pages that writes their block sums and forms the
-// page scores on the fly (each block's sum is dotted with Qbar while it is in
-// registers), the last CTA taking the top-K_p pages.  The candidate pages are row
-// *chunk (or row 0) of chunk_pages [n_chunks][n_c].  With a page index only the
-// queries are read, and the scores come from the index's block sums.
+// S1: one cooperative launch reads the queries and the candidate pages once, writing
+// their block sums and forming the page scores and the top-K_p pages on the way.  The
+// candidate pages are row *chunk (or row 0) of chunk_pages [n_chunks][n_c].  With a
+// page index only the queries are read, and the scores come from the index's block
+// sums of the candidates.
 wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int d,
                          const void* k_pool, int n_pool_pages, int T_p, const int32_t* chunk_pages,
                          const int32_t* chunk, int n_chunks, int n_c, int K_p, int B, wa_dtype dt,
@@ -208,19 +207,16 @@ wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int
   uint32_t* err = errw();
   if (!err) return set_error(WA_ERR_CUDA, "no device error word (is a CUDA device present?)");
   const int n_qb = ceil_div(Nq, B), nbp = ceil_div(T_p, B);
+  if (!page_index)
+    return launch_page_retrieval(dt, q, Nq, H, d, k_pool, n_pool_pages, T_p, chunk_pages, chunk, n_chunks,
+                                 n_c, K_p, B, w.q_blocksum, w.k_blocksum, w.qbar, w.q_blockmean, w.kdot,
+                                 w.counters, alpha, sel, sel_pos, err, st);
   BlockSumSeg gq;
   gq.x = q; gq.rows = Nq; gq.n_blocks = n_qb; gq.sums = w.q_blocksum; gq.nb_out = n_qb;
   WA_TRY(launch_block_sums(dt, cols, B, &gq, 1, w.counters, page_alpha_counters(cols), err, st));
-  if (page_index)
-    return launch_page_alpha(w.q_blocksum, n_qb, Nq, B, cols, page_index, chunk_pages, n_pool_pages, nbp,
-                             chunk_pages, chunk, n_chunks, n_c, T_p, H, d, K_p, w.qbar, w.q_blockmean,
-                             w.scratch, w.counters, alpha, sel, sel_pos, err, st);
-  WA_TRY(launch_qmeans(w.q_blocksum, n_qb, Nq, B, cols, w.qbar, w.q_blockmean, st));
-  BlockSumSeg g;
-  g.x = k_pool; g.ids = chunk_pages; g.chunk = chunk; g.id_rows = n_chunks; g.n_src = n_c;
-  g.n_pages = n_pool_pages; g.rows = T_p; g.n_blocks = nbp; g.sums = w.k_blocksum; g.nb_out = nbp;
-  return launch_block_sums_scored(dt, cols, B, g, w.qbar, w.kdot, w.counters, n_chunks, T_p, H, d, K_p,
-                                  alpha, sel, sel_pos, err, st);
+  return launch_page_alpha(w.q_blocksum, n_qb, Nq, B, cols, page_index, chunk_pages, n_pool_pages, nbp,
+                           chunk_pages, chunk, n_chunks, n_c, T_p, H, d, K_p, w.qbar, w.q_blockmean,
+                           w.scratch, w.counters, alpha, sel, sel_pos, err, st);
 }
 
 // Block sums of one contiguous buffer of `rows` rows (all its blocks).
@@ -270,7 +266,7 @@ wa_status wa_prompt_select(const float* e_cur, const float* e_chunks, int n_chun
 size_t wa_page_score_workspace_size(int Nq, int H, int d, int n_c, int T_p, int B) {
   if (Nq < 1 || H < 1 || d < 1 || n_c < 1 || T_p < 1 || B < 1) return 0;
   Carver c(nullptr);
-  carve_page_score(c, Nq, H, d, n_c, T_p, B, true, WA_F32);   // the larger of the two dtypes
+  carve_page_score(c, Nq, H, d, n_c, T_p, B, true);
   c.take<int32_t>(n_c);
   return c.used;
 }
@@ -289,7 +285,7 @@ wa_status wa_page_score(const void* q, int Nq, int H, int d, const void* k_pool,
   WA_TRY(check_ws(ws, ws_bytes, wa_page_score_workspace_size(Nq, H, d, n_c, T_p, B)));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Carver c(ws);
-  PageScoreWs w = carve_page_score(c, Nq, H, d, n_c, T_p, B, true, WA_F32);
+  PageScoreWs w = carve_page_score(c, Nq, H, d, n_c, T_p, B, true);
   int32_t* sel_pos = c.take<int32_t>(n_c);
   WA_TRY(run_page_score(w, q, Nq, H, d, k_pool, n_pool_pages, T_p, cand_pages, nullptr, 1, n_c, K_p, B,
                         dtype, alpha, sel, sel_pos, st));
@@ -666,7 +662,7 @@ StepWs carve_step(Carver& c, const wa_step_args* a) {
   const size_t es = elem_size(a->dtype);
   w.chunk = c.take<int32_t>(1);
   // block sums of the candidate pages, unless the page index holds them
-  w.ps = carve_page_score(c, a->Nq, a->H, a->d, a->n_c, a->T_p, a->B, a->page_index == nullptr, WA_F32);
+  w.ps = carve_page_score(c, a->Nq, a->H, a->d, a->n_c, a->T_p, a->B, a->page_index == nullptr);
   w.alpha = c.take<double>(a->n_c);
   w.sel = c.take<int32_t>(a->K_p);
   w.sel_pos = c.take<int32_t>(a->K_p);
