@@ -461,6 +461,10 @@ k_page_retrieval(const __grid_constant__ S1Args a, uint32_t* err) {
   const int32_t* cand = a.ids + static_cast<size_t>(row) * a.n_c;
   const unsigned q_target = static_cast<unsigned>(a.n_qb) * n_cons_warps;
   const int n_qbar_warps = (a.cols + 31) / 32;
+  // the Qbar warps: the CTAs right after the query-block owners (they have no query
+  // block and one candidate block fewer than the last CTAs), else the first CTAs
+  const int n_duty_ctas = (n_qbar_warps + n_cons_warps - 1) / n_cons_warps;
+  const int duty0 = G >= a.n_qb + n_duty_ctas ? a.n_qb : 0;
   if (tid == 0) {
     for (int s = 0; s < a.S; ++s) {
       mbar_init(&sh.full[s], 1);
@@ -524,19 +528,31 @@ k_page_retrieval(const __grid_constant__ S1Args a, uint32_t* err) {
     // Qbar duty of this warp (if it has one): 32 columns of Qbar and of the query block
     // means, once every query block is in
     auto qbar_duty = [&]() -> bool {
-      const int qw = blockIdx.x * n_cons_warps + cw;
-      if (qw >= n_qbar_warps) return true;
+      const int qw = (static_cast<int>(blockIdx.x) - duty0) * n_cons_warps + cw;
+      if (qw < 0 || qw >= n_qbar_warps) return true;
       if (!__all_sync(0xffffffffu, wait_count(&a.counters[0], q_target, &sh.abort_flag, a.wait_ns))) {
         if (lane == 0) atomicOr(err, WA_DEVERR_TIMEOUT);
         return false;
       }
       const int col = qw * 32 + lane;
       if (col < a.cols) {
+        // loads in batches of 16 (all in flight), then the adds in block order
+        const double* __restrict__ qs = a.qsum + col;
+        double* __restrict__ qm = a.qmean + col;
         double t = 0.0;
-        for (int i = 0; i < a.n_qb; ++i) {
-          const double v = __ldcg(a.qsum + static_cast<size_t>(i) * a.cols + col);
-          t += v;
-          a.qmean[static_cast<size_t>(i) * a.cols + col] = v / (min(a.Nq, (i + 1) * a.B) - i * a.B);
+        for (int i0 = 0; i0 < a.n_qb; i0 += 16) {
+          double v[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            v[e] = i0 + e < a.n_qb ? __ldcg(qs + static_cast<size_t>(i0 + e) * a.cols) : 0.0;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int i = i0 + e;
+            if (i < a.n_qb) {
+              t += v[e];
+              qm[static_cast<size_t>(i) * a.cols] = v[e] / (min(a.Nq, (i + 1) * a.B) - i * a.B);
+            }
+          }
         }
         a.qbar[col] = t / a.Nq;
       }
