@@ -794,6 +794,10 @@ wa_status launch_page_retrieval(wa_dtype dt, const void* q, int Nq, int H, int d
   const void* fn = dt == WA_BF16 ? reinterpret_cast<const void*>(&k_page_retrieval<__nv_bfloat16>)
                                  : reinterpret_cast<const void*>(&k_page_retrieval<float>);
   cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  // all of the unified L1 / shared memory as shared, so that kCtasPerSm rings fit an SM
+  // (the occupancy below, which sizes the cooperative grid, assumes this split)
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
   if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "page retrieval smem attr: %s", cudaGetErrorString(e));
   int per_sm = 0;
   e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
