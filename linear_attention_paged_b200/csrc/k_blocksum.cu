@@ -426,14 +426,33 @@ struct S1Args {
   uint64_t wait_ns;
 };
 
+// Bounded wait for a global counter to reach `target`, polled by one thread with a
+// pause between reads (many pollers on one word slow the L2 traffic everyone needs).
 __device__ __forceinline__ bool wait_count(const unsigned* ctr, unsigned target, int* abort_flag,
                                            uint64_t limit_ns) {
   if (ld_acquire_u32(ctr) >= target) return true;
   const uint64_t t0 = globaltimer_ns();
   for (uint32_t i = 1;; ++i) {
-    __nanosleep(64);
+    __nanosleep(256);
     if (ld_acquire_u32(ctr) >= target) return true;
-    if ((i & 63u) == 0u) {
+    if ((i & 15u) == 0u) {
+      if (*reinterpret_cast<volatile int*>(abort_flag)) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *reinterpret_cast<volatile int*>(abort_flag) = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Bounded wait for a shared-memory flag set by another warp of the CTA.
+__device__ __forceinline__ bool wait_flag(const int* flag, int* abort_flag, uint64_t limit_ns) {
+  if (*reinterpret_cast<const volatile int*>(flag)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(128);
+    if (*reinterpret_cast<const volatile int*>(flag)) return true;
+    if ((i & 15u) == 0u) {
       if (*reinterpret_cast<volatile int*>(abort_flag)) return false;
       if (globaltimer_ns() - t0 > limit_ns) {
         *reinterpret_cast<volatile int*>(abort_flag) = 1;
@@ -450,6 +469,7 @@ k_page_retrieval(const __grid_constant__ S1Args a, uint32_t* err) {
   extern __shared__ __align__(128) uint8_t smem_raw[];
   __shared__ PassShared sh;
   __shared__ int last;
+  __shared__ int qbar_in;   // set by the CTA's poller once Qbar is complete
   const int chunk_bytes = a.R * a.row_bytes;
   uint8_t* ring = smem_raw;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -471,6 +491,7 @@ k_page_retrieval(const __grid_constant__ S1Args a, uint32_t* err) {
       mbar_init(&sh.empty[s], n_cons_warps);
     }
     sh.abort_flag = 0;
+    qbar_in = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -530,7 +551,9 @@ k_page_retrieval(const __grid_constant__ S1Args a, uint32_t* err) {
     auto qbar_duty = [&]() -> bool {
       const int qw = (static_cast<int>(blockIdx.x) - duty0) * n_cons_warps + cw;
       if (qw < 0 || qw >= n_qbar_warps) return true;
-      if (!__all_sync(0xffffffffu, wait_count(&a.counters[0], q_target, &sh.abort_flag, a.wait_ns))) {
+      int ok = 1;
+      if (lane == 0) ok = wait_count(&a.counters[0], q_target, &sh.abort_flag, a.wait_ns) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) {
         if (lane == 0) atomicOr(err, WA_DEVERR_TIMEOUT);
         return false;
       }
@@ -600,9 +623,18 @@ k_page_retrieval(const __grid_constant__ S1Args a, uint32_t* err) {
         continue;
       }
       if (!have_qbar) {
-        const bool ok = __all_sync(0xffffffffu, wait_count(&a.counters[1], static_cast<unsigned>(n_qbar_warps),
-                                                           &sh.abort_flag, a.wait_ns));
-        if (!ok) {
+        // one poller per CTA (the first consumer warp); the others watch its flag
+        int ok = 1;
+        if (lane == 0) {
+          if (cw == 0) {
+            ok = wait_count(&a.counters[1], static_cast<unsigned>(n_qbar_warps), &sh.abort_flag, a.wait_ns);
+            if (ok) *reinterpret_cast<volatile int*>(&qbar_in) = 1;
+          } else {
+            ok = wait_flag(&qbar_in, &sh.abort_flag, a.wait_ns) &&
+                 ld_acquire_u32(&a.counters[1]) >= static_cast<unsigned>(n_qbar_warps);
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
           if (lane == 0) atomicOr(err, WA_DEVERR_TIMEOUT);
           alive = false;
           break;
