@@ -101,12 +101,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
       : "memory");
 }
 
-__device__ __forceinline__ unsigned ld_acquire_u32(const unsigned* p) {
-  unsigned v;
-  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
-
 __device__ __forceinline__ double bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ double bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
@@ -389,328 +383,6 @@ k_page_alpha(const double* __restrict__ qsum, int n_qb, int Nq, int B, int cols,
   }
 }
 
-// ------------------------------------------------------------------ S1 in one launch
-// Page retrieval as one cooperative launch (all CTAs resident at once), streaming the
-// queries and the candidate pages through the same bulk-copy rings as the pass above:
-//   1. the CTAs that own a query block (CTA c owns blocks c, c + G, ...) sum it first;
-//   2. consumer warps of the first few CTAs then each take 32 columns (after their own
-//      CTA's query blocks, before its candidate blocks): once every query block is in
-//      (a bounded wait on a counter), Qbar = sum / Nq and the query block means;
-//   3. every CTA streams its candidate blocks (handed out from the last CTA down, so
-//      the CTAs with query work get fewer), writes each block sum and, once Qbar is
-//      in (a second bounded wait, normally long satisfied), dots it with Qbar while it
-//      is in registers: one value per (block, consumer warp);
-//   4. the last CTA to finish adds every page's values in order, forms
-//      alpha_j = Qbar . colsum_j / (T_p sqrt(d) H) and takes the top-K_p pages.
-// The waits only depend on work that resident CTAs do before any wait of their own,
-// so they cannot deadlock; a wait that runs out records WA_DEVERR_TIMEOUT.
-struct S1Args {
-  const char* q;            // [Nq][cols]
-  const char* k_pool;       // [n_pages][T_p][cols]
-  const int32_t* ids;       // [n_chunks][n_c] pool page ids
-  const int32_t* chunk;     // nullable: row of ids
-  int n_chunks, n_c, n_pages;
-  int Nq, n_qb, T_p, nbp;
-  int cols, row_bytes, B, R, S, G;
-  double* qsum;             // [n_qb][cols]
-  double* ksum;             // [n_c][nbp][cols]
-  double* qbar;             // [cols]
-  double* qmean;            // [n_qb][cols]
-  double* kdot;             // [n_c * nbp][consumer warps]
-  unsigned* counters;       // [3]: query warps done, Qbar warps done, CTAs done (zero at launch)
-  int K_p;
-  double alpha_den;
-  double* alpha;
-  int32_t* sel;
-  int32_t* sel_pos;
-  uint64_t wait_ns;
-};
-
-// Bounded wait for a global counter to reach `target`, polled by one thread with a
-// pause between reads (many pollers on one word slow the L2 traffic everyone needs).
-__device__ __forceinline__ bool wait_count(const unsigned* ctr, unsigned target, int* abort_flag,
-                                           uint64_t limit_ns) {
-  if (ld_acquire_u32(ctr) >= target) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    __nanosleep(256);
-    if (ld_acquire_u32(ctr) >= target) return true;
-    if ((i & 15u) == 0u) {
-      if (*reinterpret_cast<volatile int*>(abort_flag)) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *reinterpret_cast<volatile int*>(abort_flag) = 1;
-        return false;
-      }
-    }
-  }
-}
-
-// Bounded wait for a shared-memory flag set by another warp of the CTA.
-__device__ __forceinline__ bool wait_flag(const int* flag, int* abort_flag, uint64_t limit_ns) {
-  if (*reinterpret_cast<const volatile int*>(flag)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  for (uint32_t i = 1;; ++i) {
-    __nanosleep(128);
-    if (*reinterpret_cast<const volatile int*>(flag)) return true;
-    if ((i & 15u) == 0u) {
-      if (*reinterpret_cast<volatile int*>(abort_flag)) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *reinterpret_cast<volatile int*>(abort_flag) = 1;
-        return false;
-      }
-    }
-  }
-}
-
-template <typename T>
-__global__ void __launch_bounds__(1024)
-k_page_retrieval(const __grid_constant__ S1Args a, uint32_t* err) {
-  constexpr int V = 16 / sizeof(T);
-  extern __shared__ __align__(128) uint8_t smem_raw[];
-  __shared__ PassShared sh;
-  __shared__ int last;
-  __shared__ int qbar_in;   // set by the CTA's poller once Qbar is complete
-  const int chunk_bytes = a.R * a.row_bytes;
-  uint8_t* ring = smem_raw;
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int n_cons_warps = (a.G + 31) >> 5;
-  const int G = gridDim.x;
-  const int n_k = a.n_c * a.nbp;
-  int row = a.chunk ? *a.chunk : 0;
-  if (row < 0 || row >= a.n_chunks) row = 0;
-  const int32_t* cand = a.ids + static_cast<size_t>(row) * a.n_c;
-  const unsigned q_target = static_cast<unsigned>(a.n_qb) * n_cons_warps;
-  const int n_qbar_warps = (a.cols + 31) / 32;
-  // the Qbar warps: the CTAs right after the query-block owners (they have no query
-  // block and one candidate block fewer than the last CTAs), else the first CTAs
-  const int n_duty_ctas = (n_qbar_warps + n_cons_warps - 1) / n_cons_warps;
-  const int duty0 = G >= a.n_qb + n_duty_ctas ? a.n_qb : 0;
-  if (tid == 0) {
-    for (int s = 0; s < a.S; ++s) {
-      mbar_init(&sh.full[s], 1);
-      mbar_init(&sh.empty[s], n_cons_warps);
-    }
-    sh.abort_flag = 0;
-    qbar_in = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
-  // unit k of this CTA: its query blocks first, then its candidate blocks
-  const int my_q = blockIdx.x < a.n_qb ? (a.n_qb - 1 - blockIdx.x) / G + 1 : 0;
-  const int kfirst = G - 1 - blockIdx.x;
-  const int my_k = kfirst < n_k ? (n_k - 1 - kfirst) / G + 1 : 0;
-  auto unit = [&](int k, bool& is_q, int& page, int& pos, int& b, int& r0, int& r1) {
-    if (k < my_q) {
-      is_q = true; page = 0; pos = 0; b = blockIdx.x + k * G;
-      r0 = b * a.B; r1 = min(a.Nq, r0 + a.B);
-    } else {
-      is_q = false;
-      const int u = kfirst + (k - my_q) * G;
-      pos = u / a.nbp; b = u % a.nbp;
-      page = cand[pos];
-      r0 = b * a.B; r1 = min(a.T_p, r0 + a.B);
-    }
-  };
-  int issued = 0;
-  if (warp == 0) {
-    if (lane == 0) {
-      int c = 0;
-      bool go = true;
-      for (int k = 0; k < my_q + my_k && go; ++k) {
-        bool is_q; int page, pos, b, r0, r1;
-        unit(k, is_q, page, pos, b, r0, r1);
-        if (!is_q && (page < 0 || page >= a.n_pages)) { atomicOr(err, WA_DEVERR_PAGE_ID); page = 0; }
-        const char* base = is_q ? a.q + static_cast<size_t>(r0) * a.row_bytes
-                                : a.k_pool + (static_cast<size_t>(page) * a.T_p + r0) * a.row_bytes;
-        for (int r = r0; r < r1; r += a.R, ++c) {
-          const int st = c % a.S;
-          const int w = mbar_wait_bounded(&sh.empty[st], ((c / a.S) & 1) ^ 1, &sh.abort_flag, a.wait_ns);
-          if (w != kWaitOk) {
-            if (w == kWaitTimeout) atomicOr(err, WA_DEVERR_TIMEOUT);
-            go = false;
-            break;
-          }
-          const uint32_t bytes = static_cast<uint32_t>(min(a.R, r1 - r) * a.row_bytes);
-          mbar_arrive_expect_tx(&sh.full[st], bytes);
-          bulk_g2s(ring + static_cast<size_t>(st) * chunk_bytes,
-                   base + static_cast<size_t>(r - r0) * a.row_bytes, bytes, &sh.full[st]);
-          issued = c + 1;
-        }
-      }
-    }
-  } else if (warp <= n_cons_warps) {
-    const int grp = tid - 32;
-    const int cw = warp - 1;                   // consumer warp index
-    const bool active = grp < a.G;
-    double qb[V];
-    bool have_qbar = false;
-    int c = 0;
-    bool alive = true;
-    // Qbar duty of this warp (if it has one): 32 columns of Qbar and of the query block
-    // means, once every query block is in
-    auto qbar_duty = [&]() -> bool {
-      const int qw = (static_cast<int>(blockIdx.x) - duty0) * n_cons_warps + cw;
-      if (qw < 0 || qw >= n_qbar_warps) return true;
-      int ok = 1;
-      if (lane == 0) ok = wait_count(&a.counters[0], q_target, &sh.abort_flag, a.wait_ns) ? 1 : 0;
-      if (!__shfl_sync(0xffffffffu, ok, 0)) {
-        if (lane == 0) atomicOr(err, WA_DEVERR_TIMEOUT);
-        return false;
-      }
-      const int col = qw * 32 + lane;
-      if (col < a.cols) {
-        // loads in batches of 16 (all in flight), then the adds in block order
-        const double* __restrict__ qs = a.qsum + col;
-        double* __restrict__ qm = a.qmean + col;
-        double t = 0.0;
-        for (int i0 = 0; i0 < a.n_qb; i0 += 16) {
-          double v[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            v[e] = i0 + e < a.n_qb ? __ldcg(qs + static_cast<size_t>(i0 + e) * a.cols) : 0.0;
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int i = i0 + e;
-            if (i < a.n_qb) {
-              t += v[e];
-              qm[static_cast<size_t>(i) * a.cols] = v[e] / (min(a.Nq, (i + 1) * a.B) - i * a.B);
-            }
-          }
-        }
-        a.qbar[col] = t / a.Nq;
-      }
-      __threadfence();
-      __syncwarp();
-      if (lane == 0) atomicAdd(&a.counters[1], 1u);
-      return true;
-    };
-    for (int k = 0; k < my_q + my_k && alive; ++k) {
-      if (k == my_q && !qbar_duty()) { alive = false; break; }
-      bool is_q; int page, pos, b, r0, r1;
-      unit(k, is_q, page, pos, b, r0, r1);
-      double acc[V];
-#pragma unroll
-      for (int v = 0; v < V; ++v) acc[v] = 0.0;
-      for (int r = r0; r < r1; r += a.R, ++c) {
-        const int st = c % a.S;
-        const bool got = __all_sync(0xffffffffu, mbar_wait_bounded(&sh.full[st], (c / a.S) & 1,
-                                                                   &sh.abort_flag, a.wait_ns) == kWaitOk);
-        if (!got) { alive = false; break; }
-        if (active) {
-          const int nr = min(a.R, r1 - r);
-          const uint8_t* src = ring + static_cast<size_t>(st) * chunk_bytes + grp * 16;
-#pragma unroll 4
-          for (int rr = 0; rr < nr; ++rr) {
-            const uint4 w = *reinterpret_cast<const uint4*>(src + static_cast<size_t>(rr) * a.row_bytes);
-            add16<T>(w, acc);
-          }
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.empty[st]);
-      }
-      if (!alive) break;
-      double* out = is_q ? a.qsum + static_cast<size_t>(b) * a.cols
-                         : a.ksum + (static_cast<size_t>(pos) * a.nbp + b) * a.cols;
-      if (active) {
-#pragma unroll
-        for (int v = 0; v < V; ++v) out[grp * V + v] = acc[v];
-      }
-      if (is_q) {
-        // this warp's part of a query block is in: count it
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) atomicAdd(&a.counters[0], 1u);
-        continue;
-      }
-      if (!have_qbar) {
-        // one poller per CTA (the first consumer warp); the others watch its flag
-        int ok = 1;
-        if (lane == 0) {
-          if (cw == 0) {
-            ok = wait_count(&a.counters[1], static_cast<unsigned>(n_qbar_warps), &sh.abort_flag, a.wait_ns);
-            if (ok) *reinterpret_cast<volatile int*>(&qbar_in) = 1;
-          } else {
-            ok = wait_flag(&qbar_in, &sh.abort_flag, a.wait_ns) &&
-                 ld_acquire_u32(&a.counters[1]) >= static_cast<unsigned>(n_qbar_warps);
-          }
-        }
-        if (!__shfl_sync(0xffffffffu, ok, 0)) {
-          if (lane == 0) atomicOr(err, WA_DEVERR_TIMEOUT);
-          alive = false;
-          break;
-        }
-#pragma unroll
-        for (int v = 0; v < V; ++v) qb[v] = active ? __ldcg(a.qbar + grp * V + v) : 0.0;
-        have_qbar = true;
-      }
-      double dot = 0.0;
-#pragma unroll
-      for (int v = 0; v < V; ++v) dot += acc[v] * qb[v];
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-      if (lane == 0) a.kdot[(static_cast<size_t>(pos) * a.nbp + b) * n_cons_warps + cw] = dot;
-    }
-    // a CTA without candidate blocks still owes its Qbar duty
-    if (alive && my_k == 0 && !qbar_duty()) alive = false;
-  }
-  __syncthreads();
-  if (sh.abort_flag) {
-    if (warp == 0 && lane == 0) {
-      int never = 0;
-      for (int c = issued > a.S ? issued - a.S : 0; c < issued; ++c)
-        if (mbar_wait_bounded(&sh.full[c % a.S], (c / a.S) & 1, &never, a.wait_ns) == kWaitTimeout)
-          atomicOr(err, WA_DEVERR_TIMEOUT);
-    }
-    return;
-  }
-  __threadfence();
-  __syncthreads();
-  if (tid == 0) last = atomicAdd(&a.counters[2], 1u) == static_cast<unsigned>(G) - 1;
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  const int nw = blockDim.x >> 5;
-  const int per_page = a.nbp * n_cons_warps;
-  for (int c = warp; c < a.n_c; c += nw) {
-    const double* kd = a.kdot + static_cast<size_t>(c) * per_page;
-    double t = 0.0;
-    for (int e = lane; e < per_page; e += 32) t += __ldcg(kd + e);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
-    if (lane == 0) a.alpha[c] = t / a.alpha_den;
-  }
-  unsigned char* chosen = smem_raw;   // the ring is idle now: n_c flags
-  for (int c = tid; c < a.n_c; c += blockDim.x) chosen[c] = 0;
-  __syncthreads();
-  if (warp != 0) return;
-  for (int k = 0; k < a.K_p; ++k) {
-    double best = -DBL_MAX;
-    int bi = INT_MAX;
-    for (int c = lane; c < a.n_c; c += 32) {
-      if (chosen[c]) continue;
-      const double v = const_cast<const volatile double*>(a.alpha)[c];
-      if (bi == INT_MAX || v > best) { best = v; bi = c; }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const double ob = __shfl_xor_sync(0xffffffffu, best, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (oi != INT_MAX && (bi == INT_MAX || ob > best || (ob == best && oi < bi))) { best = ob; bi = oi; }
-    }
-    if (lane == 0 && bi != INT_MAX) chosen[bi] = 1;
-    __syncwarp();
-  }
-  if (lane == 0) {
-    int k = 0;
-    for (int c = 0; c < a.n_c && k < a.K_p; ++c)
-      if (chosen[c]) {
-        a.sel[k] = cand[c];
-        if (a.sel_pos) a.sel_pos[k] = c;
-        ++k;
-      }
-  }
-}
-
 int g_n_sm = 0;
 int n_sm() {
   if (g_n_sm == 0) {
@@ -783,81 +455,6 @@ wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* seg
   }
   if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "block sums smem attr: %s", cudaGetErrorString(e));
   return check_launch("block_sums");
-}
-
-size_t page_retrieval_kdot_doubles(int cols, int n_c, int T_p, int B, wa_dtype dt) {
-  const int G = cols * (dt == WA_BF16 ? 2 : 4) / 16;
-  return static_cast<size_t>(n_c) * ((T_p + B - 1) / B) * ((G + 31) / 32);
-}
-
-wa_status launch_page_retrieval(wa_dtype dt, const void* q, int Nq, int H, int d, const void* k_pool,
-                                int n_pages, int T_p, const int32_t* ids, const int32_t* chunk,
-                                int n_chunks, int n_c, int K_p, int B, double* qsum, double* ksum,
-                                double* qbar, double* qmean, double* kdot, unsigned* counters,
-                                double* alpha, int32_t* sel, int32_t* sel_pos, uint32_t* err,
-                                cudaStream_t st) {
-  S1Args a{};
-  const int es = dt == WA_BF16 ? 2 : 4;
-  a.q = static_cast<const char*>(q);
-  a.k_pool = static_cast<const char*>(k_pool);
-  a.ids = ids; a.chunk = chunk; a.n_chunks = n_chunks < 1 ? 1 : n_chunks; a.n_c = n_c; a.n_pages = n_pages;
-  a.Nq = Nq; a.n_qb = (Nq + B - 1) / B; a.T_p = T_p; a.nbp = (T_p + B - 1) / B;
-  a.cols = H * d; a.row_bytes = a.cols * es; a.B = B;
-  if (a.row_bytes % 16 != 0 || reinterpret_cast<uintptr_t>(q) % 16 || reinterpret_cast<uintptr_t>(k_pool) % 16)
-    return set_error(WA_ERR_UNSUPPORTED, "page retrieval needs 16-byte aligned rows");
-  int R = 1;
-  while (R * 2 <= B && B % (R * 2) == 0 && (R * 2) * a.row_bytes <= kChunkBytesMax) R *= 2;
-  a.R = R;
-  const int chunk_bytes = R * a.row_bytes;
-  a.G = a.row_bytes / 16;
-  if (a.G > 992) return set_error(WA_ERR_UNSUPPORTED, "page retrieval: rows longer than 15872 bytes");
-  int S = kRingBytes / chunk_bytes;
-  if (S > kMaxStages) S = kMaxStages;
-  if (S < 2) S = 2;
-  a.S = S;
-  const size_t smem = static_cast<size_t>(S) * chunk_bytes;
-  if (static_cast<size_t>(n_c) > smem) return set_error(WA_ERR_UNSUPPORTED, "page retrieval: too many candidates");
-  a.qsum = qsum; a.ksum = ksum; a.qbar = qbar; a.qmean = qmean; a.kdot = kdot; a.counters = counters;
-  a.K_p = K_p;
-  a.alpha_den = static_cast<double>(T_p) * sqrt(static_cast<double>(d)) * H;
-  a.alpha = alpha; a.sel = sel; a.sel_pos = sel_pos;
-  a.wait_ns = wait_limit_ns();
-  const int threads = 32 + ((a.G + 31) / 32) * 32;
-  const void* fn = dt == WA_BF16 ? reinterpret_cast<const void*>(&k_page_retrieval<__nv_bfloat16>)
-                                 : reinterpret_cast<const void*>(&k_page_retrieval<float>);
-  cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  // all of the unified L1 / shared memory as shared, so that kCtasPerSm rings fit an SM
-  // (the occupancy below, which sizes the cooperative grid, assumes this split)
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
-  if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "page retrieval smem attr: %s", cudaGetErrorString(e));
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, fn, threads, smem);
-  if (e != cudaSuccess || per_sm < 1)
-    return set_error(WA_ERR_CUDA, "page retrieval occupancy: %s", cudaGetErrorString(e));
-  if (per_sm > kCtasPerSm) per_sm = kCtasPerSm;
-  int grid = per_sm * n_sm();
-  const int n_qbar_warps = (a.cols + 31) / 32;
-  const int n_cw = (a.G + 31) / 32;
-  // the Qbar warps sit in the first CTAs
-  if ((n_qbar_warps + n_cw - 1) / n_cw > grid)
-    return set_error(WA_ERR_UNSUPPORTED, "page retrieval: too many columns for the grid");
-  e = cudaMemsetAsync(counters, 0, 3 * sizeof(unsigned), st);
-  if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "page retrieval counters: %s", cudaGetErrorString(e));
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(threads);
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeCooperative;
-  attr[0].val.cooperative = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (dt == WA_BF16) e = cudaLaunchKernelEx(&cfg, k_page_retrieval<__nv_bfloat16>, a, err);
-  else e = cudaLaunchKernelEx(&cfg, k_page_retrieval<float>, a, err);
-  if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "page retrieval launch: %s", cudaGetErrorString(e));
-  return check_launch("page_retrieval");
 }
 
 size_t page_alpha_scratch_doubles(int cols, int n_c) {

@@ -173,9 +173,8 @@ struct PageScoreWs {
   double* qbar;         // [cols]
   double* q_blockmean;  // [n_qb][cols]
   double* k_blocksum;   // [n_c][nbp][cols] by candidate position (nullable: page index)
-  double* kdot;         // page-score dot products per (candidate block, warp)
-  double* scratch;      // page-score kernel scratch (page index path)
-  unsigned* counters;   // completion counters
+  double* scratch;      // column-sum parts and partial dot products of the page scores
+  unsigned* counters;   // completion counters of the page-score kernel
 };
 
 PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, int B, bool k_blocks) {
@@ -186,18 +185,15 @@ PageScoreWs carve_page_score(Carver& c, int Nq, int H, int d, int n_c, int T_p, 
   w.qbar = c.take<double>(cols);
   w.q_blockmean = c.take<double>(static_cast<size_t>(n_qb) * cols);
   w.k_blocksum = k_blocks ? c.take<double>(static_cast<size_t>(n_c) * ceil_div(T_p, B) * cols) : nullptr;
-  // sized for float32 rows, the larger per-row warp count of the two dtypes
-  w.kdot = k_blocks ? c.take<double>(page_retrieval_kdot_doubles(cols, n_c, T_p, B, WA_F32)) : nullptr;
-  w.scratch = k_blocks ? nullptr : c.take<double>(page_alpha_scratch_doubles(cols, n_c));
-  w.counters = c.take<unsigned>(page_alpha_counters(cols) > 3 ? page_alpha_counters(cols) : 3);
+  w.scratch = c.take<double>(page_alpha_scratch_doubles(cols, n_c));
+  w.counters = c.take<unsigned>(page_alpha_counters(cols));
   return w;
 }
 
-// S1: one cooperative launch reads the queries and the candidate pages once, writing
-// their block sums and forming the page scores and the top-K_p pages on the way.  The
-// candidate pages are row *chunk (or row 0) of chunk_pages [n_chunks][n_c].  With a
-// page index only the queries are read, and the scores come from the index's block
-// sums of the candidates.
+// One pass over the queries and the candidate pages (block sums, float64), then the
+// page scores and the top-K_p pages from those sums.  The candidate pages are row
+// *chunk (or row 0) of chunk_pages [n_chunks][n_c].  With a page index the pass reads
+// only the queries and the scores read the index's block sums of the candidates.
 wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int d,
                          const void* k_pool, int n_pool_pages, int T_p, const int32_t* chunk_pages,
                          const int32_t* chunk, int n_chunks, int n_c, int K_p, int B, wa_dtype dt,
@@ -207,16 +203,20 @@ wa_status run_page_score(const PageScoreWs& w, const void* q, int Nq, int H, int
   uint32_t* err = errw();
   if (!err) return set_error(WA_ERR_CUDA, "no device error word (is a CUDA device present?)");
   const int n_qb = ceil_div(Nq, B), nbp = ceil_div(T_p, B);
-  if (!page_index)
-    return launch_page_retrieval(dt, q, Nq, H, d, k_pool, n_pool_pages, T_p, chunk_pages, chunk, n_chunks,
-                                 n_c, K_p, B, w.q_blocksum, w.k_blocksum, w.qbar, w.q_blockmean, w.kdot,
-                                 w.counters, alpha, sel, sel_pos, err, st);
-  BlockSumSeg gq;
-  gq.x = q; gq.rows = Nq; gq.n_blocks = n_qb; gq.sums = w.q_blocksum; gq.nb_out = n_qb;
-  WA_TRY(launch_block_sums(dt, cols, B, &gq, 1, w.counters, page_alpha_counters(cols), err, st));
-  return launch_page_alpha(w.q_blocksum, n_qb, Nq, B, cols, page_index, chunk_pages, n_pool_pages, nbp,
-                           chunk_pages, chunk, n_chunks, n_c, T_p, H, d, K_p, w.qbar, w.q_blockmean,
-                           w.scratch, w.counters, alpha, sel, sel_pos, err, st);
+  BlockSumSeg seg[2];
+  seg[0].x = q; seg[0].rows = Nq; seg[0].n_blocks = n_qb; seg[0].sums = w.q_blocksum; seg[0].nb_out = n_qb;
+  int n_segs = 1;
+  if (!page_index) {
+    BlockSumSeg& g = seg[1];
+    g.x = k_pool; g.ids = chunk_pages; g.chunk = chunk; g.id_rows = n_chunks; g.n_src = n_c;
+    g.n_pages = n_pool_pages; g.rows = T_p; g.n_blocks = nbp; g.sums = w.k_blocksum; g.nb_out = nbp;
+    n_segs = 2;
+  }
+  WA_TRY(launch_block_sums(dt, cols, B, seg, n_segs, w.counters, page_alpha_counters(cols), err, st));
+  return launch_page_alpha(w.q_blocksum, n_qb, Nq, B, cols, page_index ? page_index : w.k_blocksum,
+                           page_index ? chunk_pages : nullptr, n_pool_pages, nbp, chunk_pages, chunk,
+                           n_chunks, n_c, T_p, H, d, K_p, w.qbar, w.q_blockmean, w.scratch, w.counters,
+                           alpha, sel, sel_pos, err, st);
 }
 
 // Block sums of one contiguous buffer of `rows` rows (all its blocks).

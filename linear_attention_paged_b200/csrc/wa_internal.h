@@ -66,18 +66,6 @@ struct BlockSumSeg {
 };
 wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* segs, int n_segs,
                             unsigned* counter, int n_counters, uint32_t* err, cudaStream_t st);
-// S1 in one cooperative launch: block sums of the queries (qsum) and of the candidate
-// pages (ksum, by position), Qbar and the query block means, the page scores formed
-// on the fly (kdot: page_retrieval_kdot_doubles) and the top-K_p pages (sel: pool ids
-// of row *chunk of ids, sel_pos: positions), ascending.  counters: 3 words (zeroed
-// by the launch).
-size_t page_retrieval_kdot_doubles(int cols, int n_c, int T_p, int B, wa_dtype dt);
-wa_status launch_page_retrieval(wa_dtype dt, const void* q, int Nq, int H, int d, const void* k_pool,
-                                int n_pages, int T_p, const int32_t* ids, const int32_t* chunk,
-                                int n_chunks, int n_c, int K_p, int B, double* qsum, double* ksum,
-                                double* qbar, double* qmean, double* kdot, unsigned* counters,
-                                double* alpha, int32_t* sel, int32_t* sel_pos, uint32_t* err,
-                                cudaStream_t st);
 // Page scores from block sums: Qbar = sum of qsum rows / Nq (written to qbar, and the
 // query block means to qmean when non-null), column sums of each candidate page's
 // block sums (ksum rows of page kpage[row][j], or of position j when kpage is null),
