@@ -14,6 +14,8 @@ Each function follows one step of the method as the WorldAttention pages state i
      select_pages          and the top-K_p choice of pages
   S2 gather_pages       -- §3.2 "Active KV construction"; summary step (4): the chosen
                            pages joined into K_active, V_active
+  key_block_bounds      -- §3.3 "Inter- and intra-chunk sparse granularity" (history blocks
+                           of B_inter tokens, the current chunk's blocks of B_intra)
   S3 block_select       -- §3.3 "Head-level sparsity adaptation" (minimal block set whose
                            cumulative mass reaches tau_h); summary step (5), coarse
                            selection over pooled blocks
@@ -38,6 +40,11 @@ Readings where the pages are silent (each one is listed in the design notes):
   * E_K, E_V are shared by all heads, shape [L][r]; no extra scaling.
   * Keys of both branches are the retrieved history; with k_cur/v_cur the sparse
     branch also takes the current chunk's own keys (after the history); no causal mask.
+  * Key block sizes (§3.3 "Inter- and intra-chunk sparse granularity"): the history
+    is cut into blocks of B_inter tokens (128 in the pages, B by default) that tile the
+    concatenated history K_active, so a block may span two adjacent pages; the current
+    chunk's own keys and the queries use blocks of B (B_intra = 64).  One softmax runs
+    over all key blocks of a row, whatever their size.
   * O = sigmoid(g) * O_sp + (1 - sigmoid(g)) * O_lin, per token and head (or two gates).
   * Cube order (its formula is lost): cubes in raster order of their corners, tokens
     in raster order inside a cube, the last cube along a side cut short when the side
@@ -151,16 +158,41 @@ def gather_pages(pool, page_ids: Iterable[int]):
 
 
 # ----------------------------------------------------------------------------- S3
+def block_bounds(n: int, B: int, start: int = 0) -> list:
+    """[start + b*B, start + min(n, (b+1)*B)) for the ceil(n/B) blocks of n tokens."""
+    return [(start + b, start + min(n, b + B)) for b in range(0, n, B)]
+
+
+def key_block_bounds(L_hist: int, B_inter: int, L_cur: int = 0, B_intra: Optional[int] = None) -> list:
+    """Key blocks of the sparse branch (§3.3 "Inter- and intra-chunk sparse
+    granularity"): the retrieved history's L_hist tokens in blocks of B_inter, then
+    the current chunk's own L_cur tokens in blocks of B_intra."""
+    return block_bounds(L_hist, B_inter) + block_bounds(L_cur, B_intra or B_inter, start=L_hist)
+
+
+def block_means_at(x, bounds) -> np.ndarray:
+    """Mean over the rows of each block [s, e) of ``bounds``.  x: [N][H][d] -> [n][H][d]."""
+    X = f64(x)
+    out = np.empty((len(bounds),) + X.shape[1:], dtype=np.float64)
+    for b, (s0, e0) in enumerate(bounds):
+        out[b] = X[s0:e0].mean(axis=0)
+    return out
+
+
 def block_means(x, B: int) -> np.ndarray:
     """Mean over the valid rows of each block of B consecutive tokens.
     x: [N][H][d] -> [ceil(N/B)][H][d]; the last block may hold fewer than B rows."""
-    X = f64(x)
-    N = X.shape[0]
-    nb = (N + B - 1) // B
-    out = np.empty((nb,) + X.shape[1:], dtype=np.float64)
-    for b in range(nb):
-        out[b] = X[b * B:min(N, (b + 1) * B)].mean(axis=0)
-    return out
+    return block_means_at(x, block_bounds(f64(x).shape[0], B))
+
+
+def expand_blocks(kept_row, bounds, B: int) -> list:
+    """The B-token blocks (of the key sequence) that the kept blocks of ``bounds`` cover,
+    ascending: the same key set at the granularity of B."""
+    out = set()
+    for j in kept_row:
+        s0, e0 = bounds[j]
+        out.update(range(s0 // B, (e0 - 1) // B + 1))
+    return sorted(out)
 
 
 def softmax(s: np.ndarray) -> np.ndarray:
@@ -199,20 +231,21 @@ def select_row(scores: np.ndarray, tau: float) -> tuple:
     return kept, margin
 
 
-def block_scores(q, k_act, B: int) -> np.ndarray:
-    """Pooled block scores s[h][i][j] = qbar_{h,i} . kbar_{h,j} / sqrt(d)."""
+def block_scores(q, k_act, B: int, key_bounds=None) -> np.ndarray:
+    """Pooled block scores s[h][i][j] = qbar_{h,i} . kbar_{h,j} / sqrt(d); query blocks
+    of B, key blocks of B or ``key_bounds``."""
     qb = block_means(q, B)                 # [n_qb][H][d]
-    kb = block_means(k_act, B)             # [n_kb][H][d]
+    kb = block_means(k_act, B) if key_bounds is None else block_means_at(k_act, key_bounds)
     d = qb.shape[2]
     # per head: [n_qb][d] @ [d][n_kb]
     return np.stack([qb[:, h, :] @ kb[:, h, :].T for h in range(qb.shape[1])]) / math.sqrt(d)
 
 
-def block_select(q, k_act, tau, B: int, scores: Optional[np.ndarray] = None):
+def block_select(q, k_act, tau, B: int, scores: Optional[np.ndarray] = None, key_bounds=None):
     """Per (head, query block): the kept key blocks (ascending) and the margin.
 
     Returns (kept[h][i] -> list, margin[h][i] -> float)."""
-    s = block_scores(q, k_act, B) if scores is None else scores
+    s = block_scores(q, k_act, B, key_bounds) if scores is None else scores
     H, n_qb, _ = s.shape
     tau = f64(tau)
     kept = [[None] * n_qb for _ in range(H)]
@@ -258,7 +291,8 @@ def linear_attention(q, k_til, v_til, rows: Optional[np.ndarray] = None) -> np.n
 
 
 # ----------------------------------------------------------------------------- S5
-def sparse_attention_block(q, k_act, v_act, h: int, i: int, kept_blocks, B: int) -> np.ndarray:
+def sparse_attention_block(q, k_act, v_act, h: int, i: int, kept_blocks, B: int,
+                           key_bounds=None) -> np.ndarray:
     """Exact attention of the rows of query block i, head h, over the keys of the kept
     key blocks only (§3.3 sparse branch; A.1.3: a block is computed whole or skipped).
     Two passes: scores, then softmax-weighted values.  -> [rows][d]."""
@@ -266,7 +300,8 @@ def sparse_attention_block(q, k_act, v_act, h: int, i: int, kept_blocks, B: int)
     Nq = Q.shape[0]
     L = k_act.shape[0]
     r0, r1 = i * B, min(Nq, (i + 1) * B)
-    keys = np.concatenate([np.arange(j * B, min(L, (j + 1) * B)) for j in kept_blocks])
+    kb = block_bounds(L, B) if key_bounds is None else key_bounds
+    keys = np.concatenate([np.arange(kb[j][0], kb[j][1]) for j in kept_blocks])
     Kh = f64(k_act[keys, h, :] if not hasattr(k_act, "detach") else k_act[keys, h, :])
     Vh = f64(v_act[keys, h, :] if not hasattr(v_act, "detach") else v_act[keys, h, :])
     d = Q.shape[2]
@@ -277,7 +312,7 @@ def sparse_attention_block(q, k_act, v_act, h: int, i: int, kept_blocks, B: int)
     return w @ Vh
 
 
-def sparse_attention(q, k_act, v_act, kept, B: int) -> np.ndarray:
+def sparse_attention(q, k_act, v_act, kept, B: int, key_bounds=None) -> np.ndarray:
     """O_sp for every (query block, head): [Nq][H][d]."""
     Q = f64(q)
     Nq, H, d = Q.shape
@@ -285,7 +320,7 @@ def sparse_attention(q, k_act, v_act, kept, B: int) -> np.ndarray:
     for h in range(H):
         for i in range(len(kept[h])):
             out[i * B:min(Nq, (i + 1) * B), h, :] = sparse_attention_block(
-                Q, k_act, v_act, h, i, kept[h][i], B)
+                Q, k_act, v_act, h, i, kept[h][i], B, key_bounds)
     return out
 
 
@@ -307,8 +342,13 @@ def gate_fuse2(o_sp, o_lin, g_sp, g_lin) -> np.ndarray:
 
 
 # ----------------------------------------------------------------------------- step
-def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tuple]] = None) -> dict:
+def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tuple]] = None,
+             B_inter: Optional[int] = None) -> dict:
     """The whole decode step S0..S6 on one input dict (see the workload module).
+
+    ``B_inter`` (default B) is the block size of the retrieved history in the sparse
+    branch (main text §3.3, "Inter- and intra-chunk sparse granularity": 128 for the
+    history pages, B = 64 for the current chunk); queries always use blocks of B.
 
     With ``rows_of_blocks`` = [(h, i), ...] only those (head, query block) outputs are
     computed (the selection is still computed for every row); otherwise all of O.
@@ -338,11 +378,15 @@ def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tupl
     v_act = gather_pages(v_pool, sel)
     res["k_act"], res["v_act"] = k_act, v_act
     k_sp, v_sp = k_act, v_act
+    L_hist = k_act.shape[0]
+    L_cur = 0
     if inp.get("k_cur") is not None:
         k_sp = np.concatenate([f64(k_act), f64(inp["k_cur"])], axis=0)
         v_sp = np.concatenate([f64(v_act), f64(inp["v_cur"])], axis=0)
-    kept, margin = block_select(inp["q"], k_sp, inp["tau"], B)
-    res["kept"], res["block_margin"] = kept, margin
+        L_cur = k_sp.shape[0] - L_hist
+    kbounds = key_block_bounds(L_hist, B_inter or B, L_cur, B)
+    kept, margin = block_select(inp["q"], k_sp, inp["tau"], B, key_bounds=kbounds)
+    res["kept"], res["block_margin"], res["key_bounds"] = kept, margin, kbounds
     kt, vt = linear_project(k_act, v_act, inp["e_k"], inp["e_v"])
     res["k_til"], res["v_til"] = kt, vt
     Q = f64(inp["q"])
@@ -350,7 +394,7 @@ def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tupl
     g = f64(inp["gate"])
     g_lin = f64(inp["gate_lin"]) if inp.get("gate_lin") is not None else None
     if rows_of_blocks is None:
-        o_sp = sparse_attention(Q, k_sp, v_sp, kept, B)
+        o_sp = sparse_attention(Q, k_sp, v_sp, kept, B, kbounds)
         o_lin = linear_attention(Q, kt, vt)
         res["o_sp"], res["o_lin"] = o_sp, o_lin
         res["o"] = gate_fuse(o_sp, o_lin, g) if g_lin is None else gate_fuse2(o_sp, o_lin, g, g_lin)
@@ -358,7 +402,7 @@ def hsa_step(inp: dict, B: int, K_p: int, rows_of_blocks: Optional[Sequence[tupl
         outs = {}
         for (h, i) in rows_of_blocks:
             r0, r1 = i * B, min(Nq, (i + 1) * B)
-            osp = sparse_attention_block(Q, k_sp, v_sp, h, i, kept[h][i], B)
+            osp = sparse_attention_block(Q, k_sp, v_sp, h, i, kept[h][i], B, kbounds)
             olin = linear_attention(Q[r0:r1, h:h + 1, :], kt[:, h:h + 1, :], vt[:, h:h + 1, :])[:, 0, :]
             G = sigmoid(g[r0:r1, h])[:, None]
             Gl = (1.0 - G) if g_lin is None else sigmoid(g_lin[r0:r1, h])[:, None]

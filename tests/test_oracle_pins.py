@@ -455,3 +455,86 @@ def test_cube_order_groups_are_cubes(grid, cube):
                             for w in range(w0, w0 + cw)}
         corners.append((t0, h0, w0))
     assert corners == sorted(corners)              # cubes in raster order of their corners
+
+
+# --------------------------------------------- mixed key-block granularity (§3.3)
+def test_key_block_bounds_hand_example_and_page_shape():
+    # 10 history tokens in blocks of 4, then 5 chunk tokens in blocks of 2
+    assert O.key_block_bounds(10, 4, 5, 2) == [(0, 4), (4, 8), (8, 10), (10, 12), (12, 14), (14, 15)]
+    assert O.key_block_bounds(8, 4) == [(0, 4), (4, 8)]
+    # the one-layer shape: 4 pages of 12,480 tokens in 128-token blocks = 390 blocks (no
+    # ragged block); block 97 spans pages 0 and 1; then 4680 chunk tokens in 74 blocks of 64
+    kb = O.key_block_bounds(4 * 12480, 128, 4680, 64)
+    assert len(kb) == 390 + 74
+    assert kb[97] == (12416, 12544) and kb[97][0] < 12480 < kb[97][1]
+    assert kb[389] == (49792, 49920) and kb[390] == (49920, 49984)
+    assert kb[-1] == (49920 + 4672, 49920 + 4680)
+    # expansion to 64-token blocks: a 128-block covers two, a chunk block one
+    assert O.expand_blocks([97, 390], kb, 64) == [194, 195, 780]
+    assert O.expand_blocks([2], O.key_block_bounds(10, 4), 2) == [4]
+
+
+def test_mixed_block_means_closed_form():
+    # x[n] = n in every entry: the mean of rows [s, e) is (s + e - 1) / 2
+    n = 200
+    x = np.arange(n, dtype=np.float64).reshape(n, 1, 1) * np.ones((1, 2, 3))
+    kb = O.key_block_bounds(150, 128, 50, 64)   # blocks (0,128), (128,150), (150,200)
+    m = O.block_means_at(x, kb)
+    np.testing.assert_array_equal(m[:, 1, 2], [63.5, 138.5, 174.5])
+    # a block spanning two 64-token halves has the mean of the two halves' means
+    m64 = O.block_means(x[:128], 64)
+    np.testing.assert_array_equal(m[0], 0.5 * (m64[0] + m64[1]))
+
+
+def test_mixed_granularity_tau_one_is_dense_attention():
+    """With tau = 1 every block is kept whatever its size: the sparse branch is textbook
+    attention over the history followed by the chunk's own keys."""
+    cfg = W.C0.with_(T_p=192, Nq=72, intra=True, tau_const=1.0)
+    inp = W.make_inputs(cfg)
+    res = O.hsa_step(inp, cfg.B, cfg.K_p, B_inter=128)
+    kb = res["key_bounds"]
+    assert len(kb) == (cfg.L // 128) + 2 and all(e - s == 128 for s, e in kb[:cfg.L // 128])
+    k_all = np.concatenate([O.f64(res["k_act"]), O.f64(inp["k_cur"])])
+    v_all = np.concatenate([O.f64(res["v_act"]), O.f64(inp["v_cur"])])
+    q = O.f64(inp["q"])[:, 0, :]
+    np.testing.assert_allclose(res["o_sp"][:, 0, :], sdpa(q, k_all[:, 0, :], v_all[:, 0, :]),
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_mixed_granularity_selection_brute_force():
+    """Per row: scores of mixed-size blocks from pairwise dot products (mean over the
+    query block's rows and the key block's rows), then the kept set is the smallest set
+    of blocks whose softmax mass reaches tau, the largest mass among those."""
+    r = rng(31)
+    H, d, B = 2, 4, 4
+    for trial in range(12):
+        L_hist, L_cur, Nq = int(r.integers(9, 24)), int(r.integers(1, 9)), int(r.integers(3, 10))
+        q = r.normal(size=(Nq, H, d))
+        k = r.normal(size=(L_hist + L_cur, H, d)) * r.uniform(0.3, 3)
+        kb = O.key_block_bounds(L_hist, 8, L_cur, B)
+        if len(kb) > 10:
+            continue
+        tau = np.full(H, r.uniform(0.2, 0.95))
+        kept, margin = O.block_select(q, k, tau, B, key_bounds=kb)
+        for h in range(H):
+            for i in range(-(-Nq // B)):
+                rows = range(i * B, min(Nq, (i + 1) * B))
+                s = np.array([sum(float(q[a, h] @ k[b, h]) for a in rows for b in range(s0, e0))
+                              / (len(rows) * (e0 - s0) * math.sqrt(d)) for (s0, e0) in kb])
+                p = np.exp(s - s.max()); p /= p.sum()
+                feasible = [c for m in range(1, len(kb) + 1) for c in itertools.combinations(range(len(kb)), m)
+                            if p[list(c)].sum() >= tau[h]]
+                best = min(len(c) for c in feasible)
+                best_mass = max(p[list(c)].sum() for c in feasible if len(c) == best)
+                if margin[h, i] > 1e-9:
+                    assert len(kept[h][i]) == best
+                    assert p[kept[h][i]].sum() == pytest.approx(best_mass, abs=1e-12)
+
+
+def test_mixed_granularity_equal_sizes_is_uniform():
+    cfg = _intra_cfg(tau_const=0.7)
+    inp = W.make_inputs(cfg)
+    a = O.hsa_step(inp, cfg.B, cfg.K_p)
+    b = O.hsa_step(inp, cfg.B, cfg.K_p, B_inter=cfg.B)
+    assert a["kept"] == b["kept"]
+    np.testing.assert_array_equal(a["o"], b["o"])
