@@ -70,9 +70,11 @@ def load_peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
 
 
-def workload_desc(cfg):
+def workload_desc(cfg, b_inter=0):
     intra = (f"; sparse branch also over the chunk's own {cfg.Nq} keys (intra-chunk keys)"
              if cfg.intra else "")
+    if b_inter and b_inter != cfg.B:
+        intra += f"; history selected in blocks of {b_inter} tokens (inter-chunk granularity)"
     return (f"{cfg.name}: one HSA decode step (chunk-layer), H={cfg.H}, d={cfg.d}, T_p={cfg.T_p} "
             f"(8 frames x 1560 tokens), n_c={cfg.n_c} candidate pages, Nq={cfg.Nq}, K_p={cfg.K_p} "
             f"-> L={cfg.L}, B={cfg.B}, r={cfg.r}, tau_h=0.80+0.15h/11, bf16{intra}")
@@ -261,6 +263,8 @@ def run_ours(args, rank, world, local_rank):
     base = W.C1 if args.heads is None else W.C1.with_(name=f"c1_layer_bf16_h{args.heads}", H=args.heads)
     if args.intra:
         base = base.with_(name=base.name + "_intra", intra=True)
+    if args.b_inter:
+        base = base.with_(name=base.name + f"_inter{args.b_inter}")
     cfg = base.with_(seed=replicas.rank_seed(base.seed, rank))   # each rank: its own layer
     inp = W.make_inputs(cfg, device="cuda", gen_device="cuda")
     tau = inp["tau"].cuda()
@@ -268,18 +272,18 @@ def run_ours(args, rank, world, local_rank):
 
     step = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"], inp["e_v"],
                       tau, inp["gate"], cfg.K_p, cfg.B, fused_gather=True, keep_intermediates=True,
-                      k_cur=inp.get("k_cur"), v_cur=inp.get("v_cur"))
+                      k_cur=inp.get("k_cur"), v_cur=inp.get("v_cur"), B_inter=args.b_inter)
     step()
     torch.cuda.synchronize()
     flags = wa.wa_device_error()
     if flags:
         raise RuntimeError(f"device error flags 0x{flags:x}")
     flops, kept_frac = selected_flops(step.inter["blk_mask"], cfg)
-    # per step: pick_chunk, candidate-page row sums, page-score dots, alpha/top-k, block
-    # scores, block choice, pairing, work items, sparse attention, combine on the
-    # caller's stream; query row sums and means, then projection, split reduction and
-    # linear branch on the side stream
-    launches_per_step = 15 + (1 if cfg.intra else 0)   # + block sums of the chunk's keys
+    # per step: the block-sum pass over the queries and candidate pages, page scores
+    # and top-k, block scores, block choice, pairing, work items, sparse attention and
+    # combine on the caller's stream; projection, split reduction and linear branch on
+    # the side stream
+    launches_per_step = 11 + (1 if cfg.intra else 0)   # + block sums of the chunk's keys
 
     n_ev = 8  # WA_STEP_EVENTS
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
@@ -405,7 +409,7 @@ def run_ours(args, rank, world, local_rank):
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
             "ms_per_chunk_layer": ms_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": workload_desc(cfg),
+            "config": {"workload": workload_desc(cfg, args.b_inter),
                        "l2": "no flush: each step reads >600 MB (candidate keys + selected K/V), "
                              "larger than the 126 MB L2",
                        "parallelism": f"replicas x{world} (one layer per rank, no collective)"},
@@ -569,6 +573,9 @@ def main():
     ap.add_argument("--config", choices=["c1", "c4"], default="c1",
                     help="c1: one-layer step (default); c4: the full denoise stack")
     ap.add_argument("--layers", type=int, default=30, help="c4: layers")
+    ap.add_argument("--b-inter", type=int, default=0, choices=[0, 64, 128],
+                    help="c1: block size of the history in block selection (128: inter-chunk "
+                         "granularity; the chunk's own keys keep 64)")
     ap.add_argument("--intra", action="store_true",
                     help="c1: add the chunk's own keys to the sparse branch (intra-chunk keys)")
     ap.add_argument("--chunks", type=int, default=20, help="c4: chunks")

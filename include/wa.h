@@ -367,6 +367,16 @@ typedef struct wa_step_args {
      linear branch stays over the history.  Needs K_p*T_p % B == 0. */
   const void* k_cur;
   const void* v_cur;
+  /* optional inter-chunk granularity (main text §3.3, "Inter- and intra-chunk sparse
+     granularity": blocks of 128 tokens for the retrieved history pages, 64 for the
+     current chunk): the block size of the history in block selection, 0 or B (the
+     default: B everywhere) or 2*B.  With 2*B the history's selection blocks are
+     consecutive 2B-token windows of the concatenated history (K_active; a block may
+     span two adjacent pages), the chunk's own keys and the queries keep blocks of B,
+     and one softmax runs over all key blocks of a row.  blk_mask_out stays at B-token
+     granularity (a kept history block sets its two B-token blocks).  2*B needs
+     K_p*T_p % B == 0. */
+  int B_inter;
 } wa_step_args;
 
 /* Stage boundaries recorded into wa_step_args.stage_events:

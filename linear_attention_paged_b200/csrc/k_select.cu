@@ -122,18 +122,24 @@ k_block_scores(const double* __restrict__ qmean, KeyMeans km, int n_qb, int n_kb
   for (int rr = warp; rr < 32; rr += blockDim.x >> 5) {
     const int j = j0 + rr, i = i0 + rr;
     const double* ksrc = nullptr;
+    const double* ksrc2 = nullptr;   // second B-row half of a 2B-row history block
+    auto sub_row = [&](int jj) -> size_t {
+      if (km.page_pos) return static_cast<size_t>(km.page_pos[jj / km.nbp]) * km.nbp + jj % km.nbp;
+      return static_cast<size_t>(jj);
+    };
     if (j < n_kb) {
       if (km.data2 && j >= km.n_kb1) {
         ksrc = km.data2 + static_cast<size_t>(j - km.n_kb1) * cols + h * d;
+      } else if (km.pair) {
+        ksrc = km.data + sub_row(2 * j) * cols + h * d;
+        if (2 * j + 1 < km.n_sub) ksrc2 = km.data + sub_row(2 * j + 1) * cols + h * d;
       } else {
-        size_t row = j;
-        if (km.page_pos) row = static_cast<size_t>(km.page_pos[j / km.nbp]) * km.nbp + j % km.nbp;
-        ksrc = km.data + row * cols + h * d;
+        ksrc = km.data + sub_row(j) * cols + h * d;
       }
     }
     const double* qsrc = i < n_qb ? qmean + static_cast<size_t>(i) * cols + h * d : nullptr;
     for (int c = lane; c < d; c += 32) {
-      kc[rr * (d + 1) + c] = ksrc ? ksrc[c] : 0.0;
+      kc[rr * (d + 1) + c] = ksrc ? (ksrc2 ? ksrc[c] + ksrc2[c] : ksrc[c]) : 0.0;
       qs[rr * d + c] = qsrc ? qsrc[c] : 0.0;
     }
   }
@@ -161,7 +167,8 @@ k_block_scores(const double* __restrict__ qmean, KeyMeans km, int n_qb, int n_kb
       const int jj = j - km.n_kb1;
       den = static_cast<double>(min(km.L2, (jj + 1) * B) - jj * B) * sqrt_d;
     } else if (km.is_sum) {
-      den = static_cast<double>(min(km.L, (j + 1) * B) - j * B) * sqrt_d;
+      const int Bk = km.pair ? 2 * B : B;   // rows of a history block
+      den = static_cast<double>(min(km.L, (j + 1) * Bk) - j * Bk) * sqrt_d;
     }
 #pragma unroll
     for (int u = 0; u < 2; ++u) {
@@ -185,12 +192,14 @@ __device__ __forceinline__ bool before(double ka, int ia, double kb, int ib) {
 __global__ void __launch_bounds__(kChooseThreads)
 k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int lg_np, int W,
                const float* __restrict__ tau, int32_t* __restrict__ blk_idx,
-               int32_t* __restrict__ blk_cnt, uint32_t* __restrict__ blk_mask) {
+               int32_t* __restrict__ blk_cnt, uint32_t* __restrict__ blk_mask, int n_h, int n_sub,
+               int W_mask) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int NP = 1 << lg_np;
   double* key = reinterpret_cast<double*>(smem_raw);          // [NP]
   int* idx = reinterpret_cast<int*>(key + NP);                 // [NP]
-  uint32_t* maskw = reinterpret_cast<uint32_t*>(idx + NP);     // [W]
+  uint32_t* maskw = reinterpret_cast<uint32_t*>(idx + NP);     // [W] (selection blocks)
+  uint32_t* maskx = maskw + W;                                  // [W_mask] (n_h > 0: B-row blocks)
   __shared__ double wred[kChooseThreads / 32];
   __shared__ int ired[kChooseThreads / 32];
   const int h = blockIdx.y, i = blockIdx.x;
@@ -202,6 +211,7 @@ k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int lg_np,
     idx[e] = e < n_kb ? e : INT_MAX;
   }
   for (int w = tid; w < W; w += kChooseThreads) maskw[w] = 0u;
+  for (int w = tid; w < W_mask && n_h > 0; w += kChooseThreads) maskx[w] = 0u;
   __syncthreads();
   for (int k = 2; k <= NP; k <<= 1) {
     for (int js = k >> 1; js > 0; js >>= 1) {
@@ -272,10 +282,23 @@ k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int lg_np,
   for (int t = tid; t < m; t += kChooseThreads) {
     const int j = idx[t];
     atomicOr(&maskw[j >> 5], 1u << (j & 31));
+    if (n_h > 0) {
+      // the same keys at B-row granularity: a 2B-row history block covers B-row blocks
+      // 2j and 2j + 1, a chunk block one
+      if (j < n_h) {
+        atomicOr(&maskx[(2 * j) >> 5], 1u << ((2 * j) & 31));
+        if (2 * j + 1 < n_sub) atomicOr(&maskx[(2 * j + 1) >> 5], 1u << ((2 * j + 1) & 31));
+      } else {
+        const int x = n_sub + (j - n_h);
+        atomicOr(&maskx[x >> 5], 1u << (x & 31));
+      }
+    }
   }
   __syncthreads();
-  if (blk_mask)
-    for (int w = tid; w < W; w += kChooseThreads) blk_mask[rowid * W + w] = maskw[w];
+  if (blk_mask) {
+    const uint32_t* src = n_h > 0 ? maskx : maskw;
+    for (int w = tid; w < W_mask; w += kChooseThreads) blk_mask[rowid * W_mask + w] = src[w];
+  }
   if (blk_cnt && tid == 0) blk_cnt[rowid] = m;
   if (blk_idx && warp == 0) {
     const int wpl = (W + 31) / 32;
@@ -328,11 +351,13 @@ size_t block_scores_bytes(int H, int n_qb, int n_kb) {
 }
 
 wa_status launch_block_select(const double* q_blockmean, int Nq, int H, int d, int B,
-                              KeyMeans km, int n_kb, const float* tau, double* scores,
+                              KeyMeans km, int n_kb, int n_kb_mask, const float* tau, double* scores,
                               int32_t* blk_idx, int32_t* blk_cnt, uint32_t* blk_mask,
                               cudaStream_t st) {
   const int n_qb = (Nq + B - 1) / B;
   const int W = (n_kb + 31) / 32;
+  const int W_mask = (n_kb_mask + 31) / 32;
+  if (km.pair && !km.is_sum) return set_error(WA_ERR_UNSUPPORTED, "2B-row history blocks need block sums");
   const size_t smem_s = (32 * static_cast<size_t>(d + 1) + 32 * static_cast<size_t>(d)) *
                         sizeof(double);
   cudaError_t e = cudaFuncSetAttribute(k_block_scores, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -342,12 +367,13 @@ wa_status launch_block_select(const double* q_blockmean, int Nq, int H, int d, i
       q_blockmean, km, n_qb, n_kb, H, d, B, scores);
   int lg = 5;
   while ((1 << lg) < n_kb) ++lg;
-  const size_t smem_c = (static_cast<size_t>(1) << lg) * 12 + static_cast<size_t>(W) * 4 + 16;
+  const size_t smem_c = (static_cast<size_t>(1) << lg) * 12 + static_cast<size_t>(W + W_mask) * 4 + 16;
   e = cudaFuncSetAttribute(k_block_choose, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem_c));
   if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "block_choose smem attr: %s", cudaGetErrorString(e));
-  k_block_choose<<<dim3(n_qb, H), kChooseThreads, smem_c, st>>>(scores, n_qb, n_kb, lg, W, tau,
-                                                                blk_idx, blk_cnt, blk_mask);
+  k_block_choose<<<dim3(n_qb, H), kChooseThreads, smem_c, st>>>(
+      scores, n_qb, n_kb, lg, W, tau, blk_idx, blk_cnt, blk_mask, km.pair ? km.n_kb1 : 0, km.n_sub,
+      km.pair ? W_mask : W);
   return check_launch("block_select");
 }
 

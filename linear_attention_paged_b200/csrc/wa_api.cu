@@ -473,7 +473,7 @@ wa_status wa_block_select(const void* q, int Nq, int H, int d, const void* k_act
     km.data = k_blockmean;
     km.is_sum = 0;
   }
-  return launch_block_select(w.qmean, Nq, H, d, B, km, n_kb, tau, w.scores, blk_idx, blk_cnt,
+  return launch_block_select(w.qmean, Nq, H, d, B, km, n_kb, n_kb, tau, w.scores, blk_idx, blk_cnt,
                              blk_mask, st);
 }
 
@@ -640,6 +640,10 @@ wa_status validate_step(const wa_step_args* a) {
     return set_error(WA_ERR_UNSUPPORTED, "the page index needs fused_gather and T_p %% B == 0");
   WA_REQUIRE(static_cast<long long>(a->n_pool_pages) * a->T_p < (1LL << 31), "pool too large");
   WA_REQUIRE(!a->k_cur == !a->v_cur, "k_cur and v_cur are given together");
+  WA_REQUIRE(a->B_inter == 0 || a->B_inter == a->B || a->B_inter == 2 * a->B,
+             "B_inter must be 0, B or 2*B (got %d)", a->B_inter);
+  if (a->B_inter == 2 * a->B && L % a->B != 0)
+    return set_error(WA_ERR_UNSUPPORTED, "B_inter = 2*B needs K_p*T_p %% B == 0");
   if (a->k_cur) {
     if (L % a->B != 0)
       return set_error(WA_ERR_UNSUPPORTED, "the chunk's keys need K_p*T_p %% B == 0");
@@ -761,6 +765,16 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
     km.data2 = w.cur_sum; km.n_kb1 = L / a->B; km.L2 = a->Nq;
   }
 
+  // inter-chunk granularity: the history's selection blocks pair up B-row block sums
+  int n_sel = n_kb;   // selection blocks (= mask blocks unless paired)
+  if (a->B_inter == 2 * a->B) {
+    km.pair = 1;
+    km.n_sub = L / a->B;
+    const int n_h = (km.n_sub + 1) / 2;
+    n_sel = n_h + (a->k_cur ? ceil_div(a->Nq, a->B) : 0);
+    km.n_kb1 = n_h;
+  }
+
   mark(2);
   uint32_t* mask = a->blk_mask_out ? a->blk_mask_out : w.mask;
   void* kt = a->k_til_out ? a->k_til_out : w.k_til;
@@ -787,8 +801,8 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
     mark_side(5);
     cudaEventRecord(side->join, side->stream);
     // S3: block selection
-    WA_TRY(launch_block_select(w.ps.q_blockmean, a->Nq, a->H, a->d, a->B, km, n_kb, a->tau, w.scores,
-                               nullptr, nullptr, mask, st));
+    WA_TRY(launch_block_select(w.ps.q_blockmean, a->Nq, a->H, a->d, a->B, km, n_sel, n_kb, a->tau,
+                               w.scores, nullptr, nullptr, mask, st));
     mark(3);
     WA_TRY(launch_attn_worklist(a->Nq, a->H, a->d, a->B, sparse_key_rows(a), mask, w.attn, st));
     cudaStreamWaitEvent(st, side->join, 0);
@@ -797,8 +811,8 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
     WA_TRY(launch_attn_sparse(a->q, a->Nq, a->H, a->d, rs, a->B, mask, a->gate, w.lin, a->out, nullptr,
                               w.attn, err, st));
   } else {
-    WA_TRY(launch_block_select(w.ps.q_blockmean, a->Nq, a->H, a->d, a->B, km, n_kb, a->tau, w.scores,
-                               nullptr, nullptr, mask, st));
+    WA_TRY(launch_block_select(w.ps.q_blockmean, a->Nq, a->H, a->d, a->B, km, n_sel, n_kb, a->tau,
+                               w.scores, nullptr, nullptr, mask, st));
     mark(3);
     WA_TRY(launch_simt_project(static_cast<const float*>(rs.k), rs.page_ids, rs.page_rows,
                                rs.n_pages, static_cast<const float*>(a->e_k), L, cols, a->r,

@@ -102,12 +102,20 @@ struct KeyMeans {
   const double* data2 = nullptr;
   int n_kb1 = 0;
   int L2 = 0;
+  // history blocks of 2B rows (inter-chunk granularity; needs is_sum): block j < n_kb1
+  // is the sum of B-row blocks 2j and 2j + 1 (the latter when < n_sub) of `data`
+  int pair = 0;
+  int n_sub = 0;
 };
 // S3: float64 pooled block scores into `scores` [H][n_qb][n_kb], then per (head,
 // query block) the shortest descending prefix reaching tau_h.
 size_t block_scores_bytes(int H, int n_qb, int n_kb);
+// With km.pair the n_kb selection blocks are mixed (history blocks of 2B rows, then
+// chunk blocks of B); blk_idx / blk_cnt count them, and blk_mask is written at B-row
+// granularity (n_kb_mask blocks: the history's n_sub, then the chunk's) for the
+// attention kernel.  Without it n_kb_mask == n_kb.
 wa_status launch_block_select(const double* q_blockmean, int Nq, int H, int d, int B,
-                              KeyMeans km, int n_kb, const float* tau, double* scores,
+                              KeyMeans km, int n_kb, int n_kb_mask, const float* tau, double* scores,
                               int32_t* blk_idx, int32_t* blk_cnt, uint32_t* blk_mask,
                               cudaStream_t st);
 

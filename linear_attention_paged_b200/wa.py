@@ -54,6 +54,7 @@ class StepArgs(ctypes.Structure):
         ("page_index", P),
         ("gate_lin", P),
         ("k_cur", P), ("v_cur", P),
+        ("B_inter", c_int),
     ]
 
 
@@ -365,7 +366,7 @@ class HSAStep:
     def __init__(self, q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 4,
                  B: int = 64, e_cur=None, e_chunks=None, fused_gather: bool = True,
                  keep_intermediates: bool = False, out=None, page_index=None, gate_lin=None,
-                 k_cur=None, v_cur=None):
+                 k_cur=None, v_cur=None, B_inter: int = 0):
         _need_cuda(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, e_cur, e_chunks, gate_lin,
                    k_cur, v_cur)
         Nq, H, d = q.shape
@@ -394,6 +395,7 @@ class HSAStep:
         a.page_index = _p(page_index)
         a.gate_lin = _p(gate_lin)
         a.k_cur, a.v_cur = _p(k_cur), _p(v_cur)
+        a.B_inter = int(B_inter)
         self._keep += [page_index, gate_lin, k_cur, v_cur]
         self.inter = {}
         if keep_intermediates:
@@ -427,11 +429,11 @@ class HSAStep:
 
 def wa_hsa_step(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p: int = 4, B: int = 64,
                 e_cur=None, e_chunks=None, fused_gather: bool = True, keep_intermediates: bool = False,
-                stream=None, page_index=None, gate_lin=None, k_cur=None, v_cur=None):
+                stream=None, page_index=None, gate_lin=None, k_cur=None, v_cur=None, B_inter: int = 0):
     """One HSA decode step; returns ``out`` (and the intermediates when asked)."""
     st = HSAStep(q, k_pool, v_pool, chunk_pages, e_k, e_v, tau, gate, K_p, B, e_cur, e_chunks,
                  fused_gather, keep_intermediates, page_index=page_index, gate_lin=gate_lin,
-                 k_cur=k_cur, v_cur=v_cur)
+                 k_cur=k_cur, v_cur=v_cur, B_inter=B_inter)
     out = st(stream)
     return (out, st.inter) if keep_intermediates else out
 

@@ -286,25 +286,32 @@ def sparse_blocks(cfg):
     return -(-(cfg.L + (cfg.Nq if cfg.intra else 0)) // cfg.B)
 
 
-def _full_size_step(wa, cfg, samples, gen_device="cuda"):
+def expanded_kept(res, B):
+    """The oracle's kept blocks at B-token granularity (what the step's mask holds)."""
+    kb = res["key_bounds"]
+    return [[O.expand_blocks(row, kb, B) for row in kh] for kh in res["kept"]]
+
+
+def _full_size_step(wa, cfg, samples, gen_device="cuda", B_inter=0):
     inp = W.make_inputs(cfg, device="cuda", gen_device=gen_device)
     e_cur = inp.get("e_cur")
     step = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"], inp["e_v"],
                       inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B, e_cur=e_cur,
                       e_chunks=inp.get("e_chunks"), fused_gather=True, keep_intermediates=True,
-                      k_cur=inp.get("k_cur"), v_cur=inp.get("v_cur"))
+                      k_cur=inp.get("k_cur"), v_cur=inp.get("v_cur"), B_inter=B_inter)
     out = step()
     torch.cuda.synchronize()
-    res = O.hsa_step(inp, cfg.B, cfg.K_p, rows_of_blocks=samples)
+    res = O.hsa_step(inp, cfg.B, cfg.K_p, rows_of_blocks=samples, B_inter=B_inter or None)
     if "chunk" in res:
         assert int(step.inter["chunk"].item()) == res["chunk"]
     np.testing.assert_allclose(to64(step.inter["alpha"]), res["alpha"], rtol=1e-9, atol=1e-13)
     if res["page_margin"] >= MARGIN_F64:
         assert step.inter["sel"].cpu().tolist() == res["sel"]
     n_kb = sparse_blocks(cfg)
-    compare_selection(mask_to_sets(step.inter["blk_mask"], n_kb), res["kept"], res["block_margin"],
-                      f"{cfg.name} masks")
-    print(f"[info] {cfg.name} kept fraction per head: {np.round(kept_fraction(res['kept'], n_kb), 3)}")
+    compare_selection(mask_to_sets(step.inter["blk_mask"], n_kb), expanded_kept(res, cfg.B),
+                      res["block_margin"], f"{cfg.name} masks")
+    print(f"[info] {cfg.name} kept fraction per head: "
+          f"{np.round(kept_fraction(res['kept'], len(res['key_bounds'])), 3)}")
     assert_close(step.inter["k_til"], res["k_til"], "bf16", f"{cfg.name} K~")
     assert_close(step.inter["v_til"], res["v_til"], "bf16", f"{cfg.name} V~")
     for (h, i), blk in res["blocks"].items():
@@ -355,6 +362,40 @@ def test_full_size_narrow_projection_step(wa):
     cfg = W.C1.with_(name="c1_narrow_proj", H=3, d=64, r=128, seed=43)
     samples = [(0, 0), (2, cfg.n_qb - 1), (1, 36)]
     _full_size_step(wa, cfg, samples)
+
+
+def test_full_size_layer_step_inter_intra_granularity(wa):
+    """C1 with the chunk's own keys, history blocks of 128 tokens (390 of them, some
+    spanning two pages) and chunk blocks of 64 (74, the last one 8 rows)."""
+    cfg = W.C1.with_(name="c1_inter128", intra=True)
+    samples = [(0, 0), (11, cfg.n_qb - 1), (6, 33)]
+    _full_size_step(wa, cfg, samples, B_inter=128)
+
+
+MIXED_SMALL = [SMALL_BF16.with_(name="mixed_bf16"),
+               W.HSAConfig("mixed_f32_odd", H=2, d=64, T_p=192, n_c=4, Nq=150, K_p=3, B=64, r=48,
+                           dtype="f32", seed=15, recipe="offset"),
+               SMALL_BF16_D64.with_(name="mixed_bf16_d64_odd", T_p=576, K_p=3)]
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "gathered"])
+@pytest.mark.parametrize("intra", [True, False], ids=["intra", "history"])
+@pytest.mark.parametrize("cfg", MIXED_SMALL, ids=lambda c: c.name)
+def test_hsa_step_inter_granularity_small(wa, cfg, intra, fused):
+    """History blocks of 2B = 128 tokens (an odd number of 64-token blocks leaves a
+    64-token last history block), with or without the chunk's own keys in blocks of 64."""
+    cfg = cfg.with_(intra=intra)
+    inp = inputs(cfg)
+    out, inter = wa.wa_hsa_step(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"],
+                                inp["e_v"], inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B,
+                                fused_gather=fused, keep_intermediates=True, k_cur=inp.get("k_cur"),
+                                v_cur=inp.get("v_cur"), B_inter=128)
+    res = O.hsa_step(inp, cfg.B, cfg.K_p, B_inter=128)
+    n_kb = sparse_blocks(cfg)
+    compare_selection(mask_to_sets(inter["blk_mask"], n_kb), expanded_kept(res, cfg.B),
+                      res["block_margin"], f"{cfg.name} masks (B_inter 128)")
+    assert_close(out, res["o"], dkey(cfg), f"{cfg.name} step O (B_inter 128, {'intra' if intra else 'history'})")
+    check_device_ok(wa)
 
 
 def test_full_size_stress_step(wa):
