@@ -395,6 +395,12 @@ def run_ours(args, rank, world, local_rank):
         del kc
     del ka, va
 
+    # the full denoise stack (spec config 5) on the same GPU, after the one-layer
+    # figures: every rank runs its own stack
+    c4 = None
+    if not args.no_c4 and args.heads is None and not args.intra and not args.b_inter:
+        c4 = c4_measure(args, rank, world, local_rank)
+
     line = None
     if rank == 0:
         cpu = None
@@ -443,6 +449,10 @@ def run_ours(args, rank, world, local_rank):
                             "on their own streams overlapping the previous/next step"}
                     if e2e_steps else None),
             "cpu_baseline": cpu,
+            "c4_denoise_stack": ({"value": c4["frames_per_s"], "unit": "frames/s", "ms_total": c4["ms_total"],
+                                  "ms_per_step": c4["ms_per_step"], "steps": c4["steps"],
+                                  "workload": c4["workload"], "clocks": c4["clocks"],
+                                  "gpu_launches": c4["gpu_launches"]} if c4 else None),
             "clocks": clocks,
             "gpu_launches": launches_per_step * args.steps,
             "context": {"pages_end_to_end_fps_h100": 22.0, "pages_e2e_speedup_h100": 2.21,
@@ -454,7 +464,7 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
-def run_c4(args, rank, world, local_rank):
+def c4_measure(args, rank, world, local_rank):
     """Full denoise stack: `layers` layers x 4 denoising steps per chunk x `chunks`
     chunks of 3 frames.  Each layer owns a 16-page pool (8 history pages = the
     candidate chunk, 8 pages of room for appended chunks), its E_K/E_V and tau, and
@@ -462,11 +472,7 @@ def run_c4(args, rank, world, local_rank):
     gates cycle through a resident set of pre-drawn tensors), then every layer's
     new 4680-token KV is appended to its pool with the index refreshed.  The index
     of the history pages is built before timing (it belongs to the cache state);
-    appends and all steps are timed."""
-    from linear_attention_paged_b200 import build as wb
-    if rank == 0:
-        wb.build()
-    replicas.barrier(world)
+    appends and all steps are timed.  Returns the figures of rank 0 (None elsewhere)."""
     from linear_attention_paged_b200 import wa, workloads as W
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
@@ -533,22 +539,41 @@ def run_c4(args, rank, world, local_rank):
     clocks = clk.stop()
     total_ms = replicas.max_over_ranks(e0.elapsed_time(e1), world, dev)
     frames = world * FRAMES_PER_CHUNK * n_chunks
+    del layers, qs, gs
+    torch.cuda.empty_cache()
+    if rank != 0:
+        return None
+    n_step_calls = n_chunks * n_steps * n_layers
+    # per step: block sums of the queries and the page scores from the index, block
+    # scores and choice, pairing and work items, sparse attention and combine; on the
+    # side stream projection, split reduction and linear branch; per append: two
+    # copies and the index refresh
+    return {"frames_per_s": frames / (total_ms / 1000.0), "ms_total": total_ms,
+            "ms_per_step": total_ms / n_step_calls, "steps": n_step_calls,
+            "workload": f"c4 full denoise stack: {n_layers} layers x {n_steps} denoising steps "
+                        f"x {n_chunks} chunks of 3 frames, one-layer shapes as C1, pool of "
+                        f"16 pages per layer with a float64 page index; each chunk's KV "
+                        f"appended to every layer's pool (index refreshed) inside the "
+                        f"timed region; queries/gates cycle through {n_rot} resident draws",
+            "clocks": clocks, "gpu_launches": n_step_calls * 11 + n_chunks * n_layers * 3}
+
+
+def run_c4(args, rank, world, local_rank):
+    from linear_attention_paged_b200 import build as wb
     if rank == 0:
-        n_step_calls = n_chunks * n_steps * n_layers
+        wb.build()
+    replicas.barrier(world)
+    c4 = c4_measure(args, rank, world, local_rank)
+    if rank == 0:
         line = {
-            "metric": METRIC, "value": frames / (total_ms / 1000.0), "unit": "frames/s", "n_gpus": world,
-            "steps": n_step_calls, "warmup": n_steps * n_layers, "ms_per_step": total_ms / n_step_calls,
-            "ms_total": total_ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "metric": METRIC, "value": c4["frames_per_s"], "unit": "frames/s", "n_gpus": world,
+            "steps": c4["steps"], "warmup": c4["steps"] // args.chunks, "ms_per_step": c4["ms_per_step"],
+            "ms_total": c4["ms_total"], "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"c4 full denoise stack: {n_layers} layers x {n_steps} denoising steps "
-                                   f"x {n_chunks} chunks of 3 frames, one-layer shapes as C1, pool of "
-                                   f"16 pages per layer with a float64 page index; each chunk's KV "
-                                   f"appended to every layer's pool (index refreshed) inside the "
-                                   f"timed region; queries/gates cycle through {n_rot} resident draws",
+            "config": {"workload": c4["workload"],
                        "l2": "no flush: each step reads >300 MB of selected K/V",
                        "parallelism": f"replicas x{world} (independent layer stacks, no collective)"},
-            "clocks": clocks,
-            "gpu_launches": n_step_calls * 14 + n_chunks * n_layers * 3,
+            "clocks": c4["clocks"], "gpu_launches": c4["gpu_launches"],
         }
         print(json.dumps(line), flush=True)
     return 0
@@ -573,6 +598,8 @@ def main():
     ap.add_argument("--config", choices=["c1", "c4"], default="c1",
                     help="c1: one-layer step (default); c4: the full denoise stack")
     ap.add_argument("--layers", type=int, default=30, help="c4: layers")
+    ap.add_argument("--no-c4", action="store_true",
+                    help="c1: skip the full denoise stack figure added to the line")
     ap.add_argument("--b-inter", type=int, default=0, choices=[0, 64, 128],
                     help="c1: block size of the history in block selection (128: inter-chunk "
                          "granularity; the chunk's own keys keep 64)")
