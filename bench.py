@@ -50,8 +50,9 @@ from linear_attention_paged_b200 import replicas  # noqa: E402
 
 METRIC = "HSA ms/chunk-layer & attention frames/s; % of BF16 tensor / HBM roofline"
 # DRAM bytes per launch of the sparse-branch attention kernel per head, from one ncu
-# capture of the 6-head C1 launch (355.8 MB / 6); set to None when the kernel changes
-ATTN_DRAM_BYTES_PER_HEAD = 355.8e6 / 6
+# capture of the 6-head C1 launch with work items grouped by two heads (161.5 MB read +
+# 15.0 MB written) / 6; set to None when the kernel or its item order changes
+ATTN_DRAM_BYTES_PER_HEAD = (161521408 + 14956544) / 6
 FRAMES_PER_CHUNK = 3
 CHUNK_LAYERS_PER_CHUNK = 30 * 4
 # stage -> (start event, end event) of the events wa_hsa_step records; the
