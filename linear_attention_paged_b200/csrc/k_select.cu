@@ -179,107 +179,69 @@ k_block_scores(const double* __restrict__ qmean, KeyMeans km, int n_qb, int n_kb
 }
 
 // ------------------------------------------------------------------ S3 choice
-// CTA = one (head, query block) row of 256 threads, each holding E consecutive
-// positions of the row in registers (E = 4 up to 1024 key blocks).  A bitonic sort
-// orders the scores descending (ascending block on ties): compare-exchange stages of
-// stride < E run inside a thread, strides < 32E across the lanes of a warp
-// (shuffles), and only the six stages of stride >= 32E go through shared memory.
-// Then the softmax masses exp(s - max)/Z, a block-wide scan of the masses in sorted
-// order, the first position whose prefix reaches tau_h, and the mask and the
-// ascending index list.
+// CTA = one (head, query block) row: bitonic sort of the scores (descending,
+// ascending block on ties), softmax masses exp(s - max)/Z, a block-wide scan of the
+// masses in sorted order, the first position whose prefix reaches tau_h, then the
+// mask and the ascending index list.
 constexpr int kChooseThreads = 256;
 
 __device__ __forceinline__ bool before(double ka, int ia, double kb, int ib) {
   return ka > kb || (ka == kb && ia < ib);
 }
 
-template <int E>
 __global__ void __launch_bounds__(kChooseThreads)
-k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int W,
+k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int lg_np, int W,
                const float* __restrict__ tau, int32_t* __restrict__ blk_idx,
                int32_t* __restrict__ blk_cnt, uint32_t* __restrict__ blk_mask, int n_h, int n_sub,
                int W_mask) {
-  constexpr int NP = kChooseThreads * E;
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  double* xk = reinterpret_cast<double*>(smem_raw);            // [NP] exchange of the wide stages
-  int* xi = reinterpret_cast<int*>(xk + NP);                    // [NP]
-  uint32_t* maskw = reinterpret_cast<uint32_t*>(xi + NP);      // [W] (selection blocks)
+  const int NP = 1 << lg_np;
+  double* key = reinterpret_cast<double*>(smem_raw);          // [NP]
+  int* idx = reinterpret_cast<int*>(key + NP);                 // [NP]
+  uint32_t* maskw = reinterpret_cast<uint32_t*>(idx + NP);     // [W] (selection blocks)
   uint32_t* maskx = maskw + W;                                  // [W_mask] (n_h > 0: B-row blocks)
   __shared__ double wred[kChooseThreads / 32];
   __shared__ int ired[kChooseThreads / 32];
-  __shared__ double row_max;
   const int h = blockIdx.y, i = blockIdx.x;
   const size_t rowid = static_cast<size_t>(h) * n_qb + i;
   const double* srow = scores + rowid * n_kb;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int e0 = tid * E;
-  double kv[E];
-  int iv[E];
-#pragma unroll
-  for (int s = 0; s < E; ++s) {
-    const int e = e0 + s;
-    kv[s] = e < n_kb ? srow[e] : -INFINITY;
-    iv[s] = e < n_kb ? e : INT_MAX;
+  for (int e = tid; e < NP; e += kChooseThreads) {
+    key[e] = e < n_kb ? srow[e] : -INFINITY;
+    idx[e] = e < n_kb ? e : INT_MAX;
   }
   for (int w = tid; w < W; w += kChooseThreads) maskw[w] = 0u;
   for (int w = tid; w < W_mask && n_h > 0; w += kChooseThreads) maskx[w] = 0u;
-  // the position e = e0 + s keeps the element its side of the pair wants: the first
-  // in sort order at the lower position of an ascending (k-bit 0) run, else the second
-  auto settle = [&](int s, int j, int k, double pk, int pi) {
-    const int e = e0 + s;
-    const bool wants_first = ((e & j) == 0) == ((e & k) == 0);
-    const bool mine_first = before(kv[s], iv[s], pk, pi);
-    if (wants_first != mine_first) { kv[s] = pk; iv[s] = pi; }
-  };
+  __syncthreads();
   for (int k = 2; k <= NP; k <<= 1) {
-    for (int j = k >> 1; j > 0; j >>= 1) {
-      if (j < E) {
-#pragma unroll
-        for (int s = 0; s < E; ++s) {
-          if (s & j) continue;
-          const int a = s, b = s | j;
-          const bool up = ((e0 + a) & k) == 0;
-          const bool swap = up ? before(kv[b], iv[b], kv[a], iv[a]) : before(kv[a], iv[a], kv[b], iv[b]);
-          if (swap) {
-            const double tk = kv[a]; kv[a] = kv[b]; kv[b] = tk;
-            const int ti = iv[a]; iv[a] = iv[b]; iv[b] = ti;
-          }
-        }
-      } else if (j < 32 * E) {
-        const int lm = j / E;
-#pragma unroll
-        for (int s = 0; s < E; ++s) {
-          const double pk = __shfl_xor_sync(0xffffffffu, kv[s], lm);
-          const int pi = __shfl_xor_sync(0xffffffffu, iv[s], lm);
-          settle(s, j, k, pk, pi);
-        }
-      } else {
-        __syncthreads();   // the previous exchange is read by everyone
-#pragma unroll
-        for (int s = 0; s < E; ++s) { xk[e0 + s] = kv[s]; xi[e0 + s] = iv[s]; }
-        __syncthreads();
-#pragma unroll
-        for (int s = 0; s < E; ++s) {
-          const int p = (e0 + s) ^ j;
-          settle(s, j, k, xk[p], xi[p]);
-        }
+    for (int js = k >> 1; js > 0; js >>= 1) {
+      for (int p = tid; p < (NP >> 1); p += kChooseThreads) {
+        const int a = ((p & ~(js - 1)) << 1) | (p & (js - 1));   // bit js of a is 0
+        const int b = a | js;
+        const double ka = key[a], kb = key[b];
+        const int ia = idx[a], ib = idx[b];
+        const bool swap = (a & k) == 0 ? before(kb, ib, ka, ia) : before(ka, ia, kb, ib);
+        if (swap) { key[a] = kb; key[b] = ka; idx[a] = ib; idx[b] = ia; }
       }
+      __syncthreads();
     }
   }
-  // thread t now holds sorted positions [t*E, t*E + E)
-  if (tid == 0) row_max = kv[0];
-  __syncthreads();
   const double th = static_cast<double>(tau[h]);
   int m = n_kb;
   if (th < 1.0) {
-    const double smax = row_max;
-    // z_t = exp(s_t - max); Z = sum (per thread in order, then warps in order)
-    double p[E];
+    // every thread takes the maximum before thread 0 overwrites key[0] with its
+    // exponential below (without this barrier a warp running ahead changes the
+    // maximum that slower warps read, and the masses of their blocks come out wrong)
+    const double smax = key[0];
+    __syncthreads();
+    const int per = NP / kChooseThreads > 0 ? NP / kChooseThreads : 1;
+    const int t0 = tid * per;
+    // z_t = exp(s_t - max), kept in place of the sorted scores
     double zl = 0.0;
-#pragma unroll
-    for (int s = 0; s < E; ++s) {
-      p[s] = (e0 + s) < n_kb ? exp(kv[s] - smax) : 0.0;
-      zl += p[s];
+    for (int t = t0; t < t0 + per && t < NP; ++t) {
+      const double z = t < n_kb ? exp(key[t] - smax) : 0.0;
+      key[t] = z;
+      zl += z;
     }
     zl = warp_sum(zl);
     if (lane == 0) wred[warp] = zl;
@@ -288,10 +250,10 @@ k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int W,
     for (int w = 0; w < kChooseThreads / 32; ++w) Z += wred[w];
     __syncthreads();
     double pl = 0.0;
-#pragma unroll
-    for (int s = 0; s < E; ++s) {
-      p[s] = p[s] / Z;
-      pl += p[s];
+    for (int t = t0; t < t0 + per && t < NP; ++t) {
+      const double pv = key[t] / Z;
+      key[t] = pv;
+      pl += pv;
     }
     // exclusive prefix of the per-thread sums, in thread order
     double incl = pl;
@@ -305,10 +267,9 @@ k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int W,
     double c = incl - pl;
     for (int w = 0; w < warp; ++w) c += wred[w];
     int first = INT_MAX;
-#pragma unroll
-    for (int s = 0; s < E; ++s) {
-      c += p[s];
-      if (first == INT_MAX && e0 + s < n_kb && c >= th) first = e0 + s;
+    for (int t = t0; t < t0 + per && t < n_kb; ++t) {
+      c += key[t];
+      if (c >= th) { first = t; break; }
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
@@ -318,10 +279,8 @@ k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int W,
     for (int w = 0; w < kChooseThreads / 32; ++w) first = min(first, ired[w]);
     if (first != INT_MAX) m = first + 1;
   }
-#pragma unroll
-  for (int s = 0; s < E; ++s) {
-    if (e0 + s >= m) break;
-    const int j = iv[s];
+  for (int t = tid; t < m; t += kChooseThreads) {
+    const int j = idx[t];
     atomicOr(&maskw[j >> 5], 1u << (j & 31));
     if (n_h > 0) {
       // the same keys at B-row granularity: a 2B-row history block covers B-row blocks
@@ -406,26 +365,15 @@ wa_status launch_block_select(const double* q_blockmean, int Nq, int H, int d, i
   if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "block_scores smem attr: %s", cudaGetErrorString(e));
   k_block_scores<<<dim3((n_kb + 31) / 32, (n_qb + 31) / 32, H), 256, smem_s, st>>>(
       q_blockmean, km, n_qb, n_kb, H, d, B, scores);
-  // E positions per thread: the row padded to 256 * E >= n_kb
-  int E = 4;
-  while (kChooseThreads * E < n_kb) E *= 2;
-  const size_t smem_c = static_cast<size_t>(kChooseThreads) * E * 12 + static_cast<size_t>(W + W_mask) * 4 + 16;
-  const int n_h = km.pair ? km.n_kb1 : 0;
-  const int W_out = km.pair ? W_mask : W;
-  auto launch = [&](auto kern) -> cudaError_t {
-    cudaError_t r = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem_c));
-    if (r != cudaSuccess) return r;
-    kern<<<dim3(n_qb, H), kChooseThreads, smem_c, st>>>(scores, n_qb, n_kb, W, tau, blk_idx, blk_cnt,
-                                                        blk_mask, n_h, km.n_sub, W_out);
-    return cudaSuccess;
-  };
-  if (E == 4) e = launch(k_block_choose<4>);
-  else if (E == 8) e = launch(k_block_choose<8>);
-  else if (E == 16) e = launch(k_block_choose<16>);
-  else if (E == 32) e = launch(k_block_choose<32>);
-  else return set_error(WA_ERR_UNSUPPORTED, "block selection: at most 8192 key blocks");
+  int lg = 5;
+  while ((1 << lg) < n_kb) ++lg;
+  const size_t smem_c = (static_cast<size_t>(1) << lg) * 12 + static_cast<size_t>(W + W_mask) * 4 + 16;
+  e = cudaFuncSetAttribute(k_block_choose, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(smem_c));
   if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "block_choose smem attr: %s", cudaGetErrorString(e));
+  k_block_choose<<<dim3(n_qb, H), kChooseThreads, smem_c, st>>>(
+      scores, n_qb, n_kb, lg, W, tau, blk_idx, blk_cnt, blk_mask, km.pair ? km.n_kb1 : 0, km.n_sub,
+      km.pair ? W_mask : W);
   return check_launch("block_select");
 }
 
