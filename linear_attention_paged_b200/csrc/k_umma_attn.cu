@@ -92,7 +92,7 @@ struct Shared {
   uint64_t s_full;        // S_t computed
   uint64_t s_free;        // S_t loaded by all eight softmax warps
   uint64_t p_full[2];     // P_t of group g stored, one arrival per warp of the group
-  uint64_t o_done[2];     // O_g += P_t V_t complete, one barrier per group
+  uint64_t o_done;        // O_g += P_t V_t complete (both groups)
   uint64_t drain[2];      // abort path: every MMA of issuer 0 (S) / 1 (P V) complete
   uint64_t wait_ns;       // bound of every wait (wa_set_wait_limit_ns)
   uint32_t tmem_base;
@@ -230,8 +230,7 @@ k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CU
     mbar_init(&sh.s_free, 8);
     mbar_init(&sh.p_full[0], 4);
     mbar_init(&sh.p_full[1], 4);
-    mbar_init(&sh.o_done[0], 1);
-    mbar_init(&sh.o_done[1], 1);
+    mbar_init(&sh.o_done, 1);
     mbar_init(&sh.drain[0], 1);
     mbar_init(&sh.drain[1], 1);
     sh.wait_ns = wait_ns;
@@ -359,13 +358,7 @@ k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CU
         // group 1 has no block in an odd list's last iteration
         const int n_grp = (u == n_it - 1 && odd_tail) ? 1 : 2;
         bool ok = true;
-        for (int g = 0; g < 2; ++g) {
-          if (g >= n_grp) {
-            // no block for group 1 in an odd list's last iteration: its barrier still
-            // completes (once the MMAs issued so far are done)
-            mma_commit(&sh.o_done[g]);
-            break;
-          }
+        for (int g = 0; g < n_grp; ++g) {
           if (!wait_bar(&sh.p_full[g], u & 1, sh, err)) { ok = false; break; }
           tc_fence_after();
           const uint32_t v_base = smem_u32(Vs(vs)) + g * (kBN * 128);
@@ -375,10 +368,10 @@ k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CU
             mma_ts(tbase + kColO + g * D, tbase + kColP + g * (kBN / 2) + kk * 8, bdesc,
                    C::kIdescO, (u > 0 || kk > 0) ? 1u : 0u);
           }
-          mma_commit(&sh.o_done[g]);   // this group's P may be overwritten, its O rescaled
         }
         if (!ok) break;
         mma_commit(&sh.v_empty[vs]);
+        mma_commit(&sh.o_done);
       }
     }
   } else if (warp >= 4) {
@@ -409,7 +402,7 @@ k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CU
     // completed t-1 or t phases: its parity is unambiguous.
     auto wait_pv = [&](int t) -> bool {
       if (t == 0) return true;
-      const bool w = __all_sync(0xffffffffu, wait_bar(&sh.o_done[g], (t - 1) & 1, sh, err));
+      const bool w = __all_sync(0xffffffffu, wait_bar(&sh.o_done, (t - 1) & 1, sh, err));
       tc_fence_after();
       return w;
     };
@@ -512,11 +505,7 @@ k_umma_attention(const __nv_bfloat16* __restrict__ q, const __grid_constant__ CU
     // writes half of the columns of  w_0 O_0 + w_1 O_1  and  l = w_0 l_0 + w_1 l_1
     sh.xch[0][g][row] = m_run;
     sh.xch[1][g][row] = l_run;
-    // each group waited for its own P V MMAs; across this barrier (with the tcgen05
-    // fences) the other group's accumulator is complete too
-    tc_fence_before();
     asm volatile("bar.sync 1, 256;" ::: "memory");
-    tc_fence_after();
     const float m_o = sh.xch[0][g ^ 1][row], l_o = sh.xch[1][g ^ 1][row];
     const float m0 = g ? m_o : m_run, m1 = g ? m_run : m_o;
     const float l0 = g ? l_o : l_run, l1 = g ? l_run : l_o;
