@@ -37,7 +37,8 @@ Readings where the pages are silent (each one is listed in the design notes):
     does a row whose cumulative mass never reaches tau_h.
   * Block pooling is the mean over the valid rows of a block; a block's score is
     q-bar . k-bar / sqrt(d); the mass is the softmax of one (head, query block) row.
-  * E_K, E_V are shared by all heads, shape [L][r]; no extra scaling.
+  * E_K, E_V are shared by all heads, shape [L][r], unless given per head ([H][L][r],
+    the main text's K~^(h) read as one projection per head); no extra scaling.
   * Keys of both branches are the retrieved history; with k_cur/v_cur the sparse
     branch also takes the current chunk's own keys (after the history); no causal mask.
   * Key block sizes (§3.3 "Inter- and intra-chunk sparse granularity"): the history
@@ -258,14 +259,20 @@ def block_select(q, k_act, tau, B: int, scores: Optional[np.ndarray] = None, key
 
 # ----------------------------------------------------------------------------- S4
 def linear_project(k_act, v_act, e_k, e_v):
-    """K~ = E_K^T K, V~ = E_V^T V per head (§3.3 linear branch; E shared by heads).
-    k_act, v_act: [L][H][d]; e_k, e_v: [L][r] -> K~, V~: [r][H][d]."""
+    """K~ = E_K^T K, V~ = E_V^T V per head (§3.3 linear branch, K~^(h) = E_K^T K^(h)).
+    k_act, v_act: [L][H][d]; e_k, e_v: [L][r] shared by the heads, or [H][L][r] one
+    per head -> K~, V~: [r][H][d]."""
     K = f64(k_act)
     V = f64(v_act)
     EK = f64(e_k)
     EV = f64(e_v)
-    # sum over l of E[l][c] * X[l][h][:], as one [r][L] @ [L][H*d] product
     L, H, d = K.shape
+    if EK.ndim == 3:
+        # one E per head: K~[:, h, :] = E_K[h]^T K[:, h, :]
+        kt = np.stack([EK[h].T @ K[:, h, :] for h in range(H)], axis=1)
+        vt = np.stack([EV[h].T @ V[:, h, :] for h in range(H)], axis=1)
+        return kt, vt
+    # sum over l of E[l][c] * X[l][h][:], as one [r][L] @ [L][H*d] product
     kt = (EK.T @ K.reshape(L, H * d)).reshape(-1, H, d)
     vt = (EV.T @ V.reshape(L, H * d)).reshape(-1, H, d)
     return kt, vt

@@ -538,3 +538,35 @@ def test_mixed_granularity_equal_sizes_is_uniform():
     b = O.hsa_step(inp, cfg.B, cfg.K_p, B_inter=cfg.B)
     assert a["kept"] == b["kept"]
     np.testing.assert_array_equal(a["o"], b["o"])
+
+
+# ----------------------------------------------- per-head Linformer projections (§3.3)
+def test_linear_branch_per_head_row_selection():
+    """One E per head (K~^(h) = E_K^(h)T K^(h)): with a different row selection per head
+    and per branch, each head's linear branch is textbook attention over its own
+    selected rows -- which pins the head each E goes with and its orientation."""
+    r = rng(41)
+    Nq, L, H, d, rr = 5, 18, 3, 4, 6
+    q = r.normal(size=(Nq, H, d)); k = r.normal(size=(L, H, d)); v = r.normal(size=(L, H, d))
+    EK = np.zeros((H, L, rr)); EV = np.zeros((H, L, rr))
+    sel_k = [r.choice(L, rr, replace=False) for _ in range(H)]
+    sel_v = [r.choice(L, rr, replace=False) for _ in range(H)]
+    for h in range(H):
+        EK[h, sel_k[h], np.arange(rr)] = 1
+        EV[h, sel_v[h], np.arange(rr)] = 1
+    kt, vt = O.linear_project(k, v, EK, EV)
+    o = O.linear_attention(q, kt, vt)
+    for h in range(H):
+        np.testing.assert_allclose(o[:, h], sdpa(q[:, h], k[sel_k[h], h], v[sel_v[h], h]),
+                                   rtol=1e-12, atol=1e-12)
+
+
+def test_linear_branch_per_head_identity_is_dense_attention():
+    r = rng(42)
+    Nq, L, H, d = 4, 9, 2, 3
+    q = r.normal(size=(Nq, H, d)); k = r.normal(size=(L, H, d)); v = r.normal(size=(L, H, d))
+    E = np.stack([np.eye(L)] * H)
+    kt, vt = O.linear_project(k, v, E, E)
+    o = O.linear_attention(q, kt, vt)
+    for h in range(H):
+        np.testing.assert_allclose(o[:, h], sdpa(q[:, h], k[:, h], v[:, h]), rtol=1e-12, atol=1e-12)
