@@ -233,6 +233,15 @@ WA_API wa_status wa_linear_project(const void* k_act, const void* v_act, const v
                             void* k_til, void* v_til, void* ws, size_t ws_bytes,
                             void* stream);
 
+/* The same with one projection per head (main text §3.3, "Linear branch", writes
+ * K~^(h) = E_K^T K^(h)): e_k, e_v are [H][L][r] with e_head_stride = L*r elements
+ * (0 falls back to wa_linear_project: one E for every head).  The workspace is at most
+ * wa_linear_project_workspace_size's.  INVALID_ARG: any other stride. */
+WA_API wa_status wa_linear_project_heads(const void* k_act, const void* v_act, const void* e_k,
+                                         const void* e_v, int L, int H, int d, int r,
+                                         wa_dtype dtype, long long e_head_stride, void* k_til,
+                                         void* v_til, void* ws, size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------------------
  * The S4a projection for callers that cannot allocate device memory.  The paper
  * has no counterpart to this entry point.
@@ -377,6 +386,10 @@ typedef struct wa_step_args {
      granularity (a kept history block sets its two B-token blocks).  2*B needs
      K_p*T_p % B == 0. */
   int B_inter;
+  /* optional per-head projections (main text §3.3, "Linear branch", K~^(h)): 0 (the
+     default) when e_k / e_v are one [K_p*T_p][r] matrix for every head, or
+     K_p*T_p*r when they are [H][K_p*T_p][r], one matrix per head (elements). */
+  long long e_head_stride;
 } wa_step_args;
 
 /* Stage boundaries recorded into wa_step_args.stage_events:

@@ -24,10 +24,12 @@ __device__ __forceinline__ long long row_of(const RowSource& rs, int l, int B, b
 }
 
 __global__ void k_simt_project(const float* __restrict__ x, RowSource rs, const float* __restrict__ e,
-                               int L, int cols, int r, float* __restrict__ out, uint32_t* err) {
+                               int L, int cols, int r, int d, long long e_head_stride,
+                               float* __restrict__ out, uint32_t* err) {
   const int col = blockIdx.x * blockDim.x + threadIdx.x;
   const int c = blockIdx.y;
   if (col >= cols) return;
+  e += static_cast<long long>(col / d) * e_head_stride;   // this column's head's E (0: shared)
   double acc = 0.0;
   bool bad = false;
   for (int l = 0; l < L; ++l) {
@@ -141,15 +143,15 @@ k_simt_attention(int mode, const float* __restrict__ q, int Nq, int H, RowSource
 }  // namespace
 
 wa_status launch_simt_project(const float* x, const int32_t* page_ids, int page_rows, int n_pages,
-                              const float* e, int L, int cols, int r, float* out,
-                              uint32_t* err, cudaStream_t st) {
+                              const float* e, int L, int cols, int r, int d, long long e_head_stride,
+                              float* out, uint32_t* err, cudaStream_t st) {
   RowSource rs;
   rs.page_ids = page_ids;
   rs.page_rows = page_rows;
   rs.n_pages = n_pages;
   rs.L = L;
   dim3 grid((cols + 127) / 128, r);
-  k_simt_project<<<grid, 128, 0, st>>>(x, rs, e, L, cols, r, out, err);
+  k_simt_project<<<grid, 128, 0, st>>>(x, rs, e, L, cols, r, d, e_head_stride, out, err);
   return check_launch("simt_project");
 }
 

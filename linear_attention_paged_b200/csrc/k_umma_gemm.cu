@@ -64,7 +64,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 k_umma_project(const __grid_constant__ CUtensorMap tmEK, const __grid_constant__ CUtensorMap tmEV,
                const __grid_constant__ CUtensorMap tmXK, const __grid_constant__ CUtensorMap tmXV,
                RowSource rs, int L, int cols, int n_split, float* __restrict__ part,
-               uint32_t* err, uint64_t wait_ns) {
+               uint32_t* err, uint64_t wait_ns, int d, int e_head_rows) {
   using C = GCfg<NSUB, TN>;
   extern __shared__ uint8_t smem_dyn[];
   __shared__ GShared sh;
@@ -81,6 +81,9 @@ k_umma_project(const __grid_constant__ CUtensorMap tmEK, const __grid_constant__
   const int nk = kb1 > kb0 ? kb1 - kb0 : 0;
   const CUtensorMap* tE = m ? &tmEV : &tmEK;
   const CUtensorMap* tX = m ? &tmXV : &tmXK;
+  // one E per head (e_head_rows = L): a tile lies within one head (TN <= d), whose E
+  // rows start at head * L of the [H*L][r] view
+  const int e_row0 = e_head_rows ? (nt * TN / d) * e_head_rows : 0;
 
   if (tid == 0) {
     for (int s = 0; s < C::kStages; ++s) { mbar_init(&sh.full[s], 1); mbar_init(&sh.empty[s], 1); }
@@ -117,7 +120,7 @@ k_umma_project(const __grid_constant__ CUtensorMap tmEK, const __grid_constant__
         uint8_t* As = tiles + s * C::kStageBytes;
         uint8_t* Bs = As + C::kABytes;
         mbar_arrive_expect_tx(&sh.full[s], C::kStageBytes);
-        for (int p = 0; p < C::kR / 64; ++p) tma_load_2d(As + p * 8192, tE, &sh.full[s], p * 64, l0);
+        for (int p = 0; p < C::kR / 64; ++p) tma_load_2d(As + p * 8192, tE, &sh.full[s], p * 64, e_row0 + l0);
         for (int p = 0; p < TN / 64; ++p)
           tma_load_2d(Bs + p * 8192, tX, &sh.full[s], nt * TN + p * 64, row);
         issued = t + 1;
@@ -223,8 +226,14 @@ int pick_tn(int cols) {
   return 0;
 }
 
-int pick_splits(int L, int r, int cols) {
+// with one E per head a tile must lie within one head: width d at most
+int pick_tn_for(int cols, int d, bool e_per_head) {
   const int tn = pick_tn(cols);
+  return (e_per_head && tn > d) ? d : tn;
+}
+
+int pick_splits(int L, int r, int cols, int tn_override = 0) {
+  const int tn = tn_override ? tn_override : pick_tn(cols);
   const int tiles = 2 * (cols / tn);
   const int n_kb = (L + kKB - 1) / kKB;
   int s = 148 / tiles;
@@ -237,36 +246,42 @@ int pick_splits(int L, int r, int cols) {
 template <int NSUB, int TN>
 void launch_proj(dim3 grid, cudaStream_t st, const CUtensorMap& a, const CUtensorMap& b,
                  const CUtensorMap& c, const CUtensorMap& d, RowSource rs, int L, int cols,
-                 int n_split, float* part, uint32_t* err) {
+                 int n_split, float* part, uint32_t* err, int dh = 128, int e_head_rows = 0) {
   using C = GCfg<NSUB, TN>;
   cudaFuncSetAttribute(k_umma_project<NSUB, TN>, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmem);
   k_umma_project<NSUB, TN><<<grid, kThreads, C::kSmem, st>>>(a, b, c, d, rs, L, cols, n_split,
-                                                             part, err, wait_limit_ns());
+                                                             part, err, wait_limit_ns(), dh,
+                                                             e_head_rows);
 }
 
 }  // namespace
 
-size_t umma_project_ws_bytes(int L, int H, int d, int r) {
+size_t umma_project_ws_bytes(int L, int H, int d, int r, bool e_per_head) {
   const int cols = H * d;
-  if (pick_tn(cols) == 0) return 0;
-  return 2ull * pick_splits(L, r, cols) * r * cols * sizeof(float);
+  const int tn = pick_tn_for(cols, d, e_per_head);
+  if (tn == 0) return 0;
+  return 2ull * pick_splits(L, r, cols, tn) * r * cols * sizeof(float);
 }
 
 wa_status launch_umma_project(const void* k, const void* v, RowSource rs, const void* e_k,
                               const void* e_v, int L, int H, int d, int r, void* k_til,
-                              void* v_til, void* ws, uint32_t* err, cudaStream_t st) {
+                              void* v_til, void* ws, uint32_t* err, cudaStream_t st,
+                              bool e_per_head) {
   const int cols = H * d;
-  const int tn = pick_tn(cols);
+  const int tn = pick_tn_for(cols, d, e_per_head);
   if (tn == 0) return set_error(WA_ERR_UNSUPPORTED, "projection needs H*d %% 64 == 0");
   if (r != 128 && r != 256) return set_error(WA_ERR_UNSUPPORTED, "bf16 projection needs r in {128, 256}");
   if (rs.page_ids && rs.page_rows % kKB != 0)
     return set_error(WA_ERR_UNSUPPORTED, "paged projection needs T_p %% 64 == 0");
-  const int n_split = pick_splits(L, r, cols);
+  const int n_split = pick_splits(L, r, cols, tn);
   const uint64_t rows = rs.page_ids ? static_cast<uint64_t>(rs.n_pages) * rs.page_rows
                                     : static_cast<uint64_t>(L);
+  // E as a 2-D [rows][r] tensor: L rows, or H * L rows when there is one E per head
+  const uint64_t e_rows = e_per_head ? static_cast<uint64_t>(H) * L : static_cast<uint64_t>(L);
+  const int e_head_rows = e_per_head ? L : 0;
   alignas(64) CUtensorMap tek, tev, txk, txv;
-  if (!make_tmap_bf16_2d(&tek, e_k, r, L, static_cast<uint64_t>(r) * 2, 64, 64) ||
-      !make_tmap_bf16_2d(&tev, e_v, r, L, static_cast<uint64_t>(r) * 2, 64, 64) ||
+  if (!make_tmap_bf16_2d(&tek, e_k, r, e_rows, static_cast<uint64_t>(r) * 2, 64, 64) ||
+      !make_tmap_bf16_2d(&tev, e_v, r, e_rows, static_cast<uint64_t>(r) * 2, 64, 64) ||
       !make_tmap_bf16_2d(&txk, k, cols, rows, static_cast<uint64_t>(cols) * 2, 64, 64) ||
       !make_tmap_bf16_2d(&txv, v, cols, rows, static_cast<uint64_t>(cols) * 2, 64, 64))
     return set_error(WA_ERR_CUDA, "cuTensorMapEncodeTiled failed for the projection operands");
@@ -274,13 +289,13 @@ wa_status launch_umma_project(const void* k, const void* v, RowSource rs, const 
   dim3 grid(2 * (cols / tn), n_split);
   const int nsub = r / 128;
   if (nsub == 2) {
-    if (tn == 256) launch_proj<2, 256>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
-    else if (tn == 128) launch_proj<2, 128>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
-    else launch_proj<2, 64>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
+    if (tn == 256) launch_proj<2, 256>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err, d, e_head_rows);
+    else if (tn == 128) launch_proj<2, 128>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err, d, e_head_rows);
+    else launch_proj<2, 64>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err, d, e_head_rows);
   } else {
-    if (tn == 256) launch_proj<1, 256>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
-    else if (tn == 128) launch_proj<1, 128>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
-    else launch_proj<1, 64>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err);
+    if (tn == 256) launch_proj<1, 256>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err, d, e_head_rows);
+    else if (tn == 128) launch_proj<1, 128>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err, d, e_head_rows);
+    else launch_proj<1, 64>(grid, st, tek, tev, txk, txv, rs, L, cols, n_split, part, err, d, e_head_rows);
   }
   wa_status s = check_launch("umma_project");
   if (s != WA_OK) return s;

@@ -499,10 +499,37 @@ wa_status wa_linear_project(const void* k_act, const void* v_act, const void* e_
   if (dtype == WA_BF16)
     return launch_umma_project(k_act, v_act, rs, e_k, e_v, L, H, d, r, k_til, v_til, ws, err, st);
   WA_TRY(launch_simt_project(static_cast<const float*>(k_act), nullptr, L, 1,
-                             static_cast<const float*>(e_k), L, H * d, r,
+                             static_cast<const float*>(e_k), L, H * d, r, d, 0,
                              static_cast<float*>(k_til), err, st));
   return launch_simt_project(static_cast<const float*>(v_act), nullptr, L, 1,
-                             static_cast<const float*>(e_v), L, H * d, r,
+                             static_cast<const float*>(e_v), L, H * d, r, d, 0,
+                             static_cast<float*>(v_til), err, st);
+}
+
+wa_status wa_linear_project_heads(const void* k_act, const void* v_act, const void* e_k,
+                                  const void* e_v, int L, int H, int d, int r, wa_dtype dtype,
+                                  long long e_head_stride, void* k_til, void* v_til, void* ws,
+                                  size_t ws_bytes, void* stream) {
+  WA_REQUIRE(k_act && v_act && e_k && e_v && k_til && v_til, "NULL pointer");
+  WA_REQUIRE(L >= 1 && r >= 1, "sizes must be >= 1");
+  WA_TRY(check_shape(H, d, 64, dtype));
+  WA_REQUIRE(e_head_stride == 0 || e_head_stride == static_cast<long long>(L) * r,
+             "e_head_stride must be 0 (one E for all heads) or L*r (one per head)");
+  if (e_head_stride == 0)
+    return wa_linear_project(k_act, v_act, e_k, e_v, L, H, d, r, dtype, k_til, v_til, ws, ws_bytes, stream);
+  WA_TRY(check_ws(ws, ws_bytes, wa_linear_project_workspace_size(L, H, d, r, dtype)));
+  uint32_t* err = errw();
+  if (!err) return set_error(WA_ERR_CUDA, "no CUDA device");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  RowSource rs;
+  rs.k = k_act; rs.v = v_act; rs.page_rows = L; rs.n_pages = 1; rs.L = L;
+  if (dtype == WA_BF16)
+    return launch_umma_project(k_act, v_act, rs, e_k, e_v, L, H, d, r, k_til, v_til, ws, err, st, true);
+  WA_TRY(launch_simt_project(static_cast<const float*>(k_act), nullptr, L, 1,
+                             static_cast<const float*>(e_k), L, H * d, r, d, e_head_stride,
+                             static_cast<float*>(k_til), err, st));
+  return launch_simt_project(static_cast<const float*>(v_act), nullptr, L, 1,
+                             static_cast<const float*>(e_v), L, H * d, r, d, e_head_stride,
                              static_cast<float*>(v_til), err, st);
 }
 
@@ -642,6 +669,8 @@ wa_status validate_step(const wa_step_args* a) {
   WA_REQUIRE(!a->k_cur == !a->v_cur, "k_cur and v_cur are given together");
   WA_REQUIRE(a->B_inter == 0 || a->B_inter == a->B || a->B_inter == 2 * a->B,
              "B_inter must be 0, B or 2*B (got %d)", a->B_inter);
+  WA_REQUIRE(a->e_head_stride == 0 || a->e_head_stride == L * a->r,
+             "e_head_stride must be 0 (one E for all heads) or K_p*T_p*r (one per head)");
   if (a->B_inter == 2 * a->B && L % a->B != 0)
     return set_error(WA_ERR_UNSUPPORTED, "B_inter = 2*B needs K_p*T_p %% B == 0");
   if (a->k_cur) {
@@ -794,7 +823,7 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
         cudaEventRecord(static_cast<cudaEvent_t>(a->stage_events[k]), side->stream);
     };
     WA_TRY(launch_umma_project(rs.k, rs.v, rs, a->e_k, a->e_v, L, a->H, a->d, a->r, kt, vt, w.proj,
-                               err, side->stream));
+                               err, side->stream, a->e_head_stride != 0));
     mark_side(4);
     WA_TRY(launch_linear_attention(a->q, a->Nq, a->H, a->d, lin, a->B, a->gate, a->gate_lin, w.lin,
                                    nullptr, err, side->stream));
@@ -815,11 +844,11 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
                                w.scores, nullptr, nullptr, mask, st));
     mark(3);
     WA_TRY(launch_simt_project(static_cast<const float*>(rs.k), rs.page_ids, rs.page_rows,
-                               rs.n_pages, static_cast<const float*>(a->e_k), L, cols, a->r,
-                               static_cast<float*>(kt), err, st));
+                               rs.n_pages, static_cast<const float*>(a->e_k), L, cols, a->r, a->d,
+                               a->e_head_stride, static_cast<float*>(kt), err, st));
     WA_TRY(launch_simt_project(static_cast<const float*>(rs.v), rs.page_ids, rs.page_rows,
-                               rs.n_pages, static_cast<const float*>(a->e_v), L, cols, a->r,
-                               static_cast<float*>(vt), err, st));
+                               rs.n_pages, static_cast<const float*>(a->e_v), L, cols, a->r, a->d,
+                               a->e_head_stride, static_cast<float*>(vt), err, st));
     mark(4);
     WA_TRY(run_attention(a->q, a->Nq, a->H, a->d, rs, a->B, mask, kt, vt, a->r, a->gate, a->gate_lin,
                          a->dtype, a->out, nullptr, nullptr, w.lin, w.attn, st, a->stage_events));

@@ -130,9 +130,11 @@ wa_status launch_permute_rows(const void* src, void* dst, const int32_t* perm, i
                               size_t row_bytes, int inverse, uint32_t* err, cudaStream_t st);
 
 // ---------------------------------------------------------------- fp32 SIMT path
+// out[c][col] = sum_l E_h[l][c] x[l][col], h = col / d, E_h = e + h * e_head_stride
+// (e_head_stride 0: one E for every head)
 wa_status launch_simt_project(const float* x, const int32_t* page_ids, int page_rows, int n_pages,
-                              const float* e, int L, int cols, int r, float* out,
-                              uint32_t* err, cudaStream_t st);
+                              const float* e, int L, int cols, int r, int d, long long e_head_stride,
+                              float* out, uint32_t* err, cudaStream_t st);
 // mode 0: linear branch over (k_til, v_til), writes lin_ws = w * O_lin with
 //         w = 1 - sigmoid(g), or sigmoid(g_lin) when gate_lin is given (two gates)
 // mode 1: sparse branch over blk_mask, writes out = sigmoid(g)*O_sp + lin_ws
@@ -142,10 +144,13 @@ wa_status launch_simt_attention(int mode, const float* q, int Nq, int H, int d, 
                                 uint32_t* err, cudaStream_t st);
 
 // ---------------------------------------------------------------- bf16 tcgen05 path
-size_t umma_project_ws_bytes(int L, int H, int d, int r);
+// e_per_head: E_K, E_V are [H][L][r] (one projection per head); else [L][r], shared.
+// The workspace of the shared form is at least that of the per-head form.
+size_t umma_project_ws_bytes(int L, int H, int d, int r, bool e_per_head = false);
 wa_status launch_umma_project(const void* k, const void* v, RowSource rs, const void* e_k,
                               const void* e_v, int L, int H, int d, int r, void* k_til,
-                              void* v_til, void* ws, uint32_t* err, cudaStream_t st);
+                              void* v_til, void* ws, uint32_t* err, cudaStream_t st,
+                              bool e_per_head = false);
 
 // Linear branch on tcgen05 (keys = k_til/v_til [r][H][d], every block): writes
 //   lin_ws[n][h][:] = w * O_lin (fp32) and o_lin (nullable), with w = 1 - sigmoid(g),

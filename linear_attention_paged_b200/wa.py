@@ -55,6 +55,7 @@ class StepArgs(ctypes.Structure):
         ("gate_lin", P),
         ("k_cur", P), ("v_cur", P),
         ("B_inter", c_int),
+        ("e_head_stride", ctypes.c_longlong),
     ]
 
 
@@ -74,6 +75,8 @@ _SIGS = {
     "wa_linear_project": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, c_int, P, P, P,
                                   c_size_t, P]),
     "wa_linear_project_noalloc": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, c_int, P, P, P]),
+    "wa_linear_project_heads": (c_int, [P, P, P, P, c_int, c_int, c_int, c_int, c_int, ctypes.c_longlong,
+                                        P, P, P, c_size_t, P]),
     "wa_hsa_attention_workspace_size": (c_size_t, [c_int] * 7),
     "wa_hsa_attention": (c_int, [P, c_int, c_int, c_int, P, P, c_int, c_int, P, P, P, c_int, P,
                                  c_int, P, P, P, P, c_size_t, P]),
@@ -302,9 +305,20 @@ def wa_block_select(q, tau, B: int = 64, k_act=None, k_blockmean=None, L: Option
 
 # --------------------------------------------------------------------- S4a
 def wa_linear_project(k_act, v_act, e_k, e_v, stream=None):
+    """K~ = E_K^T K, V~ = E_V^T V; e_k / e_v [L][r] (shared) or [H][L][r] (one per head)."""
     _need_cuda(k_act, v_act, e_k, e_v)
     L, H, d = k_act.shape
-    r = e_k.shape[1]
+    r = e_k.shape[-1]
+    if e_k.dim() == 3:
+        k_til = _empty((r, H, d), k_act.dtype, k_act.device)
+        v_til = _empty((r, H, d), k_act.dtype, k_act.device)
+        dt = dtype_code(k_act)
+        nbytes = lib.wa_linear_project_workspace_size(L, H, d, r, dt)
+        ws = workspace(nbytes, k_act.device)
+        _check("wa_linear_project_heads", lib.wa_linear_project_heads(
+            _p(k_act), _p(v_act), _p(e_k), _p(e_v), L, H, d, r, dt, L * r, _p(k_til), _p(v_til),
+            _p(ws), nbytes, _stream(stream)))
+        return k_til, v_til
     k_til = _empty((r, H, d), k_act.dtype, k_act.device)
     v_til = _empty((r, H, d), k_act.dtype, k_act.device)
     dt = dtype_code(k_act)
@@ -374,7 +388,7 @@ class HSAStep:
         if chunk_pages.dim() == 1:
             chunk_pages = chunk_pages.reshape(1, -1)
         n_chunks, n_c = chunk_pages.shape
-        r = e_k.shape[1]
+        r = e_k.shape[-1]
         L = K_p * T_p
         n_qb, n_kb = -(-Nq // B), -(-(L + (Nq if k_cur is not None else 0)) // B)
         W = -(-n_kb // 32)
@@ -396,6 +410,7 @@ class HSAStep:
         a.gate_lin = _p(gate_lin)
         a.k_cur, a.v_cur = _p(k_cur), _p(v_cur)
         a.B_inter = int(B_inter)
+        a.e_head_stride = L * r if e_k.dim() == 3 else 0
         self._keep += [page_index, gate_lin, k_cur, v_cur]
         self.inter = {}
         if keep_intermediates:

@@ -58,6 +58,8 @@ class HSAConfig:
     hot_beta_scale: float = 7.0
     # the current chunk's own K and V ([Nq][H][d]) join the sparse branch's keys
     intra: bool = False
+    # one Linformer projection per head: e_k, e_v of shape [H][L][r]
+    e_per_head: bool = False
 
     @property
     def L(self) -> int:
@@ -197,6 +199,10 @@ def make_inputs(cfg: HSAConfig, device: str = "cpu", gen_device: Optional[str] =
         sc = 1.0 if cfg.recipe == "gauss" else inv_sqrt_d
         out["k_cur"] = (randn(Nq, H, d) * sc).to(dt).to(device)
         out["v_cur"] = (randn(Nq, H, d) * sc).to(dt).to(device)
+    if cfg.e_per_head:
+        # one E pair per head, drawn after every other input so that those keep their bits
+        e_k = randn(H, L, r) * (1.0 / math.sqrt(L))
+        e_v = randn(H, L, r) * (1.0 / math.sqrt(L))
     out["chunk_pages"] = torch.arange(P, dtype=torch.int32).reshape(cfg.n_chunks, cfg.n_c).to(device)
     out["cand"] = out["chunk_pages"][0].clone()
 

@@ -165,6 +165,23 @@ def test_linear_project(wa, cfg):
     check_device_ok(wa)
 
 
+@pytest.mark.parametrize("cfg", [SMALL_BF16, SMALL_BF16_D64, SMALL_F32], ids=lambda c: c.name)
+def test_linear_project_per_head(wa, cfg):
+    """One projection per head (e_k, e_v [H][L][r]): each head's K~, V~ against the
+    oracle; the bf16 path then tiles the columns within one head."""
+    cfg = cfg.with_(e_per_head=True)
+    inp = inputs(cfg)
+    assert inp["e_k"].dim() == 3 and inp["e_k"].shape[0] == cfg.H
+    sel = [int(x) for x in inp["cand"][: cfg.K_p].cpu()]
+    k_act = O.gather_pages(inp["k_pool"], sel)
+    v_act = O.gather_pages(inp["v_pool"], sel)
+    kt, vt = wa.wa_linear_project(k_act, v_act, inp["e_k"], inp["e_v"])
+    kr, vr = O.linear_project(k_act, v_act, inp["e_k"], inp["e_v"])
+    assert_close(kt, kr, dkey(cfg), f"{cfg.name} per-head K~")
+    assert_close(vt, vr, dkey(cfg), f"{cfg.name} per-head V~")
+    check_device_ok(wa)
+
+
 # ---------------------------------------------------------------- S4b + S5 + S6
 @pytest.mark.parametrize("cfg", [W.C0, SMALL_BF16, SMALL_BF16_D64, SMALL_STRESS, SMALL_F32],
                          ids=lambda c: c.name)
@@ -278,6 +295,20 @@ def test_hsa_step_small(wa, cfg, fused):
                       f"{cfg.name} step masks")
     assert_close(inter["k_til"], res["k_til"], dkey(cfg), f"{cfg.name} step K~")
     assert_close(out, res["o"], dkey(cfg), f"{cfg.name} step O ({'fused' if fused else 'gathered'})")
+    check_device_ok(wa)
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "gathered"])
+@pytest.mark.parametrize("cfg", [SMALL_BF16, SMALL_BF16_D64, SMALL_F32], ids=lambda c: c.name)
+def test_hsa_step_per_head_projection(wa, cfg, fused):
+    cfg = cfg.with_(e_per_head=True)
+    inp = inputs(cfg)
+    out, inter = wa.wa_hsa_step(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"],
+                                inp["e_v"], inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B,
+                                fused_gather=fused, keep_intermediates=True)
+    res = O.hsa_step(inp, cfg.B, cfg.K_p)
+    assert_close(inter["k_til"], res["k_til"], dkey(cfg), f"{cfg.name} step per-head K~")
+    assert_close(out, res["o"], dkey(cfg), f"{cfg.name} step O (per-head E, {'fused' if fused else 'gathered'})")
     check_device_ok(wa)
 
 
@@ -396,6 +427,13 @@ def test_hsa_step_inter_granularity_small(wa, cfg, intra, fused):
                       res["block_margin"], f"{cfg.name} masks (B_inter 128)")
     assert_close(out, res["o"], dkey(cfg), f"{cfg.name} step O (B_inter 128, {'intra' if intra else 'history'})")
     check_device_ok(wa)
+
+
+def test_full_size_layer_step_per_head_projection(wa):
+    """C1 with one E_K / E_V pair per head (12 x 49,920 x 256 each)."""
+    cfg = W.C1.with_(name="c1_e_per_head", e_per_head=True)
+    samples = [(0, 0), (11, cfg.n_qb - 1), (7, 21)]
+    _full_size_step(wa, cfg, samples)
 
 
 def test_full_size_stress_step(wa):
