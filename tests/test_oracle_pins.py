@@ -570,3 +570,15 @@ def test_linear_branch_per_head_identity_is_dense_attention():
     o = O.linear_attention(q, kt, vt)
     for h in range(H):
         np.testing.assert_allclose(o[:, h], sdpa(q[:, h], k[:, h], v[:, h]), rtol=1e-12, atol=1e-12)
+
+
+def test_linear_project_per_head_copies_equal_shared():
+    """A per-head E whose heads all hold the same matrix is the shared projection."""
+    r = rng(43)
+    L, H, d, rr = 11, 3, 4, 5
+    k = r.normal(size=(L, H, d)); v = r.normal(size=(L, H, d))
+    EK = r.normal(size=(L, rr)); EV = r.normal(size=(L, rr))
+    kt_s, vt_s = O.linear_project(k, v, EK, EV)
+    kt_h, vt_h = O.linear_project(k, v, np.stack([EK] * H), np.stack([EV] * H))
+    np.testing.assert_allclose(kt_h, kt_s, rtol=1e-13, atol=1e-13)
+    np.testing.assert_allclose(vt_h, vt_s, rtol=1e-13, atol=1e-13)
