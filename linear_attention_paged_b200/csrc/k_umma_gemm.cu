@@ -202,21 +202,36 @@ k_umma_project(const __grid_constant__ CUtensorMap tmEK, const __grid_constant__
 }
 
 // out_m[c][n] = bf16( sum_{split} part[m][split][c][n] ), splits summed in order.
-__global__ void k_reduce_splits(const float* __restrict__ part, int n_split, size_t per_m,
-                                __nv_bfloat16* __restrict__ out_k, __nv_bfloat16* __restrict__ out_v) {
+// One float4 per thread; the split loads are issued kBatch at a time (independent,
+// so they overlap) and added in split order.
+constexpr int kReduceThreads = 256;
+__global__ void __launch_bounds__(kReduceThreads)
+k_reduce_splits(const float* __restrict__ part, int n_split, size_t per_m,
+                __nv_bfloat16* __restrict__ out_k, __nv_bfloat16* __restrict__ out_v) {
+  constexpr int kBatch = 8;
   const size_t n4 = per_m / 4;
-  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < 2 * n4;
-       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
-    const int m = i >= n4;
-    const size_t e = (i - m * n4) * 4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int s = 0; s < n_split; ++s) {
-      const float4 v = *reinterpret_cast<const float4*>(part + (static_cast<size_t>(m) * n_split + s) * per_m + e);
-      acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
-    }
-    __nv_bfloat16* o = (m ? out_v : out_k) + e;
-    *reinterpret_cast<uint2*>(o) = make_uint2(sm100::pack_bf16x2(acc.x, acc.y), sm100::pack_bf16x2(acc.z, acc.w));
+  const size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x;
+  if (i >= 2 * n4) return;
+  const int m = i >= n4;
+  const size_t e = (i - m * n4) * 4;
+  const float* src = part + static_cast<size_t>(m) * n_split * per_m + e;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int s0 = 0; s0 < n_split; s0 += kBatch) {
+    float4 v[kBatch];
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b)
+      if (s0 + b < n_split) v[b] = __ldcs(reinterpret_cast<const float4*>(src + (s0 + b) * per_m));
+#pragma unroll
+    for (int b = 0; b < kBatch; ++b)
+      if (s0 + b < n_split) { acc.x += v[b].x; acc.y += v[b].y; acc.z += v[b].z; acc.w += v[b].w; }
   }
+  __nv_bfloat16* o = (m ? out_v : out_k) + e;
+  *reinterpret_cast<uint2*>(o) = make_uint2(sm100::pack_bf16x2(acc.x, acc.y), sm100::pack_bf16x2(acc.z, acc.w));
+}
+
+// one thread per float4 of the two outputs
+unsigned reduce_grid(size_t per_m) {
+  return static_cast<unsigned>((2 * (per_m / 4) + kReduceThreads - 1) / kReduceThreads);
 }
 
 int pick_tn(int cols) {
@@ -300,8 +315,9 @@ wa_status launch_umma_project(const void* k, const void* v, RowSource rs, const 
   wa_status s = check_launch("umma_project");
   if (s != WA_OK) return s;
   const size_t per_m = static_cast<size_t>(r) * cols;
-  k_reduce_splits<<<2 * 148, 256, 0, st>>>(part, n_split, per_m, static_cast<__nv_bfloat16*>(k_til),
-                                           static_cast<__nv_bfloat16*>(v_til));
+  k_reduce_splits<<<reduce_grid(per_m), kReduceThreads, 0, st>>>(part, n_split, per_m,
+                                                                  static_cast<__nv_bfloat16*>(k_til),
+                                                                  static_cast<__nv_bfloat16*>(v_til));
   return check_launch("reduce_splits");
 }
 
@@ -414,7 +430,8 @@ extern "C" wa_status wa_linear_project_noalloc(const void* k_act, const void* v_
   s = check_launch("umma_project (no-alloc)");
   if (s != WA_OK) return s;
   const size_t per_m = static_cast<size_t>(r) * cols;
-  k_reduce_splits<<<2 * 148, 256, 0, st>>>(part, n_split, per_m, static_cast<__nv_bfloat16*>(k_til),
-                                           static_cast<__nv_bfloat16*>(v_til));
+  k_reduce_splits<<<reduce_grid(per_m), kReduceThreads, 0, st>>>(part, n_split, per_m,
+                                                                  static_cast<__nv_bfloat16*>(k_til),
+                                                                  static_cast<__nv_bfloat16*>(v_til));
   return check_launch("reduce_splits (no-alloc)");
 }
