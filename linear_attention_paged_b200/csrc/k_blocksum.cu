@@ -230,114 +230,118 @@ k_block_sums(const __grid_constant__ PassArgs a, uint32_t* err) {
 }
 
 // ------------------------------------------------------------------ page scores
-// Grid (column slice cs of kAlphaCols columns, role y).  y == 0: Qbar for the slice
-// (sum of the query block sums / Nq; also written out, with the query block means).
-// y = 1 + j * kAlphaSplits + p: the sum over blocks [p*nbp/S, (p+1)*nbp/S) of page j's
-// block sums for the slice (a column-sum part).  Each CTA's threads take the blocks in
-// kAlphaGroups strided groups, combined in order.  The last CTA of a slice forms the
-// slice's dot product of Qbar with every page's column sum (parts added in order);
-// the last slice to finish adds the slices in order, forms
+// One CTA per slice of kAlphaCols columns; thread (tx, gy) takes column tx of the
+// slice and the rows gy, gy + kAlphaGroups, ... of each sum it forms:
+//   Qbar for the slice (the query block sums added / Nq; also written out, with the
+//   query block means), then, kAlphaPages pages at a time, every candidate page's
+//   column sum over its block sums (page kpage[row][j], or position j), each combined
+//   over the row groups in order and dotted with Qbar over the slice -> partial[j][cs].
+// The last CTA to finish adds the slices in order, forms
 //   alpha_j = Qbar . colsum_j / (T_p sqrt(d) H)
 // and takes the top-K_p pages (ties -> lower position), emitted in ascending position.
-constexpr int kAlphaCols = 32;
-constexpr int kAlphaGroups = 8;
-constexpr int kAlphaSplits = 4;
+constexpr int kAlphaCols = 16;
+constexpr int kAlphaThreads = 512;
+constexpr int kAlphaGroups = kAlphaThreads / kAlphaCols;   // row groups
+constexpr int kAlphaPages = 8;                             // pages whose loads are in flight together
+constexpr int kAlphaBatch = 4;                             // blocks per page per thread per batch
 
-__global__ void __launch_bounds__(kAlphaCols * kAlphaGroups)
+__global__ void __launch_bounds__(kAlphaThreads)
 k_page_alpha(const double* __restrict__ qsum, int n_qb, int Nq, int B, int cols,
              const double* __restrict__ ksum, const int32_t* __restrict__ kpage, int n_pages,
              int nbp, const int32_t* __restrict__ cand, const int32_t* __restrict__ chunk,
              int n_chunks, int n_c, int T_p, int H, int d, int K_p, double* __restrict__ qbar,
-             double* __restrict__ qmean, double* __restrict__ colpart, double* __restrict__ partial,
-             unsigned* counters, double* __restrict__ alpha, int32_t* __restrict__ sel,
-             int32_t* __restrict__ sel_pos, uint32_t* err) {
-  __shared__ double red[kAlphaGroups][kAlphaCols];
+             double* __restrict__ qmean, double* __restrict__ partial, unsigned* counter,
+             double* __restrict__ alpha, int32_t* __restrict__ sel, int32_t* __restrict__ sel_pos,
+             uint32_t* err) {
+  extern __shared__ double red[];            // [kAlphaPages][kAlphaGroups][kAlphaCols]
+  __shared__ double qb[kAlphaCols];
   __shared__ bool last;
-  extern __shared__ unsigned char chosen_sm[];   // [n_c], used by the last CTA
-  const int cs = blockIdx.x, y = blockIdx.y;
-  const int n_cs = gridDim.x;
+  const int cs = blockIdx.x, n_cs = gridDim.x;
   const int tx = threadIdx.x % kAlphaCols, gy = threadIdx.x / kAlphaCols;
   const int col = cs * kAlphaCols + tx;
   const bool cv = col < cols;
   const int lanei = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
   int row = chunk ? *chunk : 0;
   if (row < 0 || row >= n_chunks) row = 0;
-  double t = 0.0;
-  if (y == 0) {
+  // Qbar of the slice
+  {
+    double t = 0.0;
     if (cv)
       for (int i = gy; i < n_qb; i += kAlphaGroups) {
         const double v = qsum[static_cast<size_t>(i) * cols + col];
         t += v;
         if (qmean) qmean[static_cast<size_t>(i) * cols + col] = v / (min(Nq, (i + 1) * B) - i * B);
       }
-  } else {
-    const int j = (y - 1) / kAlphaSplits, p = (y - 1) % kAlphaSplits;
-    int page = j;
-    if (kpage) {
-      page = kpage[static_cast<size_t>(row) * n_c + j];
-      if (page < 0 || page >= n_pages) {
-        if (threadIdx.x == 0 && cs == 0 && p == 0) atomicOr(err, WA_DEVERR_PAGE_ID);
-        page = 0;
-      }
-    }
-    const int b0 = static_cast<int>(static_cast<long long>(p) * nbp / kAlphaSplits);
-    const int b1 = static_cast<int>(static_cast<long long>(p + 1) * nbp / kAlphaSplits);
-    const double* kp = ksum + static_cast<size_t>(page) * nbp * cols;
-    if (cv) {
-      // independent loads first (many in flight), then the adds in block order
-      constexpr int kBatch = 8;
-      for (int bb = b0 + gy; bb < b1; bb += kBatch * kAlphaGroups) {
-        double v[kBatch];
-#pragma unroll
-        for (int e = 0; e < kBatch; ++e) {
-          const int b = bb + e * kAlphaGroups;
-          v[e] = b < b1 ? kp[static_cast<size_t>(b) * cols + col] : 0.0;
-        }
-#pragma unroll
-        for (int e = 0; e < kBatch; ++e) t += v[e];
-      }
-    }
-  }
-  red[gy][tx] = t;
-  __syncthreads();
-  if (gy == 0) {
-    double s = 0.0;
-    for (int g = 0; g < kAlphaGroups; ++g) s += red[g][tx];
-    if (y == 0) {
+    red[gy * kAlphaCols + tx] = t;
+    __syncthreads();
+    if (gy == 0) {
+      double s = 0.0;
+      for (int g = 0; g < kAlphaGroups; ++g) s += red[g * kAlphaCols + tx];
       s /= Nq;
+      qb[tx] = cv ? s : 0.0;
       if (cv) qbar[col] = s;
     }
-    // Qbar of the slice (y == 0) or a column-sum part, in [y][col]
-    colpart[static_cast<size_t>(y) * n_cs * kAlphaCols + col] = s;
+    __syncthreads();
   }
-  __threadfence();
-  __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(&counters[1 + cs], 1u) == gridDim.y - 1;
-  __syncthreads();
-  if (!last) return;
-  __threadfence();
-  // the last CTA of the slice: the slice's dot product for every page
-  const double* qb = colpart + static_cast<size_t>(cs) * kAlphaCols;   // y == 0 row
-  for (int j = warp; j < n_c; j += nw) {
-    double dot = 0.0;
-    if (cs * kAlphaCols + lanei < cols) {
-      double c = 0.0;
-      for (int p = 0; p < kAlphaSplits; ++p)
-        c += __ldcg(colpart + static_cast<size_t>(1 + j * kAlphaSplits + p) * n_cs * kAlphaCols +
-                    cs * kAlphaCols + lanei);
-      dot = c * __ldcg(qb + lanei);
+  // the pages' column sums, kAlphaPages at a time; each thread issues the loads of
+  // kAlphaBatch of its blocks for every page of the group before adding them (in
+  // block order)
+  for (int j0 = 0; j0 < n_c; j0 += kAlphaPages) {
+    const double* kp[kAlphaPages];
+#pragma unroll
+    for (int jj = 0; jj < kAlphaPages; ++jj) {
+      const int j = j0 + jj;
+      int page = j < n_c ? j : 0;
+      if (kpage && j < n_c) {
+        page = kpage[static_cast<size_t>(row) * n_c + j];
+        if (page < 0 || page >= n_pages) {
+          if (threadIdx.x == 0 && cs == 0) atomicOr(err, WA_DEVERR_PAGE_ID);
+          page = 0;
+        }
+      }
+      kp[jj] = (j < n_c && cv) ? ksum + static_cast<size_t>(page) * nbp * cols + col : nullptr;
+    }
+    double acc[kAlphaPages];
+#pragma unroll
+    for (int jj = 0; jj < kAlphaPages; ++jj) acc[jj] = 0.0;
+    for (int b0 = gy; b0 < nbp; b0 += kAlphaBatch * kAlphaGroups) {
+      double v[kAlphaPages][kAlphaBatch];
+#pragma unroll
+      for (int jj = 0; jj < kAlphaPages; ++jj)
+#pragma unroll
+        for (int e = 0; e < kAlphaBatch; ++e) {
+          const int b = b0 + e * kAlphaGroups;
+          v[jj][e] = (kp[jj] && b < nbp) ? kp[jj][static_cast<size_t>(b) * cols] : 0.0;
+        }
+#pragma unroll
+      for (int jj = 0; jj < kAlphaPages; ++jj)
+#pragma unroll
+        for (int e = 0; e < kAlphaBatch; ++e) acc[jj] += v[jj][e];
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    if (lanei == 0) partial[static_cast<size_t>(j) * n_cs + cs] = dot;
+    for (int jj = 0; jj < kAlphaPages; ++jj) red[(jj * kAlphaGroups + gy) * kAlphaCols + tx] = acc[jj];
+    __syncthreads();
+    // warp jj: page j0 + jj; lanes 0-15 combine the row groups of one column each
+    if (warp < kAlphaPages && j0 + warp < n_c) {
+      double dot = 0.0;
+      if (lanei < kAlphaCols) {
+        double c = 0.0;
+        for (int g = 0; g < kAlphaGroups; ++g) c += red[(warp * kAlphaGroups + g) * kAlphaCols + lanei];
+        dot = c * qb[lanei];
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
+      if (lanei == 0) partial[static_cast<size_t>(j0 + warp) * n_cs + cs] = dot;
+    }
+    __syncthreads();
   }
   __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) last = atomicAdd(&counters[0], 1u) == static_cast<unsigned>(n_cs) - 1;
+  if (threadIdx.x == 0) last = atomicAdd(counter, 1u) == static_cast<unsigned>(n_cs) - 1;
   __syncthreads();
   if (!last) return;
   __threadfence();
-  // the last slice: alpha for every page, then the top-K_p
+  // the last CTA: alpha for every page, then the top-K_p
   const double den = static_cast<double>(T_p) * sqrt(static_cast<double>(d)) * H;
   for (int c = warp; c < n_c; c += nw) {
     // lane l adds slices l, l + 32, ... in order, then a fixed butterfly
@@ -348,7 +352,8 @@ k_page_alpha(const double* __restrict__ qsum, int n_qb, int Nq, int B, int cols,
     for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     if (lanei == 0) alpha[c] = s / den;
   }
-  unsigned char* chosen = chosen_sm;   // [n_c]
+  unsigned char* chosen = reinterpret_cast<unsigned char*>(red);   // [n_c], reuses the reduction buffer
+  __syncthreads();
   for (int c = threadIdx.x; c < n_c; c += blockDim.x) chosen[c] = 0;
   __syncthreads();
   if (warp != 0) return;
@@ -379,9 +384,11 @@ k_page_alpha(const double* __restrict__ qsum, int n_qb, int Nq, int B, int cols,
         if (sel_pos) sel_pos[k] = c;
         ++k;
       }
-    for (int i = 0; i <= n_cs; ++i) counters[i] = 0u;
+    *counter = 0u;
   }
 }
+
+constexpr size_t kAlphaSmem = static_cast<size_t>(kAlphaPages) * kAlphaGroups * kAlphaCols * sizeof(double);
 
 int g_n_sm = 0;
 int n_sm() {
@@ -459,11 +466,10 @@ wa_status launch_block_sums(wa_dtype dt, int cols, int B, const BlockSumSeg* seg
 
 size_t page_alpha_scratch_doubles(int cols, int n_c) {
   const size_t n_cs = (cols + kAlphaCols - 1) / kAlphaCols;
-  // column parts [1 + n_c * splits][n_cs * kAlphaCols] and slice dots [n_c][n_cs]
-  return (1 + static_cast<size_t>(n_c) * kAlphaSplits) * n_cs * kAlphaCols + static_cast<size_t>(n_c) * n_cs;
+  return static_cast<size_t>(n_c) * n_cs;   // slice dots [n_c][n_cs]
 }
 
-int page_alpha_counters(int cols) { return 1 + (cols + kAlphaCols - 1) / kAlphaCols; }
+int page_alpha_counters(int) { return 1; }
 
 wa_status launch_page_alpha(const double* qsum, int n_qb, int Nq, int B, int cols, const double* ksum,
                             const int32_t* kpage, int n_pages, int nbp, const int32_t* cand,
@@ -471,15 +477,15 @@ wa_status launch_page_alpha(const double* qsum, int n_qb, int Nq, int B, int col
                             int K_p, double* qbar, double* qmean, double* scratch, unsigned* counters,
                             double* alpha, int32_t* sel, int32_t* sel_pos, uint32_t* err,
                             cudaStream_t st) {
+  if (static_cast<size_t>(n_c) > kAlphaSmem)
+    return set_error(WA_ERR_UNSUPPORTED, "page scores: too many candidate pages");
   const int n_cs = (cols + kAlphaCols - 1) / kAlphaCols;
-  const long long gy = 1 + static_cast<long long>(n_c) * kAlphaSplits;
-  if (gy > 65535) return set_error(WA_ERR_UNSUPPORTED, "page scores: too many candidate pages");
-  double* colpart = scratch;
-  double* partial = scratch + (1 + static_cast<size_t>(n_c) * kAlphaSplits) * n_cs * kAlphaCols;
-  dim3 grid(n_cs, static_cast<unsigned>(gy));
-  k_page_alpha<<<grid, kAlphaCols * kAlphaGroups, n_c, st>>>(
+  cudaError_t e = cudaFuncSetAttribute(k_page_alpha, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kAlphaSmem));
+  if (e != cudaSuccess) return set_error(WA_ERR_CUDA, "page scores smem attr: %s", cudaGetErrorString(e));
+  k_page_alpha<<<n_cs, kAlphaThreads, kAlphaSmem, st>>>(
       qsum, n_qb, Nq, B, cols, ksum, kpage, n_pages, nbp, cand, chunk, n_chunks, n_c, T_p, H, d, K_p,
-      qbar, qmean, colpart, partial, counters, alpha, sel, sel_pos, err);
+      qbar, qmean, scratch, counters, alpha, sel, sel_pos, err);
   return check_launch("page_alpha");
 }
 
