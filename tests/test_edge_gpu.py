@@ -7,7 +7,9 @@ oracle (every row compared):
     page table from global memory instead of staging it in shared memory;
   * the largest key list the library takes, 8192 key blocks (524,288 keys), with pages
     of 2048 blocks: the key-list scan, the block-selection sort of 8192 scores and
-    the 256-word masks at their maximum.
+    the 256-word masks at their maximum;
+  * the smallest steps: one query row over one key block of one page (bf16 and
+    fp32), and a query tail of a single row.
 """
 import pytest
 import torch
@@ -15,7 +17,7 @@ import torch
 from oracle import hsa_oracle as O
 from linear_attention_paged_b200 import workloads as W
 from tests.helpers import MARGIN_F64, assert_close, compare_selection, mask_to_sets
-from tests.test_parity_gpu import check_device_ok
+from tests.test_parity_gpu import check_device_ok, dkey
 
 pytestmark = pytest.mark.gpu
 
@@ -39,8 +41,8 @@ def _check_step(wa, cfg, fused=True):
         assert inter["sel"].cpu().tolist() == res["sel"]
     compare_selection(mask_to_sets(inter["blk_mask"], cfg.n_kb), res["kept"], res["block_margin"],
                       f"{cfg.name} masks")
-    assert_close(inter["k_til"], res["k_til"], "bf16", f"{cfg.name} K~")
-    assert_close(out, res["o"], "bf16", f"{cfg.name} O ({'fused' if fused else 'gathered'})")
+    assert_close(inter["k_til"], res["k_til"], dkey(cfg), f"{cfg.name} K~")
+    assert_close(out, res["o"], dkey(cfg), f"{cfg.name} O ({'fused' if fused else 'gathered'})")
     check_device_ok(wa)
     return res
 
@@ -72,3 +74,19 @@ def test_step_at_the_largest_key_list(wa):
     res = _check_step(wa, cfg)
     kept = [len(row) for row in res["kept"][0]]
     print(f"[info] {cfg.name}: kept blocks per query block {kept} of {cfg.n_kb}")
+
+
+SMALLEST = [
+    W.HSAConfig("edge_one_query", H=1, d=64, T_p=64, n_c=1, Nq=1, K_p=1, B=64, r=128, dtype="bf16",
+                seed=54, recipe="offset"),
+    W.HSAConfig("edge_one_row_tail", H=1, d=128, T_p=128, n_c=2, Nq=65, K_p=1, B=64, r=128,
+                dtype="bf16", seed=55, recipe="offset"),
+    W.HSAConfig("edge_one_query_f32", H=1, d=64, T_p=64, n_c=1, Nq=1, K_p=1, B=64, r=8, dtype="f32",
+                seed=56, recipe="gauss", tau_const=0.9),
+]
+
+
+@pytest.mark.parametrize("fused", [True, False], ids=["fused", "gathered"])
+@pytest.mark.parametrize("cfg", SMALLEST, ids=lambda c: c.name)
+def test_smallest_steps(wa, cfg, fused):
+    _check_step(wa, cfg, fused)
