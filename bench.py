@@ -22,8 +22,9 @@ the launching stream), the roofline of the dominant kernel (the block-sparse
 attention, counting selected-block FLOPs only), the HBM fraction of the page
 scoring pass, an end-to-end number through the public API with pinned host
 buffers (H2D of the step's q and gate, D2H of its output, inside the timed
-region), the clock record, and the fp64 oracle timed on the host cores on a
-bounded sample of the same workload (rank 0, N=1 only).
+region), the clock record, the same step with two gates, the page tier's
+host-to-device rate, and the fp64 oracle timed on the host cores on a bounded
+sample of the same workload (rank 0, N=1 only).
 
 --impl reference times that oracle alone (the reference arm: the method is
 described only in prose, so there is no upstream implementation to install).
@@ -396,6 +397,28 @@ def run_ours(args, rank, world, local_rank):
         del kc
     del ka, va
 
+    # two-gate fusion (O = G_lin * O_lin + G_sp * O_sp, gates from independent logits):
+    # the same step with a second, seeded gate
+    two_gate_ms = None
+    if not cfg.intra and not args.b_inter:
+        g_lin = torch.randn(inp["gate"].shape, generator=torch.Generator().manual_seed(cfg.seed + 6)).to(dev)
+        step2 = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"],
+                           inp["e_v"], tau, inp["gate"], cfg.K_p, cfg.B, fused_gather=True, gate_lin=g_lin)
+        for _ in range(3):
+            step2()
+        ts_, te_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ts_.record(stream)
+        for _ in range(n_g):
+            step2()
+        te_.record(stream)
+        torch.cuda.synchronize()
+        two_gate_ms = ts_.elapsed_time(te_) / n_g
+        del step2, g_lin
+
+    # L1 <-> L2 page tier: the candidate pages in pinned host memory, K_p device slots;
+    # each request brings in K_p pages that are not resident (host -> device copies)
+    tier = tier_measure(inp, cfg, dev, stream)
+
     # the full denoise stack (spec config 5) on the same GPU, after the one-layer
     # figures: every rank runs its own stack
     c4 = None
@@ -443,6 +466,9 @@ def run_ours(args, rank, world, local_rank):
                                   "achieved": perm_gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                                   "frac": perm_gbs / float(peaks["hbm_gbs"]), "bytes_per_launch": perm_bytes,
                                   "ms_per_launch": perm_ms} if perm_ms else None),
+            "two_gate_step": ({"ms_per_step": two_gate_ms, "frames_per_s": frames_per_s(two_gate_ms),
+                               "steps": n_g} if two_gate_ms else None),
+            "page_tier": tier,
             "stage_ms": {k: round(v, 4) for k, v in stage_ms.items()},
             "e2e": ({"value": frames_per_s(e2e_ms, world), "unit": "frames/s", "ms_per_step": e2e_ms,
                      "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
@@ -463,6 +489,47 @@ def run_ours(args, rank, world, local_rank):
         }
         print(json.dumps(line), flush=True)
     return 0
+
+
+def tier_measure(inp, cfg, dev, stream, rounds=4):
+    """Host -> device page traffic of the L1 <-> L2 tier: the n_c candidate pages in
+    pinned host memory, K_p device slots, requests alternating between two disjoint
+    sets of K_p pages so that every request misses; GB/s of page bytes moved."""
+    from linear_attention_paged_b200 import wa
+    n_pages = cfg.n_c
+    if n_pages < 2 * cfg.K_p:
+        return None
+    shape = tuple(inp["k_pool"].shape[1:])
+    host_k = torch.empty((n_pages,) + shape, dtype=inp["k_pool"].dtype).pin_memory()
+    host_v = torch.empty_like(host_k).pin_memory()
+    host_k.copy_(inp["k_pool"][:n_pages])
+    host_v.copy_(inp["v_pool"][:n_pages])
+    slot_k = torch.empty((cfg.K_p,) + shape, dtype=host_k.dtype, device=dev)
+    slot_v = torch.empty_like(slot_k)
+    t = wa.Tier(host_k, host_v, slot_k, slot_v)
+    sets = [list(range(cfg.K_p)), list(range(cfg.K_p, 2 * cfg.K_p))]
+    t.ensure(sets[1], stream)
+    t.release(stream)
+    torch.cuda.synchronize()
+    page_bytes = 2 * host_k[0].numel() * host_k.element_size()
+    ms = []
+    for r in range(rounds):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        t.ensure(sets[r % 2], stream)
+        e1.record(stream)
+        t.release(stream)
+        torch.cuda.synchronize()
+        ms.append(e0.elapsed_time(e1))
+    stats = t.stats()
+    t.close()
+    moved = cfg.K_p * page_bytes
+    return {"what": f"wa_tier_ensure of {cfg.K_p} non-resident pages (K and V) from pinned host memory "
+                    f"into device slots, {rounds} requests alternating between two page sets",
+            "bytes_per_request": moved, "ms_per_request": sum(ms) / len(ms), "ms_best": min(ms),
+            "achieved_gbs": moved / (sum(ms) / len(ms) * 1e-3) / 1e9, "unit": "GB/s",
+            "pcie_gen5_x16_nominal_gbs": 64.0, "misses": stats["misses"], "hits": stats["hits"],
+            "bytes_h2d": stats["bytes_h2d"]}
 
 
 def c4_measure(args, rank, world, local_rank):
