@@ -6,7 +6,7 @@
 // and the page scores alpha_j = (1/H) sum_h Qbar_h . Kbar_{h,j} / sqrt(d) with the
 // top-K_p pages, formed from those sums.
 //
-// The pass streams every block once.  Each CTA is persistent (two per SM) and walks
+// The pass streams every block once.  Each CTA is persistent (three per SM) and walks
 // a fixed list of blocks; one producer thread copies each block, a few rows at a
 // time, into a ring of shared-memory stages with cp.async.bulk (the rows of a block
 // are contiguous in memory, so one bulk copy moves whole rows), and the consumer
