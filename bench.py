@@ -22,9 +22,9 @@ the launching stream), the roofline of the dominant kernel (the block-sparse
 attention, counting selected-block FLOPs only), the HBM fraction of the page
 scoring pass, an end-to-end number through the public API with pinned host
 buffers (H2D of the step's q and gate, D2H of its output, inside the timed
-region), the clock record, the same step with two gates, the page tier's
-host-to-device rate, and the fp64 oracle timed on the host cores on a bounded
-sample of the same workload (rank 0, N=1 only).
+region), the clock record, the same step with two gates and over a 120-page pool
+(long history), the page tier's host-to-device rate, and the fp64 oracle timed on
+the host cores on a bounded sample of the same workload (rank 0, N=1 only).
 
 --impl reference times that oracle alone (the reference arm: the method is
 described only in prose, so there is no upstream implementation to install).
@@ -419,6 +419,13 @@ def run_ours(args, rank, world, local_rank):
     # each request brings in K_p pages that are not resident (host -> device copies)
     tier = tier_measure(inp, cfg, dev, stream)
 
+    # long history (config 4 of the workloads): a 120-page pool, the candidate chunk
+    # chosen by prompt embeddings, then the same step; its time against C1's shows
+    # whether retrieval grows with the history
+    c3 = None
+    if not args.no_c3 and args.heads is None and not args.intra and not args.b_inter:
+        c3 = c3_measure(dev, stream, n_g)
+
     # the full denoise stack (spec config 5) on the same GPU, after the one-layer
     # figures: every rank runs its own stack
     c4 = None
@@ -466,6 +473,7 @@ def run_ours(args, rank, world, local_rank):
                                   "achieved": perm_gbs, "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                                   "frac": perm_gbs / float(peaks["hbm_gbs"]), "bytes_per_launch": perm_bytes,
                                   "ms_per_launch": perm_ms} if perm_ms else None),
+            "c3_long_history": c3,
             "two_gate_step": ({"ms_per_step": two_gate_ms, "frames_per_s": frames_per_s(two_gate_ms),
                                "steps": n_g} if two_gate_ms else None),
             "page_tier": tier,
@@ -489,6 +497,45 @@ def run_ours(args, rank, world, local_rank):
         }
         print(json.dumps(line), flush=True)
     return 0
+
+
+def c3_measure(dev, stream, n_steps):
+    """The step over a 120-page pool (15 chunks of 8 pages, 9.2 GB of K and V) with
+    the candidate chunk picked by cosine similarity of prompt embeddings (S0)."""
+    from linear_attention_paged_b200 import wa, workloads as W
+    cfg = W.C3
+    inp = W.make_inputs(cfg, device="cuda", gen_device="cuda")
+    step = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"], inp["e_v"],
+                      inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B, e_cur=inp["e_cur"],
+                      e_chunks=inp["e_chunks"], fused_gather=True)
+    for _ in range(3):
+        step()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
+    for e in ev:
+        e.record(stream)
+    torch.cuda.synchronize()
+    arr, keep = ctypes_void_array(ev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n_steps):
+        step()
+    e1.record(stream)
+    step.args.stage_events = arr     # one more step with stage events, outside the timing
+    step()
+    step.args.stage_events = None
+    torch.cuda.synchronize()
+    flags = wa.wa_device_error()
+    if flags:
+        raise RuntimeError(f"device error flags 0x{flags:x}")
+    ms = e0.elapsed_time(e1) / n_steps
+    pool_bytes = 2 * inp["k_pool"].numel() * inp["k_pool"].element_size()
+    del step, inp, keep
+    torch.cuda.empty_cache()
+    return {"workload": f"{cfg.name}: C1 shapes over a pool of {cfg.n_pool_pages} pages "
+                        f"({pool_bytes / 1e9:.1f} GB of K and V), prompt embeddings of {cfg.prompt_dim} "
+                        f"pick the candidate chunk among {cfg.n_chunks}",
+            "ms_per_step": ms, "frames_per_s": frames_per_s(ms), "steps": n_steps,
+            "page_retrieval_ms": ev[0].elapsed_time(ev[1])}
 
 
 def tier_measure(inp, cfg, dev, stream, rounds=4):
@@ -668,6 +715,8 @@ def main():
     ap.add_argument("--layers", type=int, default=30, help="c4: layers")
     ap.add_argument("--no-c4", action="store_true",
                     help="c1: skip the full denoise stack figure added to the line")
+    ap.add_argument("--no-c3", action="store_true",
+                    help="c1: skip the long-history (120-page pool) figure added to the line")
     ap.add_argument("--b-inter", type=int, default=0, choices=[0, 64, 128],
                     help="c1: block size of the history in block selection (128: inter-chunk "
                          "granularity; the chunk's own keys keep 64)")
