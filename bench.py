@@ -22,9 +22,10 @@ the launching stream), the roofline of the dominant kernel (the block-sparse
 attention, counting selected-block FLOPs only), the HBM fraction of the page
 scoring pass, an end-to-end number through the public API with pinned host
 buffers (H2D of the step's q and gate, D2H of its output, inside the timed
-region), the clock record, the same step with two gates and over a 120-page pool
-(long history), the page tier's host-to-device rate, and the fp64 oracle timed on
-the host cores on a bounded sample of the same workload (rank 0, N=1 only).
+region), the clock record, the same step with two gates, over a 120-page pool
+(long history) and on the head-adaptive stress inputs, the page tier's
+host-to-device rate, and the fp64 oracle timed on the host cores on a bounded
+sample of the same workload (rank 0, N=1 only).
 
 --impl reference times that oracle alone (the reference arm: the method is
 described only in prose, so there is no upstream implementation to install).
@@ -51,9 +52,10 @@ from linear_attention_paged_b200 import replicas  # noqa: E402
 
 METRIC = "HSA ms/chunk-layer & attention frames/s; % of BF16 tensor / HBM roofline"
 # DRAM bytes per launch of the sparse-branch attention kernel per head, from one ncu
-# capture of the 6-head C1 launch with work items grouped by two heads (161.5 MB read +
-# 15.0 MB written) / 6; set to None when the kernel or its item order changes
-ATTN_DRAM_BYTES_PER_HEAD = (161521408 + 14956544) / 6
+# capture of the 6-head C1 launch with the work items longest first over all heads
+# (332.2 MB read + 22.2 MB written) / 6; set to None when the kernel or its item order
+# changes
+ATTN_DRAM_BYTES_PER_HEAD = (332163328 + 22242560) / 6
 FRAMES_PER_CHUNK = 3
 CHUNK_LAYERS_PER_CHUNK = 30 * 4
 # stage -> (start event, end event) of the events wa_hsa_step records; the
@@ -422,9 +424,15 @@ def run_ours(args, rank, world, local_rank):
     # long history (config 4 of the workloads): a 120-page pool, the candidate chunk
     # chosen by prompt embeddings, then the same step; its time against C1's shows
     # whether retrieval grows with the history
-    c3 = None
+    c3 = c2 = None
     if not args.no_c3 and args.heads is None and not args.intra and not args.b_inter:
-        c3 = c3_measure(dev, stream, n_g)
+        c3 = config_measure(W.C3, dev, stream, n_g, peak_t)
+        c3["workload"] = (f"{W.C3.name}: one-layer shapes over a pool of {W.C3.n_pool_pages} pages "
+                          f"({c3['pool_gb']:.1f} GB of K and V); prompt embeddings of {W.C3.prompt_dim} "
+                          f"pick the candidate chunk among {W.C3.n_chunks}")
+        c2 = config_measure(W.C2, dev, stream, n_g, peak_t)
+        c2["workload"] = (f"{W.C2.name}: one-layer shapes, Student-t values, 1-32 planted hot key "
+                          f"blocks per head, tau_h ~ U[0.5, 0.99] (kept fractions from about 1 % to 100 %)")
 
     # the full denoise stack (spec config 5) on the same GPU, after the one-layer
     # figures: every rank runs its own stack
@@ -474,6 +482,7 @@ def run_ours(args, rank, world, local_rank):
                                   "frac": perm_gbs / float(peaks["hbm_gbs"]), "bytes_per_launch": perm_bytes,
                                   "ms_per_launch": perm_ms} if perm_ms else None),
             "c3_long_history": c3,
+            "c2_head_adaptive_stress": c2,
             "two_gate_step": ({"ms_per_step": two_gate_ms, "frames_per_s": frames_per_s(two_gate_ms),
                                "steps": n_g} if two_gate_ms else None),
             "page_tier": tier,
@@ -499,15 +508,15 @@ def run_ours(args, rank, world, local_rank):
     return 0
 
 
-def c3_measure(dev, stream, n_steps):
-    """The step over a 120-page pool (15 chunks of 8 pages, 9.2 GB of K and V) with
-    the candidate chunk picked by cosine similarity of prompt embeddings (S0)."""
+def config_measure(cfg, dev, stream, n_steps, peak_t):
+    """The step on another full-size workload (the long-history pool with prompt-level
+    chunk selection, or the head-adaptive stress inputs): ms per step, and the sparse
+    branch's selected-block FLOP rate from one more step with stage events."""
     from linear_attention_paged_b200 import wa, workloads as W
-    cfg = W.C3
     inp = W.make_inputs(cfg, device="cuda", gen_device="cuda")
     step = wa.HSAStep(inp["q"], inp["k_pool"], inp["v_pool"], inp["chunk_pages"], inp["e_k"], inp["e_v"],
-                      inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B, e_cur=inp["e_cur"],
-                      e_chunks=inp["e_chunks"], fused_gather=True)
+                      inp["tau"].cuda(), inp["gate"], cfg.K_p, cfg.B, e_cur=inp.get("e_cur"),
+                      e_chunks=inp.get("e_chunks"), fused_gather=True, keep_intermediates=True)
     for _ in range(3):
         step()
     ev = [torch.cuda.Event(enable_timing=True) for _ in range(8)]
@@ -528,14 +537,16 @@ def c3_measure(dev, stream, n_steps):
     if flags:
         raise RuntimeError(f"device error flags 0x{flags:x}")
     ms = e0.elapsed_time(e1) / n_steps
+    flops, kept = selected_flops(step.inter["blk_mask"], cfg)
+    attn_ms = ev[6].elapsed_time(ev[7])
     pool_bytes = 2 * inp["k_pool"].numel() * inp["k_pool"].element_size()
     del step, inp, keep
     torch.cuda.empty_cache()
-    return {"workload": f"{cfg.name}: C1 shapes over a pool of {cfg.n_pool_pages} pages "
-                        f"({pool_bytes / 1e9:.1f} GB of K and V), prompt embeddings of {cfg.prompt_dim} "
-                        f"pick the candidate chunk among {cfg.n_chunks}",
-            "ms_per_step": ms, "frames_per_s": frames_per_s(ms), "steps": n_steps,
-            "page_retrieval_ms": ev[0].elapsed_time(ev[1])}
+    return {"pool_gb": pool_bytes / 1e9, "ms_per_step": ms, "frames_per_s": frames_per_s(ms),
+            "steps": n_steps, "page_retrieval_ms": ev[0].elapsed_time(ev[1]),
+            "sparse_branch_gate_ms": attn_ms, "kept_fraction": kept,
+            "sparse_tflops": flops / (attn_ms * 1e-3) / 1e12,
+            "sparse_frac_of_peak": flops / (attn_ms * 1e-3) / 1e12 / peak_t}
 
 
 def tier_measure(inp, cfg, dev, stream, rounds=4):
@@ -716,7 +727,7 @@ def main():
     ap.add_argument("--no-c4", action="store_true",
                     help="c1: skip the full denoise stack figure added to the line")
     ap.add_argument("--no-c3", action="store_true",
-                    help="c1: skip the long-history (120-page pool) figure added to the line")
+                    help="c1: skip the long-history (120-page pool) and stress figures added to the line")
     ap.add_argument("--b-inter", type=int, default=0, choices=[0, 64, 128],
                     help="c1: block size of the history in block selection (128: inter-chunk "
                          "granularity; the chunk's own keys keep 64)")
