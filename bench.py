@@ -20,7 +20,7 @@ runs its own layer: weak scaling, no data-path collective).
 The JSON line also carries: per-stage ms (CUDA events recorded by the library on
 the launching stream), the roofline of the dominant kernel (the block-sparse
 attention, counting selected-block FLOPs only), the HBM fraction of the page
-scoring pass, an end-to-end number through the public API with pinned host
+retrieval stage and of its block-sum pass alone, an end-to-end number through the public API with pinned host
 buffers (H2D of the step's q and gate, D2H of its output, inside the timed
 region), the clock record, the same step with two gates, over a 120-page pool
 (long history) and on the head-adaptive stress inputs, the page tier's
@@ -378,6 +378,23 @@ def run_ours(args, rank, world, local_rank):
     gather_ms = gs.elapsed_time(ge) / n_g
     gather_bytes = 2 * 2 * ka.numel() * ka.element_size()
     gather_gbs = gather_bytes / (gather_ms * 1e-3) / 1e9
+    # S1's HBM pass on its own: the float64 block sums of the candidate pages (the same
+    # kernel the step runs, here through the page-index entry point), K read once
+    cand_pages = inp["chunk_pages"][0].to(torch.int32).contiguous()
+    pidx = torch.zeros((inp["k_pool"].shape[0], cfg.T_p // cfg.B, cfg.H, cfg.d), dtype=torch.float64,
+                       device=dev)
+    for _ in range(3):
+        wa.wa_pool_index(inp["k_pool"], cand_pages, cfg.B, page_index=pidx)
+    bs_, be_ = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    bs_.record(stream)
+    for _ in range(n_g):
+        wa.wa_pool_index(inp["k_pool"], cand_pages, cfg.B, page_index=pidx)
+    be_.record(stream)
+    torch.cuda.synchronize()
+    pass_ms = bs_.elapsed_time(be_) / n_g
+    pass_bytes = cand_pages.numel() * cfg.T_p * cfg.H * cfg.d * inp["k_pool"].element_size()
+    pass_gbs = pass_bytes / (pass_ms * 1e-3) / 1e9
+    del pidx
     # cube-tile token order: the active keys (K_p pages) re-ordered page by page into
     # (8, 2, 4) cubes of an 8-frame 30 x 52 latent page, one row gather over L rows
     perm_ms = perm_gbs = perm_bytes = None
@@ -473,6 +490,11 @@ def run_ours(args, rank, world, local_rank):
             "hbm_page_scoring": {"achieved": hbm_achieved, "peak": float(peaks["hbm_gbs"]),
                                  "unit": "GB/s", "frac": hbm_achieved / float(peaks["hbm_gbs"]),
                                  "bytes_per_launch": page_bytes},
+            "hbm_block_sum_pass": {"kernel": "k_block_sums over the candidate pages (S1's HBM pass, "
+                                             "through wa_pool_index)", "achieved": pass_gbs,
+                                   "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
+                                   "frac": pass_gbs / float(peaks["hbm_gbs"]),
+                                   "bytes_per_launch": pass_bytes, "ms_per_launch": pass_ms},
             "hbm_gather": {"kernel": "k_gather (non-fused S2)", "achieved": gather_gbs,
                            "peak": float(peaks["hbm_gbs"]), "unit": "GB/s",
                            "frac": gather_gbs / float(peaks["hbm_gbs"]), "bytes_per_launch": gather_bytes,
