@@ -20,12 +20,12 @@ runs its own layer: weak scaling, no data-path collective).
 The JSON line also carries: per-stage ms (CUDA events recorded by the library on
 the launching stream), the roofline of the dominant kernel (the block-sparse
 attention, counting selected-block FLOPs only), the HBM fraction of the page
-retrieval stage and of its block-sum pass alone, an end-to-end number through the public API with pinned host
-buffers (H2D of the step's q and gate, D2H of its output, inside the timed
-region), the clock record, the same step with two gates, over a 120-page pool
-(long history) and on the head-adaptive stress inputs, the page tier's
-host-to-device rate, and the fp64 oracle timed on the host cores on a bounded
-sample of the same workload (rank 0, N=1 only).
+retrieval stage and of its block-sum pass alone, an end-to-end number through the
+public API with pinned host buffers (H2D of the step's q and gate, D2H of its
+output, inside the timed region), the clock record, the same step with two gates,
+over a 120-page pool (long history) and on the head-adaptive stress inputs, the
+page tier's host-to-device rate, and the fp64 oracle timed on the host cores on a
+bounded sample of the same workload (rank 0, N=1 only).
 
 --impl reference times that oracle alone (the reference arm: the method is
 described only in prose, so there is no upstream implementation to install).
