@@ -109,10 +109,16 @@ bool make_tmap_bf16_2d(void* tmap, const void* base, uint64_t inner, uint64_t ou
 // A second stream (and the fork / join events) per host thread and device, on
 // which the decode step runs the projection and the linear branch concurrently with
 // block selection.  Created on first use; no device memory is allocated.
+// The step's internal streams: `stream` takes the projection and the linear branch;
+// `hi` (the device's highest stream priority) takes block selection and the work
+// list, so that when both have CTAs waiting for an SM the selection side, which the
+// sparse branch waits for first, is served first.
 struct SideStream {
   cudaStream_t stream = nullptr;
   cudaEvent_t fork = nullptr;
   cudaEvent_t join = nullptr;
+  cudaStream_t hi = nullptr;
+  cudaEvent_t hi_join = nullptr;
 };
 thread_local SideStream t_side[64];
 
@@ -122,9 +128,13 @@ wa_status side_stream(SideStream** out) {
     return set_error(WA_ERR_CUDA, "cudaGetDevice failed");
   SideStream& s = t_side[dev];
   if (!s.stream) {
+    int least = 0, greatest = 0;
+    cudaDeviceGetStreamPriorityRange(&least, &greatest);
     if (cudaStreamCreateWithFlags(&s.stream, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithPriority(&s.hi, cudaStreamNonBlocking, greatest) != cudaSuccess ||
         cudaEventCreateWithFlags(&s.fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess)
+        cudaEventCreateWithFlags(&s.join, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&s.hi_join, cudaEventDisableTiming) != cudaSuccess)
       return set_error(WA_ERR_CUDA, "could not create the side stream");
   }
   *out = &s;
@@ -812,8 +822,8 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
   lin.k = kt; lin.v = vt; lin.page_rows = a->r; lin.n_pages = 1; lin.L = a->r;
   if (a->dtype == WA_BF16) {
     // S4a + S4b (HBM-bound projection, then the linear branch) on a side stream,
-    // concurrently with S3 and the work list (latency-bound) on this stream; the
-    // sparse branch joins both.
+    // concurrently with S3 and the work list (latency-bound) on a high-priority one;
+    // the sparse branch, on this stream, joins both.
     SideStream* side = nullptr;
     WA_TRY(side_stream(&side));
     cudaEventRecord(side->fork, st);
@@ -829,11 +839,15 @@ wa_status wa_hsa_step(const wa_step_args* a, void* ws, size_t ws_bytes, void* st
                                    nullptr, err, side->stream));
     mark_side(5);
     cudaEventRecord(side->join, side->stream);
-    // S3: block selection
+    // S3: block selection, then the work list
+    cudaStreamWaitEvent(side->hi, side->fork, 0);
     WA_TRY(launch_block_select(w.ps.q_blockmean, a->Nq, a->H, a->d, a->B, km, n_sel, n_kb, a->tau,
-                               w.scores, nullptr, nullptr, mask, st));
-    mark(3);
-    WA_TRY(launch_attn_worklist(a->Nq, a->H, a->d, a->B, sparse_key_rows(a), mask, w.attn, st));
+                               w.scores, nullptr, nullptr, mask, side->hi));
+    if (a->stage_events && a->stage_events[3])
+      cudaEventRecord(static_cast<cudaEvent_t>(a->stage_events[3]), side->hi);
+    WA_TRY(launch_attn_worklist(a->Nq, a->H, a->d, a->B, sparse_key_rows(a), mask, w.attn, side->hi));
+    cudaEventRecord(side->hi_join, side->hi);
+    cudaStreamWaitEvent(st, side->hi_join, 0);
     cudaStreamWaitEvent(st, side->join, 0);
     mark(6);
     // S5 + S6
