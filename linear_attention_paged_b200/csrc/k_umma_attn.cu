@@ -765,7 +765,8 @@ k_pair_heads(const uint32_t* __restrict__ mask, int n_qb, int W, int4* __restric
 }
 
 // Two work items per pair -- both halves of a split key list, or the whole list
-// and an empty placeholder -- ordered longest first over all heads, by a counting
+// and an empty placeholder (placed after every real item, so that a launch over the
+// first n_pairs items covers them all) -- ordered longest first over all heads, by a counting
 // sort (order among equal lengths is arbitrary: it affects only the schedule, never a
 // result).  One CTA.  Ordering by head group first (so that a group's keys and values
 // stay in L2 while its items run) halved the launch's DRAM reads but made the sparse
@@ -781,9 +782,9 @@ k_make_items(const int4* __restrict__ pairs, int n_pairs, int shift, int split_m
   __shared__ int wsum[32];
   for (int e = threadIdx.x; e < kLenBins; e += blockDim.x) hist[e] = 0;
   __syncthreads();
-  // long first: the longest lists in the lowest bins; the last bin also takes the
-  // empty placeholders
-  auto bin_of = [&](int len) { return kLenBins - 1 - min(kLenBins - 1, len >> shift); };
+  // long first: the longest lists in the lowest bins; the last bin holds only the
+  // empty placeholders, so every real item comes before them
+  auto bin_of = [&](int len) { return kLenBins - 2 - min(kLenBins - 2, len >> shift); };
   for (int p = threadIdx.x; p < n_pairs; p += blockDim.x) {
     const int cnt = pairs[p].w;
     if (cnt >= split_min) {
@@ -961,19 +962,23 @@ wa_status launch_attn_sparse(const void* q, int Nq, int H, int d, RowSource rs, 
   alignas(64) CUtensorMap tk, tv, tk2, tv2;
   wa_status e = make_maps(H, d, rs, &tk, &tv, &tk2, &tv2);
   if (e != WA_OK) return e;
-  const int grid = 2 * s.n_pairs;
   float* lin_rw = const_cast<float*>(lin_ws);
   const int split_min = split_min_for(s.n_pairs);
+  // nothing split: the first n_pairs items are the whole lists and no CTA combines
+  const bool split = split_min != INT_MAX;
+  const int grid = split ? 2 * s.n_pairs : s.n_pairs;
   if (d == 128) {
     launch_attn_kernel<128>(grid, st, q, tk, tv, tk2, tv2, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
                             s.part, gate, 0.f, lin_rw, out, o_sp, err);
-    k_combine<128><<<dim3(s.n_pairs, kBM / 32), 2 * 128, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate, lin_ws,
-                                                                  static_cast<__nv_bfloat16*>(out), o_sp);
+    if (split)
+      k_combine<128><<<dim3(s.n_pairs, kBM / 32), 2 * 128, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate,
+                                                                    lin_ws, static_cast<__nv_bfloat16*>(out), o_sp);
   } else {
     launch_attn_kernel<64>(grid, st, q, tk, tv, tk2, tv2, 1, Nq, H, rs, blk_mask, s.W, s.n_qb, s.pairs, s.items,
                            s.part, gate, 0.f, lin_rw, out, o_sp, err);
-    k_combine<64><<<dim3(s.n_pairs, kBM / 32), 2 * 64, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate, lin_ws,
-                                                                static_cast<__nv_bfloat16*>(out), o_sp);
+    if (split)
+      k_combine<64><<<dim3(s.n_pairs, kBM / 32), 2 * 64, 0, st>>>(s.pairs, s.part, Nq, H, split_min, gate,
+                                                                  lin_ws, static_cast<__nv_bfloat16*>(out), o_sp);
   }
   return check_launch("sparse attention");
 }
