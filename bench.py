@@ -284,10 +284,13 @@ def run_ours(args, rank, world, local_rank):
         raise RuntimeError(f"device error flags 0x{flags:x}")
     flops, kept_frac = selected_flops(step.inter["blk_mask"], cfg)
     # per step: the block-sum pass over the queries and candidate pages, page scores
-    # and top-k, block scores, block choice, pairing, work items, sparse attention and
-    # combine on the caller's stream; projection, split reduction and linear branch on
-    # the side stream
-    launches_per_step = 11 + (1 if cfg.intra else 0)   # + block sums of the chunk's keys
+    # and top-k, block scores, block choice, pairing, work items, the sparse attention
+    # and (when key lists are split, i.e. the tile pairs fill fewer than two waves of
+    # one CTA per SM) the combine; projection, split reduction and linear branch
+    n_pairs = cfg.H * ((cfg.n_qb + 1) // 2)
+    n_sm = torch.cuda.get_device_properties(dev).multi_processor_count
+    launches_per_step = (10 + (1 if n_pairs < 2 * n_sm else 0)
+                         + (1 if cfg.intra else 0))   # + block sums of the chunk's keys
 
     n_ev = 8  # WA_STEP_EVENTS
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(n_ev)] for _ in range(args.steps)]
