@@ -53,9 +53,9 @@ from linear_attention_paged_b200 import replicas  # noqa: E402
 METRIC = "HSA ms/chunk-layer & attention frames/s; % of BF16 tensor / HBM roofline"
 # DRAM bytes per launch of the sparse-branch attention kernel per head, from one ncu
 # capture of the 6-head C1 launch with the work items longest first over all heads
-# (332.2 MB read + 22.2 MB written) / 6; set to None when the kernel or its item order
+# (330.7 MB read + 22.6 MB written) / 6; set to None when the kernel or its item order
 # changes
-ATTN_DRAM_BYTES_PER_HEAD = (332163328 + 22242560) / 6
+ATTN_DRAM_BYTES_PER_HEAD = (330707456 + 22639360) / 6
 FRAMES_PER_CHUNK = 3
 CHUNK_LAYERS_PER_CHUNK = 30 * 4
 # stage -> (start event, end event) of the events wa_hsa_step records; the
