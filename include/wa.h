@@ -396,8 +396,10 @@ typedef struct wa_step_args {
  *   0 start | 1 after S0+S1 (page retrieval) | 2 after S2 (gather; = 1 when fused)
  *   3 after S3 (block selection) | 4 after S4a (projection) | 5 after S4b (linear
  *   branch) | 6 after the work list | 7 after S5+S6 (sparse branch + gate).
- * With bf16 inputs S4a and S4b run on a second stream that forks after event 2 and
- * joins before event 6, so events 4 and 5 are recorded on that stream. */
+ * With bf16 inputs the step forks two internal streams after event 2 and joins them
+ * before event 6: S4a and S4b run on one (events 4 and 5 are recorded there), S3 and
+ * the work list on the other, which has the device's highest stream priority (event 3
+ * is recorded there).  Events on different streams compare by time as usual. */
 #define WA_STEP_EVENTS 8
 
 WA_API size_t wa_hsa_step_workspace_size(const wa_step_args* a);
