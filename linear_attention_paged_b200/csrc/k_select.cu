@@ -324,6 +324,203 @@ k_block_choose(const double* __restrict__ scores, int n_qb, int n_kb, int lg_np,
   }
 }
 
+// The same choice for rows of at most 1024 key blocks, without a barrier per stage of
+// the sorting network: thread g of the row's NW warps holds positions g*E .. g*E+E-1
+// in registers (NP = 32 * NW * E), strides below E compare inside a thread, strides
+// below 32 E exchange with the partner lane by shuffles, and only larger ones (the
+// last stages of the last phases when NW > 1) go through shared memory.  Padding
+// positions carry score -inf and their own position as index, so the order stays
+// strict.  The masses, their prefix and the cut follow the block kernel above (sums
+// in another grouping: float64 rounding only).
+template <int E>
+__device__ __forceinline__ void ce_lane(double (&key)[E], int (&idx)[E], int a, int b, bool asc) {
+  // a < b inside the thread; asc: position a must hold the element that comes first
+  const bool b_first = key[b] > key[a] || (key[b] == key[a] && idx[b] < idx[a]);
+  const bool a_first = key[a] > key[b] || (key[a] == key[b] && idx[a] < idx[b]);
+  if (asc ? b_first : a_first) {
+    const double tk = key[a]; key[a] = key[b]; key[b] = tk;
+    const int ti = idx[a]; idx[a] = idx[b]; idx[b] = ti;
+  }
+}
+
+template <int E, int NW>
+__global__ void __launch_bounds__(32 * NW)
+k_block_choose_net(const double* __restrict__ scores, int n_qb, int n_kb, int W,
+                   const float* __restrict__ tau, int32_t* __restrict__ blk_idx,
+                   int32_t* __restrict__ blk_cnt, uint32_t* __restrict__ blk_mask, int n_h,
+                   int n_sub, int W_mask) {
+  constexpr int NT = 32 * NW;
+  constexpr int NP = NT * E;
+  constexpr int LGE = E >= 8 ? 3 : E >= 4 ? 2 : E >= 2 ? 1 : 0;
+  static_assert(E <= 8 && NP <= 1024, "positions per thread / row length");
+  __shared__ double xk[NW > 1 ? E * NT : 1];   // exchange of the cross-warp stages,
+  __shared__ int xi[NW > 1 ? E * NT : 1];      // position g*E+e at [e][g]
+  __shared__ double red_d[NW];
+  __shared__ int red_i[NW];
+  __shared__ uint32_t maskw[32];                 // selection blocks (n_kb <= 1024)
+  extern __shared__ uint32_t maskx[];            // [W_mask] (n_h > 0: B-row blocks)
+  const int h = blockIdx.y, i = blockIdx.x, g = threadIdx.x, lane = g & 31, warp = g >> 5;
+  const size_t rowid = static_cast<size_t>(h) * n_qb + i;
+  const double* srow = scores + rowid * n_kb;
+  const int p0 = g * E;
+  double key[E];
+  int idx[E];
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    key[e] = p0 + e < n_kb ? srow[p0 + e] : -INFINITY;
+    idx[e] = p0 + e;
+  }
+  for (int w = g; w < 32; w += NT) maskw[w] = 0u;
+  for (int w = g; w < W_mask && n_h > 0; w += NT) maskx[w] = 0u;
+  // phases k <= E: every stride is inside the thread
+#pragma unroll
+  for (int lk = 1; lk <= LGE; ++lk) {
+    const int k = 1 << lk;
+#pragma unroll
+    for (int lj = lk - 1; lj >= 0; --lj) {
+      const int j = 1 << lj;
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if ((e & j) == 0) ce_lane<E>(key, idx, e, e | j, ((p0 + e) & k) == 0);
+    }
+  }
+  // phases k > E: strides across threads (shared memory, then shuffles), then inside
+  for (int k = 2 * E; k <= NP; k <<= 1) {
+    const bool asc = (p0 & k) == 0;   // the same for the thread's E positions
+    for (int j = k >> 1; j >= E; j >>= 1) {
+      const int gm = j / E;           // partner thread g ^ gm
+      const bool keep_first = ((g & gm) == 0) == asc;
+      if (NW > 1 && gm >= 32) {
+        __syncthreads();              // the previous exchange has been read
+#pragma unroll
+        for (int e = 0; e < E; ++e) { xk[e * NT + g] = key[e]; xi[e * NT + g] = idx[e]; }
+        __syncthreads();
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const double ok = xk[e * NT + (g ^ gm)];
+          const int oi = xi[e * NT + (g ^ gm)];
+          const bool other_first = ok > key[e] || (ok == key[e] && oi < idx[e]);
+          if (keep_first == other_first) { key[e] = ok; idx[e] = oi; }
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < E; ++e) {
+          const double ok = __shfl_xor_sync(0xffffffffu, key[e], gm);
+          const int oi = __shfl_xor_sync(0xffffffffu, idx[e], gm);
+          const bool other_first = ok > key[e] || (ok == key[e] && oi < idx[e]);
+          if (keep_first == other_first) { key[e] = ok; idx[e] = oi; }
+        }
+      }
+    }
+#pragma unroll
+    for (int lj = LGE - 1; lj >= 0; --lj) {
+      const int j = 1 << lj;
+#pragma unroll
+      for (int e = 0; e < E; ++e)
+        if ((e & j) == 0) ce_lane<E>(key, idx, e, e | j, asc);
+    }
+  }
+  const double th = static_cast<double>(tau[h]);
+  int m = n_kb;
+  if (th < 1.0) {
+    if (g == 0) red_d[0] = key[0];    // position 0: the largest score
+    __syncthreads();
+    const double smax = red_d[0];
+    __syncthreads();
+    // z_t = exp(s_t - max) in place of the sorted scores, then p_t = z_t / Z
+    double zl = 0.0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const double z = p0 + e < n_kb ? exp(key[e] - smax) : 0.0;
+      key[e] = z;
+      zl += z;
+    }
+    zl = warp_sum(zl);
+    if (lane == 0) red_d[warp] = zl;
+    __syncthreads();
+    double Z = 0.0;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) Z += red_d[w];
+    __syncthreads();
+    double pl = 0.0;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      key[e] = key[e] / Z;
+      pl += key[e];
+    }
+    // exclusive prefix of the per-thread sums, in thread order
+    double incl = pl;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const double y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) red_d[warp] = incl;
+    double c = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) c = 0.0;
+    __syncthreads();
+    for (int w = 0; w < warp; ++w) c += red_d[w];
+    int first = INT_MAX;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      if (p0 + e < n_kb && first == INT_MAX) {
+        c += key[e];
+        if (c >= th) first = p0 + e;
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) first = min(first, __shfl_xor_sync(0xffffffffu, first, o));
+    if (lane == 0) red_i[warp] = first;
+    __syncthreads();
+    first = INT_MAX;
+#pragma unroll
+    for (int w = 0; w < NW; ++w) first = min(first, red_i[w]);
+    if (first != INT_MAX) m = first + 1;
+  }
+  __syncthreads();
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    if (p0 + e >= m) continue;
+    const int j = idx[e];
+    atomicOr(&maskw[j >> 5], 1u << (j & 31));
+    if (n_h > 0) {
+      // the same keys at B-row granularity: a 2B-row history block covers B-row blocks
+      // 2j and 2j + 1, a chunk block one
+      if (j < n_h) {
+        atomicOr(&maskx[(2 * j) >> 5], 1u << ((2 * j) & 31));
+        if (2 * j + 1 < n_sub) atomicOr(&maskx[(2 * j + 1) >> 5], 1u << ((2 * j + 1) & 31));
+      } else {
+        const int x = n_sub + (j - n_h);
+        atomicOr(&maskx[x >> 5], 1u << (x & 31));
+      }
+    }
+  }
+  __syncthreads();
+  if (blk_mask) {
+    const uint32_t* src = n_h > 0 ? maskx : maskw;
+    for (int w = g; w < W_mask; w += NT) blk_mask[rowid * W_mask + w] = src[w];
+  }
+  if (warp == 0) {
+    // W <= 32: one mask word per lane of the first warp
+    const uint32_t bits0 = lane < W ? maskw[lane] : 0u;
+    const int cnt = __popc(bits0);
+    int incl = cnt;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    const int total = __shfl_sync(0xffffffffu, incl, 31);
+    if (blk_cnt && lane == 0) blk_cnt[rowid] = total;
+    if (blk_idx) {
+      int32_t* out = blk_idx + rowid * n_kb;
+      int pos = incl - cnt;
+      for (uint32_t bits = bits0; bits != 0u; bits &= bits - 1u) out[pos++] = lane * 32 + __ffs(bits) - 1;
+      for (int t = total + lane; t < n_kb; t += 32) out[t] = -1;
+    }
+  }
+}
+
 }  // namespace
 
 // ==================================================================== launchers
@@ -367,6 +564,26 @@ wa_status launch_block_select(const double* q_blockmean, int Nq, int H, int d, i
       q_blockmean, km, n_qb, n_kb, H, d, B, scores);
   int lg = 5;
   while ((1 << lg) < n_kb) ++lg;
+  const int wm = km.pair ? W_mask : W;
+  if (lg <= 10) {
+    // rows of at most 1024 key blocks: the network in registers, 1, 2 or 4 warps a row
+    const size_t smem_w = static_cast<size_t>(W_mask) * 4;
+    const dim3 grid(n_qb, H);
+    const int nh = km.pair ? km.n_kb1 : 0;
+#define WA_CHOOSE(E_, NW_) \
+  k_block_choose_net<E_, NW_><<<grid, 32 * NW_, smem_w, st>>>(scores, n_qb, n_kb, W, tau, blk_idx, \
+                                                              blk_cnt, blk_mask, nh, km.n_sub, wm)
+    switch (lg) {
+      case 5: WA_CHOOSE(1, 1); break;
+      case 6: WA_CHOOSE(2, 1); break;
+      case 7: WA_CHOOSE(4, 1); break;
+      case 8: WA_CHOOSE(8, 1); break;
+      case 9: WA_CHOOSE(8, 2); break;
+      default: WA_CHOOSE(8, 4); break;
+    }
+#undef WA_CHOOSE
+    return check_launch("block_select");
+  }
   const size_t smem_c = (static_cast<size_t>(1) << lg) * 12 + static_cast<size_t>(W + W_mask) * 4 + 16;
   e = cudaFuncSetAttribute(k_block_choose, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            static_cast<int>(smem_c));

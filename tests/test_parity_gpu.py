@@ -151,6 +151,42 @@ def test_block_select_limits(wa):
                     assert gpu[h][i] == [int(np.argmax(s[h, i]))]
 
 
+@pytest.mark.parametrize("n_kb", [1, 7, 32, 33, 64, 100, 128, 200, 256, 300, 512, 700, 1024, 1025,
+                                  1500])
+def test_block_select_key_list_lengths(wa, n_kb):
+    """The block choice at every class of key-list length: rows of up to 1024 blocks
+    are sorted by one warp (1 to 32 positions per lane), longer ones by a whole CTA.
+    Every row of a key block is the same, so a block's mean is exact; repeated blocks
+    give bit-identical scores on both sides (exact ties, broken towards the lower
+    block) and zero blocks scores of +-0.  Every row must match the oracle exactly."""
+    g = torch.Generator().manual_seed(500 + n_kb)
+    H, d, B = 2, 64, 64
+    Nq = 3 * B - 5
+    q = torch.randn(Nq, H, d, generator=g).to(torch.bfloat16)
+    rows = torch.randn(n_kb, H, d, generator=g)
+    for j in range(n_kb):
+        if j % 5 == 4:
+            rows[j] = rows[j // 2]
+        if j % 7 == 6:
+            rows[j] = 0.0
+    k_act = rows.to(torch.bfloat16).repeat_interleave(B, dim=0)
+    n_qb = -(-Nq // B)
+    for tau_vals in ((0.9, 0.3), (0.6, 0.97), (1e-9, 1.0)):
+        tau = torch.tensor(tau_vals, dtype=torch.float32)
+        kept, _ = O.block_select(q, k_act, tau, B)
+        idx, cnt, mask = wa.wa_block_select(q.cuda(), tau.cuda(), B, k_act=k_act.cuda())
+        gpu = mask_to_sets(mask, n_kb)
+        idx_c, cnt_c = idx.cpu().numpy(), cnt.cpu().numpy()
+        for h in range(H):
+            for i in range(n_qb):
+                assert gpu[h][i] == kept[h][i], (n_kb, tau_vals, h, i)
+                c = int(cnt_c[h, i])
+                assert c == len(kept[h][i])
+                assert idx_c[h, i, :c].tolist() == kept[h][i]
+                assert (idx_c[h, i, c:] == -1).all()
+    check_device_ok(wa)
+
+
 # ---------------------------------------------------------------- S4a
 @pytest.mark.parametrize("cfg", [W.C0, SMALL_BF16, SMALL_BF16_D64, SMALL_F32], ids=lambda c: c.name)
 def test_linear_project(wa, cfg):
